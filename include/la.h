@@ -1,0 +1,144 @@
+/*
+ * la.h — C ABI of the Lightning Attention layer kernel for NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  The linear-attention layer of the hybrid Lightning Attention + MLA stack
+ * described in "Ling and Ring 2.6 Technical Report" (Chinese translation,
+ * garden.houmin.site/digest/ling-ring-2.6): §2.1, Fig. 2 places a "Linear Attention Kernel" between
+ * QK-Norm/RoPE and a grouped RMSNorm with a sigmoid gate; §4.1.1 ("Context Parallel for Lightning
+ * Attention") describes it as an RNN-style recurrence whose per-rank hidden state is shaped
+ * [B,H,D,D].  The recurrence itself is the decayed causal linear attention of Lightning Attention
+ * (TransNormerLLM, the report's reference 7), which the pages name but do not print:
+ *
+ *     S_t = lambda_h * S_{t-1} + k_t^T v_t          (S is d x d, S_{-1} = 0)
+ *     o_t = q_t S_t  =  sum_{s<=t} lambda_h^(t-s) (q_t . k_s) v_s
+ *
+ * with lambda_h = exp(-slope_h).  No softmax, normaliser or scale is applied inside the kernel (the
+ * report normalises the output afterwards, in the grouped RMSNorm of Fig. 2).
+ *
+ * Conventions shared by every entry point.
+ *   - All tensor pointers are DEVICE pointers (cudaMalloc / PyTorch CUDA memory) unless a
+ *     parameter says otherwise.  The caller owns every buffer; the library keeps no allocations,
+ *     handles or global state between calls.
+ *   - Activations q, k, v, out are laid out token-major, [B, N, H, d] contiguous (d innermost),
+ *     as a fused QKV projection writes them.  Element type is bf16 (LA_BF16) or fp32 (LA_F32).
+ *   - The recurrent state is always fp32, [B, H, d, d] contiguous, S[b][h][i][j] with i over the
+ *     key dimension and j over the value dimension.
+ *   - slopes: fp32[H] device array, slope_h >= 0, the decay is lambda_h = exp(-slope_h).
+ *   - stream: a cudaStream_t passed as void*; NULL means the legacy default stream.  Calls are
+ *     stream-ordered and asynchronous: a return of LA_OK means the work was enqueued.
+ *   - Base pointers of q, k, v, out must be 16-byte aligned (tensor-memory-accelerator rule);
+ *     otherwise LA_ERR_ALIGN.  out must not overlap q, k or v (LA_ERR_ALIAS).
+ *   - Argument errors are reported synchronously before anything is enqueued.  Launch errors
+ *     map to LA_ERR_CUDA.  Nothing in the library calls exit(), abort() or a device trap.
+ *   - All sizes and index arithmetic are 64-bit.
+ */
+#ifndef LA_H_
+#define LA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LA_VERSION 1000 /* major*1000 + minor */
+
+typedef enum {
+  LA_OK = 0,
+  LA_ERR_NULL = -1,        /* a required pointer is NULL */
+  LA_ERR_SHAPE = -2,       /* B, N, H or d out of range (N >= 1, d in {64,128}, ...) */
+  LA_ERR_DTYPE = -3,       /* dtype not LA_BF16 / LA_F32 */
+  LA_ERR_ALIGN = -4,       /* a base pointer is not 16-byte aligned */
+  LA_ERR_OVERFLOW = -5,    /* B*N*H*d or a byte size does not fit the 64-bit / tensor-map limits */
+  LA_ERR_WORKSPACE = -6,   /* workspace too small (see la_prefill_workspace_bytes) */
+  LA_ERR_CUDA = -7,        /* a CUDA runtime/driver call failed */
+  LA_ERR_TIMEOUT = -8,     /* a device-side bounded wait gave up (reported by la_workspace_status) */
+  LA_ERR_UNSUPPORTED = -9, /* valid arguments, but no kernel for this combination (e.g. chunk) */
+  LA_ERR_ALIAS = -10       /* out overlaps an input */
+} la_status;
+
+typedef enum { LA_BF16 = 0, LA_F32 = 1 } la_dtype;
+
+/* Which prefill kernel runs.  AUTO picks the tensor-core chunked kernel for bf16 with d = 128 and
+ * the recurrent kernel otherwise.  RECURRENT forces the token-by-token CUDA-core kernel (any dtype
+ * and d), which is also the fp32 path; TENSOR forces the chunked tcgen05 kernel (bf16, d = 128). */
+typedef enum { LA_PATH_AUTO = 0, LA_PATH_TENSOR = 1, LA_PATH_RECURRENT = 2 } la_path;
+
+/* Problem descriptor for la_prefill. */
+typedef struct {
+  int64_t B;        /* batch (independent sequences), >= 1 */
+  int64_t N;        /* tokens per sequence, >= 1 */
+  int64_t H;        /* heads, >= 1 */
+  int64_t d;        /* head dimension, d_k = d_v = d, 64 or 128 */
+  int32_t dtype;    /* la_dtype of q, k, v, out */
+  int32_t chunk;    /* chunk length C of the tensor-core path: 0 = default (128); 128 supported */
+  int32_t segments; /* segments per sequence: 0 = automatic; >= 1 explicit (clamped to chunks) */
+  int32_t path;     /* la_path */
+} la_desc;
+
+/* Bytes of device workspace la_prefill needs for this descriptor (0 if none).  The workspace holds
+ * the segment-state ring, the scan flags, a work counter and a device status word. */
+size_t la_prefill_workspace_bytes(const la_desc* desc);
+
+/*
+ * la_prefill — the whole prefill of one layer: o for every token and the final state.
+ *
+ * Chunked evaluation of the recurrence above ("chunk QKV", Fig. 10 of §4.1.1): within a chunk of
+ * C tokens the intra-chunk term (Q K^T ⊙ M) V with M_ij = lambda^(i-j) (i >= j, else 0) and the
+ * inter-chunk term diag(lambda^(i+1)) Q KV are tensor-core contractions; the fp32 state is carried
+ * as KV <- lambda^C KV + (K ⊙ lambda^(C-1-i))^T V.  Long sequences are cut into segments whose
+ * local states are combined by a decayed prefix scan, the single-GPU form of the report's
+ * "local recurrence, then global correction" (§4.1.1, Fig. 10: local h, fused update h / O).
+ *
+ *   desc       problem shape and options (host pointer, read during the call only)
+ *   q, k, v    [B, N, H, d] device, dtype desc->dtype, read only
+ *   slopes     fp32[H] device, read only
+ *   out        [B, N, H, d] device, dtype desc->dtype, written (o_t for every token)
+ *   state_out  fp32 [B, H, d, d] device, written (S_{N-1}); may be NULL if not wanted
+ *   workspace  device scratch of at least la_prefill_workspace_bytes(desc) bytes, 256-byte aligned,
+ *              used exclusively by this call until it completes on `stream`.  May be NULL: the
+ *              library then allocates and frees it on `stream` (cudaMallocAsync/cudaFreeAsync).
+ *   stream     cudaStream_t as void*
+ *
+ * Returns LA_OK when enqueued.  A device-side timeout of the segment scan (a bounded wait that
+ * gave up; it cannot occur unless the GPU is starved for seconds) is recorded in the workspace's
+ * status word, readable with la_workspace_status().
+ */
+la_status la_prefill(const la_desc* desc, const void* q, const void* k, const void* v,
+                     const float* slopes, void* out, float* state_out, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/*
+ * la_decode_step — one generated token for B sequences: for every (b, h)
+ *     S <- lambda_h S + k^T v   (in place, fp32),   o = q S   (read out after the update)
+ * This is the per-token RNN-style update of §4.1.1; the state it continues is la_prefill's
+ * state_out (prefix caching in the report's serving path).
+ *
+ *   B, H, d       batch, heads, head dim (64 or 128)
+ *   dtype         la_dtype of q, k, v, out
+ *   q, k, v       [B, H, d] device, read only
+ *   slopes        fp32[H] device
+ *   state_inout   fp32 [B, H, d, d] device, read and written in place
+ *   out           [B, H, d] device, written
+ *   stream        cudaStream_t as void*
+ */
+la_status la_decode_step(int64_t B, int64_t H, int64_t d, int32_t dtype, const void* q,
+                         const void* k, const void* v, const float* slopes, float* state_inout,
+                         void* out, void* stream);
+
+/* Synchronises `stream`, then returns the device status word of a workspace that la_prefill
+ * used: LA_OK, or LA_ERR_TIMEOUT if a bounded device wait gave up during the last call. */
+la_status la_workspace_status(const void* workspace, void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* la_status_string(int status);
+
+/* LA_VERSION of the built library. */
+int la_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_H_ */

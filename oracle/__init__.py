@@ -1,0 +1,156 @@
+"""fp64 CPU oracle of the Lightning Attention layer kernel — TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may import this
+package.  The product path (``long_context_attention_la_b200``) never imports it, and this package
+imports nothing from the product: the two share no code.
+
+The arithmetic lives in ``la_oracle.c`` (plain C, fp64, OpenMP over heads).  This module only
+compiles it (``build()``) and marshals numpy arrays through ``ctypes``.
+
+Source of the method: "Ling and Ring 2.6 Technical Report" (Chinese translation,
+garden.houmin.site), §4.1.1 (linear attention as an RNN-style recurrence with a [B,H,D,D] state)
+and §2.1 Fig. 2 (kernel placement, no normaliser inside); the decayed recurrence
+``S_t = lambda S_{t-1} + k_t^T v_t, o_t = q_t S_t`` is Lightning Attention's (the report's
+reference 7), which the pages name without printing it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "la_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "libla_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+BF16 = 0
+F32 = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile la_oracle.c into oracle/_build/libla_oracle.so (gcc, -O2, no fast-math)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    return compile_source(_SRC, _LIB_PATH)
+
+
+def open_library(path: str):
+    """ctypes handle of a compiled oracle library with its signatures declared."""
+    lib = ctypes.CDLL(path)
+    i64, p, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+    lib.la_oracle_prefill.argtypes = [i64, i64, i64, i64, i32, p, p, p, p, p, i64, p, i64,
+                                      p, p, p, i32]
+    lib.la_oracle_prefill.restype = i32
+    lib.la_oracle_decode.argtypes = [i64, i64, i64, i32, p, p, p, p, p, p, i32]
+    lib.la_oracle_decode.restype = i32
+    lib.orc_num_threads.argtypes = [i32]
+    lib.orc_num_threads.restype = i32
+    return lib
+
+
+def compile_source(src: str, out_path: str) -> str:
+    """Compile an oracle C source with the oracle's own flags (used by build() and by the tests
+    that check the pins reject deliberately broken copies of the source)."""
+    tmp = out_path + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-shared", "-fPIC",
+           "-std=c11", "-o", tmp, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out_path)
+    return out_path
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = open_library(build())
+    return _lib
+
+
+def num_threads(requested: int = 0) -> int:
+    """OpenMP threads the oracle uses for a call with ``nthreads=requested``."""
+    return int(_load().orc_num_threads(int(requested)))
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    # bf16 tensors are passed as their raw uint16 bit patterns.
+    if a.dtype == np.uint16:
+        return BF16
+    if a.dtype == np.float32:
+        return F32
+    raise TypeError(f"oracle inputs must be uint16 (bf16 bits) or float32, got {a.dtype}")
+
+
+def _ptr(a):
+    return None if a is None else ctypes.c_void_p(a.ctypes.data)
+
+
+def prefill(q, k, v, slopes, heads=None, t_sel=None, state_in=None, nthreads: int = 0, lib=None):
+    """Run the fp64 recurrence.
+
+    q, k, v: [B, N, H, d] arrays, uint16 (bf16 bits) or float32, C-contiguous.
+    slopes: float32[H] (decay lambda_h = exp(-slope_h)).
+    heads: optional int64 list of flat head indices b*H+h to evaluate (default: all, in order).
+    t_sel: optional sorted int64 list of token indices whose outputs to record (default: all).
+    state_in: optional float64 [n_heads, d, d] initial state (default zero).
+    lib: optional handle from open_library() (default: the built oracle).
+    Returns (o, state): o float64 [n_heads, n_t, d], state float64 [n_heads, d, d].
+    """
+    q = np.ascontiguousarray(q)
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    if not (q.shape == k.shape == v.shape) or q.ndim != 4:
+        raise ValueError("q, k, v must share one [B, N, H, d] shape")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    B, N, H, d = q.shape
+    slopes = np.ascontiguousarray(slopes, dtype=np.float32)
+    if slopes.shape != (H,):
+        raise ValueError("slopes must be float32[H]")
+    heads_a = None if heads is None else np.ascontiguousarray(heads, dtype=np.int64)
+    n_sel = B * H if heads_a is None else int(heads_a.size)
+    t_a = None if t_sel is None else np.ascontiguousarray(t_sel, dtype=np.int64)
+    if t_a is not None and (np.any(np.diff(t_a) <= 0) or (t_a.size and (t_a[0] < 0 or t_a[-1] >= N))):
+        raise ValueError("t_sel must be strictly increasing token indices in [0, N)")
+    n_t = N if t_a is None else int(t_a.size)
+    o = np.zeros((n_sel, n_t, d), dtype=np.float64)
+    state = np.zeros((n_sel, d, d), dtype=np.float64)
+    sin = None
+    if state_in is not None:
+        sin = np.ascontiguousarray(state_in, dtype=np.float64)
+        if sin.shape != (n_sel, d, d):
+            raise ValueError("state_in must be float64 [n_heads, d, d]")
+    rc = (lib or _load()).la_oracle_prefill(B, N, H, d, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+                                   _ptr(slopes), _ptr(heads_a), 0 if heads_a is None else n_sel,
+                                   _ptr(t_a), n_t, _ptr(o), _ptr(state), _ptr(sin), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("la_oracle_prefill rejected its arguments")
+    return o, state
+
+
+def decode(q, k, v, slopes, state, nthreads: int = 0):
+    """One decode step.  q, k, v: [B, H, d] (uint16 bf16 bits or float32); state: float64
+    [B, H, d, d], updated IN PLACE.  Returns o float64 [B, H, d]."""
+    q = np.ascontiguousarray(q)
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    if not (q.shape == k.shape == v.shape) or q.ndim != 3:
+        raise ValueError("q, k, v must share one [B, H, d] shape")
+    B, H, d = q.shape
+    if state.dtype != np.float64 or state.shape != (B, H, d, d) or not state.flags.c_contiguous:
+        raise ValueError("state must be a C-contiguous float64 [B, H, d, d] array")
+    slopes = np.ascontiguousarray(slopes, dtype=np.float32)
+    o = np.zeros((B, H, d), dtype=np.float64)
+    rc = _load().la_oracle_decode(B, H, d, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(slopes), _ptr(state), _ptr(o), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("la_oracle_decode rejected its arguments")
+    return o

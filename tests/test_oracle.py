@@ -1,0 +1,240 @@
+"""Pins of the fp64 oracle against things other than itself (CPU only).
+
+The report (Ling and Ring 2.6 Technical Report, Chinese translation, garden.houmin.site) prints
+no numeric example for the kernel, so the oracle is pinned by:
+  * hand-derived worked examples (tests/golden/hand_cases.json);
+  * the textbook O(N^2) form  o_t = sum_{s<=t} lambda^(t-s) (q_t . k_s) v_s  (numpy, fp64, with
+    lambda^(t-s) from exp, not from repeated multiplication), and the state
+    S = sum_s lambda^(N-1-s) k_s^T v_s;
+  * closed forms: lambda = 1 is a causal cumulative sum of outer products; lambda = 0 keeps only
+    the diagonal; N = 1 is (q.k) v;
+  * invariants: linearity in v and q, prefix causality, decode-after-prefill, resume from a state.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_attention_la_b200 import synth
+from tests.helpers import oracle_bits
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_cases.json")
+
+
+def _f32(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+def _rand(B, N, H, d, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    return tuple(_f32(rng.standard_normal((B, N, H, d)) * scale) for _ in range(3))
+
+
+def brute_force(q, k, v, slopes):
+    """O(N^2) decayed masked attention in fp64 (independent of the recurrence)."""
+    q = q.astype(np.float64)
+    k = k.astype(np.float64)
+    v = v.astype(np.float64)
+    B, N, H, d = q.shape
+    o = np.zeros((B, N, H, d))
+    st = np.zeros((B, H, d, d))
+    t = np.arange(N)
+    for b in range(B):
+        for h in range(H):
+            s = float(np.float32(slopes[h]))
+            diff = t[:, None] - t[None, :]
+            decay = np.where(diff >= 0, np.exp(-np.maximum(diff, 0) * s), 0.0)
+            A = (q[b, :, h, :] @ k[b, :, h, :].T) * decay
+            o[b, :, h, :] = A @ v[b, :, h, :]
+            w = np.exp(-(N - 1 - t) * s)
+            st[b, h] = (k[b, :, h, :] * w[:, None]).T @ v[b, :, h, :]
+    return o, st
+
+
+def run_oracle(q, k, v, slopes, **kw):
+    B, N, H, d = q.shape
+    o, st = oracle.prefill(q, k, v, _f32(slopes), **kw)
+    return o.reshape(B, H, -1, d).transpose(0, 2, 1, 3), st.reshape(B, H, d, d)
+
+
+def test_oracle_builds():
+    assert os.path.exists(oracle.build())
+    assert oracle.num_threads(3) == 3
+
+
+@pytest.mark.parametrize("case", json.load(open(GOLDEN))["cases"], ids=lambda c: c["name"])
+def test_hand_cases(case):
+    B, N, H, d = case["B"], case["N"], case["H"], case["d"]
+    q = _f32(case["q"]).reshape(B, N, H, d)
+    k = _f32(case["k"]).reshape(B, N, H, d)
+    v = _f32(case["v"]).reshape(B, N, H, d)
+    o, st = run_oracle(q, k, v, case["slopes"])
+    exp_o = np.asarray(case["o"], dtype=np.float64).reshape(B, N, H, d)
+    exp_s = np.asarray(case["state"], dtype=np.float64).reshape(B, H, d, d)
+    np.testing.assert_allclose(o, exp_o, rtol=case["rtol"], atol=0)
+    np.testing.assert_allclose(st, exp_s, rtol=case["rtol"], atol=0)
+
+
+@pytest.mark.parametrize("B,N,H,d,seed", [(1, 1, 1, 4, 0), (2, 37, 3, 4, 1), (1, 300, 2, 64, 2),
+                                          (1, 512, 1, 4, 3), (2, 129, 4, 8, 4)])
+def test_brute_force(B, N, H, d, seed):
+    q, k, v = _rand(B, N, H, d, seed)
+    sl = synth.slopes(H).numpy()
+    o, st = run_oracle(q, k, v, sl)
+    ob, sb = brute_force(q, k, v, sl)
+    scale_o = np.max(np.abs(ob))
+    scale_s = np.max(np.abs(sb))
+    assert np.max(np.abs(o - ob)) <= 1e-12 * max(scale_o, 1.0) * np.sqrt(N)
+    assert np.max(np.abs(st - sb)) <= 1e-12 * max(scale_s, 1.0) * np.sqrt(N)
+
+
+def test_brute_force_wide_slopes():
+    # Slopes spanning no decay to fast decay in one call, with per-head checks.
+    B, N, H, d = 1, 200, 4, 16
+    q, k, v = _rand(B, N, H, d, 11)
+    sl = np.array([0.0, 1e-3, 0.3, 2.0], dtype=np.float32)
+    o, st = run_oracle(q, k, v, sl)
+    ob, sb = brute_force(q, k, v, sl)
+    for h in range(H):
+        np.testing.assert_allclose(o[:, :, h], ob[:, :, h], rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(st[:, h], sb[:, h], rtol=1e-11, atol=1e-11)
+
+
+def test_lambda_one_is_causal_cumsum():
+    B, N, H, d = 1, 64, 2, 8
+    q, k, v = _rand(B, N, H, d, 5)
+    sl = np.zeros(H, dtype=np.float32)
+    o, st = run_oracle(q, k, v, sl)
+    qd, kd, vd = (x.astype(np.float64) for x in (q, k, v))
+    outer = np.einsum("bnhi,bnhj->bnhij", kd, vd)
+    C = np.cumsum(outer, axis=1)
+    expect = np.einsum("bnhi,bnhij->bnhj", qd, C)
+    np.testing.assert_allclose(o, expect, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(st, C[:, -1], rtol=1e-12, atol=1e-12)
+
+
+def test_lambda_zero_keeps_diagonal():
+    B, N, H, d = 2, 17, 2, 8
+    q, k, v = _rand(B, N, H, d, 6)
+    sl = np.full(H, 1e4, dtype=np.float32)  # exp(-1e4) underflows to exactly 0 in double
+    o, st = run_oracle(q, k, v, sl)
+    qd, kd, vd = (x.astype(np.float64) for x in (q, k, v))
+    diag = np.einsum("bnhi,bnhi->bnh", qd, kd)[..., None] * vd
+    np.testing.assert_allclose(o, diag, rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(st, np.einsum("bhi,bhj->bhij", kd[:, -1], vd[:, -1]), rtol=0, atol=0)
+
+
+def test_single_token():
+    q, k, v = _rand(3, 1, 2, 16, 7)
+    o, st = run_oracle(q, k, v, synth.slopes(2).numpy())
+    qd, kd, vd = (x.astype(np.float64) for x in (q, k, v))
+    np.testing.assert_allclose(o[:, 0], np.einsum("bhi,bhi->bh", qd[:, 0], kd[:, 0])[..., None]
+                               * vd[:, 0], rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(st, np.einsum("bhi,bhj->bhij", kd[:, 0], vd[:, 0]), rtol=0, atol=0)
+
+
+def test_linearity():
+    q, k, v = _rand(1, 50, 2, 8, 8)
+    sl = synth.slopes(2).numpy()
+    o, st = run_oracle(q, k, v, sl)
+    o2, st2 = run_oracle(q, k, _f32(2 * v), sl)          # scaling by 2 is exact
+    np.testing.assert_array_equal(o2, 2 * o)
+    np.testing.assert_array_equal(st2, 2 * st)
+    o3, _ = run_oracle(_f32(2 * q), k, v, sl)
+    np.testing.assert_array_equal(o3, 2 * o)
+    # additivity in v (catches a dropped term that scaling alone would not); values on a 2^-10
+    # grid so that v + w is exact in float32
+    _, _, w = _rand(1, 50, 2, 8, 9)
+    vg = _f32(np.round(v * 1024) / 1024)
+    wg = _f32(np.round(w * 1024) / 1024)
+    assert np.array_equal(_f32(vg + wg).astype(np.float64), vg.astype(np.float64) + wg)
+    og, _ = run_oracle(q, k, vg, sl)
+    oa, _ = run_oracle(q, k, wg, sl)
+    ob, _ = run_oracle(q, k, _f32(vg + wg), sl)
+    np.testing.assert_allclose(ob, og + oa, rtol=1e-12, atol=1e-12)
+
+
+def test_prefix_causality():
+    q, k, v = _rand(2, 90, 2, 8, 10)
+    sl = synth.slopes(2).numpy()
+    o, _ = run_oracle(q, k, v, sl)
+    o_short, _ = run_oracle(*(np.ascontiguousarray(x[:, :33]) for x in (q, k, v)), sl)
+    np.testing.assert_array_equal(o[:, :33], o_short)
+
+
+def test_bf16_bits_upcast_exactly():
+    t = torch.randn(1, 20, 2, 8, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    bits = oracle_bits(t)
+    as_f32 = t.float().numpy()
+    sl = synth.slopes(2).numpy()
+    o1, s1 = run_oracle(bits, bits, bits, sl)
+    o2, s2 = run_oracle(as_f32, as_f32, as_f32, sl)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(s1, s2)
+
+
+def test_decode_equals_prefill():
+    B, N, H, d = 2, 12, 3, 8
+    q, k, v = _rand(B, N, H, d, 12)
+    sl = synth.slopes(H).numpy()
+    o, st = run_oracle(q, k, v, sl)
+    S = np.zeros((B, H, d, d))
+    for t in range(N):
+        ot = oracle.decode(q[:, t], k[:, t], v[:, t], sl, S)
+        np.testing.assert_array_equal(ot, o[:, t])
+    np.testing.assert_array_equal(S, st)
+
+
+def test_resume_from_state():
+    B, N, H, d = 1, 40, 2, 8
+    q, k, v = _rand(B, N, H, d, 13)
+    sl = synth.slopes(H).numpy()
+    o, st = run_oracle(q, k, v, sl)
+    n1 = 15
+    _, s1 = oracle.prefill(*(np.ascontiguousarray(x[:, :n1]) for x in (q, k, v)), sl)
+    o2, s2 = oracle.prefill(*(np.ascontiguousarray(x[:, n1:]) for x in (q, k, v)), sl, state_in=s1)
+    np.testing.assert_array_equal(o2.reshape(B, H, -1, d).transpose(0, 2, 1, 3), o[:, n1:])
+    np.testing.assert_array_equal(s2.reshape(B, H, d, d), st)
+
+
+def test_head_and_token_selection():
+    B, N, H, d = 2, 30, 3, 4
+    q, k, v = _rand(B, N, H, d, 14)
+    sl = synth.slopes(H).numpy()
+    o_all, st_all = oracle.prefill(q, k, v, sl)
+    heads = [5, 1, 3]
+    tsel = [0, 7, 29]
+    o_sel, st_sel = oracle.prefill(q, k, v, sl, heads=heads, t_sel=tsel, nthreads=2)
+    np.testing.assert_array_equal(o_sel, o_all[heads][:, tsel])
+    np.testing.assert_array_equal(st_sel, st_all[heads])
+
+
+def test_thread_count_invariance():
+    q, k, v = _rand(1, 64, 8, 8, 15)
+    sl = synth.slopes(8).numpy()
+    a = oracle.prefill(q, k, v, sl, nthreads=1)
+    b = oracle.prefill(q, k, v, sl, nthreads=4)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_rejects_bad_arguments():
+    q, k, v = _rand(1, 4, 2, 4, 16)
+    with pytest.raises(ValueError):
+        oracle.prefill(q, k, v, np.zeros(3, np.float32))
+    with pytest.raises(ValueError):
+        oracle.prefill(q, k, v, np.zeros(2, np.float32), t_sel=[3, 1])
+    with pytest.raises(TypeError):
+        oracle.prefill(q.astype(np.float64), k, v, np.zeros(2, np.float32))
+
+
+def test_slope_schedule_values():
+    # Decays quoted for the schedule s_h = 2^(-8(h+1)/H): H=64 -> 0.39972 .. 0.99610,
+    # H=2 -> 0.93941, 0.99610.
+    lam64 = np.exp(-synth.slopes(64).double().numpy())
+    lam2 = np.exp(-synth.slopes(2).double().numpy())
+    assert abs(lam64[0] - 0.39972) < 1e-5 and abs(lam64[63] - 0.99610) < 1e-5
+    assert abs(lam2[0] - 0.93941) < 1e-5 and abs(lam2[1] - 0.99610) < 1e-5
