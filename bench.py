@@ -1,0 +1,424 @@
+"""Benchmark of the Lightning Attention layer kernel (prefill + decode step) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill_32k|prefill_4k|prefill_256k]
+
+One step = one whole pass of the hot path over one batch of synthetic input:
+  * la_prefill of the prefill workload (default: B=2, N=32768, H=64, d=128, bf16, seed 1), which
+    writes o for every token and the final fp32 state;
+  * one la_decode_step of 256 sequences x 64 heads x d=128 on a resident fp32 state (2 GiB).
+The JSON line's ``value`` is prefill tokens/s (tokens = B*N positions, all 64 heads) summed over
+ranks; the decode step is reported under ``decode`` as state GB/s.  Under torchrun each rank runs
+an independent replica (weak scaling, no collective on the data path).
+
+Timing: W untimed warm-up steps, then K steps between a barrier + device synchronize on both
+sides, CUDA events on the launching stream, max over ranks.  Inputs are larger than L2 (4 GiB of
+prefill activations, 2 GiB of decode state), so no flush is needed between steps.
+
+``--impl reference`` times the fp64 CPU oracle (test infrastructure) on the host cores instead:
+a bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from long_context_attention_la_b200 import synth  # noqa: E402
+
+METRIC = "lightning-attn prefill tok/s & TFLOP/s (H=64,d=128); decode state GB/s vs peak"
+DECODE = dict(B=256, H=64, d=128)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# --------------------------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------------------------
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--id={self.index}",
+               "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+               "--format=csv,noheader,nounits", "-lms", "100"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            if self.thread:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                s, m = float(parts[0]), float(parts[1])
+                bits = int(parts[3], 16)
+            except ValueError:
+                continue
+            sm.append(s)
+            mx = m
+            for b, name in REASON_BITS.items():
+                if bits & b and name != "gpu_idle":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# --------------------------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_teardown(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on the host cores, bounded sample
+# --------------------------------------------------------------------------------------------
+def oracle_sample(w, seconds_target=15.0):
+    """Times the oracle on n_threads heads x n_tok tokens of the workload's distribution.
+    Returns (tok/s scaled to the workload's all-heads token, cores, description)."""
+    import numpy as np
+
+    import oracle
+    cores = oracle.num_threads()
+    n_heads = cores
+    # ~2 * 2 * d^2 fp64 flops per token-head; aim at about seconds_target of CPU time
+    n_tok = min(w.N, 8192)
+    q, k, v = synth.draw_qkv(1, n_tok, n_heads, w.d, dist=w.dist, seed=w.seed, dtype=w.dtype)
+    bits = [x.view(torch.int16).numpy().view(np.uint16) for x in (q, k, v)]
+    sl = synth.slopes(w.H).numpy()[:n_heads] if n_heads <= w.H else np.resize(
+        synth.slopes(w.H).numpy(), n_heads)
+    t0 = time.perf_counter()
+    oracle.prefill(*bits, sl.astype(np.float32), nthreads=cores)
+    dt = time.perf_counter() - t0
+    reps = max(1, int(seconds_target / max(dt, 1e-3)))
+    reps = min(reps, 64)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.prefill(*bits, sl.astype(np.float32), nthreads=cores)
+    dt = (time.perf_counter() - t0) / reps
+    token_heads_per_s = n_heads * n_tok / dt
+    desc = (f"fp64 oracle, {n_heads} heads x {n_tok} tokens of the {w.name} distribution "
+            f"({reps} reps, {dt:.2f} s each); tok/s = token-heads/s / H={w.H}")
+    return token_heads_per_s / w.H, cores, desc
+
+
+# --------------------------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------------------------
+def run_ours(args):
+    from long_context_attention_la_b200 import build as labuild
+    from long_context_attention_la_b200 import la
+
+    labuild.build()
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[args.workload]
+    B, N, H, d = w.B, w.N, w.H, w.d
+    q, k, v = synth.draw_qkv(B, N, H, d, dist=w.dist, seed=w.seed + 1000 * rank, dtype=w.dtype,
+                             device=dev)
+    sl = synth.slopes(H, dev)
+    out = torch.empty_like(q)
+    st = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+    desc = la.make_desc(B, N, H, d, w.dtype)
+    ws_bytes = la.la_prefill_workspace_bytes(desc)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+
+    Bd, Hd, dd = DECODE["B"], DECODE["H"], DECODE["d"]
+    dstate = torch.randn(Bd, Hd, dd, dd, dtype=torch.float32, device=dev) * 0.05
+    gdec = synth.decode_token_generator(4 + 1000 * rank, dev)
+    dq, dk, dv = synth.draw_decode_token(gdec, Bd, Hd, dd, device=dev)
+    dout = torch.empty_like(dq)
+    dsl = synth.slopes(Hd, dev)
+
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+
+    def prefill_call():
+        rc = la.la_prefill(desc, q.data_ptr(), k.data_ptr(), v.data_ptr(), sl.data_ptr(),
+                           out.data_ptr(), st.data_ptr(), ws.data_ptr(), ws_bytes, sp)
+        if rc != la.LA_OK:
+            raise la.LaError(rc, "la_prefill")
+
+    def decode_call():
+        rc = la.la_decode_step(Bd, Hd, dd, la.LA_BF16, dq.data_ptr(), dk.data_ptr(),
+                               dv.data_ptr(), dsl.data_ptr(), dstate.data_ptr(),
+                               dout.data_ptr(), sp)
+        if rc != la.LA_OK:
+            raise la.LaError(rc, "la_decode_step")
+
+    for _ in range(args.warmup):
+        prefill_call()
+        decode_call()
+    torch.cuda.synchronize(dev)
+    st_rc = la.la_workspace_status(ws.data_ptr(), sp)
+    if st_rc != la.LA_OK:
+        raise la.LaError(st_rc, "device status after warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_all0 = torch.cuda.Event(enable_timing=True)
+    t_all1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t_all0.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            prefill_call()
+            ev[i][1].record(stream)
+            decode_call()
+            ev[i][2].record(stream)
+        t_all1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    total_ms = t_all0.elapsed_time(t_all1)
+    pre_ms = sum(a.elapsed_time(b) for a, b, _ in ev) / K
+    dec_ms = sum(b.elapsed_time(c) for _, b, c in ev) / K
+    st_rc = la.la_workspace_status(ws.data_ptr(), sp)
+    if st_rc != la.LA_OK:
+        raise la.LaError(st_rc, "device status after the timed steps")
+
+    total_ms = max_over_ranks(total_ms, world)
+    pre_ms_max = max_over_ranks(pre_ms, world)
+    dec_ms_max = max_over_ranks(dec_ms, world)
+
+    # ---- e2e: host buffers through the C ABI, copies inside the timed region ----
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        hk = torch.empty_like(hq).pin_memory()
+        hv = torch.empty_like(hq).pin_memory()
+        hq.copy_(q.cpu())
+        hk.copy_(k.cpu())
+        hv.copy_(v.cpu())
+        hout = torch.empty_like(hq).pin_memory()
+        hst = torch.empty(st.shape, dtype=st.dtype, pin_memory=True)
+        hdq = torch.empty(dq.shape, dtype=dq.dtype, pin_memory=True)
+        hdk = torch.empty_like(hdq).pin_memory()
+        hdv = torch.empty_like(hdq).pin_memory()
+        hdq.copy_(dq.cpu())
+        hdk.copy_(dk.cpu())
+        hdv.copy_(dv.cpu())
+        hdout = torch.empty_like(hdq).pin_memory()
+        n_e2e = max(1, min(K, 3))
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            dq.copy_(hdq, non_blocking=True)
+            dk.copy_(hdk, non_blocking=True)
+            dv.copy_(hdv, non_blocking=True)
+            prefill_call()
+            decode_call()
+            hout.copy_(out, non_blocking=True)
+            hst.copy_(st, non_blocking=True)
+            hdout.copy_(dout, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
+        bi = 3 * q.numel() * q.element_size() + 3 * dq.numel() * dq.element_size()
+        bo = out.numel() * out.element_size() + st.numel() * 4 + dout.numel() * dout.element_size()
+        e2e = {"value": world * B * N / (e2e_ms * 1e-3), "unit": "tok/s",
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms,
+               "steps": n_e2e}
+
+    if rank == 0:
+        hbm_peak, tc_peak, peak_kind = load_peaks()
+        tokens = B * N
+        tok_s = world * tokens / (pre_ms_max * 1e-3)
+        # algorithmic bytes of one prefill launch: read q, k, v and write o (bf16), write state
+        pre_bytes = 4 * B * N * H * d * 2 + B * H * d * d * 4
+        achieved = pre_bytes / (pre_ms_max * 1e-3) / 1e9
+        canon = 4.0 * d * d * B * N * H  # recurrent-form flops
+        executed = (4.0 * d * d + 4.0 * 128 * d) * B * N * H  # full 128 x 128 tiles
+        dec_bytes = 2 * Bd * Hd * dd * dd * 4 + 4 * Bd * Hd * dd * 2
+        dec_gbs = dec_bytes / (dec_ms_max * 1e-3) / 1e9
+        cpu = None
+        if world == 1 and not args.no_cpu:
+            try:
+                v_cpu, cores, sample = oracle_sample(w)
+                cpu = {"value": v_cpu, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                       "sample": sample}
+            except Exception as exc:  # pragma: no cover - reported, not fatal
+                cpu = {"value": None, "unit": "tok/s", "cores": None, "kind": "oracle",
+                       "sample": f"failed: {exc}"}
+        line = {
+            "metric": METRIC, "value": tok_s, "unit": "tok/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{w.name}: B={B} N={N} H={H} d={d} bf16 + decode step "
+                                   f"B={Bd} H={Hd} d={dd} (fp32 state)",
+                       "global_batch": world * B, "seq_len": N, "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "prefill": {"ms": pre_ms_max, "tok_s": tok_s,
+                        "tflops_canonical": world * canon / (pre_ms_max * 1e-3) / 1e12,
+                        "tflops_executed_c128": world * executed / (pre_ms_max * 1e-3) / 1e12,
+                        "hbm_gbs": achieved},
+            "decode": {"ms": dec_ms_max, "state_gbs": dec_gbs, "frac_of_measured": dec_gbs / hbm_peak,
+                       "frac_of_8tbs": dec_gbs / 8000.0, "tok_s": world * Bd / (dec_ms_max * 1e-3)},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": None,
+                         "kernel": "chunked_prefill_kernel", "peak_kind": peak_kind},
+            "cpu_baseline": cpu,
+            "clocks": clk.summary(),
+            "e2e": e2e,
+            "gpu_launches": 2 * K,
+        }
+        print(json.dumps(line), flush=True)
+    dist_teardown(world)
+
+
+# --------------------------------------------------------------------------------------------
+# reference arm: the fp64 oracle on the host cores
+# --------------------------------------------------------------------------------------------
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    w = synth.WORKLOADS[args.workload]
+    cores = oracle.num_threads()
+    n_heads = cores
+    n_tok = min(w.N, 4096)
+    q, k, v = synth.draw_qkv(1, n_tok, n_heads, w.d, dist=w.dist, seed=w.seed, dtype=w.dtype)
+    bits = [x.view(torch.int16).numpy().view(np.uint16) for x in (q, k, v)]
+    sl = np.resize(synth.slopes(w.H).numpy(), n_heads).astype(np.float32)
+    for _ in range(args.warmup):
+        oracle.prefill(*bits, sl, nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.prefill(*bits, sl, nthreads=cores)
+    dt = (time.perf_counter() - t0) / args.steps
+    tok_s = n_heads * n_tok / dt / w.H
+    sample = (f"fp64 oracle, {n_heads} heads x {n_tok} tokens of the {w.name} distribution per "
+              f"step; tok/s = token-heads/s / H={w.H}")
+    line = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tok/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{w.name}: B={w.B} N={w.N} H={w.H} d={w.d} (sampled)",
+                       "global_batch": w.B, "seq_len": w.N, "parallelism": "host cores"},
+            "cpu_baseline": {"value": tok_s, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": tok_s, "unit": "tok/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["prefill_32k", "prefill_4k", "prefill_256k"],
+                    default="prefill_32k")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer e2e leg")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

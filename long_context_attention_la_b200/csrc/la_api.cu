@@ -1,0 +1,174 @@
+// la_api.cu — the C ABI declared in include/la.h: argument validation, kernel selection and
+// workspace handling.  No torch types cross this boundary; every pointer is a plain device
+// pointer owned by the caller.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "la.h"
+#include "la_internal.h"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// a * b without signed overflow; false if it would exceed INT64_MAX.
+bool mul_ok(int64_t a, int64_t b, int64_t* out) {
+  if (a < 0 || b < 0) return false;
+  if (a != 0 && b > INT64_MAX / a) return false;
+  *out = a * b;
+  return true;
+}
+
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+bool use_tensor_path(const la_desc* d) {
+  if (d->path == LA_PATH_RECURRENT) return false;
+  if (d->path == LA_PATH_TENSOR) return true;
+  return d->dtype == LA_BF16 && d->d == la::kHeadDim;
+}
+
+// Validates a prefill descriptor; on success writes the element count of one activation tensor.
+la_status check_desc(const la_desc* d, int64_t* numel) {
+  if (d == nullptr) return LA_ERR_NULL;
+  if (d->dtype != LA_BF16 && d->dtype != LA_F32) return LA_ERR_DTYPE;
+  if (d->B < 1 || d->N < 1 || d->H < 1 || (d->d != 64 && d->d != 128)) return LA_ERR_SHAPE;
+  if (d->path != LA_PATH_AUTO && d->path != LA_PATH_TENSOR && d->path != LA_PATH_RECURRENT)
+    return LA_ERR_UNSUPPORTED;
+  if (d->segments < 0) return LA_ERR_SHAPE;
+  int64_t t = 0, bytes = 0;
+  if (!mul_ok(d->B, d->N, &t) || !mul_ok(t, d->H, &t) || !mul_ok(t, d->d, &t))
+    return LA_ERR_OVERFLOW;
+  if (!mul_ok(t, d->dtype == LA_BF16 ? 2 : 4, &bytes)) return LA_ERR_OVERFLOW;
+  int64_t st = 0;
+  if (!mul_ok(d->B, d->H, &st) || !mul_ok(st, d->d * d->d * 4, &st)) return LA_ERR_OVERFLOW;
+  if (d->B * d->H > INT32_MAX) return LA_ERR_OVERFLOW;  // grid / flat-head index range
+  if (use_tensor_path(d)) {
+    if (d->dtype != LA_BF16 || d->d != la::kHeadDim) return LA_ERR_UNSUPPORTED;
+    if (d->chunk != 0 && d->chunk != la::kChunk) return LA_ERR_UNSUPPORTED;
+    // tensor-map coordinates are 32-bit; byte strides below 2^40
+    if (d->N > INT32_MAX - la::kChunk || d->H > INT32_MAX || d->B > INT32_MAX)
+      return LA_ERR_OVERFLOW;
+    int64_t row = 0;
+    if (!mul_ok(d->N, d->H * d->d * 2, &row) || row >= (int64_t(1) << 40)) return LA_ERR_OVERFLOW;
+  } else if (d->chunk != 0 && d->chunk != 1) {
+    return LA_ERR_UNSUPPORTED;  // the recurrent path has no chunking
+  }
+  *numel = t;
+  return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t la_prefill_workspace_bytes(const la_desc* desc) {
+  int64_t numel = 0;
+  if (check_desc(desc, &numel) != LA_OK) return 0;
+  if (!use_tensor_path(desc)) return 0;
+  const la::SegmentPlan plan =
+      la::plan_segments(desc->B, desc->N, desc->H, desc->segments, device_sms() > 0 ? device_sms() : 148);
+  return la::workspace_layout(desc->B, desc->H, plan).total;
+}
+
+la_status la_prefill(const la_desc* desc, const void* q, const void* k, const void* v,
+                     const float* slopes, void* out, float* state_out, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  int64_t numel = 0;
+  const la_status st = check_desc(desc, &numel);
+  if (st != LA_OK) return st;
+  if (!q || !k || !v || !slopes || !out) return LA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_ALIGN;
+  if (state_out != nullptr && !aligned16(state_out)) return LA_ERR_ALIGN;
+  const size_t bytes = static_cast<size_t>(numel) * (desc->dtype == LA_BF16 ? 2 : 4);
+  if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) ||
+      overlaps(out, bytes, v, bytes))
+    return LA_ERR_ALIAS;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  la::PrefillArgs a{desc->B, desc->N, desc->H, desc->d, desc->dtype, q, k, v, slopes, out,
+                    state_out};
+  if (!use_tensor_path(desc)) {
+    return la::launch_recurrent_prefill(a, s) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+  }
+  const int sms = device_sms();
+  if (sms <= 0) return LA_ERR_CUDA;
+  const la::SegmentPlan plan = la::plan_segments(desc->B, desc->N, desc->H, desc->segments, sms);
+  const size_t need = la::workspace_layout(desc->B, desc->H, plan).total;
+  void* ws = workspace;
+  bool owned = false;
+  if (ws == nullptr) {
+    if (cudaMallocAsync(&ws, need, s) != cudaSuccess) return LA_ERR_CUDA;
+    owned = true;
+  } else {
+    if (workspace_bytes < need) return LA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return LA_ERR_ALIGN;
+  }
+  const cudaError_t e = la::launch_chunked_prefill(a, plan, ws, s, sms);
+  if (owned) cudaFreeAsync(ws, s);
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status la_decode_step(int64_t B, int64_t H, int64_t d, int32_t dtype, const void* q,
+                         const void* k, const void* v, const float* slopes, float* state_inout,
+                         void* out, void* stream) {
+  if (dtype != LA_BF16 && dtype != LA_F32) return LA_ERR_DTYPE;
+  if (B < 1 || H < 1 || (d != 64 && d != 128)) return LA_ERR_SHAPE;
+  if (!q || !k || !v || !slopes || !state_inout || !out) return LA_ERR_NULL;
+  int64_t bh = 0, n = 0, sb = 0;
+  if (!mul_ok(B, H, &bh) || bh > INT32_MAX || !mul_ok(bh, d, &n) || !mul_ok(bh, d * d * 4, &sb))
+    return LA_ERR_OVERFLOW;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      !aligned16(state_inout))
+    return LA_ERR_ALIGN;
+  const size_t bytes = static_cast<size_t>(n) * (dtype == LA_BF16 ? 2 : 4);
+  if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) ||
+      overlaps(out, bytes, v, bytes) || overlaps(out, bytes, state_inout, static_cast<size_t>(sb)))
+    return LA_ERR_ALIAS;
+  la::DecodeArgs a{B, H, d, dtype, q, k, v, slopes, state_inout, out};
+  return la::launch_decode(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? LA_OK
+                                                                                 : LA_ERR_CUDA;
+}
+
+la_status la_workspace_status(const void* workspace, void* stream) {
+  if (workspace == nullptr) return LA_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LA_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, static_cast<const uint8_t*>(workspace) + la::kWsStatus, sizeof v,
+                 cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LA_ERR_CUDA;
+  return v == 0 ? LA_OK : static_cast<la_status>(v);
+}
+
+const char* la_status_string(int status) {
+  switch (status) {
+    case LA_OK: return "ok";
+    case LA_ERR_NULL: return "a required pointer is NULL";
+    case LA_ERR_SHAPE: return "shape out of range (B, N, H >= 1; d in {64, 128})";
+    case LA_ERR_DTYPE: return "unknown dtype";
+    case LA_ERR_ALIGN: return "pointer not 16-byte aligned (workspace: 256-byte)";
+    case LA_ERR_OVERFLOW: return "size exceeds the 64-bit or tensor-map limits";
+    case LA_ERR_WORKSPACE: return "workspace smaller than la_prefill_workspace_bytes()";
+    case LA_ERR_CUDA: return "a CUDA call failed";
+    case LA_ERR_TIMEOUT: return "a bounded device wait expired";
+    case LA_ERR_UNSUPPORTED: return "no kernel for this combination of options";
+    case LA_ERR_ALIAS: return "output overlaps an input";
+    default: return "unknown status";
+  }
+}
+
+int la_version(void) { return LA_VERSION; }
+
+}  // extern "C"

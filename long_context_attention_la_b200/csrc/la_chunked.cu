@@ -1,0 +1,864 @@
+// la_chunked.cu — chunked Lightning Attention prefill on the sm_100a tensor cores.
+//
+// Method ("Ling and Ring 2.6 Technical Report", Chinese translation, garden.houmin.site;
+// §4.1.1 Context Parallel for Lightning Attention, Fig. 10): each (b, h) sequence is evaluated as
+// chunks of C = 128 tokens ("chunk QKV").  For chunk c with rows i, j in [0, C):
+//     S      = Q K^T                                   (tensor cores, fp32 in TMEM)
+//     P_ij   = lambda^(i-j) S_ij  (i >= j), 0 otherwise  (CUDA cores, bf16 back into TMEM)
+//     O      = P V + diag(lambda^(i+1)) Q KV_in          (two tensor-core accumulators)
+//     KV_out = lambda^n KV_in + (K ⊙ lambda^(n-1-j))^T V  (tensor cores, fp32 state in TMEM)
+// where n is the chunk's token count and KV_in the d x d state before the chunk.  Long sequences
+// are cut into segments ("local recurrence, then global correction"): a segment first computes its
+// local state h (the "local h" of Fig. 10) from K, V alone, obtains its incoming state from its
+// predecessor through a decayed prefix scan over segments (S_{k+1} = lambda^L S_k + h_k, the
+// "fused update h"), and then runs its output chunks starting from that state (the "fused
+// update O", folded into the inter-chunk term instead of a separate correction pass).
+//
+// Execution: one persistent CTA per SM (512 threads, ~226 KB shared memory, all 512 TMEM
+// columns).  Work units (segment, b, h) are taken in segment-major order from an atomic counter,
+// so a unit only ever waits on units that running CTAs already hold.  Roles:
+//   warp 0       TMA producer (two-stage ring of Q/K/V tiles)
+//   warp 1       tcgen05.mma issuer
+//   warp 2       TMEM allocator
+//   warps 4-7    P = decay-mask(S) into TMEM, and K -> K~ (row-scaled) in shared memory
+//   warps 8-11   state: look-back scan, KV -> bf16 operand, decay rescale, final state
+//   warps 12-15  output epilogue: O = O_intra + lambda^(i+1) O_inter -> bf16 -> TMA store
+// Every wait (mbarrier or scan flag) is bounded in time; on expiry the CTA records
+// LA_ERR_TIMEOUT in the workspace status word, unwinds, frees its TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "la_internal.h"
+#include "la_sm100.cuh"
+
+namespace la {
+namespace {
+
+constexpr int C = kChunk;      // 128 tokens per chunk
+constexpr int D = kHeadDim;    // 128
+constexpr int kThreads = 512;
+constexpr uint32_t kTileBytes = C * D * 2;           // one bf16 [128 x 128] tile
+constexpr uint32_t kHalfBytes = kTileBytes / 2;      // [128 rows x 64 cols], 128-byte rows
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kTileBytes;
+constexpr uint32_t kOffV = 2 * kTileBytes;
+constexpr uint32_t kStageBytes = 3 * kTileBytes;     // 96 KiB
+constexpr uint32_t kOffKVb = 2 * kStageBytes;        // bf16 state operand, 32 KiB
+constexpr uint32_t kOffCtrl = kOffKVb + kTileBytes;  // barriers and unit ring
+constexpr uint32_t kCtrlBytes = 1024;
+constexpr uint32_t kSmemBytes = kOffCtrl + kCtrlBytes;
+constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;   // slack for 1024-byte alignment
+
+// TMEM columns (128 lanes x 512 columns of 32 bit).
+constexpr uint32_t kColS = 0;        // S (fp32, 128 cols); P (bf16 pairs) aliases cols 0..63
+constexpr uint32_t kColOintra = 128;
+constexpr uint32_t kColOinter = 256;
+constexpr uint32_t kColKV = 384;     // carried state / segment-local state h
+
+constexpr int32_t kErrTimeout = -8;  // LA_ERR_TIMEOUT
+
+struct UnitInfo {
+  int32_t bh;       // flat head b*H + h, or -1 = no more work
+  int32_t seg;      // segment index k
+  int32_t c0;       // first chunk of the segment
+  int32_t nc;       // chunks in the segment
+  int32_t len;      // tokens in the segment
+  int32_t flags;    // bit 0: compute the local state first; bit 1: last segment of the sequence
+  int32_t pad[2];
+};
+
+struct Ctrl {
+  uint64_t full[2];
+  uint64_t empty[2];
+  uint64_t kt_ready[2];
+  uint64_t unit_full[2];
+  uint64_t unit_empty[2];
+  uint64_t s_full;
+  uint64_t p_ready;
+  uint64_t o_full;
+  uint64_t o_free;
+  uint64_t kv_done;
+  uint64_t kvb_ready;
+  uint64_t kv_free;
+  uint64_t h_done;
+  uint64_t mma_final;
+  uint32_t tmem_base;
+  uint32_t abort;
+  uint32_t pad[2];
+  UnitInfo units[2];
+};
+static_assert(sizeof(Ctrl) <= kCtrlBytes, "control block too large");
+
+struct Params {
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  CUtensorMap tm_o;
+  const float* slopes;
+  float* state_out;
+  uint32_t* counter;
+  int32_t* status;
+  uint32_t* flags;
+  float* ring;
+  int64_t N, H, BH;
+  int64_t n_chunks, seg_chunks, segments, units;
+  uint64_t timeout_ns;
+};
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// All 128 threads of a warpgroup agree on `ok` (logical AND) at named barrier `id`.
+__device__ __forceinline__ bool wg_all(bool ok, uint32_t id) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(ok ? 1u : 0u), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int32_t ld_volatile_s32(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.volatile.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Byte offset of 16-byte chunk `c16` (0..7) of row `r` in a [rows x 64] bf16 half-tile stored
+// with the 128-byte swizzle (8-row, 1024-byte atoms; chunk index XOR row-in-atom).
+__device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t c16) {
+  return (r >> 3) * 1024u + (r & 7u) * 128u + ((c16 ^ (r & 7u)) << 4);
+}
+
+__device__ __forceinline__ void decode_unit(const Params& p, int64_t u, UnitInfo& ui) {
+  const int64_t k = u / p.BH;
+  const int64_t bh = u % p.BH;
+  const int64_t c0 = k * p.seg_chunks;
+  const int64_t nc = min(p.seg_chunks, p.n_chunks - c0);
+  const int64_t end = min(p.N, (c0 + nc) * C);
+  ui.bh = static_cast<int32_t>(bh);
+  ui.seg = static_cast<int32_t>(k);
+  ui.c0 = static_cast<int32_t>(c0);
+  ui.nc = static_cast<int32_t>(nc);
+  ui.len = static_cast<int32_t>(end - c0 * C);
+  ui.flags = (k + 1 < p.segments ? 1 : 0) | (k + 1 == p.segments ? 2 : 0);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    chunked_prefill_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + kOffCtrl);
+  volatile uint32_t* abort_flag = &ctrl->abort;
+  const uint32_t smem_base = smem_u32(smem);
+
+  const uint32_t warp = threadIdx.x >> 5;
+  const uint32_t lane = threadIdx.x & 31;
+  const uint64_t T = p.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&ctrl->full[s], 1);
+      mbar_init(&ctrl->empty[s], 2);
+      mbar_init(&ctrl->kt_ready[s], 128);
+      mbar_init(&ctrl->unit_full[s], 1);
+      mbar_init(&ctrl->unit_empty[s], 1 + 3 * 128);
+    }
+    mbar_init(&ctrl->s_full, 1);
+    mbar_init(&ctrl->p_ready, 128);
+    mbar_init(&ctrl->o_full, 1);
+    mbar_init(&ctrl->o_free, 128);
+    mbar_init(&ctrl->kv_done, 1);
+    mbar_init(&ctrl->kvb_ready, 128);
+    mbar_init(&ctrl->kv_free, 128);
+    mbar_init(&ctrl->h_done, 1);
+    mbar_init(&ctrl->mma_final, 1);
+    ctrl->abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+    tma_prefetch_desc(&p.tm_o);
+  }
+  if (warp == 2) {
+    tmem_alloc(&ctrl->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+
+  if (warp == 0) {
+    // =========================================================================================
+    // TMA producer
+    // =========================================================================================
+    if (lane == 0) {
+      const uint64_t pol_first = policy_evict_first();
+      const uint64_t pol_last = policy_evict_last();
+      uint32_t g = 0;
+      uint32_t j = 0;
+      uint32_t issued[2] = {0, 0};  // fills issued per stage (for the abort drain)
+      bool ok = true;
+      while (ok) {
+        const uint32_t slot = j & 1;
+        if (!mbar_wait_bounded(&ctrl->unit_empty[slot], ((j >> 1) & 1) ^ 1, abort_flag, T)) {
+          ok = false;
+          break;
+        }
+        const int64_t u = static_cast<int64_t>(atomicAdd(p.counter, 1u));
+        UnitInfo ui;
+        if (u < p.units) {
+          decode_unit(p, u, ui);
+        } else {
+          ui.bh = -1;
+          ui.seg = ui.c0 = ui.nc = ui.len = ui.flags = 0;
+        }
+        ctrl->units[slot] = ui;
+        mbar_arrive(&ctrl->unit_full[slot]);
+        if (ui.bh < 0) break;
+        const int32_t b = static_cast<int32_t>(ui.bh / p.H);
+        const int32_t h = static_cast<int32_t>(ui.bh % p.H);
+        const int passes = (ui.flags & 1) ? 2 : 1;
+        for (int pass = 0; pass < passes && ok; ++pass) {
+          const bool local_state_pass = (passes == 2 && pass == 0);
+          for (int32_t c = 0; c < ui.nc; ++c) {
+            const uint32_t s = g & 1;
+            if (!mbar_wait_bounded(&ctrl->empty[s], ((g >> 1) & 1) ^ 1, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            uint8_t* st = smem + s * kStageBytes;
+            const int32_t n0 = (ui.c0 + c) * C;
+            const uint64_t kv_pol = local_state_pass ? pol_last : pol_first;
+            if (local_state_pass) {
+              mbar_arrive_expect_tx(&ctrl->full[s], 2 * kTileBytes);
+            } else {
+              mbar_arrive_expect_tx(&ctrl->full[s], 3 * kTileBytes);
+              tma_load_4d(st + kOffQ, &p.tm_q, &ctrl->full[s], 0, h, n0, b, pol_first);
+              tma_load_4d(st + kOffQ + kHalfBytes, &p.tm_q, &ctrl->full[s], 64, h, n0, b,
+                          pol_first);
+            }
+            tma_load_4d(st + kOffK, &p.tm_k, &ctrl->full[s], 0, h, n0, b, kv_pol);
+            tma_load_4d(st + kOffK + kHalfBytes, &p.tm_k, &ctrl->full[s], 64, h, n0, b, kv_pol);
+            tma_load_4d(st + kOffV, &p.tm_v, &ctrl->full[s], 0, h, n0, b, kv_pol);
+            tma_load_4d(st + kOffV + kHalfBytes, &p.tm_v, &ctrl->full[s], 64, h, n0, b, kv_pol);
+            issued[s] += 1;
+            ++g;
+          }
+        }
+        ++j;
+      }
+      if (!ok) {
+        // Let every fill already issued land before the CTA's shared memory goes away.
+        for (uint32_t s = 0; s < 2; ++s) {
+          if (issued[s] > 0) {
+            const uint32_t last_parity = (issued[s] - 1) & 1;
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&ctrl->full[s], last_parity) && globaltimer_ns() - t0 < T) {
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // =========================================================================================
+    // tcgen05.mma issuer
+    // =========================================================================================
+    if (lane == 0) {
+      constexpr uint32_t idS = make_idesc_bf16(128, 128, 0, 0);   // Q (K-major) x K (K-major)
+      constexpr uint32_t idQK = make_idesc_bf16(128, 128, 0, 1);  // Q x KVb (MN-major)
+      constexpr uint32_t idPV = make_idesc_bf16(128, 128, 0, 1);  // P (TMEM) x V (MN-major)
+      constexpr uint32_t idKV = make_idesc_bf16(128, 128, 1, 1);  // K~^T (MN) x V (MN)
+      uint32_t g = 0, j = 0;
+      uint32_t n_kvb = 0, n_ofree = 0, n_p = 0;
+      bool ok = true;
+      while (ok) {
+        const uint32_t slot = j & 1;
+        if (!mbar_wait_bounded(&ctrl->unit_full[slot], (j >> 1) & 1, abort_flag, T)) break;
+        const UnitInfo ui = ctrl->units[slot];
+        mbar_arrive(&ctrl->unit_empty[slot]);
+        if (ui.bh < 0) break;
+        // the state region must be free of the previous unit's read-out
+        if (!mbar_wait_bounded(&ctrl->kv_free, j & 1, abort_flag, T)) break;
+        tc_fence_after();
+        if (ui.flags & 1) {
+          // local segment state h = sum_j lambda^(L-1-j) k_j^T v_j into the KV columns
+          for (int32_t c = 0; c < ui.nc && ok; ++c) {
+            const uint32_t s = g & 1;
+            const uint32_t ph = (g >> 1) & 1;
+            if (!mbar_wait_bounded(&ctrl->full[s], ph, abort_flag, T) ||
+                !mbar_wait_bounded(&ctrl->kt_ready[s], ph, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t kb = smem_base + s * kStageBytes + kOffK;
+            const uint32_t vb = smem_base + s * kStageBytes + kOffV;
+#pragma unroll
+            for (uint32_t kk = 0; kk < 8; ++kk) {
+              umma_ss(tmem + kColKV, make_sdesc_sw128(kb + kk * 2048, kHalfBytes, 1024),
+                      make_sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idKV,
+                      (c > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&ctrl->empty[s]);
+            mbar_arrive(&ctrl->empty[s]);
+            ++g;
+          }
+          if (!ok) break;
+          umma_commit(&ctrl->h_done);
+        }
+        for (int32_t c = 0; c < ui.nc && ok; ++c) {
+          const uint32_t s = g & 1;
+          const uint32_t ph = (g >> 1) & 1;
+          if (!mbar_wait_bounded(&ctrl->full[s], ph, abort_flag, T)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t qb = smem_base + s * kStageBytes + kOffQ;
+          const uint32_t kb = smem_base + s * kStageBytes + kOffK;
+          const uint32_t vb = smem_base + s * kStageBytes + kOffV;
+          const uint32_t kvb = smem_base + kOffKVb;
+          // S = Q K^T
+#pragma unroll
+          for (uint32_t kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+            umma_ss(tmem + kColS, make_sdesc_sw128(qb + off, 16, 1024),
+                    make_sdesc_sw128(kb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&ctrl->s_full);
+          // O_inter = Q KV_in (needs the bf16 state operand and a free O accumulator)
+          if (!mbar_wait_bounded(&ctrl->kvb_ready, n_kvb & 1, abort_flag, T) ||
+              !mbar_wait_bounded(&ctrl->o_free, n_ofree & 1, abort_flag, T)) {
+            ok = false;
+            break;
+          }
+          ++n_kvb;
+          ++n_ofree;
+          tc_fence_after();
+#pragma unroll
+          for (uint32_t kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+            umma_ss(tmem + kColOinter, make_sdesc_sw128(qb + off, 16, 1024),
+                    make_sdesc_sw128(kvb + kk * 2048, kHalfBytes, 1024), idQK,
+                    kk > 0 ? 1u : 0u);
+          }
+          // O_intra = P V, P read from TMEM
+          if (!mbar_wait_bounded(&ctrl->p_ready, n_p & 1, abort_flag, T)) {
+            ok = false;
+            break;
+          }
+          ++n_p;
+          tc_fence_after();
+#pragma unroll
+          for (uint32_t kk = 0; kk < 8; ++kk) {
+            umma_ts(tmem + kColOintra, tmem + kColS + kk * 8,
+                    make_sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idPV, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&ctrl->o_full);
+          // KV <- lambda^n KV (done by the state warps) + K~^T V
+          if (!mbar_wait_bounded(&ctrl->kt_ready[s], ph, abort_flag, T)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (uint32_t kk = 0; kk < 8; ++kk) {
+            umma_ss(tmem + kColKV, make_sdesc_sw128(kb + kk * 2048, kHalfBytes, 1024),
+                    make_sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idKV, 1u);
+          }
+          umma_commit(&ctrl->kv_done);
+          umma_commit(&ctrl->empty[s]);
+          ++g;
+        }
+        ++j;
+      }
+      // all issued MMAs must finish before TMEM is released
+      umma_commit(&ctrl->mma_final);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(&ctrl->mma_final, 0) && globaltimer_ns() - t0 < T) {
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 8) {
+    // =========================================================================================
+    // P = decay-mask(S) -> TMEM (bf16), K -> K~ in shared memory
+    // =========================================================================================
+    const uint32_t wq = warp & 3;
+    const uint32_t i = wq * 32 + lane;  // row of the chunk (query token / key token)
+    const uint32_t trow = tmem + ((wq * 32) << 16);
+    uint32_t g = 0, j = 0, n_s = 0;
+    while (true) {
+      const uint32_t slot = j & 1;
+      bool ok = mbar_wait_bounded(&ctrl->unit_full[slot], (j >> 1) & 1, abort_flag, T);
+      if (!wg_all(ok, 1)) break;
+      const UnitInfo ui = ctrl->units[slot];
+      mbar_arrive(&ctrl->unit_empty[slot]);
+      if (ui.bh < 0) break;
+      const float alpha = p.slopes[ui.bh % p.H] * kLog2e;  // lambda^n = exp2(-alpha n)
+      const bool fast = alpha * 31.f <= 120.f;
+      float bm[32];  // 2^(alpha m) = lambda^(-m), m = 0..31
+#pragma unroll
+      for (int m = 0; m < 32; ++m) bm[m] = fast ? exp2f(alpha * static_cast<float>(m)) : 0.f;
+
+      auto scale_k_row = [&](uint32_t s, float w) {
+        uint8_t* kt = smem + s * kStageBytes + kOffK;
+#pragma unroll
+        for (uint32_t half = 0; half < 2; ++half) {
+          uint8_t* row = kt + half * kHalfBytes + (i >> 3) * 1024u + (i & 7u) * 128u;
+#pragma unroll
+          for (uint32_t c = 0; c < 8; ++c) {
+            uint4* q4 = reinterpret_cast<uint4*>(row + ((c ^ (i & 7u)) << 4));
+            uint4 x = *q4;
+            x.x = pack_bf16x2(bf16lo_to_f32(x.x) * w, bf16hi_to_f32(x.x) * w);
+            x.y = pack_bf16x2(bf16lo_to_f32(x.y) * w, bf16hi_to_f32(x.y) * w);
+            x.z = pack_bf16x2(bf16lo_to_f32(x.z) * w, bf16hi_to_f32(x.z) * w);
+            x.w = pack_bf16x2(bf16lo_to_f32(x.w) * w, bf16hi_to_f32(x.w) * w);
+            *q4 = x;
+          }
+        }
+      };
+
+      if (ui.flags & 1) {
+        for (int32_t c = 0; c < ui.nc; ++c) {
+          const uint32_t s = g & 1;
+          ok = mbar_wait_bounded(&ctrl->full[s], (g >> 1) & 1, abort_flag, T);
+          if (!wg_all(ok, 1)) goto wg1_out;
+          const int32_t pos = c * C + static_cast<int32_t>(i);  // token within the segment
+          const float w = pos < ui.len ? exp2f(-alpha * static_cast<float>(ui.len - 1 - pos)) : 0.f;
+          scale_k_row(s, w);
+          fence_proxy_async_smem();
+          mbar_arrive(&ctrl->kt_ready[s]);
+          ++g;
+        }
+      }
+      for (int32_t c = 0; c < ui.nc; ++c) {
+        const uint32_t s = g & 1;
+        const int32_t n_c = min(C, ui.len - c * C);  // tokens in this chunk
+        ok = mbar_wait_bounded(&ctrl->s_full, n_s & 1, abort_flag, T);
+        if (!wg_all(ok, 1)) goto wg1_out;
+        ++n_s;
+        tc_fence_after();
+        // ---- P ----
+#pragma unroll
+        for (uint32_t jb = 0; jb < 4; ++jb) {
+          uint32_t pk[16];
+          if (jb <= wq) {
+            uint32_t r[32];
+            tmem_ld32(trow + kColS + jb * 32, r);
+            tmem_wait_ld();
+            const int32_t dbase = static_cast<int32_t>(i) - static_cast<int32_t>(jb * 32);
+            const float a = exp2f(-alpha * static_cast<float>(dbase));
+#pragma unroll
+            for (int m = 0; m < 32; m += 2) {
+              float f0, f1;
+              if (fast) {
+                f0 = a * bm[m];
+                f1 = a * bm[m + 1];
+              } else {
+                f0 = exp2f(-alpha * static_cast<float>(dbase - m));
+                f1 = exp2f(-alpha * static_cast<float>(dbase - m - 1));
+              }
+              float x0 = __uint_as_float(r[m]) * f0;
+              float x1 = __uint_as_float(r[m + 1]) * f1;
+              if (jb == wq) {
+                if (m > static_cast<int>(lane)) x0 = 0.f;
+                if (m + 1 > static_cast<int>(lane)) x1 = 0.f;
+              }
+              pk[m >> 1] = pack_bf16x2(x0, x1);
+            }
+          } else {
+#pragma unroll
+            for (int m = 0; m < 16; ++m) pk[m] = 0u;
+          }
+          tmem_st16(trow + kColS + jb * 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&ctrl->p_ready);
+        // ---- K~ = diag(lambda^(n-1-i)) K for the state update ----
+        {
+          const float w = static_cast<int32_t>(i) < n_c
+                              ? exp2f(-alpha * static_cast<float>(n_c - 1 - static_cast<int32_t>(i)))
+                              : 0.f;
+          scale_k_row(s, w);
+          fence_proxy_async_smem();
+          mbar_arrive(&ctrl->kt_ready[s]);
+        }
+        ++g;
+      }
+      ++j;
+    }
+  wg1_out:;
+  } else if (warp >= 8 && warp < 12) {
+    // =========================================================================================
+    // state: look-back scan over segments, bf16 operand, decay rescale, final state
+    // =========================================================================================
+    const uint32_t wq = warp & 3;
+    const uint32_t i = wq * 32 + lane;  // key-dimension row of the state
+    const uint32_t trow = tmem + ((wq * 32) << 16);
+    uint8_t* kvb = smem + kOffKVb;
+    uint32_t j = 0, n_kvd = 0, n_h = 0;
+    tc_fence_before();
+    mbar_arrive(&ctrl->kv_free);  // the KV columns start out free
+
+    // bf16 copy of 32 state columns [32 cb, 32 cb + 32) of row i into the MN-major operand
+    auto write_kvb = [&](uint32_t cb, const float (&x)[32]) {
+      const uint32_t half = cb >> 1;
+#pragma unroll
+      for (uint32_t q = 0; q < 4; ++q) {
+        const uint32_t c16 = (cb & 1) * 4 + q;
+        uint4 w;
+        w.x = pack_bf16x2(x[8 * q + 0], x[8 * q + 1]);
+        w.y = pack_bf16x2(x[8 * q + 2], x[8 * q + 3]);
+        w.z = pack_bf16x2(x[8 * q + 4], x[8 * q + 5]);
+        w.w = pack_bf16x2(x[8 * q + 6], x[8 * q + 7]);
+        *reinterpret_cast<uint4*>(kvb + half * kHalfBytes + sw128_off(i, c16)) = w;
+      }
+    };
+
+    while (true) {
+      const uint32_t slot = j & 1;
+      bool ok = mbar_wait_bounded(&ctrl->unit_full[slot], (j >> 1) & 1, abort_flag, T);
+      if (!wg_all(ok, 2)) break;
+      const UnitInfo ui = ctrl->units[slot];
+      mbar_arrive(&ctrl->unit_empty[slot]);
+      if (ui.bh < 0) break;
+      const float alpha = p.slopes[ui.bh % p.H] * kLog2e;
+      const int64_t bh = ui.bh;
+      const int32_t k = ui.seg;
+
+      if (ui.flags & 1) {
+        ok = mbar_wait_bounded(&ctrl->h_done, n_h & 1, abort_flag, T);
+        if (!wg_all(ok, 2)) break;
+        ++n_h;
+        tc_fence_after();
+      }
+      // incoming state of this segment: published by segment k-1 of the same sequence
+      if (k > 0) {
+        const uint32_t* fl = p.flags + bh * 2 + ((k - 1) & 1);
+        const uint64_t t0 = globaltimer_ns();
+        ok = true;
+        while (ld_acquire_u32(fl) != static_cast<uint32_t>(k)) {
+          if (*abort_flag || ld_volatile_s32(p.status) != 0 || globaltimer_ns() - t0 > T) {
+            ok = false;
+            *abort_flag = 1u;
+            break;
+          }
+        }
+        if (!wg_all(ok, 2)) break;
+      }
+      const float4* ring_in =
+          reinterpret_cast<const float4*>(p.ring + (bh * 2 + ((k - 1) & 1)) * (D * D));
+      float4* ring_out = reinterpret_cast<float4*>(p.ring + (bh * 2 + (k & 1)) * (D * D));
+      const float lam_len = exp2f(-alpha * static_cast<float>(ui.len));
+      const float lam_n0 = exp2f(-alpha * static_cast<float>(min(C, ui.len)));
+#pragma unroll 1
+      for (uint32_t cb = 0; cb < 4; ++cb) {
+        float sin[32];
+        if (k > 0) {
+#pragma unroll
+          for (uint32_t q = 0; q < 8; ++q) {
+            const float4 x = __ldcg(ring_in + (cb * 8 + q) * 128 + i);
+            sin[4 * q + 0] = x.x;
+            sin[4 * q + 1] = x.y;
+            sin[4 * q + 2] = x.z;
+            sin[4 * q + 3] = x.w;
+          }
+        } else {
+#pragma unroll
+          for (int m = 0; m < 32; ++m) sin[m] = 0.f;
+        }
+        if (ui.flags & 1) {
+          // inclusive state S_{k+1} = lambda^L S_k + h_k, published for segment k+1
+          uint32_t r[32];
+          tmem_ld32(trow + kColKV + cb * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (uint32_t q = 0; q < 8; ++q) {
+            float4 x;
+            x.x = fmaf(lam_len, sin[4 * q + 0], __uint_as_float(r[4 * q + 0]));
+            x.y = fmaf(lam_len, sin[4 * q + 1], __uint_as_float(r[4 * q + 1]));
+            x.z = fmaf(lam_len, sin[4 * q + 2], __uint_as_float(r[4 * q + 2]));
+            x.w = fmaf(lam_len, sin[4 * q + 3], __uint_as_float(r[4 * q + 3]));
+            __stcg(ring_out + (cb * 8 + q) * 128 + i, x);
+          }
+        }
+        write_kvb(cb, sin);
+        uint32_t r2[32];
+#pragma unroll
+        for (int m = 0; m < 32; ++m) r2[m] = __float_as_uint(lam_n0 * sin[m]);
+        tmem_st32(trow + kColKV + cb * 32, r2);
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      if (ui.flags & 1) {
+        __threadfence();
+        named_bar_sync(2, 128);
+        if (wq == 0 && lane == 0) {
+          __threadfence();
+          st_release_u32(p.flags + bh * 2 + (k & 1), static_cast<uint32_t>(k + 1));
+        }
+      }
+      mbar_arrive(&ctrl->kvb_ready);
+
+      // carry the state through the segment's chunks
+      bool good = true;
+      for (int32_t c = 0; c < ui.nc; ++c) {
+        ok = mbar_wait_bounded(&ctrl->kv_done, n_kvd & 1, abort_flag, T);
+        if (!wg_all(ok, 2)) {
+          good = false;
+          break;
+        }
+        ++n_kvd;
+        tc_fence_after();
+        if (c + 1 < ui.nc) {
+          const int32_t n_next = min(C, ui.len - (c + 1) * C);
+          const float lam_next = exp2f(-alpha * static_cast<float>(n_next));
+#pragma unroll 1
+          for (uint32_t cb = 0; cb < 4; ++cb) {
+            uint32_t r[32];
+            tmem_ld32(trow + kColKV + cb * 32, r);
+            tmem_wait_ld();
+            float x[32];
+#pragma unroll
+            for (int m = 0; m < 32; ++m) x[m] = __uint_as_float(r[m]);
+            write_kvb(cb, x);
+#pragma unroll
+            for (int m = 0; m < 32; ++m) r[m] = __float_as_uint(lam_next * x[m]);
+            tmem_st32(trow + kColKV + cb * 32, r);
+          }
+          tmem_wait_st();
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(&ctrl->kvb_ready);
+        } else if ((ui.flags & 2) && p.state_out != nullptr) {
+          float4* so = reinterpret_cast<float4*>(p.state_out + (bh * D + i) * D);
+#pragma unroll 1
+          for (uint32_t cb = 0; cb < 4; ++cb) {
+            uint32_t r[32];
+            tmem_ld32(trow + kColKV + cb * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (uint32_t q = 0; q < 8; ++q) {
+              so[cb * 8 + q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                           __uint_as_float(r[4 * q + 2]),
+                                           __uint_as_float(r[4 * q + 3]));
+            }
+          }
+        }
+      }
+      if (!good) break;
+      tc_fence_before();
+      mbar_arrive(&ctrl->kv_free);
+      ++j;
+    }
+  } else if (warp >= 12) {
+    // =========================================================================================
+    // output epilogue
+    // =========================================================================================
+    const uint32_t wq = warp & 3;
+    const uint32_t i = wq * 32 + lane;  // token row of the chunk
+    const uint32_t trow = tmem + ((wq * 32) << 16);
+    const uint64_t pol_first = policy_evict_first();
+    uint32_t g = 0, j = 0, n_o = 0;
+    tc_fence_before();
+    mbar_arrive(&ctrl->o_free);  // the O accumulators start out free
+    while (true) {
+      const uint32_t slot = j & 1;
+      bool ok = mbar_wait_bounded(&ctrl->unit_full[slot], (j >> 1) & 1, abort_flag, T);
+      if (!wg_all(ok, 3)) break;
+      const UnitInfo ui = ctrl->units[slot];
+      mbar_arrive(&ctrl->unit_empty[slot]);
+      if (ui.bh < 0) break;
+      const float alpha = p.slopes[ui.bh % p.H] * kLog2e;
+      const float f = exp2f(-alpha * static_cast<float>(i + 1));  // lambda^(i+1)
+      const int32_t b = static_cast<int32_t>(ui.bh / p.H);
+      const int32_t h = static_cast<int32_t>(ui.bh % p.H);
+      if (ui.flags & 1) g += static_cast<uint32_t>(ui.nc);  // the local-state pass stores nothing
+      bool good = true;
+      for (int32_t c = 0; c < ui.nc; ++c) {
+        const uint32_t s = g & 1;
+        ok = mbar_wait_bounded(&ctrl->o_full, n_o & 1, abort_flag, T);
+        if (!wg_all(ok, 3)) {
+          good = false;
+          break;
+        }
+        ++n_o;
+        tc_fence_after();
+        uint8_t* ob = smem + s * kStageBytes + kOffQ;  // Q tile is dead: stage the output there
+#pragma unroll 1
+        for (uint32_t cb = 0; cb < 4; ++cb) {
+          uint32_t ra[32], re[32];
+          tmem_ld32(trow + kColOintra + cb * 32, ra);
+          tmem_ld32(trow + kColOinter + cb * 32, re);
+          tmem_wait_ld();
+          const uint32_t half = cb >> 1;
+#pragma unroll
+          for (uint32_t q = 0; q < 4; ++q) {
+            float o[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              o[e] = fmaf(f, __uint_as_float(re[8 * q + e]), __uint_as_float(ra[8 * q + e]));
+            uint4 w;
+            w.x = pack_bf16x2(o[0], o[1]);
+            w.y = pack_bf16x2(o[2], o[3]);
+            w.z = pack_bf16x2(o[4], o[5]);
+            w.w = pack_bf16x2(o[6], o[7]);
+            *reinterpret_cast<uint4*>(ob + half * kHalfBytes + sw128_off(i, (cb & 1) * 4 + q)) =
+                w;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&ctrl->o_free);
+        fence_proxy_async_smem();
+        named_bar_sync(3, 128);
+        if (wq == 0 && lane == 0) {
+          const int32_t n0 = (ui.c0 + c) * C;
+          tma_store_4d(&p.tm_o, ob, 0, h, n0, b, pol_first);
+          tma_store_4d(&p.tm_o, ob + kHalfBytes, 64, h, n0, b, pol_first);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          mbar_arrive(&ctrl->empty[s]);
+        }
+        ++g;
+      }
+      if (!good) break;
+      ++j;
+    }
+    if (wq == 0 && lane == 0) bulk_wait_group0();
+  }
+
+  // ===========================================================================================
+  // teardown
+  // ===========================================================================================
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0 && ctrl->abort) atomicExch(p.status, kErrTimeout);
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+bool encode_map(CUtensorMap* map, const void* base, int64_t B, int64_t N, int64_t H) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (encode == nullptr) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr) {
+      return false;
+    }
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2,
+                                 static_cast<cuuint64_t>(H) * D * 2,
+                                 static_cast<cuuint64_t>(N) * H * D * 2};
+  const cuuint32_t box[4] = {64, 1, C, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
+                            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+SegmentPlan plan_segments(int64_t B, int64_t N, int64_t H, int requested_segments, int num_sms) {
+  SegmentPlan pl{};
+  pl.n_chunks = (N + C - 1) / C;
+  const int64_t bh = B * H;
+  int64_t want;
+  if (requested_segments > 0) {
+    want = requested_segments;
+  } else if (bh >= 2 * static_cast<int64_t>(num_sms)) {
+    want = 1;  // enough independent sequences: no scan needed
+  } else {
+    // Segments of about 4 chunks keep the K, V tiles of the local-state pass resident in L2
+    // until the output pass of the same segment re-reads them.
+    want = (pl.n_chunks + 3) / 4;
+  }
+  want = std::max<int64_t>(1, std::min<int64_t>(want, pl.n_chunks));
+  pl.seg_chunks = (pl.n_chunks + want - 1) / want;
+  pl.segments = (pl.n_chunks + pl.seg_chunks - 1) / pl.seg_chunks;
+  pl.units = pl.segments * bh;
+  return pl;
+}
+
+WorkspaceLayout workspace_layout(int64_t B, int64_t H, const SegmentPlan& plan) {
+  WorkspaceLayout w{};
+  const int64_t bh = B * H;
+  w.header_bytes = 256;
+  w.flags_off = 256;
+  w.flags_bytes = plan.segments > 1 ? static_cast<size_t>(bh) * 2 * sizeof(uint32_t) : 0;
+  w.ring_off = (w.flags_off + w.flags_bytes + 255) / 256 * 256;
+  w.ring_bytes =
+      plan.segments > 1 ? static_cast<size_t>(bh) * 2 * D * D * sizeof(float) : 0;
+  w.total = w.ring_off + w.ring_bytes;
+  return w;
+}
+
+cudaError_t launch_chunked_prefill(const PrefillArgs& a, const SegmentPlan& plan,
+                                   void* workspace, cudaStream_t stream, int num_sms) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    e = cudaFuncSetAttribute(chunked_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemAlloc));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  Params prm{};
+  if (!encode_map(&prm.tm_q, a.q, a.B, a.N, a.H) || !encode_map(&prm.tm_k, a.k, a.B, a.N, a.H) ||
+      !encode_map(&prm.tm_v, a.v, a.B, a.N, a.H) || !encode_map(&prm.tm_o, a.out, a.B, a.N, a.H)) {
+    return cudaErrorInvalidValue;
+  }
+  const WorkspaceLayout wl = workspace_layout(a.B, a.H, plan);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  prm.slopes = a.slopes;
+  prm.state_out = a.state_out;
+  prm.counter = reinterpret_cast<uint32_t*>(ws + kWsCounter);
+  prm.status = reinterpret_cast<int32_t*>(ws + kWsStatus);
+  prm.flags = reinterpret_cast<uint32_t*>(ws + wl.flags_off);
+  prm.ring = reinterpret_cast<float*>(ws + wl.ring_off);
+  prm.N = a.N;
+  prm.H = a.H;
+  prm.BH = a.B * a.H;
+  prm.n_chunks = plan.n_chunks;
+  prm.seg_chunks = plan.seg_chunks;
+  prm.segments = plan.segments;
+  prm.units = plan.units;
+  prm.timeout_ns = 2000000000ull;  // 2 s per wait
+
+  // counter, status and scan flags start at zero for every call
+  e = cudaMemsetAsync(ws, 0, wl.flags_off + wl.flags_bytes, stream);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = std::min<int64_t>(plan.units, num_sms);
+  chunked_prefill_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, stream>>>(prm);
+  return cudaGetLastError();
+}
+
+}  // namespace la

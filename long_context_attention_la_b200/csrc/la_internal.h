@@ -1,0 +1,77 @@
+// la_internal.h — launch interfaces shared by the C ABI (la_api.cu) and the kernel files.
+// Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace la {
+
+enum DType : int { kBF16 = 0, kF32 = 1 };
+
+struct PrefillArgs {
+  int64_t B, N, H, d;
+  int dtype;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* slopes;
+  void* out;
+  float* state_out;  // may be null
+};
+
+struct DecodeArgs {
+  int64_t B, H, d;
+  int dtype;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* slopes;
+  float* state;
+  void* out;
+};
+
+// Token-by-token CUDA-core prefill (any dtype, d in {64, 128}); one CTA per (b, h).
+cudaError_t launch_recurrent_prefill(const PrefillArgs& a, cudaStream_t stream);
+
+// Fused decode step; one CTA per (b, h).
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------------------------
+// Chunked tensor-core prefill (bf16, d = 128, chunk C = 128).
+// ---------------------------------------------------------------------------------------------
+constexpr int kChunk = 128;
+constexpr int kHeadDim = 128;
+
+// How a prefill is cut into work units: each (b, h) sequence of N tokens becomes `segments`
+// segments of `seg_chunks` chunks (the last may be shorter); one unit = one (segment, b, h).
+struct SegmentPlan {
+  int64_t n_chunks;    // ceil(N / C)
+  int64_t seg_chunks;  // chunks per segment
+  int64_t segments;    // ceil(n_chunks / seg_chunks)
+  int64_t units;       // segments * B * H
+};
+
+SegmentPlan plan_segments(int64_t B, int64_t N, int64_t H, int requested_segments, int num_sms);
+
+// Workspace layout of the chunked prefill (byte offsets from the workspace base).
+struct WorkspaceLayout {
+  size_t header_bytes;  // [0, 256): counter, status
+  size_t flags_off;     // uint32 [B*H*2] scan flags
+  size_t flags_bytes;
+  size_t ring_off;      // float [B*H*2][d*d] segment-state ring (two slots per sequence)
+  size_t ring_bytes;
+  size_t total;
+};
+
+WorkspaceLayout workspace_layout(int64_t B, int64_t H, const SegmentPlan& plan);
+
+// Offsets inside the 256-byte header.
+constexpr size_t kWsCounter = 0;   // uint32 work-unit counter
+constexpr size_t kWsStatus = 64;   // uint32 device status (0 = ok, else a la_status code)
+
+cudaError_t launch_chunked_prefill(const PrefillArgs& a, const SegmentPlan& plan,
+                                   void* workspace, cudaStream_t stream, int num_sms);
+
+}  // namespace la

@@ -1,0 +1,232 @@
+// la_recurrent.cu — token-by-token CUDA-core kernels: the fp32 prefill path and the decode step.
+//
+// Both evaluate the RNN-style form of linear attention ("Ling and Ring 2.6 Technical Report",
+// §4.1.1, Context Parallel for Lightning Attention: a recurrence over the sequence with a per-head
+// [D,D] hidden state), with Lightning Attention's per-head decay lambda = exp(-slope):
+//     S <- lambda S + k^T v,    o = q S.
+//
+// Decay precision.  A plain fp32 multiply by a rounded lambda carries the rounding of lambda
+// into every step (after n steps the relative error of lambda^n grows like n * 2^-24).  The kernels
+// therefore split lambda = lam_hi + lam_lo (both fp32, computed from an fp64 exp) and apply
+//     S' = lam_hi * S + (k v + lam_lo * S)
+// with two fused multiply-adds, so the decay is exact to fp32 rounding of each step.
+#include <cuda_bf16.h>
+
+#include "la_internal.h"
+
+namespace la {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ float load_as_f32(const T* p, int64_t i);
+template <>
+__device__ __forceinline__ float load_as_f32<float>(const float* p, int64_t i) {
+  return p[i];
+}
+template <>
+__device__ __forceinline__ float load_as_f32<__nv_bfloat16>(const __nv_bfloat16* p, int64_t i) {
+  return __bfloat162float(p[i]);
+}
+
+template <typename T>
+__device__ __forceinline__ void store_from_f32(T* p, int64_t i, float x);
+template <>
+__device__ __forceinline__ void store_from_f32<float>(float* p, int64_t i, float x) {
+  p[i] = x;
+}
+template <>
+__device__ __forceinline__ void store_from_f32<__nv_bfloat16>(__nv_bfloat16* p, int64_t i,
+                                                              float x) {
+  p[i] = __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ void split_decay(float slope, float& hi, float& lo) {
+  const double lam = exp(-static_cast<double>(slope));
+  hi = static_cast<float>(lam);
+  lo = static_cast<float>(lam - static_cast<double>(hi));
+}
+
+// ---------------------------------------------------------------------------------------------
+// Recurrent prefill.  One CTA per flat head (b*H + h), 4*D threads.  Thread t owns the state
+// column j = t % D for rows [rg*R, rg*R + R), rg = t / D, R = D / 4; the read-out o_j is summed
+// over the four row groups through shared memory.  q, k, v of the next token are prefetched into
+// registers while the current token is processed.
+// ---------------------------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(4 * D) recurrent_prefill_kernel(
+    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+    const float* __restrict__ slopes, T* __restrict__ out, float* __restrict__ state_out,
+    int64_t N, int64_t H) {
+  constexpr int R = D / 4;
+  __shared__ float tok[2][3][D];
+  __shared__ float red[4][D];
+
+  const int tid = threadIdx.x;
+  const int j = tid % D;
+  const int rg = tid / D;
+  const int64_t flat = blockIdx.x;
+  const int64_t b = flat / H;
+  const int64_t h = flat % H;
+
+  float lam_hi, lam_lo;
+  split_decay(slopes[h], lam_hi, lam_lo);
+
+  // loader role: threads [0, 3D) each fetch one element of q, k or v of a token
+  const int which = tid / D;  // 0: q, 1: k, 2: v (3: idle)
+  const int e = tid % D;
+  const T* src = which == 0 ? q : (which == 1 ? k : v);
+  auto fetch = [&](int64_t t) -> float {
+    return load_as_f32<T>(src, ((b * N + t) * H + h) * D + e);
+  };
+
+  float S[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) S[r] = 0.f;
+
+  if (which < 3 && N > 0) tok[0][which][e] = fetch(0);
+  float pf = 0.f;
+  if (which < 3 && N > 1) pf = fetch(1);
+  __syncthreads();
+
+  for (int64_t t = 0; t < N; ++t) {
+    const int buf = static_cast<int>(t & 1);
+    const float vj = tok[buf][2][j];
+    float acc = 0.f;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int i = rg * R + r;
+      const float t1 = fmaf(tok[buf][1][i], vj, lam_lo * S[r]);
+      S[r] = fmaf(lam_hi, S[r], t1);
+      acc = fmaf(tok[buf][0][i], S[r], acc);
+    }
+    red[rg][j] = acc;
+    if (which < 3 && t + 1 < N) tok[buf ^ 1][which][e] = pf;
+    __syncthreads();
+    if (rg == 0) {
+      const float o = ((red[0][j] + red[1][j]) + red[2][j]) + red[3][j];
+      store_from_f32<T>(out, ((b * N + t) * H + h) * D + j, o);
+    }
+    if (which < 3 && t + 2 < N) pf = fetch(t + 2);
+    __syncthreads();
+  }
+
+  if (state_out != nullptr) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int i = rg * R + r;
+      state_out[(flat * D + i) * D + j] = S[r];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Decode step.  One CTA per flat head, 512 threads.  Thread t streams 128-bit quads of the fp32
+// state: column quad c4 = t % (D/4), rows r0, r0 + RS, ... with r0 = t / (D/4), RS = 512/(D/4).
+// All of a thread's state loads are issued before q, k, v are staged, so D*D*4/512 bytes per
+// thread are in flight at once; the updated state is written back in place with streaming
+// stores and the read-out o_j is reduced over the RS row slots through shared memory.
+// ---------------------------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(512) decode_kernel(const T* __restrict__ q,
+                                                     const T* __restrict__ k,
+                                                     const T* __restrict__ v,
+                                                     const float* __restrict__ slopes,
+                                                     float* __restrict__ state,
+                                                     T* __restrict__ out, int64_t H) {
+  constexpr int NT = 512;
+  constexpr int Q4 = D / 4;     // column quads per row
+  constexpr int RS = NT / Q4;   // row slots
+  constexpr int RPT = D / RS;   // rows per thread
+  __shared__ float sq[D], sk[D], sv[D];
+  __shared__ float red[RS][D];
+
+  const int tid = threadIdx.x;
+  const int c4 = tid % Q4;
+  const int r0 = tid / Q4;
+  const int64_t flat = blockIdx.x;
+  const int64_t h = flat % H;
+  float4* st = reinterpret_cast<float4*>(state + flat * D * D);
+
+  float4 s[RPT];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) s[r] = __ldcs(st + (r0 + r * RS) * Q4 + c4);
+
+  if (tid < 3 * D) {
+    const int which = tid / D, e = tid % D;
+    const T* src = which == 0 ? q : (which == 1 ? k : v);
+    const float x = load_as_f32<T>(src, flat * D + e);
+    (which == 0 ? sq : (which == 1 ? sk : sv))[e] = x;
+  }
+  float lam_hi, lam_lo;
+  split_decay(slopes[h], lam_hi, lam_lo);
+  __syncthreads();
+
+  const float v0 = sv[4 * c4 + 0], v1 = sv[4 * c4 + 1], v2 = sv[4 * c4 + 2], v3 = sv[4 * c4 + 3];
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    const int i = r0 + r * RS;
+    const float ki = sk[i], qi = sq[i];
+    float4 x = s[r];
+    x.x = fmaf(lam_hi, x.x, fmaf(ki, v0, lam_lo * x.x));
+    x.y = fmaf(lam_hi, x.y, fmaf(ki, v1, lam_lo * x.y));
+    x.z = fmaf(lam_hi, x.z, fmaf(ki, v2, lam_lo * x.z));
+    x.w = fmaf(lam_hi, x.w, fmaf(ki, v3, lam_lo * x.w));
+    a0 = fmaf(qi, x.x, a0);
+    a1 = fmaf(qi, x.y, a1);
+    a2 = fmaf(qi, x.z, a2);
+    a3 = fmaf(qi, x.w, a3);
+    __stcs(st + i * Q4 + c4, x);
+  }
+  red[r0][4 * c4 + 0] = a0;
+  red[r0][4 * c4 + 1] = a1;
+  red[r0][4 * c4 + 2] = a2;
+  red[r0][4 * c4 + 3] = a3;
+  __syncthreads();
+  if (tid < D) {
+    float o = 0.f;
+#pragma unroll
+    for (int rr = 0; rr < RS; ++rr) o += red[rr][tid];
+    store_from_f32<T>(out, flat * D + tid, o);
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_recurrent_typed(const PrefillArgs& a, cudaStream_t stream) {
+  const int64_t grid = a.B * a.H;
+  recurrent_prefill_kernel<T, D><<<static_cast<unsigned>(grid), 4 * D, 0, stream>>>(
+      static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
+      a.slopes, static_cast<T*>(a.out), a.state_out, a.N, a.H);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_decode_typed(const DecodeArgs& a, cudaStream_t stream) {
+  const int64_t grid = a.B * a.H;
+  decode_kernel<T, D><<<static_cast<unsigned>(grid), 512, 0, stream>>>(
+      static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
+      a.slopes, a.state, static_cast<T*>(a.out), a.H);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_recurrent_prefill(const PrefillArgs& a, cudaStream_t stream) {
+  if (a.dtype == kF32) {
+    return a.d == 64 ? launch_recurrent_typed<float, 64>(a, stream)
+                     : launch_recurrent_typed<float, 128>(a, stream);
+  }
+  return a.d == 64 ? launch_recurrent_typed<__nv_bfloat16, 64>(a, stream)
+                   : launch_recurrent_typed<__nv_bfloat16, 128>(a, stream);
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+  if (a.dtype == kF32) {
+    return a.d == 64 ? launch_decode_typed<float, 64>(a, stream)
+                     : launch_decode_typed<float, 128>(a, stream);
+  }
+  return a.d == 64 ? launch_decode_typed<__nv_bfloat16, 64>(a, stream)
+                   : launch_decode_typed<__nv_bfloat16, 128>(a, stream);
+}
+
+}  // namespace la

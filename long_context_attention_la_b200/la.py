@@ -1,0 +1,192 @@
+"""ctypes binding of the C ABI in include/la.h.
+
+The functions named like the C entry points (``la_prefill``, ``la_decode_step``, ...) take raw
+device pointers (ints) and return the status code, exactly like the C calls.  ``prefill`` and
+``decode_step`` are the tensor-level conveniences: they only check and marshal torch CUDA tensors
+into those calls; every step of the computation runs in the library's CUDA kernels.
+
+There is no fallback: if libla_b200.so has not been built, or the tensors are not on a CUDA
+device, these functions raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "libla_b200.so")
+
+LA_OK = 0
+LA_ERR_NULL = -1
+LA_ERR_SHAPE = -2
+LA_ERR_DTYPE = -3
+LA_ERR_ALIGN = -4
+LA_ERR_OVERFLOW = -5
+LA_ERR_WORKSPACE = -6
+LA_ERR_CUDA = -7
+LA_ERR_TIMEOUT = -8
+LA_ERR_UNSUPPORTED = -9
+LA_ERR_ALIAS = -10
+
+LA_BF16 = 0
+LA_F32 = 1
+
+LA_PATH_AUTO = 0
+LA_PATH_TENSOR = 1
+LA_PATH_RECURRENT = 2
+
+
+class la_desc(ctypes.Structure):  # noqa: N801 - mirrors the C type name
+    _fields_ = [("B", ctypes.c_int64), ("N", ctypes.c_int64), ("H", ctypes.c_int64),
+                ("d", ctypes.c_int64), ("dtype", ctypes.c_int32), ("chunk", ctypes.c_int32),
+                ("segments", ctypes.c_int32), ("path", ctypes.c_int32)]
+
+
+class LaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {la_status_string(status)} ({status})")
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library(path: str | None = None):
+    """The loaded libla_b200.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"{p} is missing: build it with "
+                               "`python -m long_context_attention_la_b200.build`")
+        lib = ctypes.CDLL(p)
+        vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+        lib.la_prefill_workspace_bytes.argtypes = [ctypes.POINTER(la_desc)]
+        lib.la_prefill_workspace_bytes.restype = sz
+        lib.la_prefill.argtypes = [ctypes.POINTER(la_desc), vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.la_prefill.restype = ctypes.c_int
+        lib.la_decode_step.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp]
+        lib.la_decode_step.restype = ctypes.c_int
+        lib.la_workspace_status.argtypes = [vp, vp]
+        lib.la_workspace_status.restype = ctypes.c_int
+        lib.la_status_string.argtypes = [ctypes.c_int]
+        lib.la_status_string.restype = ctypes.c_char_p
+        lib.la_version.argtypes = []
+        lib.la_version.restype = ctypes.c_int
+        if path is None:
+            _lib = lib
+        return lib
+
+
+# ------------------------------------------------------------------------------------------
+# the C entry points, one to one
+# ------------------------------------------------------------------------------------------
+def la_prefill_workspace_bytes(desc: la_desc) -> int:
+    return int(library().la_prefill_workspace_bytes(ctypes.byref(desc)))
+
+
+def la_prefill(desc: la_desc, q: int, k: int, v: int, slopes: int, out: int, state_out: int,
+               workspace: int, workspace_bytes: int, stream: int) -> int:
+    return int(library().la_prefill(ctypes.byref(desc), q, k, v, slopes, out, state_out or None,
+                                    workspace or None, workspace_bytes, stream or None))
+
+
+def la_decode_step(B: int, H: int, d: int, dtype: int, q: int, k: int, v: int, slopes: int,
+                   state_inout: int, out: int, stream: int) -> int:
+    return int(library().la_decode_step(B, H, d, dtype, q, k, v, slopes, state_inout, out,
+                                        stream or None))
+
+
+def la_workspace_status(workspace: int, stream: int) -> int:
+    return int(library().la_workspace_status(workspace, stream or None))
+
+
+def la_status_string(status: int) -> str:
+    return library().la_status_string(int(status)).decode()
+
+
+def la_version() -> int:
+    return int(library().la_version())
+
+
+# ------------------------------------------------------------------------------------------
+# tensor conveniences (argument marshalling only)
+# ------------------------------------------------------------------------------------------
+_DT = {torch.bfloat16: LA_BF16, torch.float32: LA_F32}
+
+
+def _cuda_ptr(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def make_desc(B, N, H, d, dtype, chunk=0, segments=0, path=LA_PATH_AUTO) -> la_desc:
+    return la_desc(B, N, H, d, _DT[dtype] if isinstance(dtype, torch.dtype) else int(dtype),
+                   chunk, segments, path)
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor, *,
+            out: torch.Tensor | None = None, state_out: torch.Tensor | None = None,
+            want_state: bool = True, chunk: int = 0, segments: int = 0,
+            path: int = LA_PATH_AUTO, workspace: torch.Tensor | None = None,
+            stream: torch.cuda.Stream | None = None):
+    """o, state = prefill(q, k, v, slopes): q, k, v [B, N, H, d] (bf16 or fp32, CUDA,
+    contiguous), slopes float32[H].  Returns out [B, N, H, d] and the final fp32 state
+    [B, H, d, d] (None if want_state is False and no state_out is given)."""
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share one [B, N, H, d] shape")
+    if q.dtype not in _DT or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must all be bfloat16 or all float32")
+    B, N, H, d = q.shape
+    if slopes.dtype != torch.float32 or slopes.shape != (H,):
+        raise ValueError("slopes must be float32[H]")
+    if out is None:
+        out = torch.empty_like(q)
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+    desc = make_desc(B, N, H, d, q.dtype, chunk, segments, path)
+    need = la_prefill_workspace_bytes(desc)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = 0 if workspace is None else _cuda_ptr(workspace, "workspace")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    st = la_prefill(desc, _cuda_ptr(q, "q"), _cuda_ptr(k, "k"), _cuda_ptr(v, "v"),
+                    _cuda_ptr(slopes, "slopes"), _cuda_ptr(out, "out"),
+                    0 if state_out is None else _cuda_ptr(state_out, "state_out"), ws_ptr,
+                    ws_bytes, s.cuda_stream)
+    if st != LA_OK:
+        raise LaError(st, "la_prefill")
+    return out, state_out
+
+
+def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor,
+                state: torch.Tensor, *, out: torch.Tensor | None = None,
+                stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """o = decode_step(q, k, v, slopes, state): q, k, v [B, H, d]; state fp32 [B, H, d, d] is
+    updated in place (decay, add k^T v, read out)."""
+    if q.dim() != 3 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share one [B, H, d] shape")
+    if q.dtype not in _DT or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must all be bfloat16 or all float32")
+    B, H, d = q.shape
+    if state.dtype != torch.float32 or tuple(state.shape) != (B, H, d, d):
+        raise ValueError("state must be float32 [B, H, d, d]")
+    if out is None:
+        out = torch.empty_like(q)
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    st = la_decode_step(B, H, d, _DT[q.dtype], _cuda_ptr(q, "q"), _cuda_ptr(k, "k"),
+                        _cuda_ptr(v, "v"), _cuda_ptr(slopes, "slopes"),
+                        _cuda_ptr(state, "state"), _cuda_ptr(out, "out"), s.cuda_stream)
+    if st != LA_OK:
+        raise LaError(st, "la_decode_step")
+    return out

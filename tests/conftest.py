@@ -16,6 +16,13 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: test needs a CUDA GPU (sm_100a)")
 
 
+@pytest.fixture(scope="session", autouse=True)
+def _built_library():
+    """Build libla_b200.so (in-tree, sm_100a) once per session if a source is newer."""
+    from long_context_attention_la_b200 import build
+    build.build()
+
+
 def pytest_collection_modifyitems(config, items):
     try:
         import torch
