@@ -18,7 +18,8 @@
  * Conventions shared by every entry point.
  *   - All tensor pointers are DEVICE pointers (cudaMalloc / PyTorch CUDA memory) unless a
  *     parameter says otherwise.  The caller owns every buffer; the library keeps no allocations,
- *     handles or global state between calls.
+ *     handles or global state between calls (the one exception is the fixed scratch array behind
+ *     la_prefill_noalloc).
  *   - Activations q, k, v, out are laid out token-major, [B, N, H, d] contiguous (d innermost),
  *     as a fused QKV projection writes them.  Element type is bf16 (LA_BF16) or fp32 (LA_F32).
  *   - The recurrent state is always fp32, [B, H, d, d] contiguous, S[b][h][i][j] with i over the
@@ -126,6 +127,41 @@ la_status la_prefill(const la_desc* desc, const void* q, const void* k, const vo
 la_status la_decode_step(int64_t B, int64_t H, int64_t d, int32_t dtype, const void* q,
                          const void* k, const void* v, const float* slopes, float* state_inout,
                          void* out, void* stream);
+
+/*
+ * la_prefill_noalloc — la_prefill for callers that cannot allocate device memory.
+ *
+ * The report has no counterpart to this call; it exists for callers of this library that must
+ * not call cudaMalloc (or any allocating routine) once they are running: serving loops that
+ * reserved all device memory for their own pool allocator at start-up (a stray cudaMalloc would
+ * fail, or synchronise the whole device and stall other streams), and host frameworks or plugin
+ * interfaces that hand a kernel library its inputs and outputs but no allocator.
+ *
+ * Same computation, arguments and errors as la_prefill, minus the workspace: the scratch memory
+ * (work counter, status word, scan flags and segment-state ring) is a fixed array of
+ * LA_NOALLOC_SCRATCH_BYTES bytes compiled into the library.  Every GPU that loads the library
+ * holds that array until the process exits.  The caller still passes q, k, v, slopes, out and
+ * state_out.
+ *
+ *   - Limit: problems whose scratch need (la_prefill_workspace_bytes) exceeds
+ *     LA_NOALLOC_SCRATCH_BYTES are rejected with LA_ERR_WORKSPACE before anything is enqueued.
+ *     Within the limit are every problem with B*H <= 64 (for example one sequence of the 64-head
+ *     layer at any length) and every problem that needs no segment scan (B*H at least twice the
+ *     number of SMs); the fp32 / recurrent path needs no scratch at all.
+ *   - First call on a device: it looks up the device address of the array (cudaGetSymbolAddress)
+ *     with that device current and caches it; make that first call before any stream capture.
+ *   - Sharing: all calls on a device use the same array, which keeps the previous call's
+ *     contents; each call zeroes the parts that must start at zero.  Calls whose executions
+ *     overlap on the GPU (different streams, or threads without ordering) race on the array and
+ *     give wrong results; order them on one stream or use la_prefill with separate workspaces.
+ *   - Device status: a bounded device wait that gives up (it needs the GPU to be starved for
+ *     seconds) leaves the outputs invalid and is recorded only in the array, which this call
+ *     offers no way to read; callers that must observe it use la_prefill with their own
+ *     workspace and la_workspace_status.
+ */
+#define LA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u + 4096u)
+la_status la_prefill_noalloc(const la_desc* desc, const void* q, const void* k, const void* v,
+                             const float* slopes, void* out, float* state_out, void* stream);
 
 /* Synchronises `stream`, then returns the device status word of a workspace that la_prefill
  * used: LA_OK, or LA_ERR_TIMEOUT if a bounded device wait gave up during the last call. */

@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "la.h"
 #include "la_internal.h"
@@ -139,6 +140,63 @@ la_status la_decode_step(int64_t B, int64_t H, int64_t d, int32_t dtype, const v
   la::DecodeArgs a{B, H, d, dtype, q, k, v, slopes, state_inout, out};
   return la::launch_decode(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? LA_OK
                                                                                  : LA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------------------------
+// la_prefill_noalloc: la_prefill on a scratch array compiled into the library, for callers that
+// cannot allocate device memory (see la.h).  The array is a device symbol; host code never uses
+// its name as an address, it asks the runtime for the device address once per device.
+// ---------------------------------------------------------------------------------------------
+}  // extern "C"
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 256;
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device (looked up on first use).
+la_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return LA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_noalloc_scratch) != cudaSuccess ||
+        p == nullptr)
+      return LA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+la_status la_prefill_noalloc(const la_desc* desc, const void* q, const void* k, const void* v,
+                             const float* slopes, void* out, float* state_out, void* stream) {
+  int64_t numel = 0;
+  const la_status st = check_desc(desc, &numel);
+  if (st != LA_OK) return st;
+  if (!use_tensor_path(desc)) {
+    // the recurrent kernel uses no scratch memory
+    return la_prefill(desc, q, k, v, slopes, out, state_out, nullptr, 0, stream);
+  }
+  const int sms = device_sms();
+  if (sms <= 0) return LA_ERR_CUDA;
+  const la::SegmentPlan plan = la::plan_segments(desc->B, desc->N, desc->H, desc->segments, sms);
+  const size_t need = la::workspace_layout(desc->B, desc->H, plan).total;
+  if (need > LA_NOALLOC_SCRATCH_BYTES) return LA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const la_status sa = noalloc_scratch(&scratch);
+  if (sa != LA_OK) return sa;
+  return la_prefill(desc, q, k, v, slopes, out, state_out, scratch, LA_NOALLOC_SCRATCH_BYTES,
+                    stream);
 }
 
 la_status la_workspace_status(const void* workspace, void* stream) {

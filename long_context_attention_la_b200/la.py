@@ -71,6 +71,8 @@ def library(path: str | None = None):
         lib.la_prefill_workspace_bytes.restype = sz
         lib.la_prefill.argtypes = [ctypes.POINTER(la_desc), vp, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.la_prefill.restype = ctypes.c_int
+        lib.la_prefill_noalloc.argtypes = [ctypes.POINTER(la_desc), vp, vp, vp, vp, vp, vp, vp]
+        lib.la_prefill_noalloc.restype = ctypes.c_int
         lib.la_decode_step.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp]
         lib.la_decode_step.restype = ctypes.c_int
         lib.la_workspace_status.argtypes = [vp, vp]
@@ -95,6 +97,16 @@ def la_prefill(desc: la_desc, q: int, k: int, v: int, slopes: int, out: int, sta
                workspace: int, workspace_bytes: int, stream: int) -> int:
     return int(library().la_prefill(ctypes.byref(desc), q, k, v, slopes, out, state_out or None,
                                     workspace or None, workspace_bytes, stream or None))
+
+
+def la_prefill_noalloc(desc: la_desc, q: int, k: int, v: int, slopes: int, out: int,
+                       state_out: int, stream: int) -> int:
+    """la_prefill on the library's built-in scratch array (no device allocation); see la.h."""
+    return int(library().la_prefill_noalloc(ctypes.byref(desc), q, k, v, slopes, out,
+                                            state_out or None, stream or None))
+
+
+LA_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024 + 4096
 
 
 def la_decode_step(B: int, H: int, d: int, dtype: int, q: int, k: int, v: int, slopes: int,
