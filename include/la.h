@@ -146,8 +146,9 @@ la_status la_decode_step(int64_t B, int64_t H, int64_t d, int32_t dtype, const v
  *   - Limit: problems whose scratch need (la_prefill_workspace_bytes) exceeds
  *     LA_NOALLOC_SCRATCH_BYTES are rejected with LA_ERR_WORKSPACE before anything is enqueued.
  *     Within the limit are every problem with B*H <= 64 (for example one sequence of the 64-head
- *     layer at any length) and every problem that needs no segment scan (B*H at least twice the
- *     number of SMs); the fp32 / recurrent path needs no scratch at all.
+ *     layer at any length) and every problem run with one segment per sequence (the automatic
+ *     choice once B*H exceeds half the number of SMs); the fp32 / recurrent path needs no
+ *     scratch at all.
  *   - First call on a device: it looks up the device address of the array (cudaGetSymbolAddress)
  *     with that device current and caches it; make that first call before any stream capture.
  *   - Sharing: all calls on a device use the same array, which keeps the previous call's

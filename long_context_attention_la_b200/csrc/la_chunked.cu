@@ -14,15 +14,18 @@
 // "fused update h"), and then runs its output chunks starting from that state (the "fused
 // update O", folded into the inter-chunk term instead of a separate correction pass).
 //
-// Execution: one persistent CTA per SM (512 threads, ~226 KB shared memory, all 512 TMEM
+// Execution: one persistent CTA per SM (640 threads, ~226 KB shared memory, all 512 TMEM
 // columns).  Work units (segment, b, h) are taken in segment-major order from an atomic counter,
 // so a unit only ever waits on units that running CTAs already hold.  Roles:
-//   warp 0       TMA producer (two-stage ring of Q/K/V tiles)
-//   warp 1       tcgen05.mma issuer
+//   warp 0       TMA producer: two-stage ring of Q/K/V tiles, L2 prefetch a few chunks ahead
+//   warp 1       tcgen05.mma issuer; per chunk c it issues S_c, then the state update of chunk
+//                c-1, then O_inter_c and O_intra_c, so S_c overlaps the row scaling of K_{c-1}
 //   warp 2       TMEM allocator
-//   warps 4-7    P = decay-mask(S) into TMEM, and K -> K~ (row-scaled) in shared memory
-//   warps 8-11   state: look-back scan, KV -> bf16 operand, decay rescale, final state
-//   warps 12-15  output epilogue: O = O_intra + lambda^(i+1) O_inter -> bf16 -> TMA store
+//   warps 4-11   P = decay-mask(S) into TMEM (two warps per TMEM lane quarter, alternate
+//                32-column blocks); K -> K~ (row-scaled) during the local-state pass
+//   warps 12-15  state: look-back scan, KV -> bf16 operand, decay rescale, final state, and
+//                K -> K~ during the output pass
+//   warps 16-19  output epilogue: O = O_intra + lambda^(i+1) O_inter -> bf16 -> global
 // Every wait (mbarrier or scan flag) is bounded in time; on expiry the CTA records
 // LA_ERR_TIMEOUT in the workspace status word, unwinds, frees its TMEM and exits.
 #include <cuda.h>
@@ -30,6 +33,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstdlib>
 
 #include "la_internal.h"
 #include "la_sm100.cuh"
@@ -39,7 +43,11 @@ namespace {
 
 constexpr int C = kChunk;      // 128 tokens per chunk
 constexpr int D = kHeadDim;    // 128
-constexpr int kThreads = 512;
+constexpr int kThreads = 640;  // 20 warps
+constexpr uint32_t kWarpP0 = 4;    // warps 4..11: decay mask / local-pass K scaling
+constexpr uint32_t kWarpS0 = 12;   // warps 12..15: state
+constexpr uint32_t kWarpO0 = 16;   // warps 16..19: output epilogue
+constexpr uint32_t kBarP = 1, kBarS = 2, kBarO = 3;  // named barriers of the three groups
 constexpr uint32_t kTileBytes = C * D * 2;           // one bf16 [128 x 128] tile
 constexpr uint32_t kHalfBytes = kTileBytes / 2;      // [128 rows x 64 cols], 128-byte rows
 constexpr uint32_t kOffQ = 0;
@@ -96,7 +104,7 @@ struct Params {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
-  CUtensorMap tm_o;
+  __nv_bfloat16* out;
   const float* slopes;
   float* state_out;
   uint32_t* counter;
@@ -106,20 +114,21 @@ struct Params {
   int64_t N, H, BH;
   int64_t n_chunks, seg_chunks, segments, units;
   uint64_t timeout_ns;
+  int32_t prefetch_depth;
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// All 128 threads of a warpgroup agree on `ok` (logical AND) at named barrier `id`.
-__device__ __forceinline__ bool wg_all(bool ok, uint32_t id) {
+// All `count` threads of a role group agree on `ok` (logical AND) at named barrier `id`.
+__device__ __forceinline__ bool group_all(bool ok, uint32_t id, uint32_t count) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"(ok ? 1u : 0u), "r"(id)
+      : "r"(ok ? 1u : 0u), "r"(id), "r"(count)
       : "memory");
   return r != 0;
 }
@@ -142,6 +151,28 @@ __device__ __forceinline__ int32_t ld_volatile_s32(const int32_t* p) {
 // with the 128-byte swizzle (8-row, 1024-byte atoms; chunk index XOR row-in-atom).
 __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t c16) {
   return (r >> 3) * 1024u + (r & 7u) * 128u + ((c16 ^ (r & 7u)) << 4);
+}
+
+// Multiplies the 64 bf16 of one half-row (row r of a swizzled [128 x 64] half-tile) by w, in
+// fp32 with one rounding.  Step c touches physical chunk c ^ (r & 7), so the 8 rows of a swizzle
+// atom hit 8 different 16-byte bank groups at every step.
+__device__ __forceinline__ void scale_half_row(uint8_t* half_tile, uint32_t r, float w) {
+  uint8_t* row = half_tile + (r >> 3) * 1024u + (r & 7u) * 128u;
+#pragma unroll
+  for (uint32_t c0 = 0; c0 < 8; c0 += 4) {  // four loads in flight, then four stores
+    uint4 x[4];
+#pragma unroll
+    for (uint32_t c = 0; c < 4; ++c)
+      x[c] = *reinterpret_cast<const uint4*>(row + (((c0 + c) ^ (r & 7u)) << 4));
+#pragma unroll
+    for (uint32_t c = 0; c < 4; ++c) {
+      x[c].x = pack_bf16x2(bf16lo_to_f32(x[c].x) * w, bf16hi_to_f32(x[c].x) * w);
+      x[c].y = pack_bf16x2(bf16lo_to_f32(x[c].y) * w, bf16hi_to_f32(x[c].y) * w);
+      x[c].z = pack_bf16x2(bf16lo_to_f32(x[c].z) * w, bf16hi_to_f32(x[c].z) * w);
+      x[c].w = pack_bf16x2(bf16lo_to_f32(x[c].w) * w, bf16hi_to_f32(x[c].w) * w);
+      *reinterpret_cast<uint4*>(row + (((c0 + c) ^ (r & 7u)) << 4)) = x[c];
+    }
+  }
 }
 
 __device__ __forceinline__ void decode_unit(const Params& p, int64_t u, UnitInfo& ui) {
@@ -174,13 +205,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctrl->full[s], 1);
-      mbar_init(&ctrl->empty[s], 2);
+      mbar_init(&ctrl->empty[s], 1);
       mbar_init(&ctrl->kt_ready[s], 128);
       mbar_init(&ctrl->unit_full[s], 1);
-      mbar_init(&ctrl->unit_empty[s], 1 + 3 * 128);
+      mbar_init(&ctrl->unit_empty[s], 1 + 256 + 128 + 128);
     }
     mbar_init(&ctrl->s_full, 1);
-    mbar_init(&ctrl->p_ready, 128);
+    mbar_init(&ctrl->p_ready, 256);
     mbar_init(&ctrl->o_full, 1);
     mbar_init(&ctrl->o_free, 128);
     mbar_init(&ctrl->kv_done, 1);
@@ -193,7 +224,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&p.tm_q);
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
-    tma_prefetch_desc(&p.tm_o);
   }
   if (warp == 2) {
     tmem_alloc(&ctrl->tmem_base, 512);
@@ -211,56 +241,107 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint64_t pol_first = policy_evict_first();
       const uint64_t pol_last = policy_evict_last();
-      uint32_t g = 0;
-      uint32_t j = 0;
-      uint32_t issued[2] = {0, 0};  // fills issued per stage (for the abort drain)
-      bool ok = true;
-      while (ok) {
-        const uint32_t slot = j & 1;
-        if (!mbar_wait_bounded(&ctrl->unit_empty[slot], ((j >> 1) & 1) ^ 1, abort_flag, T)) {
-          ok = false;
-          break;
-        }
+      const uint64_t pol_normal = policy_evict_normal();
+      const int32_t depth = p.prefetch_depth;  // chunk-loads brought into L2 ahead of time
+
+      // A unit is a stream of chunk-loads: nc local-state loads (K, V) if it has that pass,
+      // then nc output loads (Q, K, V).
+      auto fetch = [&](UnitInfo& ui) {
         const int64_t u = static_cast<int64_t>(atomicAdd(p.counter, 1u));
-        UnitInfo ui;
         if (u < p.units) {
           decode_unit(p, u, ui);
         } else {
           ui.bh = -1;
           ui.seg = ui.c0 = ui.nc = ui.len = ui.flags = 0;
         }
-        ctrl->units[slot] = ui;
-        mbar_arrive(&ctrl->unit_full[slot]);
-        if (ui.bh < 0) break;
+      };
+      auto n_loads = [](const UnitInfo& ui) -> int32_t {
+        return ui.bh < 0 ? 0 : ((ui.flags & 1) ? 2 * ui.nc : ui.nc);
+      };
+      // L2 prefetch of chunk-load `pos` of `ui` (the part of it that comes from DRAM)
+      auto prefetch = [&](const UnitInfo& ui, int32_t pos) {
         const int32_t b = static_cast<int32_t>(ui.bh / p.H);
         const int32_t h = static_cast<int32_t>(ui.bh % p.H);
-        const int passes = (ui.flags & 1) ? 2 : 1;
-        for (int pass = 0; pass < passes && ok; ++pass) {
-          const bool local_state_pass = (passes == 2 && pass == 0);
-          for (int32_t c = 0; c < ui.nc; ++c) {
-            const uint32_t s = g & 1;
-            if (!mbar_wait_bounded(&ctrl->empty[s], ((g >> 1) & 1) ^ 1, abort_flag, T)) {
-              ok = false;
-              break;
-            }
-            uint8_t* st = smem + s * kStageBytes;
-            const int32_t n0 = (ui.c0 + c) * C;
-            const uint64_t kv_pol = local_state_pass ? pol_last : pol_first;
-            if (local_state_pass) {
-              mbar_arrive_expect_tx(&ctrl->full[s], 2 * kTileBytes);
+        const bool two_pass = (ui.flags & 1) != 0;
+        const bool local_pass = two_pass && pos < ui.nc;
+        const int32_t c = two_pass && !local_pass ? pos - ui.nc : pos;
+        const int32_t n0 = (ui.c0 + c) * C;
+        if (!local_pass) {
+          tma_prefetch_l2_4d(&p.tm_q, 0, h, n0, b, pol_normal);
+          tma_prefetch_l2_4d(&p.tm_q, 64, h, n0, b, pol_normal);
+        }
+        if (local_pass || !two_pass) {
+          const uint64_t pol = local_pass ? pol_last : pol_normal;
+          tma_prefetch_l2_4d(&p.tm_k, 0, h, n0, b, pol);
+          tma_prefetch_l2_4d(&p.tm_k, 64, h, n0, b, pol);
+          tma_prefetch_l2_4d(&p.tm_v, 0, h, n0, b, pol);
+          tma_prefetch_l2_4d(&p.tm_v, 64, h, n0, b, pol);
+        }
+      };
+
+      uint32_t g = 0;
+      uint32_t j = 0;
+      uint32_t issued[2] = {0, 0};  // fills issued per stage (for the abort drain)
+      bool ok = true;
+      UnitInfo cur, nxt;
+      bool have_nxt = false;
+      while (ok) {
+        const uint32_t slot = j & 1;
+        if (!mbar_wait_bounded(&ctrl->unit_empty[slot], ((j >> 1) & 1) ^ 1, abort_flag, T)) {
+          ok = false;
+          break;
+        }
+        if (have_nxt) {
+          cur = nxt;
+          have_nxt = false;
+        } else {
+          fetch(cur);
+          for (int32_t q = 0; q < min(depth, n_loads(cur)); ++q) prefetch(cur, q);
+        }
+        ctrl->units[slot] = cur;
+        mbar_arrive(&ctrl->unit_full[slot]);
+        if (cur.bh < 0) break;
+        const int32_t b = static_cast<int32_t>(cur.bh / p.H);
+        const int32_t h = static_cast<int32_t>(cur.bh % p.H);
+        const int32_t n_cur = n_loads(cur);
+        for (int32_t pos = 0; pos < n_cur; ++pos) {
+          // keep `depth` chunk-loads ahead in L2, running into the next unit near the end
+          if (depth > 0) {
+            const int32_t q = pos + depth;
+            if (q < n_cur) {
+              prefetch(cur, q);
             } else {
-              mbar_arrive_expect_tx(&ctrl->full[s], 3 * kTileBytes);
-              tma_load_4d(st + kOffQ, &p.tm_q, &ctrl->full[s], 0, h, n0, b, pol_first);
-              tma_load_4d(st + kOffQ + kHalfBytes, &p.tm_q, &ctrl->full[s], 64, h, n0, b,
-                          pol_first);
+              if (!have_nxt) {
+                fetch(nxt);
+                have_nxt = true;
+              }
+              if (q - n_cur < n_loads(nxt)) prefetch(nxt, q - n_cur);
             }
-            tma_load_4d(st + kOffK, &p.tm_k, &ctrl->full[s], 0, h, n0, b, kv_pol);
-            tma_load_4d(st + kOffK + kHalfBytes, &p.tm_k, &ctrl->full[s], 64, h, n0, b, kv_pol);
-            tma_load_4d(st + kOffV, &p.tm_v, &ctrl->full[s], 0, h, n0, b, kv_pol);
-            tma_load_4d(st + kOffV + kHalfBytes, &p.tm_v, &ctrl->full[s], 64, h, n0, b, kv_pol);
-            issued[s] += 1;
-            ++g;
           }
+          const uint32_t s = g & 1;
+          if (!mbar_wait_bounded(&ctrl->empty[s], ((g >> 1) & 1) ^ 1, abort_flag, T)) {
+            ok = false;
+            break;
+          }
+          const bool local_state_pass = (cur.flags & 1) && pos < cur.nc;
+          const int32_t c = (cur.flags & 1) && !local_state_pass ? pos - cur.nc : pos;
+          uint8_t* st = smem + s * kStageBytes;
+          const int32_t n0 = (cur.c0 + c) * C;
+          const uint64_t kv_pol = local_state_pass ? pol_last : pol_first;
+          if (local_state_pass) {
+            mbar_arrive_expect_tx(&ctrl->full[s], 2 * kTileBytes);
+          } else {
+            mbar_arrive_expect_tx(&ctrl->full[s], 3 * kTileBytes);
+            tma_load_4d(st + kOffQ, &p.tm_q, &ctrl->full[s], 0, h, n0, b, pol_first);
+            tma_load_4d(st + kOffQ + kHalfBytes, &p.tm_q, &ctrl->full[s], 64, h, n0, b,
+                        pol_first);
+          }
+          tma_load_4d(st + kOffK, &p.tm_k, &ctrl->full[s], 0, h, n0, b, kv_pol);
+          tma_load_4d(st + kOffK + kHalfBytes, &p.tm_k, &ctrl->full[s], 64, h, n0, b, kv_pol);
+          tma_load_4d(st + kOffV, &p.tm_v, &ctrl->full[s], 0, h, n0, b, kv_pol);
+          tma_load_4d(st + kOffV + kHalfBytes, &p.tm_v, &ctrl->full[s], 64, h, n0, b, kv_pol);
+          issued[s] += 1;
+          ++g;
         }
         ++j;
       }
@@ -289,6 +370,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t g = 0, j = 0;
       uint32_t n_kvb = 0, n_ofree = 0, n_p = 0;
       bool ok = true;
+      // KV (+)= K~^T V for the chunk held in stage (gg & 1)
+      auto issue_state_update = [&](uint32_t gg, bool accumulate_first) {
+        const uint32_t kb = smem_base + (gg & 1) * kStageBytes + kOffK;
+        const uint32_t vb = smem_base + (gg & 1) * kStageBytes + kOffV;
+#pragma unroll
+        for (uint32_t kk = 0; kk < 8; ++kk) {
+          umma_ss(tmem + kColKV, make_sdesc_sw128(kb + kk * 2048, kHalfBytes, 1024),
+                  make_sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idKV,
+                  (accumulate_first || kk > 0) ? 1u : 0u);
+        }
+      };
       while (ok) {
         const uint32_t slot = j & 1;
         if (!mbar_wait_bounded(&ctrl->unit_full[slot], (j >> 1) & 1, abort_flag, T)) break;
@@ -309,16 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t kb = smem_base + s * kStageBytes + kOffK;
-            const uint32_t vb = smem_base + s * kStageBytes + kOffV;
-#pragma unroll
-            for (uint32_t kk = 0; kk < 8; ++kk) {
-              umma_ss(tmem + kColKV, make_sdesc_sw128(kb + kk * 2048, kHalfBytes, 1024),
-                      make_sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idKV,
-                      (c > 0 || kk > 0) ? 1u : 0u);
-            }
+            issue_state_update(g, c > 0);
             umma_commit(&ctrl->empty[s]);
-            mbar_arrive(&ctrl->empty[s]);
             ++g;
           }
           if (!ok) break;
@@ -327,6 +411,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int32_t c = 0; c < ui.nc && ok; ++c) {
           const uint32_t s = g & 1;
           const uint32_t ph = (g >> 1) & 1;
+          // The state update of the previous chunk goes first if its K~ is already scaled (it
+          // does not touch what S_c reads or writes); otherwise it follows S_c.
+          bool prev_issued = false;
+          if (c > 0 && mbar_test_wait(&ctrl->kt_ready[(g - 1) & 1], ((g - 1) >> 1) & 1)) {
+            tc_fence_after();
+            issue_state_update(g - 1, true);
+            umma_commit(&ctrl->kv_done);
+            umma_commit(&ctrl->empty[(g - 1) & 1]);
+            prev_issued = true;
+          }
           if (!mbar_wait_bounded(&ctrl->full[s], ph, abort_flag, T)) {
             ok = false;
             break;
@@ -336,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t kb = smem_base + s * kStageBytes + kOffK;
           const uint32_t vb = smem_base + s * kStageBytes + kOffV;
           const uint32_t kvb = smem_base + kOffKVb;
-          // S = Q K^T
+          // S_c = Q K^T
 #pragma unroll
           for (uint32_t kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
@@ -344,6 +438,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_sdesc_sw128(kb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
           }
           umma_commit(&ctrl->s_full);
+          // state update of the previous chunk (its K~ was scaled while S_c ran)
+          if (c > 0 && !prev_issued) {
+            const uint32_t gp = g - 1;
+            if (!mbar_wait_bounded(&ctrl->kt_ready[gp & 1], (gp >> 1) & 1, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_state_update(gp, true);
+            umma_commit(&ctrl->kv_done);
+            umma_commit(&ctrl->empty[gp & 1]);
+          }
           // O_inter = Q KV_in (needs the bf16 state operand and a free O accumulator)
           if (!mbar_wait_bounded(&ctrl->kvb_ready, n_kvb & 1, abort_flag, T) ||
               !mbar_wait_bounded(&ctrl->o_free, n_ofree & 1, abort_flag, T)) {
@@ -373,20 +479,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idPV, kk > 0 ? 1u : 0u);
           }
           umma_commit(&ctrl->o_full);
-          // KV <- lambda^n KV (done by the state warps) + K~^T V
-          if (!mbar_wait_bounded(&ctrl->kt_ready[s], ph, abort_flag, T)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (uint32_t kk = 0; kk < 8; ++kk) {
-            umma_ss(tmem + kColKV, make_sdesc_sw128(kb + kk * 2048, kHalfBytes, 1024),
-                    make_sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idKV, 1u);
-          }
-          umma_commit(&ctrl->kv_done);
-          umma_commit(&ctrl->empty[s]);
           ++g;
+        }
+        if (!ok) break;
+        // state update of the unit's last chunk
+        {
+          const uint32_t gp = g - 1;
+          if (!mbar_wait_bounded(&ctrl->kt_ready[gp & 1], (gp >> 1) & 1, abort_flag, T)) break;
+          tc_fence_after();
+          issue_state_update(gp, true);
+          umma_commit(&ctrl->kv_done);
+          umma_commit(&ctrl->empty[gp & 1]);
         }
         ++j;
       }
@@ -397,139 +500,137 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= kWarpP0 && warp < kWarpS0) {
     // =========================================================================================
-    // P = decay-mask(S) -> TMEM (bf16), K -> K~ in shared memory
+    // P = decay-mask(S) -> TMEM (bf16); K -> K~ in the local-state pass
     // =========================================================================================
-    const uint32_t wq = warp & 3;
-    const uint32_t i = wq * 32 + lane;  // row of the chunk (query token / key token)
+    const uint32_t pw = warp - kWarpP0;          // 0..7
+    const uint32_t wq = warp & 3;                // TMEM lane quarter
+    const uint32_t hf = pw >> 2;                 // column blocks hf and hf + 2
+    const uint32_t i = wq * 32 + lane;           // row of the chunk (query token)
+    const uint32_t tp = threadIdx.x - kWarpP0 * 32;  // 0..255
     const uint32_t trow = tmem + ((wq * 32) << 16);
     uint32_t g = 0, j = 0, n_s = 0;
     while (true) {
       const uint32_t slot = j & 1;
       bool ok = mbar_wait_bounded(&ctrl->unit_full[slot], (j >> 1) & 1, abort_flag, T);
-      if (!wg_all(ok, 1)) break;
+      if (!group_all(ok, kBarP, 256)) break;
       const UnitInfo ui = ctrl->units[slot];
       mbar_arrive(&ctrl->unit_empty[slot]);
       if (ui.bh < 0) break;
       const float alpha = p.slopes[ui.bh % p.H] * kLog2e;  // lambda^n = exp2(-alpha n)
-      const bool fast = alpha * 31.f <= 120.f;
-      float bm[32];  // 2^(alpha m) = lambda^(-m), m = 0..31
-#pragma unroll
-      for (int m = 0; m < 32; ++m) bm[m] = fast ? exp2f(alpha * static_cast<float>(m)) : 0.f;
-
-      auto scale_k_row = [&](uint32_t s, float w) {
-        uint8_t* kt = smem + s * kStageBytes + kOffK;
-#pragma unroll
-        for (uint32_t half = 0; half < 2; ++half) {
-          uint8_t* row = kt + half * kHalfBytes + (i >> 3) * 1024u + (i & 7u) * 128u;
-#pragma unroll
-          for (uint32_t c = 0; c < 8; ++c) {
-            uint4* q4 = reinterpret_cast<uint4*>(row + ((c ^ (i & 7u)) << 4));
-            uint4 x = *q4;
-            x.x = pack_bf16x2(bf16lo_to_f32(x.x) * w, bf16hi_to_f32(x.x) * w);
-            x.y = pack_bf16x2(bf16lo_to_f32(x.y) * w, bf16hi_to_f32(x.y) * w);
-            x.z = pack_bf16x2(bf16lo_to_f32(x.z) * w, bf16hi_to_f32(x.z) * w);
-            x.w = pack_bf16x2(bf16lo_to_f32(x.w) * w, bf16hi_to_f32(x.w) * w);
-            *q4 = x;
-          }
-        }
-      };
+      const float lam1 = ex2_approx(-alpha);                 // lambda
 
       if (ui.flags & 1) {
+        // local-state pass: K~_j = lambda^(L-1-j) k_j, two threads per row (one per half)
+        const uint32_t r = tp & 127;
+        const uint32_t half = tp >> 7;
         for (int32_t c = 0; c < ui.nc; ++c) {
           const uint32_t s = g & 1;
           ok = mbar_wait_bounded(&ctrl->full[s], (g >> 1) & 1, abort_flag, T);
-          if (!wg_all(ok, 1)) goto wg1_out;
-          const int32_t pos = c * C + static_cast<int32_t>(i);  // token within the segment
-          const float w = pos < ui.len ? exp2f(-alpha * static_cast<float>(ui.len - 1 - pos)) : 0.f;
-          scale_k_row(s, w);
+          if (!group_all(ok, kBarP, 256)) goto p_out;
+          const int32_t pos = c * C + static_cast<int32_t>(r);  // token within the segment
+          const float w =
+              pos < ui.len ? exp2f(-alpha * static_cast<float>(ui.len - 1 - pos)) : 0.f;
+          scale_half_row(smem + s * kStageBytes + kOffK + half * kHalfBytes, r, w);
           fence_proxy_async_smem();
-          mbar_arrive(&ctrl->kt_ready[s]);
+          named_bar_sync(kBarP, 256);
+          if (tp < 128) mbar_arrive(&ctrl->kt_ready[s]);
           ++g;
         }
       }
       for (int32_t c = 0; c < ui.nc; ++c) {
-        const uint32_t s = g & 1;
-        const int32_t n_c = min(C, ui.len - c * C);  // tokens in this chunk
         ok = mbar_wait_bounded(&ctrl->s_full, n_s & 1, abort_flag, T);
-        if (!wg_all(ok, 1)) goto wg1_out;
+        if (!group_all(ok, kBarP, 256)) goto p_out;
         ++n_s;
         tc_fence_after();
-        // ---- P ----
+        // P is written over S in place: P block jb -> columns [16 jb, 16 jb + 16), inside S block
+        // jb / 2.  The two warps of a lane quarter take S blocks {hf, hf + 2}; the only S blocks a
+        // P store can overwrite are 0 and 1, which the warps read first, before a barrier that
+        // precedes every P store.
+        // P_ij = lambda^(i-j) S_ij for j <= i, else 0, over S columns j = 32 jb + m.  The factor
+        // lambda^max(i-j, 0) is built per 16-column half by walking m downward from the half's
+        // last column and multiplying by lambda <= 1 once j <= i: no intermediate can overflow,
+        // for any slope, and underflow only drops terms below fp32 range.
+        auto make_p = [&](uint32_t jb, const uint32_t (&r)[32], uint32_t (&pk)[16]) {
+          const int32_t dbase = static_cast<int32_t>(i) - static_cast<int32_t>(jb * 32);
+          const int mlim = jb == wq ? static_cast<int>(lane) : 31;  // columns m > mlim: j > i
 #pragma unroll
-        for (uint32_t jb = 0; jb < 4; ++jb) {
-          uint32_t pk[16];
-          if (jb <= wq) {
-            uint32_t r[32];
-            tmem_ld32(trow + kColS + jb * 32, r);
-            tmem_wait_ld();
-            const int32_t dbase = static_cast<int32_t>(i) - static_cast<int32_t>(jb * 32);
-            const float a = exp2f(-alpha * static_cast<float>(dbase));
+          for (int h = 1; h >= 0; --h) {
+            const int mtop = 16 * h + 15;
+            float f = ex2_approx(-alpha * static_cast<float>(max(dbase - mtop, 0)));
 #pragma unroll
-            for (int m = 0; m < 32; m += 2) {
-              float f0, f1;
-              if (fast) {
-                f0 = a * bm[m];
-                f1 = a * bm[m + 1];
-              } else {
-                f0 = exp2f(-alpha * static_cast<float>(dbase - m));
-                f1 = exp2f(-alpha * static_cast<float>(dbase - m - 1));
-              }
-              float x0 = __uint_as_float(r[m]) * f0;
-              float x1 = __uint_as_float(r[m + 1]) * f1;
-              if (jb == wq) {
-                if (m > static_cast<int>(lane)) x0 = 0.f;
-                if (m + 1 > static_cast<int>(lane)) x1 = 0.f;
-              }
-              pk[m >> 1] = pack_bf16x2(x0, x1);
+            for (int m = mtop; m > 16 * h; m -= 2) {
+              const float x1 = m <= mlim ? __uint_as_float(r[m]) * f : 0.f;
+              if (dbase - m >= 0) f *= lam1;
+              const float x0 = m - 1 <= mlim ? __uint_as_float(r[m - 1]) * f : 0.f;
+              if (dbase - (m - 1) >= 0) f *= lam1;
+              pk[(m - 1) >> 1] = pack_bf16x2(x0, x1);
             }
+          }
+        };
+        {
+          uint32_t r[32];
+          uint32_t pk[16];
+          const uint32_t jb0 = hf;
+          if (jb0 <= wq) {
+            tmem_ld32(trow + kColS + jb0 * 32, r);
+            tmem_wait_ld();
+          }
+          tc_fence_before();
+          named_bar_sync(kBarP, 256);
+          tc_fence_after();
+          if (jb0 <= wq) {
+            make_p(jb0, r, pk);
           } else {
 #pragma unroll
             for (int m = 0; m < 16; ++m) pk[m] = 0u;
           }
-          tmem_st16(trow + kColS + jb * 16, pk);
+          tmem_st16(trow + kColS + jb0 * 16, pk);
+          const uint32_t jb1 = hf + 2;
+          if (jb1 <= wq) {
+            tmem_ld32(trow + kColS + jb1 * 32, r);
+            tmem_wait_ld();
+            make_p(jb1, r, pk);
+          } else {
+#pragma unroll
+            for (int m = 0; m < 16; ++m) pk[m] = 0u;
+          }
+          tmem_st16(trow + kColS + jb1 * 16, pk);
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&ctrl->p_ready);
-        // ---- K~ = diag(lambda^(n-1-i)) K for the state update ----
-        {
-          const float w = static_cast<int32_t>(i) < n_c
-                              ? exp2f(-alpha * static_cast<float>(n_c - 1 - static_cast<int32_t>(i)))
-                              : 0.f;
-          scale_k_row(s, w);
-          fence_proxy_async_smem();
-          mbar_arrive(&ctrl->kt_ready[s]);
-        }
         ++g;
       }
       ++j;
     }
-  wg1_out:;
-  } else if (warp >= 8 && warp < 12) {
+  p_out:;
+  } else if (warp >= kWarpS0 && warp < kWarpO0) {
     // =========================================================================================
-    // state: look-back scan over segments, bf16 operand, decay rescale, final state
+    // state: look-back scan over segments, bf16 operand, decay rescale, final state; K -> K~
+    // during the output pass
     // =========================================================================================
     const uint32_t wq = warp & 3;
-    const uint32_t i = wq * 32 + lane;  // key-dimension row of the state
+    const uint32_t i = wq * 32 + lane;  // key-dimension row of the state / key token of K~
     const uint32_t trow = tmem + ((wq * 32) << 16);
     uint8_t* kvb = smem + kOffKVb;
-    uint32_t j = 0, n_kvd = 0, n_h = 0;
+    uint32_t g = 0, j = 0, n_kvd = 0, n_h = 0, n_s = 0;
     tc_fence_before();
     mbar_arrive(&ctrl->kv_free);  // the KV columns start out free
 
     // bf16 copy of 32 state columns [32 cb, 32 cb + 32) of row i into the MN-major operand
-    auto write_kvb = [&](uint32_t cb, const float (&x)[32]) {
+    // (x holds fp32 bit patterns)
+    auto write_kvb = [&](uint32_t cb, const uint32_t (&x)[32]) {
       const uint32_t half = cb >> 1;
 #pragma unroll
       for (uint32_t q = 0; q < 4; ++q) {
         const uint32_t c16 = (cb & 1) * 4 + q;
         uint4 w;
-        w.x = pack_bf16x2(x[8 * q + 0], x[8 * q + 1]);
-        w.y = pack_bf16x2(x[8 * q + 2], x[8 * q + 3]);
-        w.z = pack_bf16x2(x[8 * q + 4], x[8 * q + 5]);
-        w.w = pack_bf16x2(x[8 * q + 6], x[8 * q + 7]);
+        w.x = pack_bf16x2(__uint_as_float(x[8 * q + 0]), __uint_as_float(x[8 * q + 1]));
+        w.y = pack_bf16x2(__uint_as_float(x[8 * q + 2]), __uint_as_float(x[8 * q + 3]));
+        w.z = pack_bf16x2(__uint_as_float(x[8 * q + 4]), __uint_as_float(x[8 * q + 5]));
+        w.w = pack_bf16x2(__uint_as_float(x[8 * q + 6]), __uint_as_float(x[8 * q + 7]));
         *reinterpret_cast<uint4*>(kvb + half * kHalfBytes + sw128_off(i, c16)) = w;
       }
     };
@@ -537,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (true) {
       const uint32_t slot = j & 1;
       bool ok = mbar_wait_bounded(&ctrl->unit_full[slot], (j >> 1) & 1, abort_flag, T);
-      if (!wg_all(ok, 2)) break;
+      if (!group_all(ok, kBarS, 128)) break;
       const UnitInfo ui = ctrl->units[slot];
       mbar_arrive(&ctrl->unit_empty[slot]);
       if (ui.bh < 0) break;
@@ -547,9 +648,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (ui.flags & 1) {
         ok = mbar_wait_bounded(&ctrl->h_done, n_h & 1, abort_flag, T);
-        if (!wg_all(ok, 2)) break;
+        if (!group_all(ok, kBarS, 128)) break;
         ++n_h;
         tc_fence_after();
+        g += static_cast<uint32_t>(ui.nc);  // the local-state pass used these stages
       }
       // incoming state of this segment: published by segment k-1 of the same sequence
       if (k > 0) {
@@ -563,8 +665,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
         }
-        if (!wg_all(ok, 2)) break;
+        if (!group_all(ok, kBarS, 128)) break;
       }
+      // ring layout: float4 (state row i, columns 4q..4q+3) at index q * 128 + i
       const float4* ring_in =
           reinterpret_cast<const float4*>(p.ring + (bh * 2 + ((k - 1) & 1)) * (D * D));
       float4* ring_out = reinterpret_cast<float4*>(p.ring + (bh * 2 + (k & 1)) * (D * D));
@@ -572,19 +675,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float lam_n0 = exp2f(-alpha * static_cast<float>(min(C, ui.len)));
 #pragma unroll 1
       for (uint32_t cb = 0; cb < 4; ++cb) {
-        float sin[32];
+        uint32_t sin[32];  // fp32 bits of the incoming state, columns [32 cb, 32 cb + 32)
         if (k > 0) {
 #pragma unroll
           for (uint32_t q = 0; q < 8; ++q) {
             const float4 x = __ldcg(ring_in + (cb * 8 + q) * 128 + i);
-            sin[4 * q + 0] = x.x;
-            sin[4 * q + 1] = x.y;
-            sin[4 * q + 2] = x.z;
-            sin[4 * q + 3] = x.w;
+            sin[4 * q + 0] = __float_as_uint(x.x);
+            sin[4 * q + 1] = __float_as_uint(x.y);
+            sin[4 * q + 2] = __float_as_uint(x.z);
+            sin[4 * q + 3] = __float_as_uint(x.w);
           }
         } else {
 #pragma unroll
-          for (int m = 0; m < 32; ++m) sin[m] = 0.f;
+          for (int m = 0; m < 32; ++m) sin[m] = 0u;
         }
         if (ui.flags & 1) {
           // inclusive state S_{k+1} = lambda^L S_k + h_k, published for segment k+1
@@ -594,37 +697,56 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (uint32_t q = 0; q < 8; ++q) {
             float4 x;
-            x.x = fmaf(lam_len, sin[4 * q + 0], __uint_as_float(r[4 * q + 0]));
-            x.y = fmaf(lam_len, sin[4 * q + 1], __uint_as_float(r[4 * q + 1]));
-            x.z = fmaf(lam_len, sin[4 * q + 2], __uint_as_float(r[4 * q + 2]));
-            x.w = fmaf(lam_len, sin[4 * q + 3], __uint_as_float(r[4 * q + 3]));
+            x.x = fmaf(lam_len, __uint_as_float(sin[4 * q + 0]), __uint_as_float(r[4 * q + 0]));
+            x.y = fmaf(lam_len, __uint_as_float(sin[4 * q + 1]), __uint_as_float(r[4 * q + 1]));
+            x.z = fmaf(lam_len, __uint_as_float(sin[4 * q + 2]), __uint_as_float(r[4 * q + 2]));
+            x.w = fmaf(lam_len, __uint_as_float(sin[4 * q + 3]), __uint_as_float(r[4 * q + 3]));
             __stcg(ring_out + (cb * 8 + q) * 128 + i, x);
           }
         }
         write_kvb(cb, sin);
-        uint32_t r2[32];
 #pragma unroll
-        for (int m = 0; m < 32; ++m) r2[m] = __float_as_uint(lam_n0 * sin[m]);
-        tmem_st32(trow + kColKV + cb * 32, r2);
+        for (int m = 0; m < 32; ++m) sin[m] = __float_as_uint(lam_n0 * __uint_as_float(sin[m]));
+        tmem_st32(trow + kColKV + cb * 32, sin);
       }
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       if (ui.flags & 1) {
         __threadfence();
-        named_bar_sync(2, 128);
+        named_bar_sync(kBarS, 128);
         if (wq == 0 && lane == 0) {
           __threadfence();
           st_release_u32(p.flags + bh * 2 + (k & 1), static_cast<uint32_t>(k + 1));
         }
       }
-      mbar_arrive(&ctrl->kvb_ready);
 
       // carry the state through the segment's chunks
       bool good = true;
       for (int32_t c = 0; c < ui.nc; ++c) {
+        const uint32_t s = g & 1;
+        const int32_t n_c = min(C, ui.len - c * C);  // tokens in this chunk
+        // S_c done: K_c may be rewritten; only then hand over the state operand for chunk c
+        ok = mbar_wait_bounded(&ctrl->s_full, n_s & 1, abort_flag, T);
+        if (!group_all(ok, kBarS, 128)) {
+          good = false;
+          break;
+        }
+        ++n_s;
+        mbar_arrive(&ctrl->kvb_ready);
+        // K~_c = diag(lambda^(n-1-i)) K_c for the state update
+        {
+          const float w = static_cast<int32_t>(i) < n_c
+                              ? exp2f(-alpha * static_cast<float>(n_c - 1 - static_cast<int32_t>(i)))
+                              : 0.f;
+          uint8_t* kt = smem + s * kStageBytes + kOffK;
+          scale_half_row(kt, i, w);
+          scale_half_row(kt + kHalfBytes, i, w);
+          fence_proxy_async_smem();
+          mbar_arrive(&ctrl->kt_ready[s]);
+        }
         ok = mbar_wait_bounded(&ctrl->kv_done, n_kvd & 1, abort_flag, T);
-        if (!wg_all(ok, 2)) {
+        if (!group_all(ok, kBarS, 128)) {
           good = false;
           break;
         }
@@ -638,18 +760,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t r[32];
             tmem_ld32(trow + kColKV + cb * 32, r);
             tmem_wait_ld();
-            float x[32];
+            write_kvb(cb, r);
 #pragma unroll
-            for (int m = 0; m < 32; ++m) x[m] = __uint_as_float(r[m]);
-            write_kvb(cb, x);
-#pragma unroll
-            for (int m = 0; m < 32; ++m) r[m] = __float_as_uint(lam_next * x[m]);
+            for (int m = 0; m < 32; ++m) r[m] = __float_as_uint(lam_next * __uint_as_float(r[m]));
             tmem_st32(trow + kColKV + cb * 32, r);
           }
           tmem_wait_st();
           fence_proxy_async_smem();
           tc_fence_before();
-          mbar_arrive(&ctrl->kvb_ready);
         } else if ((ui.flags & 2) && p.state_out != nullptr) {
           float4* so = reinterpret_cast<float4*>(p.state_out + (bh * D + i) * D);
 #pragma unroll 1
@@ -665,53 +783,59 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        ++g;
       }
       if (!good) break;
       tc_fence_before();
       mbar_arrive(&ctrl->kv_free);
       ++j;
     }
-  } else if (warp >= 12) {
+  } else if (warp >= kWarpO0) {
     // =========================================================================================
-    // output epilogue
+    // output epilogue: thread i owns token row i of the chunk and writes its 256-byte output row
+    // straight to global memory (no shared-memory staging, so the stage is released by the MMA
+    // warp alone)
     // =========================================================================================
     const uint32_t wq = warp & 3;
     const uint32_t i = wq * 32 + lane;  // token row of the chunk
     const uint32_t trow = tmem + ((wq * 32) << 16);
-    const uint64_t pol_first = policy_evict_first();
-    uint32_t g = 0, j = 0, n_o = 0;
+    uint32_t j = 0, n_o = 0;
     tc_fence_before();
     mbar_arrive(&ctrl->o_free);  // the O accumulators start out free
     while (true) {
       const uint32_t slot = j & 1;
       bool ok = mbar_wait_bounded(&ctrl->unit_full[slot], (j >> 1) & 1, abort_flag, T);
-      if (!wg_all(ok, 3)) break;
+      if (!group_all(ok, kBarO, 128)) break;
       const UnitInfo ui = ctrl->units[slot];
       mbar_arrive(&ctrl->unit_empty[slot]);
       if (ui.bh < 0) break;
       const float alpha = p.slopes[ui.bh % p.H] * kLog2e;
       const float f = exp2f(-alpha * static_cast<float>(i + 1));  // lambda^(i+1)
-      const int32_t b = static_cast<int32_t>(ui.bh / p.H);
-      const int32_t h = static_cast<int32_t>(ui.bh % p.H);
-      if (ui.flags & 1) g += static_cast<uint32_t>(ui.nc);  // the local-state pass stores nothing
+      const int64_t b = ui.bh / p.H;
+      const int64_t h = ui.bh % p.H;
       bool good = true;
       for (int32_t c = 0; c < ui.nc; ++c) {
-        const uint32_t s = g & 1;
         ok = mbar_wait_bounded(&ctrl->o_full, n_o & 1, abort_flag, T);
-        if (!wg_all(ok, 3)) {
+        if (!group_all(ok, kBarO, 128)) {
           good = false;
           break;
         }
         ++n_o;
         tc_fence_after();
-        uint8_t* ob = smem + s * kStageBytes + kOffQ;  // Q tile is dead: stage the output there
+        const int64_t n = static_cast<int64_t>(ui.c0 + c) * C + i;  // token of this row
+        const bool valid = n < p.N;
+        uint4* orow = reinterpret_cast<uint4*>(p.out + ((b * p.N + n) * p.H + h) * D);
 #pragma unroll 1
-        for (uint32_t cb = 0; cb < 4; ++cb) {
+        for (uint32_t cb = 0; cb < 4; ++cb) {  // 32-column blocks
           uint32_t ra[32], re[32];
           tmem_ld32(trow + kColOintra + cb * 32, ra);
           tmem_ld32(trow + kColOinter + cb * 32, re);
           tmem_wait_ld();
-          const uint32_t half = cb >> 1;
+          if (cb == 3) {
+            // every O column of this row has been read: the accumulators may be overwritten
+            tc_fence_before();
+            mbar_arrive(&ctrl->o_free);
+          }
 #pragma unroll
           for (uint32_t q = 0; q < 4; ++q) {
             float o[8];
@@ -723,28 +847,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             w.y = pack_bf16x2(o[2], o[3]);
             w.z = pack_bf16x2(o[4], o[5]);
             w.w = pack_bf16x2(o[6], o[7]);
-            *reinterpret_cast<uint4*>(ob + half * kHalfBytes + sw128_off(i, (cb & 1) * 4 + q)) =
-                w;
+            if (valid) __stcs(orow + cb * 4 + q, w);
           }
         }
-        tc_fence_before();
-        mbar_arrive(&ctrl->o_free);
-        fence_proxy_async_smem();
-        named_bar_sync(3, 128);
-        if (wq == 0 && lane == 0) {
-          const int32_t n0 = (ui.c0 + c) * C;
-          tma_store_4d(&p.tm_o, ob, 0, h, n0, b, pol_first);
-          tma_store_4d(&p.tm_o, ob + kHalfBytes, 64, h, n0, b, pol_first);
-          bulk_commit_group();
-          bulk_wait_group_read0();
-          mbar_arrive(&ctrl->empty[s]);
-        }
-        ++g;
       }
       if (!good) break;
       ++j;
     }
-    if (wq == 0 && lane == 0) bulk_wait_group0();
   }
 
   // ===========================================================================================
@@ -755,6 +864,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if (threadIdx.x == 0 && ctrl->abort) atomicExch(p.status, kErrTimeout);
   if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+// Chunk-loads the producer keeps in flight as L2 prefetches ahead of its shared-memory fills.
+// LA_PREFETCH_DEPTH overrides the default (a tuning knob; every value computes the same result).
+int32_t prefetch_depth() {
+  static int32_t v = -1;
+  if (v < 0) {
+    const char* e = getenv("LA_PREFETCH_DEPTH");
+    int32_t d = 3;
+    if (e != nullptr) d = std::max(0, std::min(16, atoi(e)));
+    v = d;
+  }
+  return v;
 }
 
 bool encode_map(CUtensorMap* map, const void* base, int64_t B, int64_t N, int64_t H) {
@@ -792,12 +914,16 @@ SegmentPlan plan_segments(int64_t B, int64_t N, int64_t H, int requested_segment
   int64_t want;
   if (requested_segments > 0) {
     want = requested_segments;
-  } else if (bh >= 2 * static_cast<int64_t>(num_sms)) {
-    want = 1;  // enough independent sequences: no scan needed
+  } else if (2 * bh > static_cast<int64_t>(num_sms)) {
+    // More than half the SMs already hold a whole sequence: splitting cannot shorten the
+    // longest unit without adding the local-state pass to every split sequence.
+    want = 1;
   } else {
-    // Segments of about 4 chunks keep the K, V tiles of the local-state pass resident in L2
-    // until the output pass of the same segment re-reads them.
-    want = (pl.n_chunks + 3) / 4;
+    // One wave of equal segments, one per SM.  All segments then finish together: each runs
+    // its local-state pass, the scan hands every segment its incoming state right after, and
+    // each runs its output pass (the last segment has no local-state pass but waits for the
+    // scan instead).  Segments keep at least 4 chunks.
+    want = std::max<int64_t>(1, std::min<int64_t>(num_sms / bh, pl.n_chunks / 4));
   }
   want = std::max<int64_t>(1, std::min<int64_t>(want, pl.n_chunks));
   pl.seg_chunks = (pl.n_chunks + want - 1) / want;
@@ -833,9 +959,10 @@ cudaError_t launch_chunked_prefill(const PrefillArgs& a, const SegmentPlan& plan
   }
   Params prm{};
   if (!encode_map(&prm.tm_q, a.q, a.B, a.N, a.H) || !encode_map(&prm.tm_k, a.k, a.B, a.N, a.H) ||
-      !encode_map(&prm.tm_v, a.v, a.B, a.N, a.H) || !encode_map(&prm.tm_o, a.out, a.B, a.N, a.H)) {
+      !encode_map(&prm.tm_v, a.v, a.B, a.N, a.H)) {
     return cudaErrorInvalidValue;
   }
+  prm.out = static_cast<__nv_bfloat16*>(a.out);
   const WorkspaceLayout wl = workspace_layout(a.B, a.H, plan);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   prm.slopes = a.slopes;
@@ -852,6 +979,7 @@ cudaError_t launch_chunked_prefill(const PrefillArgs& a, const SegmentPlan& plan
   prm.segments = plan.segments;
   prm.units = plan.units;
   prm.timeout_ns = 2000000000ull;  // 2 s per wait
+  prm.prefetch_depth = prefetch_depth();
 
   // counter, status and scan flags start at zero for every call
   e = cudaMemsetAsync(ws, 0, wl.flags_off + wl.flags_bytes, stream);
