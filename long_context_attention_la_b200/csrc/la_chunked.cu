@@ -22,9 +22,8 @@
 //                c-1, then O_inter_c and O_intra_c, so S_c overlaps the row scaling of K_{c-1}
 //   warp 2       TMEM allocator
 //   warps 4-11   P = decay-mask(S) into TMEM (two warps per TMEM lane quarter, alternate
-//                32-column blocks); K -> K~ (row-scaled) during the local-state pass
-//   warps 12-15  state: look-back scan, KV -> bf16 operand, decay rescale, final state, and
-//                K -> K~ during the output pass
+//                32-column blocks), then K -> K~ (row-scaled) in shared memory
+//   warps 12-15  state: look-back scan, KV -> bf16 operand, decay rescale, final state
 //   warps 16-19  output epilogue: O = O_intra + lambda^(i+1) O_inter -> bf16 -> global
 // Every wait (mbarrier or scan flag) is bounded in time; on expiry the CTA records
 // LA_ERR_TIMEOUT in the workspace status word, unwinds, frees its TMEM and exits.
@@ -601,6 +600,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&ctrl->p_ready);
+        {
+          // K~_c = diag(lambda^(n-1-j)) K_c for the state update (S_c, the only other reader of
+          // K_c, is complete); two threads per key row, one per half
+          const uint32_t s = g & 1;
+          const uint32_t r = tp & 127;
+          const uint32_t half = tp >> 7;
+          const int32_t n_c = min(C, ui.len - c * C);
+          const float w = static_cast<int32_t>(r) < n_c
+                              ? exp2f(-alpha * static_cast<float>(n_c - 1 - static_cast<int32_t>(r)))
+                              : 0.f;
+          scale_half_row(smem + s * kStageBytes + kOffK + half * kHalfBytes, r, w);
+          fence_proxy_async_smem();
+          named_bar_sync(kBarP, 256);
+          if (tp < 128) mbar_arrive(&ctrl->kt_ready[s]);
+        }
         ++g;
       }
       ++j;
@@ -615,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t i = wq * 32 + lane;  // key-dimension row of the state / key token of K~
     const uint32_t trow = tmem + ((wq * 32) << 16);
     uint8_t* kvb = smem + kOffKVb;
-    uint32_t g = 0, j = 0, n_kvd = 0, n_h = 0, n_s = 0;
+    uint32_t g = 0, j = 0, n_kvd = 0, n_h = 0;
     tc_fence_before();
     mbar_arrive(&ctrl->kv_free);  // the KV columns start out free
 
@@ -726,25 +740,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int32_t c = 0; c < ui.nc; ++c) {
         const uint32_t s = g & 1;
         const int32_t n_c = min(C, ui.len - c * C);  // tokens in this chunk
-        // S_c done: K_c may be rewritten; only then hand over the state operand for chunk c
-        ok = mbar_wait_bounded(&ctrl->s_full, n_s & 1, abort_flag, T);
-        if (!group_all(ok, kBarS, 128)) {
-          good = false;
-          break;
-        }
-        ++n_s;
+        // the state operand for chunk c is in place (written before the loop or by the previous
+        // iteration's update)
         mbar_arrive(&ctrl->kvb_ready);
-        // K~_c = diag(lambda^(n-1-i)) K_c for the state update
-        {
-          const float w = static_cast<int32_t>(i) < n_c
-                              ? exp2f(-alpha * static_cast<float>(n_c - 1 - static_cast<int32_t>(i)))
-                              : 0.f;
-          uint8_t* kt = smem + s * kStageBytes + kOffK;
-          scale_half_row(kt, i, w);
-          scale_half_row(kt + kHalfBytes, i, w);
-          fence_proxy_async_smem();
-          mbar_arrive(&ctrl->kt_ready[s]);
-        }
         ok = mbar_wait_bounded(&ctrl->kv_done, n_kvd & 1, abort_flag, T);
         if (!group_all(ok, kBarS, 128)) {
           good = false;
@@ -872,7 +870,7 @@ int32_t prefetch_depth() {
   static int32_t v = -1;
   if (v < 0) {
     const char* e = getenv("LA_PREFETCH_DEPTH");
-    int32_t d = 3;
+    int32_t d = 0;  // measured: prefetching ahead did not beat the two-stage TMA ring alone
     if (e != nullptr) d = std::max(0, std::min(16, atoi(e)));
     v = d;
   }
