@@ -40,6 +40,25 @@ METRIC = "lightning-attn prefill tok/s & TFLOP/s (H=64,d=128); decode state GB/s
 DECODE = dict(B=256, H=64, d=128)
 
 
+def measured_traffic():
+    """DRAM bytes per prefill launch from the committed ncu capture, or None when the kernel
+    sources changed since that capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "chunked_prefill_kernel_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["source_sha256"]:
+            return None
+        return float(rec["dram_bytes_read"]) + float(rec["dram_bytes_write"])
+    except Exception:
+        return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -350,7 +369,9 @@ def run_ours(args):
             "decode": {"ms": dec_ms_max, "state_gbs": dec_gbs, "frac_of_measured": dec_gbs / hbm_peak,
                        "frac_of_8tbs": dec_gbs / 8000.0, "tok_s": world * Bd / (dec_ms_max * 1e-3)},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved / hbm_peak, "traffic": None,
+                         "frac": achieved / hbm_peak,
+                         "traffic": measured_traffic() if args.workload == "prefill_32k" else None,
+                         "algorithmic_bytes": pre_bytes,
                          "kernel": "chunked_prefill_kernel", "peak_kind": peak_kind},
             "cpu_baseline": cpu,
             "clocks": clk.summary(),

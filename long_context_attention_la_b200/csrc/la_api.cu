@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -100,6 +101,15 @@ la_status la_prefill(const la_desc* desc, const void* q, const void* k, const vo
 
   la::PrefillArgs a{desc->B, desc->N, desc->H, desc->d, desc->dtype, q, k, v, slopes, out,
                     state_out};
+  // Failure injection for tests, read on every call: LA_DEBUG_WITHHOLD_SEGMENT=k keeps segment k
+  // of every sequence from publishing its scan state, so segment k+1 waits until its bounded
+  // wait expires (LA_DEBUG_WAIT_LIMIT_MS, default 2000) and the call reports LA_ERR_TIMEOUT
+  // through la_workspace_status.  Unset in normal use.
+  if (const char* e = getenv("LA_DEBUG_WITHHOLD_SEGMENT")) a.withhold_segment = atoi(e);
+  if (const char* e = getenv("LA_DEBUG_WAIT_LIMIT_MS")) {
+    const long ms = atol(e);
+    if (ms > 0 && ms <= 60000) a.wait_limit_ns = static_cast<uint64_t>(ms) * 1000000ull;
+  }
   if (!use_tensor_path(desc)) {
     return la::launch_recurrent_prefill(a, s) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
   }

@@ -114,6 +114,7 @@ struct Params {
   int64_t n_chunks, seg_chunks, segments, units;
   uint64_t timeout_ns;
   int32_t prefetch_depth;
+  int32_t withhold_segment;  // failure injection: this segment never publishes (-1: none)
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -729,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ui.flags & 1) {
         __threadfence();
         named_bar_sync(kBarS, 128);
-        if (wq == 0 && lane == 0) {
+        if (wq == 0 && lane == 0 && k != p.withhold_segment) {
           __threadfence();
           st_release_u32(p.flags + bh * 2 + (k & 1), static_cast<uint32_t>(k + 1));
         }
@@ -976,7 +977,8 @@ cudaError_t launch_chunked_prefill(const PrefillArgs& a, const SegmentPlan& plan
   prm.seg_chunks = plan.seg_chunks;
   prm.segments = plan.segments;
   prm.units = plan.units;
-  prm.timeout_ns = 2000000000ull;  // 2 s per wait
+  prm.timeout_ns = a.wait_limit_ns;
+  prm.withhold_segment = a.withhold_segment;
   prm.prefetch_depth = prefetch_depth();
 
   // counter, status and scan flags start at zero for every call

@@ -19,6 +19,10 @@ struct PrefillArgs {
   const float* slopes;
   void* out;
   float* state_out;  // may be null
+  // Failure injection for tests (host-side switch, see la_api.cu): the segment index whose scan
+  // flag is never published (-1: none) and the limit of every device wait.
+  int32_t withhold_segment = -1;
+  uint64_t wait_limit_ns = 2000000000ull;
 };
 
 struct DecodeArgs {
