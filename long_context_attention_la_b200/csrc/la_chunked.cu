@@ -175,6 +175,40 @@ __device__ __forceinline__ void scale_half_row(uint8_t* half_tile, uint32_t r, f
   }
 }
 
+// 4 x 4 transpose of 16-byte pieces within each group of 4 lanes: on entry lane t of a group
+// holds pieces x[0..3] of its own row; on exit it holds piece t of the group's rows 0..3.  Two
+// butterfly exchanges: swap the off-diagonal 2 x 2 blocks (partner t ^ 2), then transpose each
+// 2 x 2 block (partner t ^ 1).
+__device__ __forceinline__ uint4 shfl_xor_u4(uint4 v, int m) {
+  v.x = __shfl_xor_sync(0xffffffffu, v.x, m);
+  v.y = __shfl_xor_sync(0xffffffffu, v.y, m);
+  v.z = __shfl_xor_sync(0xffffffffu, v.z, m);
+  v.w = __shfl_xor_sync(0xffffffffu, v.w, m);
+  return v;
+}
+__device__ __forceinline__ void transpose4x4_lanes(uint4 (&x)[4], uint32_t t) {
+  const bool hi = (t & 2u) != 0;
+  uint4 a = shfl_xor_u4(hi ? x[0] : x[2], 2);
+  uint4 b = shfl_xor_u4(hi ? x[1] : x[3], 2);
+  if (hi) {
+    x[0] = a;
+    x[1] = b;
+  } else {
+    x[2] = a;
+    x[3] = b;
+  }
+  const bool odd = (t & 1u) != 0;
+  a = shfl_xor_u4(odd ? x[0] : x[1], 1);
+  b = shfl_xor_u4(odd ? x[2] : x[3], 1);
+  if (odd) {
+    x[0] = a;
+    x[2] = b;
+  } else {
+    x[1] = a;
+    x[3] = b;
+  }
+}
+
 __device__ __forceinline__ void decode_unit(const Params& p, int64_t u, UnitInfo& ui) {
   const int64_t k = u / p.BH;
   const int64_t bh = u % p.BH;
@@ -821,9 +855,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++n_o;
         tc_fence_after();
-        const int64_t n = static_cast<int64_t>(ui.c0 + c) * C + i;  // token of this row
-        const bool valid = n < p.N;
-        uint4* orow = reinterpret_cast<uint4*>(p.out + ((b * p.N + n) * p.H + h) * D);
+        // Stores go out in 4-lane groups: after a 4 x 4 exchange of 16-byte pieces among lanes
+        // 4a..4a+3 (rows i0..i0+3 of the chunk), store k writes 64 contiguous bytes of row i0 + k,
+        // so every 32-byte sector is written whole by one instruction.
+        const uint32_t t = lane & 3;
+        const int64_t n0 = static_cast<int64_t>(ui.c0 + c) * C + (i & ~3u);  // token of row i0
+        __nv_bfloat16* out_h = p.out + (b * p.N * p.H + h) * D;
+        const int64_t row_stride = p.H * D;
 #pragma unroll 1
         for (uint32_t cb = 0; cb < 4; ++cb) {  // 32-column blocks
           uint32_t ra[32], re[32];
@@ -835,18 +873,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(&ctrl->o_free);
           }
+          uint4 x[4];  // 16-byte pieces q = 0..3 of this row's 64 bytes
 #pragma unroll
           for (uint32_t q = 0; q < 4; ++q) {
             float o[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               o[e] = fmaf(f, __uint_as_float(re[8 * q + e]), __uint_as_float(ra[8 * q + e]));
-            uint4 w;
-            w.x = pack_bf16x2(o[0], o[1]);
-            w.y = pack_bf16x2(o[2], o[3]);
-            w.z = pack_bf16x2(o[4], o[5]);
-            w.w = pack_bf16x2(o[6], o[7]);
-            if (valid) __stcs(orow + cb * 4 + q, w);
+            x[q].x = pack_bf16x2(o[0], o[1]);
+            x[q].y = pack_bf16x2(o[2], o[3]);
+            x[q].z = pack_bf16x2(o[4], o[5]);
+            x[q].w = pack_bf16x2(o[6], o[7]);
+          }
+          transpose4x4_lanes(x, t);  // now x[k] = piece t of row i0 + k
+#pragma unroll
+          for (uint32_t k = 0; k < 4; ++k) {
+            if (n0 + k < p.N) {
+              uint4* dst = reinterpret_cast<uint4*>(out_h + (n0 + k) * row_stride + cb * 32) + t;
+              __stcs(dst, x[k]);
+            }
           }
         }
       }
