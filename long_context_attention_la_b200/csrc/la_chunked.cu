@@ -17,14 +17,16 @@
 // Execution: one persistent CTA per SM (640 threads, ~226 KB shared memory, all 512 TMEM
 // columns).  Work units (segment, b, h) are taken in segment-major order from an atomic counter,
 // so a unit only ever waits on units that running CTAs already hold.  Roles:
-//   warp 0       TMA producer: two-stage ring of Q/K/V tiles, L2 prefetch a few chunks ahead
-//   warp 1       tcgen05.mma issuer; per chunk c it issues S_c, then the state update of chunk
-//                c-1, then O_inter_c and O_intra_c, so S_c overlaps the row scaling of K_{c-1}
+//   warp 0       TMA producer: two-stage ring of Q/K/V tiles (optional L2 prefetch ahead)
+//   warp 1       tcgen05.mma issuer; per chunk c: S_c, O_inter_c, the state update with chunk c,
+//                O_intra_c; the stage is released when O_intra_c completes
 //   warp 2       TMEM allocator
 //   warps 4-11   P = decay-mask(S) into TMEM (two warps per TMEM lane quarter, alternate
-//                32-column blocks), then K -> K~ (row-scaled) in shared memory
-//   warps 12-15  state: look-back scan, KV -> bf16 operand, decay rescale, final state
-//   warps 16-19  output epilogue: O = O_intra + lambda^(i+1) O_inter -> bf16 -> global
+//                32-column blocks); K -> K~ in the local-state pass
+//   warps 12-15  state: look-back scan, K -> K~ (row-scaled, as soon as S_c is done) in the
+//                output pass, KV -> bf16 operand, decay rescale, final state
+//   warps 16-19  output epilogue: O = O_intra + lambda^(i+1) O_inter -> bf16 -> global, in
+//                whole 32-byte sectors
 // Every wait (mbarrier or scan flag) is bounded in time; on expiry the CTA records
 // LA_ERR_TIMEOUT in the workspace status word, unwinds, frees its TMEM and exits.
 #include <cuda.h>
@@ -445,16 +447,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int32_t c = 0; c < ui.nc && ok; ++c) {
           const uint32_t s = g & 1;
           const uint32_t ph = (g >> 1) & 1;
-          // The state update of the previous chunk goes first if its K~ is already scaled (it
-          // does not touch what S_c reads or writes); otherwise it follows S_c.
-          bool prev_issued = false;
-          if (c > 0 && mbar_test_wait(&ctrl->kt_ready[(g - 1) & 1], ((g - 1) >> 1) & 1)) {
-            tc_fence_after();
-            issue_state_update(g - 1, true);
-            umma_commit(&ctrl->kv_done);
-            umma_commit(&ctrl->empty[(g - 1) & 1]);
-            prev_issued = true;
-          }
           if (!mbar_wait_bounded(&ctrl->full[s], ph, abort_flag, T)) {
             ok = false;
             break;
@@ -472,18 +464,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_sdesc_sw128(kb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
           }
           umma_commit(&ctrl->s_full);
-          // state update of the previous chunk (its K~ was scaled while S_c ran)
-          if (c > 0 && !prev_issued) {
-            const uint32_t gp = g - 1;
-            if (!mbar_wait_bounded(&ctrl->kt_ready[gp & 1], (gp >> 1) & 1, abort_flag, T)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            issue_state_update(gp, true);
-            umma_commit(&ctrl->kv_done);
-            umma_commit(&ctrl->empty[gp & 1]);
-          }
           // O_inter = Q KV_in (needs the bf16 state operand and a free O accumulator)
           if (!mbar_wait_bounded(&ctrl->kvb_ready, n_kvb & 1, abort_flag, T) ||
               !mbar_wait_bounded(&ctrl->o_free, n_ofree & 1, abort_flag, T)) {
@@ -500,6 +480,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_sdesc_sw128(kvb + kk * 2048, kHalfBytes, 1024), idQK,
                     kk > 0 ? 1u : 0u);
           }
+          // KV += K~_c^T V_c once K_c is row-scaled (after S_c, which read K_c unscaled).  It
+          // follows O_inter_c, so kv_done also tells the state warps that the bf16 operand O_inter
+          // read is free again.
+          if (!mbar_wait_bounded(&ctrl->kt_ready[s], ph, abort_flag, T)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_state_update(g, true);
+          umma_commit(&ctrl->kv_done);
           // O_intra = P V, P read from TMEM
           if (!mbar_wait_bounded(&ctrl->p_ready, n_p & 1, abort_flag, T)) {
             ok = false;
@@ -513,18 +503,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idPV, kk > 0 ? 1u : 0u);
           }
           umma_commit(&ctrl->o_full);
+          umma_commit(&ctrl->empty[s]);
           ++g;
         }
         if (!ok) break;
-        // state update of the unit's last chunk
-        {
-          const uint32_t gp = g - 1;
-          if (!mbar_wait_bounded(&ctrl->kt_ready[gp & 1], (gp >> 1) & 1, abort_flag, T)) break;
-          tc_fence_after();
-          issue_state_update(gp, true);
-          umma_commit(&ctrl->kv_done);
-          umma_commit(&ctrl->empty[gp & 1]);
-        }
         ++j;
       }
       // all issued MMAs must finish before TMEM is released
@@ -635,21 +617,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&ctrl->p_ready);
-        {
-          // K~_c = diag(lambda^(n-1-j)) K_c for the state update (S_c, the only other reader of
-          // K_c, is complete); two threads per key row, one per half
-          const uint32_t s = g & 1;
-          const uint32_t r = tp & 127;
-          const uint32_t half = tp >> 7;
-          const int32_t n_c = min(C, ui.len - c * C);
-          const float w = static_cast<int32_t>(r) < n_c
-                              ? exp2f(-alpha * static_cast<float>(n_c - 1 - static_cast<int32_t>(r)))
-                              : 0.f;
-          scale_half_row(smem + s * kStageBytes + kOffK + half * kHalfBytes, r, w);
-          fence_proxy_async_smem();
-          named_bar_sync(kBarP, 256);
-          if (tp < 128) mbar_arrive(&ctrl->kt_ready[s]);
-        }
         ++g;
       }
       ++j;
@@ -664,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t i = wq * 32 + lane;  // key-dimension row of the state / key token of K~
     const uint32_t trow = tmem + ((wq * 32) << 16);
     uint8_t* kvb = smem + kOffKVb;
-    uint32_t g = 0, j = 0, n_kvd = 0, n_h = 0;
+    uint32_t g = 0, j = 0, n_kvd = 0, n_h = 0, n_s = 0;
     tc_fence_before();
     mbar_arrive(&ctrl->kv_free);  // the KV columns start out free
 
@@ -778,6 +745,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the state operand for chunk c is in place (written before the loop or by the previous
         // iteration's update)
         mbar_arrive(&ctrl->kvb_ready);
+        // K~_c = diag(lambda^(n-1-j)) K_c for the state update, once S_c (the only other reader of
+        // K_c) is complete; thread i scales key row i
+        ok = mbar_wait_bounded(&ctrl->s_full, n_s & 1, abort_flag, T);
+        if (!group_all(ok, kBarS, 128)) {
+          good = false;
+          break;
+        }
+        ++n_s;
+        {
+          const int32_t r = static_cast<int32_t>(i);
+          const float w = r < n_c ? exp2f(-alpha * static_cast<float>(n_c - 1 - r)) : 0.f;
+          uint8_t* kt = smem + s * kStageBytes + kOffK;
+          scale_half_row(kt, i, w);
+          scale_half_row(kt + kHalfBytes, i, w);
+          fence_proxy_async_smem();
+          mbar_arrive(&ctrl->kt_ready[s]);
+        }
         ok = mbar_wait_bounded(&ctrl->kv_done, n_kvd & 1, abort_flag, T);
         if (!group_all(ok, kBarS, 128)) {
           good = false;
