@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define LA_VERSION 1000 /* major*1000 + minor */
+#define LA_VERSION 1001 /* major*1000 + minor */
 
 typedef enum {
   LA_OK = 0,
@@ -163,6 +163,62 @@ la_status la_decode_step(int64_t B, int64_t H, int64_t d, int32_t dtype, const v
 #define LA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u + 4096u)
 la_status la_prefill_noalloc(const la_desc* desc, const void* q, const void* k, const void* v,
                              const float* slopes, void* out, float* state_out, void* stream);
+
+/* Problem descriptor for la_prefill_varlen: n_seqs sequences packed back to back along one token
+ * axis of length T. */
+typedef struct {
+  int64_t T;        /* total tokens of all sequences, >= 0 */
+  int64_t n_seqs;   /* sequences, >= 1 */
+  int64_t H;        /* heads, >= 1 */
+  int64_t d;        /* head dimension, 64 or 128 */
+  int32_t dtype;    /* la_dtype of q, k, v, out */
+  int32_t chunk;    /* as in la_desc */
+  int32_t segments; /* segments per non-empty sequence: 0 = automatic; >= 1 explicit (clamped) */
+  int32_t path;     /* la_path */
+} la_varlen_desc;
+
+/* Bytes of device workspace la_prefill_varlen needs (0 only for invalid arguments).  It depends on
+ * the sequence lengths, which set the work-unit table and the segment plan. */
+size_t la_prefill_varlen_workspace_bytes(const la_varlen_desc* desc, const int64_t* cu_seqlens);
+
+/*
+ * la_prefill_varlen — la_prefill over variable-length sequences packed along one token axis
+ * ("varlen"), each continuing from an optional initial state (a cached prefix).
+ *
+ * The report trains on packed inputs of many short sub-sequences and folds every sub-sequence's
+ * state correction into one fused launch (§4.1.2, kernel fusion for variable-length sequences);
+ * at serving time a prefill continues from a cached prefix state (§4.3, prefix caching).  Here
+ * sequence s owns tokens [cu_seqlens[s], cu_seqlens[s+1]) of the packed tensors.  For each s and
+ * head h the recurrence of la_prefill runs from S = state_in[s, h] (zero if state_in is NULL):
+ *     S <- lambda_h S + k_t^T v_t,   o_t = q_t S,   state_out[s, h] = S after the last token.
+ * A sequence of length 0 writes no output and passes its initial state through to state_out.
+ * All sequences, heads and segments go into one launch of the kernel la_prefill uses
+ * (tensor-core or recurrent, by desc->path as for la_prefill).
+ *
+ *   desc        shape and options (host pointer, read during the call only)
+ *   q, k, v     [T, H, d] device, dtype desc->dtype, read only (a [B, N, H, d] tensor is the packed
+ *               layout of B sequences of N tokens)
+ *   slopes      fp32[H] device
+ *   cu_seqlens  HOST int64[n_seqs + 1]: cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_seqs] = T;
+ *               read during the call only (the plan built from it is copied to the workspace)
+ *   state_in    fp32 [n_seqs, H, d, d] device, or NULL for zero initial states; read only
+ *   out         [T, H, d] device, written
+ *   state_out   fp32 [n_seqs, H, d, d] device, or NULL.  It may be the same pointer as state_in
+ *               (in-place continuation); any other overlap with state_in is LA_ERR_ALIAS.
+ *   workspace   device scratch of at least la_prefill_varlen_workspace_bytes(desc, cu_seqlens)
+ *               bytes, 256-byte aligned, used only by this call until it completes on `stream`;
+ *               NULL: allocated and freed on `stream` (cudaMallocAsync / cudaFreeAsync)
+ *   stream      cudaStream_t as void*
+ *
+ * Errors: LA_ERR_SHAPE for a cu_seqlens that is not a non-decreasing run from 0 to T (or other
+ * shape errors as in la_prefill), LA_ERR_ALIGN for q, k, v, out, state_in, state_out not 16-byte
+ * aligned, LA_ERR_ALIAS as above or when out overlaps q, k or v; the rest as la_prefill.  The
+ * device status word (la_workspace_status) reports a scan timeout as for la_prefill.
+ */
+la_status la_prefill_varlen(const la_varlen_desc* desc, const void* q, const void* k,
+                            const void* v, const float* slopes, const int64_t* cu_seqlens,
+                            const float* state_in, void* out, float* state_out, void* workspace,
+                            size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, then returns the device status word of a workspace that la_prefill
  * used: LA_OK, or LA_ERR_TIMEOUT if a bounded device wait gave up during the last call. */

@@ -69,15 +69,7 @@ constexpr uint32_t kColKV = 384;     // carried state / segment-local state h
 
 constexpr int32_t kErrTimeout = -8;  // LA_ERR_TIMEOUT
 
-struct UnitInfo {
-  int32_t bh;       // flat head b*H + h, or -1 = no more work
-  int32_t seg;      // segment index k
-  int32_t c0;       // first chunk of the segment
-  int32_t nc;       // chunks in the segment
-  int32_t len;      // tokens in the segment
-  int32_t flags;    // bit 0: compute the local state first; bit 1: last segment of the sequence
-  int32_t pad[2];
-};
+using UnitInfo = WorkUnit;  // one (segment, sequence, head) work unit
 
 struct Ctrl {
   uint64_t full[2];
@@ -112,6 +104,8 @@ struct Params {
   int32_t* status;
   uint32_t* flags;
   float* ring;
+  const WorkUnit* unit_table;  // variable-length plan (device), or null: units follow from N, BH
+  const float* state_in;       // fp32 [sequences, H, D, D] initial states, or null (zero)
   int64_t N, H, BH;
   int64_t n_chunks, seg_chunks, segments, units;
   uint64_t timeout_ns;
@@ -212,6 +206,20 @@ __device__ __forceinline__ void transpose4x4_lanes(uint4 (&x)[4], uint32_t t) {
 }
 
 __device__ __forceinline__ void decode_unit(const Params& p, int64_t u, UnitInfo& ui) {
+  if (p.unit_table != nullptr) {
+    const int4* src = reinterpret_cast<const int4*>(p.unit_table + u);
+    const int4 w0 = __ldg(src), w1 = __ldg(src + 1);
+    ui.bh = w0.x;
+    ui.seg = w0.y;
+    ui.c0 = w0.z;
+    ui.nc = w0.w;
+    ui.len = w1.x;
+    ui.flags = w1.y;
+    ui.b = w1.z;
+    ui.tok0 = w1.w;
+    return;
+  }
+  // fixed length: unit u = segment k of flat head bh, segment-major
   const int64_t k = u / p.BH;
   const int64_t bh = u % p.BH;
   const int64_t c0 = k * p.seg_chunks;
@@ -223,6 +231,8 @@ __device__ __forceinline__ void decode_unit(const Params& p, int64_t u, UnitInfo
   ui.nc = static_cast<int32_t>(nc);
   ui.len = static_cast<int32_t>(end - c0 * C);
   ui.flags = (k + 1 < p.segments ? 1 : 0) | (k + 1 == p.segments ? 2 : 0);
+  ui.b = static_cast<int32_t>(bh / p.H);
+  ui.tok0 = 0;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -288,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           decode_unit(p, u, ui);
         } else {
           ui.bh = -1;
-          ui.seg = ui.c0 = ui.nc = ui.len = ui.flags = 0;
+          ui.seg = ui.c0 = ui.nc = ui.len = ui.flags = ui.b = ui.tok0 = 0;
         }
       };
       auto n_loads = [](const UnitInfo& ui) -> int32_t {
@@ -296,12 +306,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // L2 prefetch of chunk-load `pos` of `ui` (the part of it that comes from DRAM)
       auto prefetch = [&](const UnitInfo& ui, int32_t pos) {
-        const int32_t b = static_cast<int32_t>(ui.bh / p.H);
+        const int32_t b = ui.b;
         const int32_t h = static_cast<int32_t>(ui.bh % p.H);
         const bool two_pass = (ui.flags & 1) != 0;
         const bool local_pass = two_pass && pos < ui.nc;
         const int32_t c = two_pass && !local_pass ? pos - ui.nc : pos;
-        const int32_t n0 = (ui.c0 + c) * C;
+        const int32_t n0 = ui.tok0 + (ui.c0 + c) * C;
         if (!local_pass) {
           tma_prefetch_l2_4d(&p.tm_q, 0, h, n0, b, pol_normal);
           tma_prefetch_l2_4d(&p.tm_q, 64, h, n0, b, pol_normal);
@@ -337,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ctrl->units[slot] = cur;
         mbar_arrive(&ctrl->unit_full[slot]);
         if (cur.bh < 0) break;
-        const int32_t b = static_cast<int32_t>(cur.bh / p.H);
+        const int32_t b = cur.b;
         const int32_t h = static_cast<int32_t>(cur.bh % p.H);
         const int32_t n_cur = n_loads(cur);
         for (int32_t pos = 0; pos < n_cur; ++pos) {
@@ -362,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool local_state_pass = (cur.flags & 1) && pos < cur.nc;
           const int32_t c = (cur.flags & 1) && !local_state_pass ? pos - cur.nc : pos;
           uint8_t* st = smem + s * kStageBytes;
-          const int32_t n0 = (cur.c0 + c) * C;
+          const int32_t n0 = cur.tok0 + (cur.c0 + c) * C;
           const uint64_t kv_pol = local_state_pass ? pol_last : pol_first;
           if (local_state_pass) {
             mbar_arrive_expect_tx(&ctrl->full[s], 2 * kTileBytes);
@@ -701,6 +711,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             sin[4 * q + 2] = __float_as_uint(x.z);
             sin[4 * q + 3] = __float_as_uint(x.w);
           }
+        } else if (p.state_in != nullptr) {
+          // the first segment continues from the caller's state: row i, columns [32 cb, +32)
+          const float4* sr = reinterpret_cast<const float4*>(p.state_in + (bh * D + i) * D) + cb * 8;
+#pragma unroll
+          for (uint32_t q = 0; q < 8; ++q) {
+            const float4 x = __ldcg(sr + q);  // coherent: state_out may be this same array
+            sin[4 * q + 0] = __float_as_uint(x.x);
+            sin[4 * q + 1] = __float_as_uint(x.y);
+            sin[4 * q + 2] = __float_as_uint(x.z);
+            sin[4 * q + 3] = __float_as_uint(x.w);
+          }
         } else {
 #pragma unroll
           for (int m = 0; m < 32; ++m) sin[m] = 0u;
@@ -828,7 +849,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ui.bh < 0) break;
       const float alpha = p.slopes[ui.bh % p.H] * kLog2e;
       const float f = exp2f(-alpha * static_cast<float>(i + 1));  // lambda^(i+1)
-      const int64_t b = ui.bh / p.H;
+      const int64_t b = ui.b;
       const int64_t h = ui.bh % p.H;
       bool good = true;
       for (int32_t c = 0; c < ui.nc; ++c) {
@@ -843,7 +864,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // 4a..4a+3 (rows i0..i0+3 of the chunk), store k writes 64 contiguous bytes of row i0 + k,
         // so every 32-byte sector is written whole by one instruction.
         const uint32_t t = lane & 3;
-        const int64_t n0 = static_cast<int64_t>(ui.c0 + c) * C + (i & ~3u);  // token of row i0
+        const int32_t r0 = c * C + static_cast<int32_t>(i & ~3u);  // row i0, from segment start
+        const int64_t n0 = static_cast<int64_t>(ui.tok0) + static_cast<int64_t>(ui.c0) * C + r0;
         __nv_bfloat16* out_h = p.out + (b * p.N * p.H + h) * D;
         const int64_t row_stride = p.H * D;
 #pragma unroll 1
@@ -872,7 +894,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           transpose4x4_lanes(x, t);  // now x[k] = piece t of row i0 + k
 #pragma unroll
           for (uint32_t k = 0; k < 4; ++k) {
-            if (n0 + k < p.N) {
+            if (r0 + static_cast<int32_t>(k) < ui.len) {  // rows past the segment end: none
               uint4* dst = reinterpret_cast<uint4*>(out_h + (n0 + k) * row_stride + cb * 32) + t;
               __stcs(dst, x[k]);
             }
@@ -973,8 +995,13 @@ WorkspaceLayout workspace_layout(int64_t B, int64_t H, const SegmentPlan& plan) 
   return w;
 }
 
-cudaError_t launch_chunked_prefill(const PrefillArgs& a, const SegmentPlan& plan,
-                                   void* workspace, cudaStream_t stream, int num_sms) {
+namespace {
+
+// Shared launch: fills the parameters common to both forms and runs the kernel.  `zero_bytes`
+// leading workspace bytes (counter, status, scan flags) are cleared first on `stream`.
+cudaError_t launch_common(const PrefillArgs& a, Params& prm, uint8_t* ws,
+                          const WorkspaceLayout& wl, int64_t units, cudaStream_t stream,
+                          int num_sms) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -985,37 +1012,124 @@ cudaError_t launch_chunked_prefill(const PrefillArgs& a, const SegmentPlan& plan
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  Params prm{};
+  // counter, status and scan flags start at zero for every call
+  e = cudaMemsetAsync(ws, 0, wl.flags_off + wl.flags_bytes, stream);
+  if (e != cudaSuccess || units == 0) return e;
   if (!encode_map(&prm.tm_q, a.q, a.B, a.N, a.H) || !encode_map(&prm.tm_k, a.k, a.B, a.N, a.H) ||
       !encode_map(&prm.tm_v, a.v, a.B, a.N, a.H)) {
     return cudaErrorInvalidValue;
   }
   prm.out = static_cast<__nv_bfloat16*>(a.out);
-  const WorkspaceLayout wl = workspace_layout(a.B, a.H, plan);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
   prm.slopes = a.slopes;
   prm.state_out = a.state_out;
+  prm.state_in = a.state_in;
   prm.counter = reinterpret_cast<uint32_t*>(ws + kWsCounter);
   prm.status = reinterpret_cast<int32_t*>(ws + kWsStatus);
   prm.flags = reinterpret_cast<uint32_t*>(ws + wl.flags_off);
   prm.ring = reinterpret_cast<float*>(ws + wl.ring_off);
   prm.N = a.N;
   prm.H = a.H;
+  prm.units = units;
+  prm.timeout_ns = a.wait_limit_ns;
+  prm.withhold_segment = a.withhold_segment;
+  prm.prefetch_depth = prefetch_depth();
+  const int64_t grid = std::min<int64_t>(units, num_sms);
+  chunked_prefill_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, stream>>>(prm);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunked_prefill(const PrefillArgs& a, const SegmentPlan& plan,
+                                   void* workspace, cudaStream_t stream, int num_sms) {
+  Params prm{};
+  prm.unit_table = nullptr;
   prm.BH = a.B * a.H;
   prm.n_chunks = plan.n_chunks;
   prm.seg_chunks = plan.seg_chunks;
   prm.segments = plan.segments;
-  prm.units = plan.units;
-  prm.timeout_ns = a.wait_limit_ns;
-  prm.withhold_segment = a.withhold_segment;
-  prm.prefetch_depth = prefetch_depth();
+  return launch_common(a, prm, static_cast<uint8_t*>(workspace), workspace_layout(a.B, a.H, plan),
+                       plan.units, stream, num_sms);
+}
 
-  // counter, status and scan flags start at zero for every call
-  e = cudaMemsetAsync(ws, 0, wl.flags_off + wl.flags_bytes, stream);
-  if (e != cudaSuccess) return e;
-  const int64_t grid = std::min<int64_t>(plan.units, num_sms);
-  chunked_prefill_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, stream>>>(prm);
-  return cudaGetLastError();
+VarlenPlan plan_varlen(const int64_t* cu, int64_t n_seqs, int64_t H, int requested_segments,
+                       int num_sms, WorkUnit* table) {
+  VarlenPlan pl;
+  int64_t nonempty = 0;
+  for (int64_t s = 0; s < n_seqs; ++s) nonempty += cu[s + 1] > cu[s] ? 1 : 0;
+  // Segments per sequence: the fixed-length rule with B*H counted over non-empty sequences, so
+  // equal lengths give the same plan as la_prefill.
+  auto segments_of = [&](int64_t n_chunks) -> int64_t {
+    int64_t want;
+    if (requested_segments > 0) {
+      want = requested_segments;
+    } else if (2 * nonempty * H > static_cast<int64_t>(num_sms)) {
+      want = 1;
+    } else {
+      want = std::max<int64_t>(1, std::min<int64_t>(num_sms / (nonempty * H), n_chunks / 4));
+    }
+    want = std::max<int64_t>(1, std::min<int64_t>(want, n_chunks));
+    const int64_t seg_chunks = (n_chunks + want - 1) / want;
+    return (n_chunks + seg_chunks - 1) / seg_chunks;
+  };
+  int64_t max_segments = 0;
+  for (int64_t s = 0; s < n_seqs; ++s) {
+    const int64_t len = cu[s + 1] - cu[s];
+    if (len <= 0) continue;
+    max_segments = std::max(max_segments, segments_of((len + C - 1) / C));
+  }
+  pl.multi_segment = max_segments > 1;
+  int64_t u = 0;
+  for (int64_t k = 0; k < max_segments; ++k) {
+    for (int64_t s = 0; s < n_seqs; ++s) {
+      const int64_t len = cu[s + 1] - cu[s];
+      if (len <= 0) continue;
+      const int64_t n_chunks = (len + C - 1) / C;
+      const int64_t segs = segments_of(n_chunks);
+      if (k >= segs) continue;
+      const int64_t seg_chunks = (n_chunks + segs - 1) / segs;
+      const int64_t c0 = k * seg_chunks;
+      const int64_t nc = std::min(seg_chunks, n_chunks - c0);
+      const int64_t end = std::min(len, (c0 + nc) * C);
+      for (int64_t h = 0; h < H; ++h, ++u) {
+        if (table == nullptr) continue;
+        WorkUnit& w = table[u];
+        w.bh = static_cast<int32_t>(s * H + h);
+        w.seg = static_cast<int32_t>(k);
+        w.c0 = static_cast<int32_t>(c0);
+        w.nc = static_cast<int32_t>(nc);
+        w.len = static_cast<int32_t>(end - c0 * C);
+        w.flags = (k + 1 < segs ? 1 : 0) | (k + 1 == segs ? 2 : 0);
+        w.b = 0;
+        w.tok0 = static_cast<int32_t>(cu[s]);
+      }
+    }
+  }
+  pl.units = u;
+  return pl;
+}
+
+VarlenWorkspace varlen_workspace_layout(int64_t n_seqs, int64_t H, const VarlenPlan& plan,
+                                        bool tensor_path) {
+  VarlenWorkspace w{};
+  SegmentPlan sp{};
+  sp.segments = plan.multi_segment ? 2 : 1;  // only "more than one segment" matters for the size
+  w.base = workspace_layout(n_seqs, H, sp);
+  w.table_off = (w.base.total + 255) / 256 * 256;
+  w.table_bytes = tensor_path ? static_cast<size_t>(plan.units) * sizeof(WorkUnit)
+                              : static_cast<size_t>(n_seqs + 1) * sizeof(int64_t);
+  w.total = w.table_off + w.table_bytes;
+  return w;
+}
+
+cudaError_t launch_chunked_prefill_varlen(const PrefillArgs& a, const VarlenPlan& plan,
+                                          const VarlenWorkspace& layout, void* workspace,
+                                          cudaStream_t stream, int num_sms) {
+  Params prm{};
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  prm.unit_table = reinterpret_cast<const WorkUnit*>(ws + layout.table_off);
+  prm.BH = a.n_seqs * a.H;
+  return launch_common(a, prm, ws, layout.base, plan.units, stream, num_sms);
 }
 
 }  // namespace la

@@ -19,6 +19,12 @@ struct PrefillArgs {
   const float* slopes;
   void* out;
   float* state_out;  // may be null
+  // Packed variable-length form (la_prefill_varlen): B = 1, N = total tokens; sequence s owns
+  // tokens [cu[s], cu[s+1]).  cu_dev is a device copy of cu (recurrent kernel), state_in an
+  // optional fp32 [n_seqs, H, d, d] initial state.  n_seqs = 0 means the fixed [B, N] form.
+  int64_t n_seqs = 0;
+  const int64_t* cu_dev = nullptr;
+  const float* state_in = nullptr;
   // Failure injection for tests (host-side switch, see la_api.cu): the segment index whose scan
   // flag is never published (-1: none) and the limit of every device wait.
   int32_t withhold_segment = -1;
@@ -47,6 +53,19 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 // ---------------------------------------------------------------------------------------------
 constexpr int kChunk = 128;
 constexpr int kHeadDim = 128;
+
+// One work unit of the chunked prefill, as the kernel reads it: one segment of one (sequence, head).
+struct WorkUnit {
+  int32_t bh;     // state / scan index: sequence * H + head (-1: no more work)
+  int32_t seg;    // segment index k within the sequence
+  int32_t c0;     // first chunk of the segment, counted from the sequence start
+  int32_t nc;     // chunks in the segment
+  int32_t len;    // tokens in the segment
+  int32_t flags;  // bit 0: compute the local state first; bit 1: last segment of the sequence
+  int32_t b;      // batch coordinate of the sequence in the [B, N, H, d] tensors
+  int32_t tok0;   // token coordinate (along N) of the sequence's first token
+};
+static_assert(sizeof(WorkUnit) == 32, "WorkUnit is read as two 16-byte words");
 
 // How a prefill is cut into work units: each (b, h) sequence of N tokens becomes `segments`
 // segments of `seg_chunks` chunks (the last may be shorter); one unit = one (segment, b, h).
@@ -77,5 +96,32 @@ constexpr size_t kWsStatus = 64;   // uint32 device status (0 = ok, else a la_st
 
 cudaError_t launch_chunked_prefill(const PrefillArgs& a, const SegmentPlan& plan,
                                    void* workspace, cudaStream_t stream, int num_sms);
+
+// Variable-length plan: the work units of every non-empty sequence, segment-major (all units of
+// segment k precede those of segment k + 1, so a unit only waits on units taken before it).
+struct VarlenPlan {
+  int64_t units = 0;
+  bool multi_segment = false;  // some sequence has more than one segment (needs flags and ring)
+};
+// Fills `table` (may be null to count only) with the units of cu[0..n_seqs]; returns the plan.
+VarlenPlan plan_varlen(const int64_t* cu, int64_t n_seqs, int64_t H, int requested_segments,
+                       int num_sms, WorkUnit* table);
+
+// Workspace of la_prefill_varlen: the fixed-length layout for n_seqs * H states, then the unit
+// table (tensor path) or a copy of cu (recurrent path).
+struct VarlenWorkspace {
+  WorkspaceLayout base;
+  size_t table_off;
+  size_t table_bytes;
+  size_t total;
+};
+VarlenWorkspace varlen_workspace_layout(int64_t n_seqs, int64_t H, const VarlenPlan& plan,
+                                        bool tensor_path);
+
+// Launches the chunked kernel over a unit table already in device memory at
+// workspace + layout.table_off.
+cudaError_t launch_chunked_prefill_varlen(const PrefillArgs& a, const VarlenPlan& plan,
+                                          const VarlenWorkspace& layout, void* workspace,
+                                          cudaStream_t stream, int num_sms);
 
 }  // namespace la

@@ -47,7 +47,8 @@ __device__ __forceinline__ void split_decay(float slope, float& hi, float& lo) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// Recurrent prefill.  One CTA per flat head (b*H + h), 4*D threads.  Thread t owns the state
+// Recurrent prefill.  One CTA per flat head (b*H + h; for packed variable-length input,
+// sequence*H + h with the sequence's tokens [cu[s], cu[s+1])), 4*D threads.  Thread t owns the state
 // column j = t % D for rows [rg*R, rg*R + R), rg = t / D, R = D / 4; the read-out o_j is summed
 // over the four row groups through shared memory.  q, k, v of the next token are prefetched into
 // registers while the current token is processed.
@@ -55,8 +56,8 @@ __device__ __forceinline__ void split_decay(float slope, float& hi, float& lo) {
 template <typename T, int D>
 __global__ void __launch_bounds__(4 * D) recurrent_prefill_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-    const float* __restrict__ slopes, T* __restrict__ out, float* __restrict__ state_out,
-    int64_t N, int64_t H) {
+    const float* __restrict__ slopes, T* __restrict__ out, float* state_out, int64_t N,
+    int64_t H, const int64_t* __restrict__ cu, const float* state_in) {
   constexpr int R = D / 4;
   __shared__ float tok[2][3][D];
   __shared__ float red[4][D];
@@ -65,8 +66,11 @@ __global__ void __launch_bounds__(4 * D) recurrent_prefill_kernel(
   const int j = tid % D;
   const int rg = tid / D;
   const int64_t flat = blockIdx.x;
-  const int64_t b = flat / H;
+  const int64_t b = flat / H;  // batch index, or sequence index of packed input
   const int64_t h = flat % H;
+  // rows [row0, row0 + len) of the token axis
+  const int64_t row0 = cu != nullptr ? cu[b] : b * N;
+  const int64_t len = cu != nullptr ? cu[b + 1] - cu[b] : N;
 
   float lam_hi, lam_lo;
   split_decay(slopes[h], lam_hi, lam_lo);
@@ -76,19 +80,22 @@ __global__ void __launch_bounds__(4 * D) recurrent_prefill_kernel(
   const int e = tid % D;
   const T* src = which == 0 ? q : (which == 1 ? k : v);
   auto fetch = [&](int64_t t) -> float {
-    return load_as_f32<T>(src, ((b * N + t) * H + h) * D + e);
+    return load_as_f32<T>(src, ((row0 + t) * H + h) * D + e);
   };
 
   float S[R];
 #pragma unroll
-  for (int r = 0; r < R; ++r) S[r] = 0.f;
+  for (int r = 0; r < R; ++r) {
+    // the initial state (a cached prefix), read before any write: state_out may be this array
+    S[r] = state_in != nullptr ? state_in[(flat * D + rg * R + r) * D + j] : 0.f;
+  }
 
-  if (which < 3 && N > 0) tok[0][which][e] = fetch(0);
+  if (which < 3 && len > 0) tok[0][which][e] = fetch(0);
   float pf = 0.f;
-  if (which < 3 && N > 1) pf = fetch(1);
+  if (which < 3 && len > 1) pf = fetch(1);
   __syncthreads();
 
-  for (int64_t t = 0; t < N; ++t) {
+  for (int64_t t = 0; t < len; ++t) {
     const int buf = static_cast<int>(t & 1);
     const float vj = tok[buf][2][j];
     float acc = 0.f;
@@ -100,13 +107,13 @@ __global__ void __launch_bounds__(4 * D) recurrent_prefill_kernel(
       acc = fmaf(tok[buf][0][i], S[r], acc);
     }
     red[rg][j] = acc;
-    if (which < 3 && t + 1 < N) tok[buf ^ 1][which][e] = pf;
+    if (which < 3 && t + 1 < len) tok[buf ^ 1][which][e] = pf;
     __syncthreads();
     if (rg == 0) {
       const float o = ((red[0][j] + red[1][j]) + red[2][j]) + red[3][j];
-      store_from_f32<T>(out, ((b * N + t) * H + h) * D + j, o);
+      store_from_f32<T>(out, ((row0 + t) * H + h) * D + j, o);
     }
-    if (which < 3 && t + 2 < N) pf = fetch(t + 2);
+    if (which < 3 && t + 2 < len) pf = fetch(t + 2);
     __syncthreads();
   }
 
@@ -193,10 +200,11 @@ __global__ void __launch_bounds__(512) decode_kernel(const T* __restrict__ q,
 
 template <typename T, int D>
 cudaError_t launch_recurrent_typed(const PrefillArgs& a, cudaStream_t stream) {
-  const int64_t grid = a.B * a.H;
+  const int64_t grid = (a.n_seqs > 0 ? a.n_seqs : a.B) * a.H;
+  if (grid == 0) return cudaSuccess;
   recurrent_prefill_kernel<T, D><<<static_cast<unsigned>(grid), 4 * D, 0, stream>>>(
       static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
-      a.slopes, static_cast<T*>(a.out), a.state_out, a.N, a.H);
+      a.slopes, static_cast<T*>(a.out), a.state_out, a.N, a.H, a.cu_dev, a.state_in);
   return cudaGetLastError();
 }
 

@@ -127,3 +127,32 @@ def window_starts(N: int, count: int = 8, length: int = 4096, seed: int = 1002):
     hi = max(N - length, 0)
     starts = torch.randint(0, hi + 1, (count,), generator=g).tolist()
     return sorted(int(s) for s in starts)
+
+
+def draw_seqlens(total: int, n_seqs: int, seed: int = 7, short_frac: float = 0.75) -> list[int]:
+    """Lengths of ``n_seqs`` packed sequences summing to ``total`` tokens, in a fragmented mix:
+    about ``short_frac`` of the sequences are short (1..256 tokens, log-uniform) and the rest
+    share the remaining tokens in random proportions.  Seeded CPU generator; returns a list."""
+    g = torch.Generator()
+    g.manual_seed(seed)
+    n_short = min(n_seqs - 1, int(round(short_frac * n_seqs))) if n_seqs > 1 else 0
+    short = torch.exp(torch.rand(n_short, generator=g, dtype=torch.float64) * math.log(256.0))
+    short = [max(1, int(x)) for x in short.tolist()]
+    while sum(short) > total // 2 and short:
+        short.pop()
+    rest = total - sum(short)
+    n_long = n_seqs - len(short)
+    w = torch.rand(n_long, generator=g, dtype=torch.float64) + 0.05
+    cuts = [int(x) for x in (w / w.sum() * rest).tolist()]
+    cuts[-1] += rest - sum(cuts)
+    lens = short + cuts
+    perm = torch.randperm(len(lens), generator=g).tolist()
+    return [lens[i] for i in perm]
+
+
+def cu_from_lengths(lengths) -> list[int]:
+    """Exclusive prefix sums [0, l0, l0 + l1, ...] (n + 1 entries)."""
+    cu = [0]
+    for x in lengths:
+        cu.append(cu[-1] + int(x))
+    return cu

@@ -40,7 +40,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert la.la_version() == 1000
+    assert la.la_version() == 1001
     for code in range(-10, 1):
         assert la.la_status_string(code) not in ("", "unknown status")
     assert la.la_status_string(-99) == "unknown status"
@@ -109,3 +109,66 @@ def test_tensor_path_workspace_covers_the_scan(lib):
     # single segment per sequence: only the header
     w1 = la.la_prefill_workspace_bytes(_desc(B=1, H=1, N=64 * 128, segments=1))
     assert w1 == 256 or w1 == 512
+
+
+# ---------------------------------------------------------------------------------------------
+# la_prefill_varlen: argument checks (CPU only; these return before any CUDA call)
+# ---------------------------------------------------------------------------------------------
+def _vdesc(**kw):
+    base = dict(T=300, n_seqs=3, H=2, d=128, dtype=la.LA_BF16, chunk=0, segments=0, path=0)
+    base.update(kw)
+    return la.la_varlen_desc(**base)
+
+
+_P = (0x1000, 0x2000, 0x3000, 0x4000)  # q, k, v, slopes
+
+
+@pytest.mark.parametrize("cu,kw,status", [
+    ([0, 100, 200, 300], dict(dtype=9), la.LA_ERR_DTYPE),
+    ([0, 100, 200, 300], dict(d=32), la.LA_ERR_SHAPE),
+    ([0, 100, 200, 300], dict(H=0), la.LA_ERR_SHAPE),
+    ([0, 100, 200, 300], dict(T=-1), la.LA_ERR_SHAPE),
+    ([1, 100, 200, 300], {}, la.LA_ERR_SHAPE),            # must start at 0
+    ([0, 100, 90, 300], {}, la.LA_ERR_SHAPE),             # must not decrease
+    ([0, 100, 200, 299], {}, la.LA_ERR_SHAPE),            # must end at T
+    ([0, 100, 200, 300], dict(chunk=64), la.LA_ERR_UNSUPPORTED),
+    ([0, 100, 200, 300], dict(dtype=la.LA_F32, path=la.LA_PATH_TENSOR), la.LA_ERR_UNSUPPORTED),
+    ([0, 100, 200, 300], dict(segments=-2), la.LA_ERR_SHAPE),
+])
+def test_varlen_rejects_bad_arguments(lib, cu, kw, status):
+    d = _vdesc(**kw)
+    assert la.la_prefill_varlen(d, *_P, cu, 0, 0x50000, 0, 0, 0, 0) == status
+    assert la.la_prefill_varlen_workspace_bytes(d, cu) == 0
+
+
+def test_varlen_null_alignment_aliasing(lib):
+    d = _vdesc()
+    cu = [0, 100, 200, 300]
+    assert lib.la_prefill_varlen(ctypes.byref(d), *_P, None, None, 0x50000, None, None, 0,
+                                 None) == la.LA_ERR_NULL
+    assert la.la_prefill_varlen(d, 0, *_P[1:], cu, 0, 0x50000, 0, 0, 0, 0) == la.LA_ERR_NULL
+    assert la.la_prefill_varlen(d, *_P, cu, 0x7008, 0x50000, 0, 0, 0, 0) == la.LA_ERR_ALIGN
+    assert la.la_prefill_varlen(d, *_P, cu, 0, 0x50000, 0x9004, 0, 0, 0) == la.LA_ERR_ALIGN
+    nbytes = 300 * 2 * 128 * 2
+    # out overlapping k
+    assert la.la_prefill_varlen(d, 0x100000, 0x100000 + nbytes, 0x100000 + 2 * nbytes, 0x4000,
+                                cu, 0, 0x100000 + nbytes + 512, 0, 0, 0, 0) == la.LA_ERR_ALIAS
+    # state_out overlapping state_in without being the same array
+    sbytes = 3 * 2 * 128 * 128 * 4
+    assert la.la_prefill_varlen(d, *_P, cu, 0x10000000, 0x50000000, 0x10000000 + sbytes // 2, 0,
+                                0, 0) == la.LA_ERR_ALIAS
+
+
+def test_varlen_workspace_sizes(lib):
+    cu = [0, 100, 200, 300]
+    # tensor path: header + a 32-byte work unit per (sequence, head, segment)
+    w = la.la_prefill_varlen_workspace_bytes(_vdesc(segments=1), cu)
+    assert w >= 256 + 3 * 2 * 32
+    # forcing several segments adds the scan flags and the state ring of every (sequence, head)
+    w2 = la.la_prefill_varlen_workspace_bytes(_vdesc(T=3000, segments=3), [0, 1000, 2000, 3000])
+    assert w2 >= 256 + 3 * 2 * 2 * 128 * 128 * 4 + 3 * 2 * 3 * 32
+    # recurrent path: header + a device copy of cu_seqlens
+    w3 = la.la_prefill_varlen_workspace_bytes(_vdesc(dtype=la.LA_F32, d=64), cu)
+    assert w3 >= 256 + 4 * 8
+    # empty sequences are allowed, including T = 0
+    assert la.la_prefill_varlen_workspace_bytes(_vdesc(T=0), [0, 0, 0, 0]) >= 256
