@@ -154,3 +154,32 @@ def decode(q, k, v, slopes, state, nthreads: int = 0):
     if rc != 0:
         raise RuntimeError("la_oracle_decode rejected its arguments")
     return o
+
+
+def _upcast(x) -> np.ndarray:
+    """Exact fp64 values of bf16 bit patterns (uint16) or float32 arrays."""
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return x.astype(np.float64)
+
+
+def gated_rmsnorm(o, gate, gamma, eps: float):
+    """The layer's step after the kernel, in fp64: a grouped RMSNorm of each head's output vector
+    followed by the sigmoid gate ("Ling and Ring 2.6 Technical Report", §2.1 Fig. 2: Linear
+    Attention Kernel -> Grouped RMSNorm, multiplied by sigmoid(Gate Projection); §4.3: the group
+    norm and sigmoid gate run as one fused operator).  Each head is one group:
+
+        y[..., j] = gamma[h, j] * o[..., j] / sqrt(mean_j(o[..., j]^2) + eps) * sigmoid(g[..., j])
+
+    o: fp64 [..., H, d] attention outputs (token-major, heads on the second-to-last axis);
+    gate: the gate pre-activation g = x W_gate with o's shape (uint16 bf16 bits or float32);
+    gamma: float32 [H, d]; eps: the RMSNorm epsilon.  Returns fp64 y with o's shape.
+    """
+    o = np.asarray(o, dtype=np.float64)
+    g = _upcast(gate)
+    gam = np.asarray(gamma, dtype=np.float32).astype(np.float64)
+    if g.shape != o.shape or gam.shape != o.shape[-2:]:
+        raise ValueError("gate must match o, gamma must be [H, d]")
+    ms = np.mean(o * o, axis=-1, keepdims=True)
+    return gam * (o / np.sqrt(ms + float(eps))) * (1.0 / (1.0 + np.exp(-g)))

@@ -238,3 +238,47 @@ def test_slope_schedule_values():
     lam2 = np.exp(-synth.slopes(2).double().numpy())
     assert abs(lam64[0] - 0.39972) < 1e-5 and abs(lam64[63] - 0.99610) < 1e-5
     assert abs(lam2[0] - 0.93941) < 1e-5 and abs(lam2[1] - 0.99610) < 1e-5
+
+
+# ---------------------------------------------------------------------------------------------
+# gated_rmsnorm: the grouped RMSNorm + sigmoid gate after the kernel
+# ---------------------------------------------------------------------------------------------
+def test_gated_rmsnorm_hand_case():
+    # one head of d = 4: o = [1, 2, 3, 4] has mean square 30/4 = 7.5; gamma = [1, 1, 2, 2];
+    # g = 0 gives sigmoid 1/2, so y = [1, 2, 6, 8] / (2 sqrt(7.5))
+    o = np.array([[[1.0, 2.0, 3.0, 4.0]]])
+    gamma = np.array([[1.0, 1.0, 2.0, 2.0]], dtype=np.float32)
+    y = oracle.gated_rmsnorm(o, np.zeros((1, 1, 4), np.float32), gamma, 0.0)
+    want = np.array([1.0, 2.0, 6.0, 8.0]) / (2.0 * np.sqrt(7.5))
+    assert np.allclose(y[0, 0], want, rtol=1e-15, atol=0)
+    # epsilon enters under the root: mean square 7.5 + 0.5 = 8
+    y = oracle.gated_rmsnorm(o, np.zeros((1, 1, 4), np.float32), gamma, 0.5)
+    assert np.allclose(y[0, 0], np.array([1.0, 2.0, 6.0, 8.0]) / (2.0 * np.sqrt(8.0)), rtol=1e-15)
+
+
+def test_gated_rmsnorm_groups_are_heads_and_gate_is_elementwise():
+    rng = np.random.default_rng(5)
+    o = rng.standard_normal((3, 2, 8))                 # [tokens, H, d]
+    g = rng.standard_normal((3, 2, 8)).astype(np.float32)
+    gamma = rng.standard_normal((2, 8)).astype(np.float32)
+    y = oracle.gated_rmsnorm(o, g, gamma, 0.0)
+    # scale invariance per head (eps = 0): scaling one head's vector leaves y unchanged
+    o2 = o.copy()
+    o2[1, 0] *= 37.0
+    assert np.allclose(oracle.gated_rmsnorm(o2, g, gamma, 0.0), y, rtol=1e-13, atol=0)
+    # each head normalised on its own: with gamma = 1 and a saturated gate, mean(y^2) = 1 per head
+    big = np.full(o.shape, 60.0, np.float32)
+    y1 = oracle.gated_rmsnorm(o, big, np.ones((2, 8), np.float32), 0.0)
+    assert np.allclose(np.mean(y1 * y1, axis=-1), 1.0, rtol=1e-13)
+    # sigmoid(g) + sigmoid(-g) = 1
+    y_neg = oracle.gated_rmsnorm(o, -g, gamma, 0.0)
+    rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True))
+    assert np.allclose(y + y_neg, gamma.astype(np.float64) * o / rms, rtol=1e-12, atol=1e-14)
+
+
+def test_gated_rmsnorm_reads_bf16_bits_exactly():
+    g = np.array([0x3F80, 0xC000, 0x0000, 0x3F00], dtype=np.uint16).reshape(1, 1, 4)  # 1,-2,0,0.5
+    o = np.ones((1, 1, 4))
+    y = oracle.gated_rmsnorm(o, g, np.ones((1, 4), np.float32), 0.0)
+    sig = 1.0 / (1.0 + np.exp(-np.array([1.0, -2.0, 0.0, 0.5])))
+    assert np.array_equal(y[0, 0], sig)
