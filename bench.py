@@ -1,12 +1,14 @@
 """Benchmark of the Lightning Attention layer kernel (prefill + decode step) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload prefill_32k|prefill_4k|prefill_256k]
+                    [--workload prefill_32k|prefill_4k|prefill_256k|varlen_64k]
 
 One step = one whole pass of the hot path over one batch of synthetic input:
   * la_prefill of the prefill workload (default: B=2, N=32768, H=64, d=128, bf16, seed 1), which
     writes o for every token and the final fp32 state;
   * one la_decode_step of 256 sequences x 64 heads x d=128 on a resident fp32 state (2 GiB).
+``--workload varlen_64k`` runs la_prefill_varlen instead: 65,536 tokens of 48 packed sequences of a
+fragmented length mix, each continuing from an fp32 initial state.
 The JSON line's ``value`` is prefill tokens/s (tokens = B*N positions, all 64 heads) summed over
 ranks; the decode step is reported under ``decode`` as state GB/s.  Under torchrun each rank runs
 an independent replica (weak scaling, no collective on the data path).
@@ -218,15 +220,48 @@ def run_ours(args):
     world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = synth.WORKLOADS[args.workload]
+    vw = synth.VARLEN_WORKLOADS.get(args.workload)
+    w = synth.WORKLOADS[args.workload] if vw is None else synth.Workload(
+        vw.name, 1, vw.T, vw.H, vw.d, vw.dtype, vw.dist, vw.seed)
     B, N, H, d = w.B, w.N, w.H, w.d
     q, k, v = synth.draw_qkv(B, N, H, d, dist=w.dist, seed=w.seed + 1000 * rank, dtype=w.dtype,
                              device=dev)
     sl = synth.slopes(H, dev)
     out = torch.empty_like(q)
-    st = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
-    desc = la.make_desc(B, N, H, d, w.dtype)
-    ws_bytes = la.la_prefill_workspace_bytes(desc)
+    extra_in = []  # further inputs copied from the host in the e2e leg
+    epi = None
+    if args.gate:
+        # fused grouped RMSNorm + sigmoid gate on the prefill output: a gate pre-activation the
+        # size of q and a norm weight per head and channel (synthetic, seeded)
+        gg = torch.Generator(device=dev)
+        gg.manual_seed(77 + 1000 * rank)
+        gate = (torch.randn((B * N, H, d), generator=gg, device=dev)).to(w.dtype)
+        gamma = (1.0 + 0.1 * torch.randn((H, d), generator=gg, device=dev)).float()
+        extra_in += [gate]
+        epi = la.la_gate_norm(gate.data_ptr(), gamma.data_ptr(), 1e-6)
+    if vw is None and args.gate:
+        # the fused epilogue is an option of the packed entry point: B sequences of N tokens
+        n_states = B
+        cu = torch.arange(0, B * N + 1, N, dtype=torch.int64, device=dev)
+        sin = None
+        st = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+        desc = la.la_varlen_desc(B * N, B, H, d, la.LA_BF16, 0, 0, la.LA_PATH_AUTO)
+        ws_bytes = la.la_prefill_varlen_workspace_bytes(desc)
+    elif vw is None:
+        n_states = B
+        st = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+        desc = la.make_desc(B, N, H, d, w.dtype)
+        ws_bytes = la.la_prefill_workspace_bytes(desc)
+    else:
+        lengths = synth.draw_seqlens(vw.T, vw.n_seqs, seed=vw.len_seed)
+        cu = torch.tensor(synth.cu_from_lengths(lengths), dtype=torch.int64, device=dev)
+        n_states = vw.n_seqs
+        sin = synth.draw_states(vw.n_seqs, H, d, seed=vw.state_seed, scale=vw.state_scale,
+                                device=dev)
+        st = torch.empty_like(sin)
+        extra_in += [sin, cu]
+        desc = la.la_varlen_desc(vw.T, vw.n_seqs, H, d, la.LA_BF16, 0, 0, la.LA_PATH_AUTO)
+        ws_bytes = la.la_prefill_varlen_workspace_bytes(desc)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
 
     Bd, Hd, dd = DECODE["B"], DECODE["H"], DECODE["d"]
@@ -239,9 +274,17 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
 
+    packed = vw is not None or args.gate
+
     def prefill_call():
-        rc = la.la_prefill(desc, q.data_ptr(), k.data_ptr(), v.data_ptr(), sl.data_ptr(),
-                           out.data_ptr(), st.data_ptr(), ws.data_ptr(), ws_bytes, sp)
+        if not packed:
+            rc = la.la_prefill(desc, q.data_ptr(), k.data_ptr(), v.data_ptr(), sl.data_ptr(),
+                               out.data_ptr(), st.data_ptr(), ws.data_ptr(), ws_bytes, sp)
+        else:
+            rc = la.la_prefill_varlen(desc, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                      sl.data_ptr(), cu.data_ptr(),
+                                      0 if sin is None else sin.data_ptr(), out.data_ptr(),
+                                      st.data_ptr(), ws.data_ptr(), ws_bytes, sp, epilogue=epi)
         if rc != la.LA_OK:
             raise la.LaError(rc, "la_prefill")
 
@@ -307,6 +350,9 @@ def run_ours(args):
         hdk.copy_(dk.cpu())
         hdv.copy_(dv.cpu())
         hdout = torch.empty_like(hdq).pin_memory()
+        hextra = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in extra_in]
+        for hx, x in zip(hextra, extra_in):
+            hx.copy_(x.cpu())
         n_e2e = max(1, min(K, 3))
         barrier(world)
         torch.cuda.synchronize(dev)
@@ -320,6 +366,8 @@ def run_ours(args):
             dq.copy_(hdq, non_blocking=True)
             dk.copy_(hdk, non_blocking=True)
             dv.copy_(hdv, non_blocking=True)
+            for x, hx in zip(extra_in, hextra):
+                x.copy_(hx, non_blocking=True)
             prefill_call()
             decode_call()
             hout.copy_(out, non_blocking=True)
@@ -328,7 +376,8 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
-        bi = 3 * q.numel() * q.element_size() + 3 * dq.numel() * dq.element_size()
+        bi = 3 * q.numel() * q.element_size() + 3 * dq.numel() * dq.element_size() + sum(
+            x.numel() * x.element_size() for x in extra_in)
         bo = out.numel() * out.element_size() + st.numel() * 4 + dout.numel() * dout.element_size()
         e2e = {"value": world * B * N / (e2e_ms * 1e-3), "unit": "tok/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms,
@@ -338,8 +387,10 @@ def run_ours(args):
         hbm_peak, tc_peak, peak_kind = load_peaks()
         tokens = B * N
         tok_s = world * tokens / (pre_ms_max * 1e-3)
-        # algorithmic bytes of one prefill launch: read q, k, v and write o (bf16), write state
-        pre_bytes = 4 * B * N * H * d * 2 + B * H * d * d * 4
+        # algorithmic bytes of one prefill launch: read q, k, v and write o (bf16), write the
+        # final states (and read the initial states of the packed workload)
+        pre_bytes = (4 + (1 if args.gate else 0)) * B * N * H * d * 2 + \
+            n_states * H * d * d * 4 * (1 if vw is None else 2)
         achieved = pre_bytes / (pre_ms_max * 1e-3) / 1e9
         canon = 4.0 * d * d * B * N * H  # recurrent-form flops
         executed = (4.0 * d * d + 4.0 * 128 * d) * B * N * H  # full 128 x 128 tiles
@@ -358,8 +409,12 @@ def run_ours(args):
             "metric": METRIC, "value": tok_s, "unit": "tok/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{w.name}: B={B} N={N} H={H} d={d} bf16 + decode step "
-                                   f"B={Bd} H={Hd} d={dd} (fp32 state)",
+            "config": {"workload": (f"{w.name}: B={B} N={N} H={H} d={d} bf16" if vw is None else
+                                    f"{vw.name}: T={vw.T} tokens in {vw.n_seqs} packed sequences "
+                                    f"(fragmented lengths), H={H} d={d} bf16, fp32 initial "
+                                    f"states") + (", fused grouped RMSNorm + sigmoid gate epilogue"
+                                                  if args.gate else "") +
+                                   f" + decode step B={Bd} H={Hd} d={dd} (fp32 state)",
                        "global_batch": world * B, "seq_len": N, "parallelism": f"replicas{world}",
                        "l2": "inputs larger than L2 (no flush)"},
             "prefill": {"ms": pre_ms_max, "tok_s": tok_s,
@@ -370,13 +425,16 @@ def run_ours(args):
                        "frac_of_8tbs": dec_gbs / 8000.0, "tok_s": world * Bd / (dec_ms_max * 1e-3)},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak,
-                         "traffic": measured_traffic() if args.workload == "prefill_32k" else None,
+                         "traffic": (measured_traffic() if args.workload == "prefill_32k"
+                                     and not args.gate else None),
                          "algorithmic_bytes": pre_bytes,
                          "kernel": "chunked_prefill_kernel", "peak_kind": peak_kind},
             "cpu_baseline": cpu,
             "clocks": clk.summary(),
             "e2e": e2e,
-            "gpu_launches": 2 * K,
+            # per step: the prefill kernel (after the planning kernel for packed input) and the
+            # decode kernel
+            "gpu_launches": (3 if packed else 2) * K,
         }
         print(json.dumps(line), flush=True)
     dist_teardown(world)
@@ -393,7 +451,9 @@ def run_reference(args):
     import numpy as np
 
     import oracle
-    w = synth.WORKLOADS[args.workload]
+    vw = synth.VARLEN_WORKLOADS.get(args.workload)
+    w = synth.WORKLOADS[args.workload] if vw is None else synth.Workload(
+        vw.name, 1, vw.T, vw.H, vw.d, vw.dtype, vw.dist, vw.seed)
     cores = oracle.num_threads()
     n_heads = cores
     n_tok = min(w.N, 4096)
@@ -428,8 +488,11 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill_32k", "prefill_4k", "prefill_256k"],
+    ap.add_argument("--workload", choices=["prefill_32k", "prefill_4k", "prefill_256k",
+                                           "varlen_64k"],
                     default="prefill_32k")
+    ap.add_argument("--gate", action="store_true",
+                    help="fuse the grouped RMSNorm + sigmoid gate into the prefill's output")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer e2e leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     args = ap.parse_args()

@@ -177,9 +177,23 @@ typedef struct {
   int32_t path;     /* la_path */
 } la_varlen_desc;
 
-/* Bytes of device workspace la_prefill_varlen needs (0 only for invalid arguments).  It depends on
- * the sequence lengths, which set the work-unit table and the segment plan. */
-size_t la_prefill_varlen_workspace_bytes(const la_varlen_desc* desc, const int64_t* cu_seqlens);
+/* Optional epilogue of la_prefill_varlen: the step the report's layer runs right after this
+ * kernel, a grouped RMSNorm of each head's output vector followed by the sigmoid gate (§2.1
+ * Fig. 2: Linear Attention Kernel -> Grouped RMSNorm, times sigmoid(Gate Projection); §4.3 fuses
+ * "group norm + sigmoid gate" into one operator).  With it, out receives, per token t and head h,
+ *     y_j = gamma[h, j] * o_j / sqrt(mean_j(o_j^2) + eps) * sigmoid(g[t, h, j])
+ * computed from the fp32 accumulator of o (each head is one norm group of d channels), rounded
+ * once to bf16.  Tensor-core path only (bf16, d = 128). */
+typedef struct {
+  const void* gate;   /* [T, H, d] device bf16: the gate pre-activation g = x W_gate, read only */
+  const float* gamma; /* fp32 [H, d] device: the norm's weight, read only */
+  float eps;          /* epsilon under the root, >= 0 (the report's RMSNorm uses 1e-6) */
+} la_gate_norm;
+
+/* Bytes of device workspace la_prefill_varlen needs (0 only for invalid arguments): an upper
+ * bound over every cu_seqlens of this shape (the work-unit table holds at most
+ * H * (n_seqs + ceil(T / 128)) units). */
+size_t la_prefill_varlen_workspace_bytes(const la_varlen_desc* desc);
 
 /*
  * la_prefill_varlen — la_prefill over variable-length sequences packed along one token axis
@@ -192,33 +206,38 @@ size_t la_prefill_varlen_workspace_bytes(const la_varlen_desc* desc, const int64
  * head h the recurrence of la_prefill runs from S = state_in[s, h] (zero if state_in is NULL):
  *     S <- lambda_h S + k_t^T v_t,   o_t = q_t S,   state_out[s, h] = S after the last token.
  * A sequence of length 0 writes no output and passes its initial state through to state_out.
- * All sequences, heads and segments go into one launch of the kernel la_prefill uses
- * (tensor-core or recurrent, by desc->path as for la_prefill).
+ * The call stays on the device: a one-block planning kernel reads cu_seqlens, checks it and
+ * writes the table of work units (one segment of one sequence and head each), then one launch
+ * of the kernel la_prefill uses (tensor-core or recurrent, by desc->path) runs them all.
  *
  *   desc        shape and options (host pointer, read during the call only)
  *   q, k, v     [T, H, d] device, dtype desc->dtype, read only (a [B, N, H, d] tensor is the packed
  *               layout of B sequences of N tokens)
  *   slopes      fp32[H] device
- *   cu_seqlens  HOST int64[n_seqs + 1]: cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_seqs] = T;
- *               read during the call only (the plan built from it is copied to the workspace)
+ *   cu_seqlens  DEVICE int64[n_seqs + 1]: cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_seqs] = T
  *   state_in    fp32 [n_seqs, H, d, d] device, or NULL for zero initial states; read only
+ *   epilogue    NULL (out receives o), or the fused norm + gate above (host pointer, read during
+ *               the call; gate and gamma 16-byte aligned, gate must not overlap out)
  *   out         [T, H, d] device, written
  *   state_out   fp32 [n_seqs, H, d, d] device, or NULL.  It may be the same pointer as state_in
  *               (in-place continuation); any other overlap with state_in is LA_ERR_ALIAS.
- *   workspace   device scratch of at least la_prefill_varlen_workspace_bytes(desc, cu_seqlens)
- *               bytes, 256-byte aligned, used only by this call until it completes on `stream`;
- *               NULL: allocated and freed on `stream` (cudaMallocAsync / cudaFreeAsync)
+ *   workspace   device scratch of at least la_prefill_varlen_workspace_bytes(desc) bytes, 256-byte
+ *               aligned, used only by this call until it completes on `stream`; NULL: allocated
+ *               and freed on `stream` (cudaMallocAsync / cudaFreeAsync)
  *   stream      cudaStream_t as void*
  *
- * Errors: LA_ERR_SHAPE for a cu_seqlens that is not a non-decreasing run from 0 to T (or other
- * shape errors as in la_prefill), LA_ERR_ALIGN for q, k, v, out, state_in, state_out not 16-byte
- * aligned, LA_ERR_ALIAS as above or when out overlaps q, k or v; the rest as la_prefill.  The
- * device status word (la_workspace_status) reports a scan timeout as for la_prefill.
+ * Errors returned by the call: shape, dtype, NULL, alignment and aliasing errors as for
+ * la_prefill (q, k, v, out, state_in, state_out must be 16-byte aligned).  cu_seqlens lives on the
+ * device, so its contents are checked there: if it is not a non-decreasing run from 0 to T, the
+ * planning kernel records LA_ERR_SHAPE in the workspace status word (la_workspace_status), no
+ * kernel touches out or state_out, and the call itself has returned LA_OK.  A scan timeout is
+ * reported the same way as for la_prefill.
  */
 la_status la_prefill_varlen(const la_varlen_desc* desc, const void* q, const void* k,
                             const void* v, const float* slopes, const int64_t* cu_seqlens,
-                            const float* state_in, void* out, float* state_out, void* workspace,
-                            size_t workspace_bytes, void* stream);
+                            const float* state_in, const la_gate_norm* epilogue, void* out,
+                            float* state_out, void* workspace, size_t workspace_bytes,
+                            void* stream);
 
 /* Synchronises `stream`, then returns the device status word of a workspace that la_prefill
  * used: LA_OK, or LA_ERR_TIMEOUT if a bounded device wait gave up during the last call. */

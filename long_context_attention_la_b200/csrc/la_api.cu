@@ -7,7 +7,6 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
-#include <vector>
 
 #include "la.h"
 #include "la_internal.h"
@@ -85,18 +84,15 @@ la_status check_desc(const la_desc* d, int64_t* numel) {
   return LA_OK;
 }
 
-// Validates a varlen descriptor and its host cu_seqlens; on success writes the element count of
-// one packed activation tensor.
-la_status check_varlen(const la_varlen_desc* d, const int64_t* cu, int64_t* numel) {
-  if (d == nullptr || cu == nullptr) return LA_ERR_NULL;
+// Validates a varlen descriptor (cu_seqlens is a device array: its contents are checked by the
+// planning kernel); on success writes the element count of one packed activation tensor.
+la_status check_varlen(const la_varlen_desc* d, int64_t* numel) {
+  if (d == nullptr) return LA_ERR_NULL;
   if (d->dtype != LA_BF16 && d->dtype != LA_F32) return LA_ERR_DTYPE;
   if (d->T < 0 || d->n_seqs < 1 || d->H < 1 || (d->d != 64 && d->d != 128)) return LA_ERR_SHAPE;
   if (d->path != LA_PATH_AUTO && d->path != LA_PATH_TENSOR && d->path != LA_PATH_RECURRENT)
     return LA_ERR_UNSUPPORTED;
   if (d->segments < 0) return LA_ERR_SHAPE;
-  if (cu[0] != 0 || cu[d->n_seqs] != d->T) return LA_ERR_SHAPE;
-  for (int64_t s = 0; s < d->n_seqs; ++s)
-    if (cu[s + 1] < cu[s]) return LA_ERR_SHAPE;
   int64_t t = 0, bytes = 0, st = 0, nh = 0;
   if (!mul_ok(d->T, d->H, &t) || !mul_ok(t, d->d, &t)) return LA_ERR_OVERFLOW;
   if (!mul_ok(t, d->dtype == LA_BF16 ? 2 : 4, &bytes)) return LA_ERR_OVERFLOW;
@@ -105,8 +101,11 @@ la_status check_varlen(const la_varlen_desc* d, const int64_t* cu, int64_t* nume
   if (use_tensor_path(d->path, d->dtype, d->d)) {
     if (d->dtype != LA_BF16 || d->d != la::kHeadDim) return LA_ERR_UNSUPPORTED;
     if (d->chunk != 0 && d->chunk != la::kChunk) return LA_ERR_UNSUPPORTED;
-    // token coordinates of the tensor maps and work units are 32-bit
+    // token coordinates of the tensor maps and work units are 32-bit, and so is the unit count
     if (d->T > INT32_MAX - la::kChunk) return LA_ERR_OVERFLOW;
+    int64_t cap = 0;
+    if (!mul_ok(d->H, d->n_seqs + (d->T + la::kChunk - 1) / la::kChunk, &cap) || cap > INT32_MAX)
+      return LA_ERR_OVERFLOW;
     int64_t row = 0;
     if (!mul_ok(d->T, d->H * d->d * 2, &row) || row >= (int64_t(1) << 40)) return LA_ERR_OVERFLOW;
   } else if (d->chunk != 0 && d->chunk != 1) {
@@ -168,24 +167,24 @@ la_status la_prefill(const la_desc* desc, const void* q, const void* k, const vo
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
-size_t la_prefill_varlen_workspace_bytes(const la_varlen_desc* desc, const int64_t* cu_seqlens) {
+size_t la_prefill_varlen_workspace_bytes(const la_varlen_desc* desc) {
   int64_t numel = 0;
-  if (check_varlen(desc, cu_seqlens, &numel) != LA_OK) return 0;
+  if (check_varlen(desc, &numel) != LA_OK) return 0;
   const bool tensor = use_tensor_path(desc->path, desc->dtype, desc->d);
   const int sms = device_sms() > 0 ? device_sms() : 148;
-  const la::VarlenPlan plan =
-      la::plan_varlen(cu_seqlens, desc->n_seqs, desc->H, desc->segments, sms, nullptr);
-  return la::varlen_workspace_layout(desc->n_seqs, desc->H, plan, tensor).total;
+  return la::varlen_workspace_layout(desc->T, desc->n_seqs, desc->H, desc->segments, sms, tensor)
+      .total;
 }
 
 la_status la_prefill_varlen(const la_varlen_desc* desc, const void* q, const void* k,
                             const void* v, const float* slopes, const int64_t* cu_seqlens,
-                            const float* state_in, void* out, float* state_out, void* workspace,
-                            size_t workspace_bytes, void* stream) {
+                            const float* state_in, const la_gate_norm* epilogue, void* out,
+                            float* state_out, void* workspace, size_t workspace_bytes,
+                            void* stream) {
   int64_t numel = 0;
-  const la_status st = check_varlen(desc, cu_seqlens, &numel);
+  const la_status st = check_varlen(desc, &numel);
   if (st != LA_OK) return st;
-  if (!q || !k || !v || !slopes || !out) return LA_ERR_NULL;
+  if (!q || !k || !v || !slopes || !out || !cu_seqlens) return LA_ERR_NULL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_ALIGN;
   if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
     return LA_ERR_ALIGN;
@@ -199,14 +198,19 @@ la_status la_prefill_varlen(const la_varlen_desc* desc, const void* q, const voi
       overlaps(state_in, state_bytes, state_out, state_bytes))
     return LA_ERR_ALIAS;
   if (state_out && bytes > 0 && overlaps(state_out, state_bytes, out, bytes)) return LA_ERR_ALIAS;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool tensor = use_tensor_path(desc->path, desc->dtype, desc->d);
+  if (epilogue != nullptr) {
+    if (!tensor) return LA_ERR_UNSUPPORTED;  // the fused norm + gate lives in the chunked kernel
+    if (!epilogue->gate || !epilogue->gamma) return LA_ERR_NULL;
+    if (!aligned16(epilogue->gate) || !aligned16(epilogue->gamma)) return LA_ERR_ALIGN;
+    if (!(epilogue->eps >= 0.f) || epilogue->eps > 3.0e38f) return LA_ERR_SHAPE;  // NaN, inf
+    if (bytes > 0 && overlaps(epilogue->gate, bytes, out, bytes)) return LA_ERR_ALIAS;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int sms = device_sms();
   if (sms <= 0) return LA_ERR_CUDA;
-
-  const int64_t n = desc->n_seqs, H = desc->H;
-  const la::VarlenPlan plan = la::plan_varlen(cu_seqlens, n, H, desc->segments, sms, nullptr);
-  const la::VarlenWorkspace layout = la::varlen_workspace_layout(n, H, plan, tensor);
+  const la::VarlenWorkspace layout =
+      la::varlen_workspace_layout(desc->T, desc->n_seqs, desc->H, desc->segments, sms, tensor);
   void* ws = workspace;
   bool owned = false;
   if (ws == nullptr) {
@@ -216,41 +220,18 @@ la_status la_prefill_varlen(const la_varlen_desc* desc, const void* q, const voi
     if (workspace_bytes < layout.total) return LA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return LA_ERR_ALIGN;
   }
-  uint8_t* table_dst = static_cast<uint8_t*>(ws) + layout.table_off;
-  cudaError_t e = cudaSuccess;
-  la::PrefillArgs a{1, desc->T, H, desc->d, desc->dtype, q, k, v, slopes, out, state_out};
-  a.n_seqs = n;
+  la::PrefillArgs a{1, desc->T, desc->H, desc->d, desc->dtype, q, k, v, slopes, out, state_out};
+  a.n_seqs = desc->n_seqs;
+  a.cu_dev = cu_seqlens;
   a.state_in = state_in;
-  apply_debug_env(a);
-  if (tensor) {
-    // The plan goes to the device with one copy from pageable host memory: the call returns once
-    // the source has been read, so the host vector may go out of scope right after.
-    std::vector<la::WorkUnit> table(static_cast<size_t>(plan.units));
-    la::plan_varlen(cu_seqlens, n, H, desc->segments, sms, table.data());
-    if (!table.empty())
-      e = cudaMemcpyAsync(table_dst, table.data(), layout.table_bytes, cudaMemcpyHostToDevice, s);
-    // Sequences without tokens have no work unit: their state passes through here.
-    for (int64_t q_ = 0; q_ < n && e == cudaSuccess && state_out != nullptr; ++q_) {
-      if (cu_seqlens[q_ + 1] != cu_seqlens[q_]) continue;
-      const size_t one = static_cast<size_t>(H) * static_cast<size_t>(desc->d * desc->d) * 4;
-      float* dst = state_out + q_ * H * desc->d * desc->d;
-      if (state_in == nullptr) {
-        e = cudaMemsetAsync(dst, 0, one, s);
-      } else if (state_in != state_out) {
-        e = cudaMemcpyAsync(dst, state_in + q_ * H * desc->d * desc->d, one,
-                            cudaMemcpyDeviceToDevice, s);
-      }
-    }
-    if (e == cudaSuccess) e = la::launch_chunked_prefill_varlen(a, plan, layout, ws, s, sms);
-  } else {
-    e = cudaMemcpyAsync(table_dst, cu_seqlens, layout.table_bytes, cudaMemcpyHostToDevice, s);
-    a.cu_dev = reinterpret_cast<const int64_t*>(table_dst);
-    if (e == cudaSuccess) {
-      // the status word is read by la_workspace_status; this path never sets it
-      e = cudaMemsetAsync(ws, 0, layout.base.header_bytes, s);
-    }
-    if (e == cudaSuccess) e = la::launch_recurrent_prefill(a, s);
+  if (epilogue != nullptr) {
+    a.gate = epilogue->gate;
+    a.gamma = epilogue->gamma;
+    a.eps = epilogue->eps;
   }
+  apply_debug_env(a);
+  const cudaError_t e =
+      la::launch_prefill_varlen(a, layout, ws, desc->segments, tensor, s, sms);
   if (owned) cudaFreeAsync(ws, s);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }

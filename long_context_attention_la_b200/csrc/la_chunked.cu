@@ -97,6 +97,7 @@ struct Params {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
+  CUtensorMap tm_gate;  // fused norm + gate only: the gate pre-activation, for L2 prefetches
   __nv_bfloat16* out;
   const float* slopes;
   float* state_out;
@@ -105,7 +106,11 @@ struct Params {
   uint32_t* flags;
   float* ring;
   const WorkUnit* unit_table;  // variable-length plan (device), or null: units follow from N, BH
+  const volatile int32_t* units_dev;  // its unit count (device), written by the planning kernel
   const float* state_in;       // fp32 [sequences, H, D, D] initial states, or null (zero)
+  const __nv_bfloat16* gate;   // fused norm + gate: gate pre-activation like out, or null
+  const float* gamma;          // fp32 [H, D] norm weight
+  float eps;
   int64_t N, H, BH;
   int64_t n_chunks, seg_chunks, segments, units;
   uint64_t timeout_ns;
@@ -207,8 +212,9 @@ __device__ __forceinline__ void transpose4x4_lanes(uint4 (&x)[4], uint32_t t) {
 
 __device__ __forceinline__ void decode_unit(const Params& p, int64_t u, UnitInfo& ui) {
   if (p.unit_table != nullptr) {
+    // written by the planning kernel earlier on the stream: coherent loads
     const int4* src = reinterpret_cast<const int4*>(p.unit_table + u);
-    const int4 w0 = __ldg(src), w1 = __ldg(src + 1);
+    const int4 w0 = __ldcg(src), w1 = __ldcg(src + 1), w2 = __ldcg(src + 2);
     ui.bh = w0.x;
     ui.seg = w0.y;
     ui.c0 = w0.z;
@@ -217,6 +223,7 @@ __device__ __forceinline__ void decode_unit(const Params& p, int64_t u, UnitInfo
     ui.flags = w1.y;
     ui.b = w1.z;
     ui.tok0 = w1.w;
+    ui.slot = w2.x;
     return;
   }
   // fixed length: unit u = segment k of flat head bh, segment-major
@@ -233,6 +240,109 @@ __device__ __forceinline__ void decode_unit(const Params& p, int64_t u, UnitInfo
   ui.flags = (k + 1 < p.segments ? 1 : 0) | (k + 1 == p.segments ? 2 : 0);
   ui.b = static_cast<int32_t>(bh / p.H);
   ui.tok0 = 0;
+  ui.slot = static_cast<int32_t>(bh);
+}
+
+// Output epilogue with the fused grouped RMSNorm and sigmoid gate ("Ling and Ring 2.6 Technical
+// Report", §2.1 Fig. 2; §4.3): thread i's row of O (one head, D channels) is one norm group,
+//     y_j = gamma_j * O_j / sqrt(mean(O^2) + eps) * sigmoid(g_j).
+// Pass 1 reads the row's fp32 accumulators once for the mean square.  Pass 2 reads them again,
+// rounds O to bf16 (the precision the unfused layer hands to its norm), exchanges 16-byte pieces
+// within each 4-lane group as the plain epilogue does, and then finishes each piece in the store
+// layout: lane t holds piece t of rows i0..i0+3, so its gate loads and stores write whole sectors
+// and its gamma slice is the same for all four rows.
+__device__ __forceinline__ float sigmoidf_fast(float x) {
+  return __fdividef(1.f, 1.f + __expf(-x));
+}
+
+__device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint32_t trow, float f,
+                                               const UnitInfo& ui, int64_t h, int64_t b,
+                                               uint32_t t, int32_t r0, int64_t n0,
+                                               int64_t row_stride) {
+  const __nv_bfloat16* gate_h = p.gate + (b * p.N * p.H + h) * D;
+  // gate pieces of 32-column block cb in the store layout: piece t of rows i0..i0+3
+  auto load_gate = [&](uint32_t cb, uint4 (&g)[4]) {
+#pragma unroll
+    for (uint32_t k = 0; k < 4; ++k) {
+      g[k] = make_uint4(0u, 0u, 0u, 0u);
+      if (r0 + static_cast<int32_t>(k) < ui.len)
+        g[k] = __ldcs(reinterpret_cast<const uint4*>(gate_h + (n0 + k) * row_stride + cb * 32) + t);
+    }
+  };
+  uint4 g_next[4];
+  load_gate(0, g_next);  // in flight during pass 1
+  float ss = 0.f;
+#pragma unroll 1
+  for (uint32_t cb = 0; cb < 8; ++cb) {  // 16-column blocks
+    uint32_t ra[16], re[16];
+    tmem_ld16(trow + kColOintra + cb * 16, ra);
+    tmem_ld16(trow + kColOinter + cb * 16, re);
+    tmem_wait_ld();
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const float o = fmaf(f, __uint_as_float(re[m]), __uint_as_float(ra[m]));
+      ss = fmaf(o, o, ss);
+    }
+  }
+  const float rinv = rsqrtf(fmaf(ss, 1.f / D, p.eps));
+  float rk[4];  // 1 / rms of rows i0 + k, held by lanes 4a + k
+  const uint32_t lane0 = (threadIdx.x & 31u) & ~3u;
+#pragma unroll
+  for (uint32_t k = 0; k < 4; ++k) rk[k] = __shfl_sync(0xffffffffu, rinv, lane0 + k);
+  __nv_bfloat16* out_h = p.out + (b * p.N * p.H + h) * D;
+#pragma unroll 1
+  for (uint32_t cb = 0; cb < 4; ++cb) {
+    uint4 x[4];  // bf16 O, pieces q = 0..3 of this row's 32 columns
+#pragma unroll
+    for (uint32_t hh = 0; hh < 2; ++hh) {
+      uint32_t ra[16], re[16];
+      tmem_ld16(trow + kColOintra + cb * 32 + hh * 16, ra);
+      tmem_ld16(trow + kColOinter + cb * 32 + hh * 16, re);
+      tmem_wait_ld();
+      if (cb == 3 && hh == 1) {
+        // every O column of this row has been read: the accumulators may be overwritten
+        tc_fence_before();
+        mbar_arrive(&ctrl->o_free);
+      }
+#pragma unroll
+      for (uint32_t qq = 0; qq < 2; ++qq) {
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          o[e] = fmaf(f, __uint_as_float(re[8 * qq + e]), __uint_as_float(ra[8 * qq + e]));
+        x[2 * hh + qq].x = pack_bf16x2(o[0], o[1]);
+        x[2 * hh + qq].y = pack_bf16x2(o[2], o[3]);
+        x[2 * hh + qq].z = pack_bf16x2(o[4], o[5]);
+        x[2 * hh + qq].w = pack_bf16x2(o[6], o[7]);
+      }
+    }
+    transpose4x4_lanes(x, t);  // now x[k] = piece t of row i0 + k
+    uint4 gx[4];
+#pragma unroll
+    for (uint32_t k = 0; k < 4; ++k) gx[k] = g_next[k];
+    if (cb + 1 < 4) load_gate(cb + 1, g_next);  // the next block's pieces load meanwhile
+    const float4 ga = __ldg(reinterpret_cast<const float4*>(p.gamma + h * D + cb * 32 + 8 * t));
+    const float4 gb = __ldg(reinterpret_cast<const float4*>(p.gamma + h * D + cb * 32 + 8 * t) + 1);
+    const float gm[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+    for (uint32_t k = 0; k < 4; ++k) {
+      if (r0 + static_cast<int32_t>(k) < ui.len) {
+        const uint32_t gw[4] = {gx[k].x, gx[k].y, gx[k].z, gx[k].w};
+        const uint32_t ow[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+        uint32_t yw[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const float y0 = gm[2 * e2] * (bf16lo_to_f32(ow[e2]) * rk[k]) *
+                           sigmoidf_fast(bf16lo_to_f32(gw[e2]));
+          const float y1 = gm[2 * e2 + 1] * (bf16hi_to_f32(ow[e2]) * rk[k]) *
+                           sigmoidf_fast(bf16hi_to_f32(gw[e2]));
+          yw[e2] = pack_bf16x2(y0, y1);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(out_h + (n0 + k) * row_stride + cb * 32) + t;
+        __stcs(dst, make_uint4(yw[0], yw[1], yw[2], yw[3]));
+      }
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -270,6 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&p.tm_q);
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
+    if (p.gate != nullptr) tma_prefetch_desc(&p.tm_gate);
   }
   if (warp == 2) {
     tmem_alloc(&ctrl->tmem_base, 512);
@@ -294,11 +405,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // then nc output loads (Q, K, V).
       auto fetch = [&](UnitInfo& ui) {
         const int64_t u = static_cast<int64_t>(atomicAdd(p.counter, 1u));
-        if (u < p.units) {
+        const int64_t units = p.units_dev != nullptr ? *p.units_dev : p.units;
+        if (u < units) {
           decode_unit(p, u, ui);
         } else {
           ui.bh = -1;
-          ui.seg = ui.c0 = ui.nc = ui.len = ui.flags = ui.b = ui.tok0 = 0;
+          ui.seg = ui.c0 = ui.nc = ui.len = ui.flags = ui.b = ui.tok0 = ui.slot = 0;
         }
       };
       auto n_loads = [](const UnitInfo& ui) -> int32_t {
@@ -364,6 +476,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (q - n_cur < n_loads(nxt)) prefetch(nxt, q - n_cur);
             }
           }
+          if (pos + 1 == n_cur && p.state_in != nullptr) {
+            // at the unit's last load, claim the next unit and bring its initial state into L2
+            // for the state warps (64 KiB per head, read when that unit starts)
+            if (!have_nxt) {
+              fetch(nxt);
+              have_nxt = true;
+            }
+            if (nxt.bh >= 0 && nxt.seg == 0)
+              bulk_prefetch_l2(p.state_in + static_cast<int64_t>(nxt.bh) * D * D, D * D * 4);
+          }
           const uint32_t s = g & 1;
           if (!mbar_wait_bounded(&ctrl->empty[s], ((g >> 1) & 1) ^ 1, abort_flag, T)) {
             ok = false;
@@ -381,6 +503,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(st + kOffQ, &p.tm_q, &ctrl->full[s], 0, h, n0, b, pol_first);
             tma_load_4d(st + kOffQ + kHalfBytes, &p.tm_q, &ctrl->full[s], 64, h, n0, b,
                         pol_first);
+          }
+          if (!local_state_pass && p.gate != nullptr) {
+            // the epilogue reads this chunk's gate rows about one chunk period from now
+            tma_prefetch_l2_4d(&p.tm_gate, 0, h, n0, b, pol_normal);
+            tma_prefetch_l2_4d(&p.tm_gate, 64, h, n0, b, pol_normal);
           }
           tma_load_4d(st + kOffK, &p.tm_k, &ctrl->full[s], 0, h, n0, b, kv_pol);
           tma_load_4d(st + kOffK + kHalfBytes, &p.tm_k, &ctrl->full[s], 64, h, n0, b, kv_pol);
@@ -433,9 +560,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const UnitInfo ui = ctrl->units[slot];
         mbar_arrive(&ctrl->unit_empty[slot]);
         if (ui.bh < 0) break;
-        // the state region must be free of the previous unit's read-out
-        if (!mbar_wait_bounded(&ctrl->kv_free, j & 1, abort_flag, T)) break;
-        tc_fence_after();
+        // A local-state pass writes the state columns first, so it waits for the previous unit's
+        // read-out.  Otherwise the state warps write them first themselves (the incoming state),
+        // after their own read-out, and every state-column MMA here waits for that; S_0 need not.
+        // Skipping the wait keeps the barrier's phases unambiguous: when this warp starts unit j,
+        // the state warps have finished unit j-2 (it waited either here or for their operand of
+        // unit j-1's first chunk), so the phase it waits for next is never two behind.  A unit
+        // without chunks gives no such operand, so it waits here too.
+        if ((ui.flags & 1) || ui.nc == 0) {
+          if (!mbar_wait_bounded(&ctrl->kv_free, j & 1, abort_flag, T)) break;
+          tc_fence_after();
+        }
         if (ui.flags & 1) {
           // local segment state h = sum_j lambda^(L-1-j) k_j^T v_j into the KV columns
           for (int32_t c = 0; c < ui.nc && ok; ++c) {
@@ -669,7 +804,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&ctrl->unit_empty[slot]);
       if (ui.bh < 0) break;
       const float alpha = p.slopes[ui.bh % p.H] * kLog2e;
-      const int64_t bh = ui.bh;
+      const int64_t bh = ui.bh;    // state_in / state_out index
+      const int64_t rs = ui.slot;  // scan flags and state ring (sequences cut into segments)
       const int32_t k = ui.seg;
 
       if (ui.flags & 1) {
@@ -681,7 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // incoming state of this segment: published by segment k-1 of the same sequence
       if (k > 0) {
-        const uint32_t* fl = p.flags + bh * 2 + ((k - 1) & 1);
+        const uint32_t* fl = p.flags + rs * 2 + ((k - 1) & 1);
         const uint64_t t0 = globaltimer_ns();
         ok = true;
         while (ld_acquire_u32(fl) != static_cast<uint32_t>(k)) {
@@ -695,8 +831,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // ring layout: float4 (state row i, columns 4q..4q+3) at index q * 128 + i
       const float4* ring_in =
-          reinterpret_cast<const float4*>(p.ring + (bh * 2 + ((k - 1) & 1)) * (D * D));
-      float4* ring_out = reinterpret_cast<float4*>(p.ring + (bh * 2 + (k & 1)) * (D * D));
+          reinterpret_cast<const float4*>(p.ring + (rs * 2 + ((k - 1) & 1)) * (D * D));
+      float4* ring_out = reinterpret_cast<float4*>(p.ring + (rs * 2 + (k & 1)) * (D * D));
       const float lam_len = exp2f(-alpha * static_cast<float>(ui.len));
       const float lam_n0 = exp2f(-alpha * static_cast<float>(min(C, ui.len)));
 #pragma unroll 1
@@ -741,6 +877,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             __stcg(ring_out + (cb * 8 + q) * 128 + i, x);
           }
         }
+        if (ui.nc == 0 && p.state_out != nullptr) {
+          // a sequence without tokens: its final state is its initial state
+          float4* so = reinterpret_cast<float4*>(p.state_out + (bh * D + i) * D) + cb * 8;
+#pragma unroll
+          for (uint32_t q = 0; q < 8; ++q)
+            so[q] = make_float4(__uint_as_float(sin[4 * q]), __uint_as_float(sin[4 * q + 1]),
+                                __uint_as_float(sin[4 * q + 2]), __uint_as_float(sin[4 * q + 3]));
+        }
         write_kvb(cb, sin);
 #pragma unroll
         for (int m = 0; m < 32; ++m) sin[m] = __float_as_uint(lam_n0 * __uint_as_float(sin[m]));
@@ -754,7 +898,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_bar_sync(kBarS, 128);
         if (wq == 0 && lane == 0 && k != p.withhold_segment) {
           __threadfence();
-          st_release_u32(p.flags + bh * 2 + (k & 1), static_cast<uint32_t>(k + 1));
+          st_release_u32(p.flags + rs * 2 + (k & 1), static_cast<uint32_t>(k + 1));
         }
       }
 
@@ -868,6 +1012,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t n0 = static_cast<int64_t>(ui.tok0) + static_cast<int64_t>(ui.c0) * C + r0;
         __nv_bfloat16* out_h = p.out + (b * p.N * p.H + h) * D;
         const int64_t row_stride = p.H * D;
+        if (p.gate != nullptr) {
+          gated_epilogue(p, ctrl, trow, f, ui, h, b, t, r0, n0, row_stride);
+          continue;
+        }
 #pragma unroll 1
         for (uint32_t cb = 0; cb < 4; ++cb) {  // 32-column blocks
           uint32_t ra[32], re[32];
@@ -997,11 +1145,11 @@ WorkspaceLayout workspace_layout(int64_t B, int64_t H, const SegmentPlan& plan) 
 
 namespace {
 
-// Shared launch: fills the parameters common to both forms and runs the kernel.  `zero_bytes`
-// leading workspace bytes (counter, status, scan flags) are cleared first on `stream`.
+// Shared launch: fills the parameters common to both forms and runs the kernel.  With
+// clear_header the counter, status word and scan flags are first cleared on `stream`.
 cudaError_t launch_common(const PrefillArgs& a, Params& prm, uint8_t* ws,
                           const WorkspaceLayout& wl, int64_t units, cudaStream_t stream,
-                          int num_sms) {
+                          int num_sms, bool clear_header = true) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1013,16 +1161,26 @@ cudaError_t launch_common(const PrefillArgs& a, Params& prm, uint8_t* ws,
     attr_set[dev] = true;
   }
   // counter, status and scan flags start at zero for every call
-  e = cudaMemsetAsync(ws, 0, wl.flags_off + wl.flags_bytes, stream);
-  if (e != cudaSuccess || units == 0) return e;
-  if (!encode_map(&prm.tm_q, a.q, a.B, a.N, a.H) || !encode_map(&prm.tm_k, a.k, a.B, a.N, a.H) ||
-      !encode_map(&prm.tm_v, a.v, a.B, a.N, a.H)) {
+  if (clear_header) {
+    e = cudaMemsetAsync(ws, 0, wl.flags_off + wl.flags_bytes, stream);
+    if (e != cudaSuccess) return e;
+  }
+  if (units == 0) return cudaSuccess;
+  // (an all-empty packed batch has N = 0 tokens: its units load nothing, but a map needs N >= 1)
+  const int64_t n_map = std::max<int64_t>(a.N, 1);
+  if (!encode_map(&prm.tm_q, a.q, a.B, n_map, a.H) || !encode_map(&prm.tm_k, a.k, a.B, n_map, a.H) ||
+      !encode_map(&prm.tm_v, a.v, a.B, n_map, a.H)) {
     return cudaErrorInvalidValue;
   }
   prm.out = static_cast<__nv_bfloat16*>(a.out);
   prm.slopes = a.slopes;
   prm.state_out = a.state_out;
   prm.state_in = a.state_in;
+  prm.gate = static_cast<const __nv_bfloat16*>(a.gate);
+  if (a.gate != nullptr && !encode_map(&prm.tm_gate, a.gate, a.B, n_map, a.H))
+    return cudaErrorInvalidValue;
+  prm.gamma = a.gamma;
+  prm.eps = a.eps;
   prm.counter = reinterpret_cast<uint32_t*>(ws + kWsCounter);
   prm.status = reinterpret_cast<int32_t*>(ws + kWsStatus);
   prm.flags = reinterpret_cast<uint32_t*>(ws + wl.flags_off);
@@ -1052,84 +1210,281 @@ cudaError_t launch_chunked_prefill(const PrefillArgs& a, const SegmentPlan& plan
                        plan.units, stream, num_sms);
 }
 
-VarlenPlan plan_varlen(const int64_t* cu, int64_t n_seqs, int64_t H, int requested_segments,
-                       int num_sms, WorkUnit* table) {
-  VarlenPlan pl;
-  int64_t nonempty = 0;
-  for (int64_t s = 0; s < n_seqs; ++s) nonempty += cu[s + 1] > cu[s] ? 1 : 0;
-  // Segments per sequence: the fixed-length rule with B*H counted over non-empty sequences, so
-  // equal lengths give the same plan as la_prefill.
-  auto segments_of = [&](int64_t n_chunks) -> int64_t {
-    int64_t want;
-    if (requested_segments > 0) {
-      want = requested_segments;
-    } else if (2 * nonempty * H > static_cast<int64_t>(num_sms)) {
-      want = 1;
-    } else {
-      want = std::max<int64_t>(1, std::min<int64_t>(num_sms / (nonempty * H), n_chunks / 4));
-    }
-    want = std::max<int64_t>(1, std::min<int64_t>(want, n_chunks));
-    const int64_t seg_chunks = (n_chunks + want - 1) / want;
-    return (n_chunks + seg_chunks - 1) / seg_chunks;
-  };
-  int64_t max_segments = 0;
-  for (int64_t s = 0; s < n_seqs; ++s) {
-    const int64_t len = cu[s + 1] - cu[s];
-    if (len <= 0) continue;
-    max_segments = std::max(max_segments, segments_of((len + C - 1) / C));
+// ---------------------------------------------------------------------------------------------
+// Variable-length plan, built on the device from cu_seqlens by one block of 1024 threads.
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanSortMax = 8192;  // sequences ordered longest first up to this count
+
+struct PlanArgs {
+  const int64_t* cu;
+  int64_t n_seqs, T, H;
+  int32_t requested, num_sms;
+  int64_t unit_cap, slot_cap;
+  WorkUnit* table;  // null: only check cu (recurrent path)
+  int32_t* status;
+  int32_t* units_out;
+};
+
+// Segments of a sequence of n_chunks chunks: the fixed-length rule of plan_segments, with B*H
+// counted over the non-empty sequences, so equal lengths plan exactly as la_prefill does.  An
+// empty sequence is one unit without chunks.
+__device__ __forceinline__ int64_t segments_of(int64_t n_chunks, int64_t nonempty_heads,
+                                               int32_t requested, int32_t sms) {
+  if (n_chunks == 0) return 1;
+  int64_t want;
+  if (requested > 0) {
+    want = requested;
+  } else if (2 * nonempty_heads > sms) {
+    want = 1;
+  } else {
+    want = max(int64_t(1), min(int64_t(sms) / nonempty_heads, n_chunks / 4));
   }
-  pl.multi_segment = max_segments > 1;
-  int64_t u = 0;
-  for (int64_t k = 0; k < max_segments; ++k) {
-    for (int64_t s = 0; s < n_seqs; ++s) {
-      const int64_t len = cu[s + 1] - cu[s];
-      if (len <= 0) continue;
-      const int64_t n_chunks = (len + C - 1) / C;
-      const int64_t segs = segments_of(n_chunks);
-      if (k >= segs) continue;
-      const int64_t seg_chunks = (n_chunks + segs - 1) / segs;
-      const int64_t c0 = k * seg_chunks;
-      const int64_t nc = std::min(seg_chunks, n_chunks - c0);
-      const int64_t end = std::min(len, (c0 + nc) * C);
-      for (int64_t h = 0; h < H; ++h, ++u) {
-        if (table == nullptr) continue;
-        WorkUnit& w = table[u];
-        w.bh = static_cast<int32_t>(s * H + h);
-        w.seg = static_cast<int32_t>(k);
-        w.c0 = static_cast<int32_t>(c0);
-        w.nc = static_cast<int32_t>(nc);
-        w.len = static_cast<int32_t>(end - c0 * C);
-        w.flags = (k + 1 < segs ? 1 : 0) | (k + 1 == segs ? 2 : 0);
-        w.b = 0;
-        w.tok0 = static_cast<int32_t>(cu[s]);
+  want = max(int64_t(1), min(want, n_chunks));
+  const int64_t seg_chunks = (n_chunks + want - 1) / want;
+  return (n_chunks + seg_chunks - 1) / seg_chunks;
+}
+
+// Exclusive block-wide prefix sum of one int64 per thread; also returns the block total.
+__device__ int64_t block_exclusive_scan(int64_t x, int64_t* total, int64_t* sh /* [33] */) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int64_t incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) sh[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int64_t v = lane < (kPlanThreads / 32) ? sh[lane] : 0;
+    int64_t vi = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(0xffffffffu, vi, o);
+      if (lane >= o) vi += y;
+    }
+    sh[lane] = vi - v;  // exclusive prefix of the warp totals
+    if (lane == 31) sh[32] = vi;
+  }
+  __syncthreads();
+  const int64_t r = sh[w] + incl - x;
+  *total = sh[32];
+  __syncthreads();
+  return r;
+}
+
+// Sorts keys[0, n) ascending in shared memory (bitonic network; n a power of two).
+__device__ void block_bitonic_sort(unsigned long long* keys, int n) {
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      __syncthreads();
+      for (int i = threadIdx.x; i < n / 2; i += kPlanThreads) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const unsigned long long x = keys[lo], y = keys[hi];
+        if ((x > y) == up) {
+          keys[lo] = y;
+          keys[hi] = x;
+        }
       }
     }
   }
-  pl.units = u;
-  return pl;
+  __syncthreads();
 }
 
-VarlenWorkspace varlen_workspace_layout(int64_t n_seqs, int64_t H, const VarlenPlan& plan,
-                                        bool tensor_path) {
+__global__ void __launch_bounds__(kPlanThreads) plan_varlen_kernel(const PlanArgs a) {
+  extern __shared__ unsigned long long order[];  // [n_pad]: (longest first, then index) keys
+  __shared__ int64_t sh[33];
+  __shared__ int bad;
+  __shared__ unsigned long long nonempty, max_seg;
+  if (threadIdx.x == 0) {
+    bad = (a.cu[0] != 0 || a.cu[a.n_seqs] != a.T) ? 1 : 0;
+    nonempty = 0;
+    max_seg = 0;
+  }
+  __syncthreads();
+  // check cu and count the non-empty sequences
+  unsigned long long my_nonempty = 0;
+  for (int64_t s = threadIdx.x; s < a.n_seqs; s += kPlanThreads) {
+    const int64_t x0 = a.cu[s], x1 = a.cu[s + 1];
+    if (x1 < x0 || x0 < 0 || x1 > a.T) bad = 1;
+    my_nonempty += x1 > x0 ? 1 : 0;
+  }
+  atomicAdd(&nonempty, my_nonempty);
+  __syncthreads();
+  if (bad) {
+    if (threadIdx.x == 0) {
+      *a.status = -2;  // LA_ERR_SHAPE
+      *a.units_out = 0;
+    }
+    return;
+  }
+  if (a.table == nullptr) {
+    if (threadIdx.x == 0) *a.units_out = 0;
+    return;
+  }
+  const int64_t nonempty_heads = max(int64_t(1), static_cast<int64_t>(nonempty)) * a.H;
+  unsigned long long my_max = 0;
+  for (int64_t s = threadIdx.x; s < a.n_seqs; s += kPlanThreads) {
+    const int64_t nch = (a.cu[s + 1] - a.cu[s] + C - 1) / C;
+    my_max = max(my_max, static_cast<unsigned long long>(
+                             segments_of(nch, nonempty_heads, a.requested, a.num_sms)));
+  }
+  atomicMax(&max_seg, my_max);
+  __syncthreads();
+  const int64_t levels = static_cast<int64_t>(max_seg);
+
+  // Within a level, sequences go longest first (ties by index), so the persistent CTAs, which
+  // take units in table order, start the long units early and finish together.  Beyond
+  // kPlanSortMax sequences the table keeps sequence order.
+  const bool sorted = a.n_seqs <= kPlanSortMax;
+  int n_pad = 1;
+  while (n_pad < a.n_seqs) n_pad <<= 1;
+  if (sorted) {
+    for (int64_t p = threadIdx.x; p < n_pad; p += kPlanThreads) {
+      if (p < a.n_seqs) {
+        const int64_t nch = (a.cu[p + 1] - a.cu[p] + C - 1) / C;
+        order[p] = (static_cast<unsigned long long>(0x7fffffff - nch) << 32) |
+                   static_cast<unsigned long long>(p);
+      } else {
+        order[p] = ~0ull;  // padding sorts last
+      }
+    }
+    block_bitonic_sort(order, n_pad);
+  }
+
+  // Units go out segment-major: all units of segment k precede those of segment k + 1, so a
+  // unit only ever waits on a unit taken before it.  Within a level: sequences in order, H heads
+  // each.  Sequences with more than one segment get a ring slot, in sequence order.
+  int64_t base = 0;
+  int status = 0;
+  for (int64_t k = 0; k < levels; ++k) {
+    int64_t slot_base = 0;
+    for (int64_t s0 = 0; s0 < a.n_seqs; s0 += kPlanThreads) {
+      const int64_t p = s0 + threadIdx.x;  // position in the level's order
+      const int64_t s = p < a.n_seqs ? (sorted ? static_cast<int64_t>(order[p] & 0xffffffffull) : p)
+                                     : a.n_seqs;
+      int64_t len = 0, nch = 0, segs = 0;
+      if (s < a.n_seqs) {
+        len = a.cu[s + 1] - a.cu[s];
+        nch = (len + C - 1) / C;
+        segs = segments_of(nch, nonempty_heads, a.requested, a.num_sms);
+      }
+      const int64_t active = (s < a.n_seqs && k < segs) ? 1 : 0;
+      const int64_t multi = (s < a.n_seqs && segs > 1) ? 1 : 0;
+      int64_t n_active = 0, n_multi = 0;
+      const int64_t pos = block_exclusive_scan(active, &n_active, sh);
+      const int64_t mpos = block_exclusive_scan(multi, &n_multi, sh);
+      if (active) {
+        const int64_t u0 = base + pos * a.H;
+        const int64_t slot = slot_base + mpos;
+        if (u0 + a.H > a.unit_cap || (multi && slot >= a.slot_cap)) {
+          status = -6;  // LA_ERR_WORKSPACE (cannot happen with the host's capacities)
+        } else {
+          const int64_t seg_chunks = nch > 0 ? (nch + segs - 1) / segs : 0;
+          const int64_t c0 = k * seg_chunks;
+          const int64_t nc = nch > 0 ? min(seg_chunks, nch - c0) : 0;
+          const int64_t end = min(len, (c0 + nc) * C);
+          WorkUnit w;
+          w.seg = static_cast<int32_t>(k);
+          w.c0 = static_cast<int32_t>(c0);
+          w.nc = static_cast<int32_t>(nc);
+          w.len = static_cast<int32_t>(end - c0 * C);
+          w.flags = (k + 1 < segs ? 1 : 0) | (k + 1 == segs ? 2 : 0);
+          w.b = 0;
+          w.tok0 = static_cast<int32_t>(a.cu[s]);
+          w.pad[0] = w.pad[1] = w.pad[2] = 0;
+          for (int64_t h = 0; h < a.H; ++h) {
+            w.bh = static_cast<int32_t>(s * a.H + h);
+            w.slot = multi ? static_cast<int32_t>(slot * a.H + h) : w.bh;
+            a.table[u0 + h] = w;
+          }
+        }
+      }
+      base += n_active * a.H;
+      slot_base += n_multi;
+    }
+  }
+  if (status != 0) atomicExch(a.status, status);
+  __syncthreads();
+  if (threadIdx.x == 0) *a.units_out = static_cast<int32_t>(min(base, a.unit_cap));
+}
+
+}  // namespace
+
+VarlenWorkspace varlen_workspace_layout(int64_t T, int64_t n_seqs, int64_t H,
+                                        int requested_segments, int num_sms, bool tensor_path) {
   VarlenWorkspace w{};
+  w.unit_cap = tensor_path ? H * (n_seqs + (T + C - 1) / C) : 0;
+  // Sequences cut into segments need a ring slot.  Automatic plans cut only when the non-empty
+  // sequences times H fit in half the SMs; an explicit request may cut every sequence.
+  if (!tensor_path || requested_segments == 1) {
+    w.slot_cap = 0;
+  } else if (requested_segments > 1) {
+    w.slot_cap = n_seqs;
+  } else {
+    w.slot_cap = std::min<int64_t>(n_seqs, std::max(0, num_sms) / std::max<int64_t>(1, 2 * H));
+  }
   SegmentPlan sp{};
-  sp.segments = plan.multi_segment ? 2 : 1;  // only "more than one segment" matters for the size
-  w.base = workspace_layout(n_seqs, H, sp);
+  sp.segments = w.slot_cap > 0 ? 2 : 1;  // only "more than one segment" matters for the size
+  w.base = workspace_layout(w.slot_cap, H, sp);
   w.table_off = (w.base.total + 255) / 256 * 256;
-  w.table_bytes = tensor_path ? static_cast<size_t>(plan.units) * sizeof(WorkUnit)
-                              : static_cast<size_t>(n_seqs + 1) * sizeof(int64_t);
-  w.total = w.table_off + w.table_bytes;
+  w.total = w.table_off + static_cast<size_t>(w.unit_cap) * sizeof(WorkUnit);
   return w;
 }
 
-cudaError_t launch_chunked_prefill_varlen(const PrefillArgs& a, const VarlenPlan& plan,
-                                          const VarlenWorkspace& layout, void* workspace,
-                                          cudaStream_t stream, int num_sms) {
-  Params prm{};
+cudaError_t launch_prefill_varlen(const PrefillArgs& a, const VarlenWorkspace& layout,
+                                  void* workspace, int requested_segments, bool tensor_path,
+                                  cudaStream_t stream, int num_sms) {
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  prm.unit_table = reinterpret_cast<const WorkUnit*>(ws + layout.table_off);
+  cudaError_t e = cudaMemsetAsync(ws, 0, layout.base.flags_off + layout.base.flags_bytes, stream);
+  if (e != cudaSuccess) return e;
+  PlanArgs pa{};
+  pa.cu = a.cu_dev;
+  pa.n_seqs = a.n_seqs;
+  pa.T = a.N;
+  pa.H = a.H;
+  pa.requested = requested_segments;
+  pa.num_sms = num_sms;
+  pa.unit_cap = layout.unit_cap;
+  pa.slot_cap = layout.slot_cap;
+  pa.table = tensor_path ? reinterpret_cast<WorkUnit*>(ws + layout.table_off) : nullptr;
+  pa.status = reinterpret_cast<int32_t*>(ws + kWsStatus);
+  pa.units_out = reinterpret_cast<int32_t*>(ws + kWsUnits);
+  size_t sort_bytes = 0;
+  if (a.n_seqs <= kPlanSortMax) {
+    int64_t n_pad = 1;
+    while (n_pad < a.n_seqs) n_pad <<= 1;
+    sort_bytes = static_cast<size_t>(n_pad) * sizeof(unsigned long long);
+  }
+  static bool plan_attr_set[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && !plan_attr_set[dev]) {
+    e = cudaFuncSetAttribute(plan_varlen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kPlanSortMax * sizeof(unsigned long long)));
+    if (e != cudaSuccess) return e;
+    plan_attr_set[dev] = true;
+  }
+  plan_varlen_kernel<<<1, kPlanThreads, sort_bytes, stream>>>(pa);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (!tensor_path) {
+    PrefillArgs r = a;
+    r.status = pa.status;
+    return launch_recurrent_prefill(r, stream);
+  }
+  Params prm{};
+  prm.unit_table = pa.table;
+  prm.units_dev = pa.units_out;
   prm.BH = a.n_seqs * a.H;
-  return launch_common(a, prm, ws, layout.base, plan.units, stream, num_sms);
+  // The plan's unit count is only known on the device: launch for the capacity (one CTA per SM
+  // at most); CTAs that find no unit exit.
+  return launch_common(a, prm, ws, layout.base, layout.unit_cap, stream, num_sms,
+                       /*clear_header=*/false);
 }
 
 }  // namespace la

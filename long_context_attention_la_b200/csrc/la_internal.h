@@ -20,11 +20,18 @@ struct PrefillArgs {
   void* out;
   float* state_out;  // may be null
   // Packed variable-length form (la_prefill_varlen): B = 1, N = total tokens; sequence s owns
-  // tokens [cu[s], cu[s+1]).  cu_dev is a device copy of cu (recurrent kernel), state_in an
-  // optional fp32 [n_seqs, H, d, d] initial state.  n_seqs = 0 means the fixed [B, N] form.
+  // tokens [cu[s], cu[s+1]) of the device array cu_dev; state_in is an optional fp32
+  // [n_seqs, H, d, d] initial state.  n_seqs = 0 means the fixed [B, N] form.  status (device)
+  // is the workspace status word, which the recurrent kernel checks before doing any work.
   int64_t n_seqs = 0;
   const int64_t* cu_dev = nullptr;
   const float* state_in = nullptr;
+  const int32_t* status = nullptr;
+  // Fused grouped RMSNorm + sigmoid gate on the output (tensor path): gate [.., H, d] bf16 and
+  // gamma fp32 [H, d]; gate == nullptr stores o itself.
+  const void* gate = nullptr;
+  const float* gamma = nullptr;
+  float eps = 0.f;
   // Failure injection for tests (host-side switch, see la_api.cu): the segment index whose scan
   // flag is never published (-1: none) and the limit of every device wait.
   int32_t withhold_segment = -1;
@@ -56,16 +63,18 @@ constexpr int kHeadDim = 128;
 
 // One work unit of the chunked prefill, as the kernel reads it: one segment of one (sequence, head).
 struct WorkUnit {
-  int32_t bh;     // state / scan index: sequence * H + head (-1: no more work)
+  int32_t bh;     // state index: sequence * H + head (-1: no more work)
   int32_t seg;    // segment index k within the sequence
   int32_t c0;     // first chunk of the segment, counted from the sequence start
-  int32_t nc;     // chunks in the segment
+  int32_t nc;     // chunks in the segment (0: an empty sequence, whose state passes through)
   int32_t len;    // tokens in the segment
   int32_t flags;  // bit 0: compute the local state first; bit 1: last segment of the sequence
   int32_t b;      // batch coordinate of the sequence in the [B, N, H, d] tensors
   int32_t tok0;   // token coordinate (along N) of the sequence's first token
+  int32_t slot;   // scan-flag / state-ring index of a sequence cut into segments (per head)
+  int32_t pad[3];
 };
-static_assert(sizeof(WorkUnit) == 32, "WorkUnit is read as two 16-byte words");
+static_assert(sizeof(WorkUnit) == 48, "WorkUnit is read as three 16-byte words");
 
 // How a prefill is cut into work units: each (b, h) sequence of N tokens becomes `segments`
 // segments of `seg_chunks` chunks (the last may be shorter); one unit = one (segment, b, h).
@@ -97,31 +106,26 @@ constexpr size_t kWsStatus = 64;   // uint32 device status (0 = ok, else a la_st
 cudaError_t launch_chunked_prefill(const PrefillArgs& a, const SegmentPlan& plan,
                                    void* workspace, cudaStream_t stream, int num_sms);
 
-// Variable-length plan: the work units of every non-empty sequence, segment-major (all units of
-// segment k precede those of segment k + 1, so a unit only waits on units taken before it).
-struct VarlenPlan {
-  int64_t units = 0;
-  bool multi_segment = false;  // some sequence has more than one segment (needs flags and ring)
-};
-// Fills `table` (may be null to count only) with the units of cu[0..n_seqs]; returns the plan.
-VarlenPlan plan_varlen(const int64_t* cu, int64_t n_seqs, int64_t H, int requested_segments,
-                       int num_sms, WorkUnit* table);
-
-// Workspace of la_prefill_varlen: the fixed-length layout for n_seqs * H states, then the unit
-// table (tensor path) or a copy of cu (recurrent path).
+// Variable-length form.  Capacities the host sizes the workspace with (cu_seqlens stays on the
+// device, so only its shape is known here): at most H * (n_seqs + ceil(T / C)) work units, and
+// ring slots for the sequences that may be cut into segments.
 struct VarlenWorkspace {
-  WorkspaceLayout base;
-  size_t table_off;
-  size_t table_bytes;
+  int64_t unit_cap;     // work units
+  int64_t slot_cap;     // sequences with a state-ring slot (times H heads each)
+  WorkspaceLayout base; // header, scan flags and ring for slot_cap * H states
+  size_t table_off;     // work-unit table
   size_t total;
 };
-VarlenWorkspace varlen_workspace_layout(int64_t n_seqs, int64_t H, const VarlenPlan& plan,
-                                        bool tensor_path);
+VarlenWorkspace varlen_workspace_layout(int64_t T, int64_t n_seqs, int64_t H,
+                                        int requested_segments, int num_sms, bool tensor_path);
 
-// Launches the chunked kernel over a unit table already in device memory at
-// workspace + layout.table_off.
-cudaError_t launch_chunked_prefill_varlen(const PrefillArgs& a, const VarlenPlan& plan,
-                                          const VarlenWorkspace& layout, void* workspace,
-                                          cudaStream_t stream, int num_sms);
+// Offset of the device-written work-unit count in the workspace header.
+constexpr size_t kWsUnits = 128;
+
+// Clears the header and flags, runs the one-block planning kernel (checks cu, writes the unit
+// table and count; with tensor_path false it only checks cu), then the prefill kernel.
+cudaError_t launch_prefill_varlen(const PrefillArgs& a, const VarlenWorkspace& layout,
+                                  void* workspace, int requested_segments, bool tensor_path,
+                                  cudaStream_t stream, int num_sms);
 
 }  // namespace la

@@ -57,7 +57,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(4 * D) recurrent_prefill_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const float* __restrict__ slopes, T* __restrict__ out, float* state_out, int64_t N,
-    int64_t H, const int64_t* __restrict__ cu, const float* state_in) {
+    int64_t H, const int64_t* __restrict__ cu, const float* state_in, const int32_t* status) {
   constexpr int R = D / 4;
   __shared__ float tok[2][3][D];
   __shared__ float red[4][D];
@@ -65,6 +65,8 @@ __global__ void __launch_bounds__(4 * D) recurrent_prefill_kernel(
   const int tid = threadIdx.x;
   const int j = tid % D;
   const int rg = tid / D;
+  // packed input whose cu_seqlens failed the device check: touch nothing
+  if (status != nullptr && *status != 0) return;
   const int64_t flat = blockIdx.x;
   const int64_t b = flat / H;  // batch index, or sequence index of packed input
   const int64_t h = flat % H;
@@ -204,7 +206,7 @@ cudaError_t launch_recurrent_typed(const PrefillArgs& a, cudaStream_t stream) {
   if (grid == 0) return cudaSuccess;
   recurrent_prefill_kernel<T, D><<<static_cast<unsigned>(grid), 4 * D, 0, stream>>>(
       static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
-      a.slopes, static_cast<T*>(a.out), a.state_out, a.N, a.H, a.cu_dev, a.state_in);
+      a.slopes, static_cast<T*>(a.out), a.state_out, a.N, a.H, a.cu_dev, a.state_in, a.status);
   return cudaGetLastError();
 }
 

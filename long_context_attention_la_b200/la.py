@@ -51,6 +51,10 @@ class la_varlen_desc(ctypes.Structure):  # noqa: N801 - mirrors the C type name
                 ("segments", ctypes.c_int32), ("path", ctypes.c_int32)]
 
 
+class la_gate_norm(ctypes.Structure):  # noqa: N801 - mirrors the C type name
+    _fields_ = [("gate", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("eps", ctypes.c_float)]
+
+
 class LaError(RuntimeError):
     def __init__(self, status: int, what: str = ""):
         self.status = status
@@ -79,10 +83,10 @@ def library(path: str | None = None):
         lib.la_prefill.restype = ctypes.c_int
         lib.la_prefill_noalloc.argtypes = [ctypes.POINTER(la_desc), vp, vp, vp, vp, vp, vp, vp]
         lib.la_prefill_noalloc.restype = ctypes.c_int
-        lib.la_prefill_varlen_workspace_bytes.argtypes = [ctypes.POINTER(la_varlen_desc), vp]
+        lib.la_prefill_varlen_workspace_bytes.argtypes = [ctypes.POINTER(la_varlen_desc)]
         lib.la_prefill_varlen_workspace_bytes.restype = sz
         lib.la_prefill_varlen.argtypes = [ctypes.POINTER(la_varlen_desc), vp, vp, vp, vp, vp, vp,
-                                          vp, vp, vp, sz, vp]
+                                          ctypes.POINTER(la_gate_norm), vp, vp, vp, sz, vp]
         lib.la_prefill_varlen.restype = ctypes.c_int
         lib.la_decode_step.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp]
         lib.la_decode_step.restype = ctypes.c_int
@@ -120,25 +124,21 @@ def la_prefill_noalloc(desc: la_desc, q: int, k: int, v: int, slopes: int, out: 
 LA_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024 + 4096
 
 
-def _i64_array(values) -> ctypes.Array:
-    vals = [int(x) for x in values]
-    return (ctypes.c_int64 * len(vals))(*vals)
+def la_prefill_varlen_workspace_bytes(desc: la_varlen_desc) -> int:
+    return int(library().la_prefill_varlen_workspace_bytes(ctypes.byref(desc)))
 
 
-def la_prefill_varlen_workspace_bytes(desc: la_varlen_desc, cu_seqlens) -> int:
-    """cu_seqlens: host sequence of n_seqs + 1 ints (or a ctypes int64 array)."""
-    cu = cu_seqlens if isinstance(cu_seqlens, ctypes.Array) else _i64_array(cu_seqlens)
-    return int(library().la_prefill_varlen_workspace_bytes(ctypes.byref(desc), cu))
-
-
-def la_prefill_varlen(desc: la_varlen_desc, q: int, k: int, v: int, slopes: int, cu_seqlens,
+def la_prefill_varlen(desc: la_varlen_desc, q: int, k: int, v: int, slopes: int, cu_seqlens: int,
                       state_in: int, out: int, state_out: int, workspace: int,
-                      workspace_bytes: int, stream: int) -> int:
-    """cu_seqlens is a HOST sequence of n_seqs + 1 ints; the pointers are device addresses."""
-    cu = cu_seqlens if isinstance(cu_seqlens, ctypes.Array) else _i64_array(cu_seqlens)
-    return int(library().la_prefill_varlen(ctypes.byref(desc), q, k, v, slopes, cu,
-                                           state_in or None, out, state_out or None,
-                                           workspace or None, workspace_bytes, stream or None))
+                      workspace_bytes: int, stream: int,
+                      epilogue: la_gate_norm | None = None) -> int:
+    """All pointers are device addresses; cu_seqlens is a device int64[n_seqs + 1]; epilogue is
+    the optional fused norm + gate (la_gate_norm)."""
+    return int(library().la_prefill_varlen(ctypes.byref(desc), q, k, v, slopes, cu_seqlens or None,
+                                           state_in or None,
+                                           None if epilogue is None else ctypes.byref(epilogue),
+                                           out, state_out or None, workspace or None,
+                                           workspace_bytes, stream or None))
 
 
 def la_decode_step(B: int, H: int, d: int, dtype: int, q: int, k: int, v: int, slopes: int,
@@ -215,26 +215,31 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Ten
 
 def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor,
                    cu_seqlens, *, state_in: torch.Tensor | None = None,
+                   gate: torch.Tensor | None = None, gamma: torch.Tensor | None = None,
+                   eps: float = 1e-6,
                    out: torch.Tensor | None = None, state_out: torch.Tensor | None = None,
                    want_state: bool = True, chunk: int = 0, segments: int = 0,
                    path: int = LA_PATH_AUTO, workspace: torch.Tensor | None = None,
                    stream: torch.cuda.Stream | None = None):
     """o, state = prefill_varlen(q, k, v, slopes, cu_seqlens): q, k, v [T, H, d] hold n_seqs
     sequences back to back, sequence s at tokens [cu_seqlens[s], cu_seqlens[s+1]).  cu_seqlens is
-    a host sequence of ints (a list, numpy array or CPU tensor).  state_in: optional fp32
-    [n_seqs, H, d, d] initial states (state_out may be the same tensor).  Returns out [T, H, d]
-    and the final fp32 states [n_seqs, H, d, d]."""
+    a CUDA int64 tensor of n_seqs + 1 entries (a host list or array is copied to the device
+    first).  state_in: optional fp32 [n_seqs, H, d, d] initial states (state_out may be the same
+    tensor).  gate [T, H, d] bf16 and gamma fp32 [H, d] switch on the fused grouped RMSNorm +
+    sigmoid gate, so out holds gamma * o / rms(o) * sigmoid(gate) per head.
+    Returns out [T, H, d] and the final fp32 states [n_seqs, H, d, d].  An invalid
+    cu_seqlens is reported by the device: check la_workspace_status(workspace) when it is not
+    known to be valid."""
     if q.dim() != 3 or q.shape != k.shape or q.shape != v.shape:
         raise ValueError("q, k, v must share one [T, H, d] shape")
     if q.dtype not in _DT or k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("q, k, v must all be bfloat16 or all float32")
-    if isinstance(cu_seqlens, torch.Tensor):
-        if cu_seqlens.is_cuda:
-            raise ValueError("cu_seqlens must be on the host")
-        cu_seqlens = cu_seqlens.tolist()
-    cu = _i64_array(cu_seqlens)
+    if not (isinstance(cu_seqlens, torch.Tensor) and cu_seqlens.is_cuda):
+        cu_seqlens = torch.as_tensor(cu_seqlens, dtype=torch.int64).to(q.device)
+    if cu_seqlens.dtype != torch.int64 or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be int64 [n_seqs + 1]")
     T, H, d = q.shape
-    n = len(cu) - 1
+    n = cu_seqlens.numel() - 1
     if n < 1:
         raise ValueError("cu_seqlens needs at least two entries")
     if slopes.dtype != torch.float32 or slopes.shape != (H,):
@@ -246,19 +251,28 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: to
         out = torch.empty_like(q)
     if state_out is None and want_state:
         state_out = torch.empty((n, H, d, d), dtype=torch.float32, device=q.device)
+    epi = None
+    if gate is not None or gamma is not None:
+        if gate is None or gamma is None:
+            raise ValueError("the fused norm + gate needs both gate and gamma")
+        if gate.shape != q.shape or gate.dtype != q.dtype:
+            raise ValueError("gate must match q's [T, H, d] shape and dtype")
+        if gamma.dtype != torch.float32 or tuple(gamma.shape) != (H, d):
+            raise ValueError("gamma must be float32 [H, d]")
+        epi = la_gate_norm(_cuda_ptr(gate, "gate"), _cuda_ptr(gamma, "gamma"), float(eps))
     desc = la_varlen_desc(T, n, H, d, _DT[q.dtype], chunk, segments, path)
-    need = la_prefill_varlen_workspace_bytes(desc, cu)
+    need = la_prefill_varlen_workspace_bytes(desc)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = 0 if workspace is None else _cuda_ptr(workspace, "workspace")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     s = stream if stream is not None else torch.cuda.current_stream(q.device)
     st = la_prefill_varlen(desc, _cuda_ptr(q, "q"), _cuda_ptr(k, "k"), _cuda_ptr(v, "v"),
-                           _cuda_ptr(slopes, "slopes"), cu,
+                           _cuda_ptr(slopes, "slopes"), _cuda_ptr(cu_seqlens, "cu_seqlens"),
                            0 if state_in is None else _cuda_ptr(state_in, "state_in"),
                            _cuda_ptr(out, "out"),
                            0 if state_out is None else _cuda_ptr(state_out, "state_out"),
-                           ws_ptr, ws_bytes, s.cuda_stream)
+                           ws_ptr, ws_bytes, s.cuda_stream, epi)
     if st != LA_OK:
         raise LaError(st, "la_prefill_varlen")
     return out, state_out

@@ -156,3 +156,34 @@ def cu_from_lengths(lengths) -> list[int]:
     for x in lengths:
         cu.append(cu[-1] + int(x))
     return cu
+
+
+@dataclass(frozen=True)
+class VarlenWorkload:
+    """A packed batch of ``n_seqs`` sequences (lengths from ``draw_seqlens(T, n_seqs, len_seed)``)
+    with initial states N(0,1) * ``state_scale`` (seed ``state_seed``); q, k, v drawn as
+    ``draw_qkv(1, T, H, d, dist, seed)``."""
+    name: str
+    T: int
+    n_seqs: int
+    H: int
+    d: int
+    dtype: torch.dtype
+    dist: str
+    seed: int
+    len_seed: int
+    state_seed: int
+    state_scale: float = 0.1
+
+
+VARLEN_WORKLOADS = {
+    "varlen_64k": VarlenWorkload("varlen_64k", 65536, 48, 64, 128, torch.bfloat16, "silu_qk", 82,
+                                 81, 83),
+}
+
+
+def draw_states(n: int, H: int, d: int, *, seed: int, scale: float, device="cpu") -> torch.Tensor:
+    """fp32 [n, H, d, d] initial states: N(0,1) * scale from one generator on ``device``."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return torch.randn((n, H, d, d), generator=g, device=device, dtype=torch.float32) * scale

@@ -112,7 +112,8 @@ def test_tensor_path_workspace_covers_the_scan(lib):
 
 
 # ---------------------------------------------------------------------------------------------
-# la_prefill_varlen: argument checks (CPU only; these return before any CUDA call)
+# la_prefill_varlen: host-side argument checks (CPU only; these return before any CUDA call).
+# cu_seqlens is a device array; its contents are checked on the device (GPU tests).
 # ---------------------------------------------------------------------------------------------
 def _vdesc(**kw):
     base = dict(T=300, n_seqs=3, H=2, d=128, dtype=la.LA_BF16, chunk=0, segments=0, path=0)
@@ -121,54 +122,70 @@ def _vdesc(**kw):
 
 
 _P = (0x1000, 0x2000, 0x3000, 0x4000)  # q, k, v, slopes
+_CU = 0x6000
 
 
-@pytest.mark.parametrize("cu,kw,status", [
-    ([0, 100, 200, 300], dict(dtype=9), la.LA_ERR_DTYPE),
-    ([0, 100, 200, 300], dict(d=32), la.LA_ERR_SHAPE),
-    ([0, 100, 200, 300], dict(H=0), la.LA_ERR_SHAPE),
-    ([0, 100, 200, 300], dict(T=-1), la.LA_ERR_SHAPE),
-    ([1, 100, 200, 300], {}, la.LA_ERR_SHAPE),            # must start at 0
-    ([0, 100, 90, 300], {}, la.LA_ERR_SHAPE),             # must not decrease
-    ([0, 100, 200, 299], {}, la.LA_ERR_SHAPE),            # must end at T
-    ([0, 100, 200, 300], dict(chunk=64), la.LA_ERR_UNSUPPORTED),
-    ([0, 100, 200, 300], dict(dtype=la.LA_F32, path=la.LA_PATH_TENSOR), la.LA_ERR_UNSUPPORTED),
-    ([0, 100, 200, 300], dict(segments=-2), la.LA_ERR_SHAPE),
+@pytest.mark.parametrize("kw,status", [
+    (dict(dtype=9), la.LA_ERR_DTYPE), (dict(d=32), la.LA_ERR_SHAPE), (dict(H=0), la.LA_ERR_SHAPE),
+    (dict(T=-1), la.LA_ERR_SHAPE), (dict(n_seqs=0), la.LA_ERR_SHAPE),
+    (dict(chunk=64), la.LA_ERR_UNSUPPORTED), (dict(path=5), la.LA_ERR_UNSUPPORTED),
+    (dict(dtype=la.LA_F32, path=la.LA_PATH_TENSOR), la.LA_ERR_UNSUPPORTED),
+    (dict(segments=-2), la.LA_ERR_SHAPE), (dict(T=1 << 40, H=1 << 20), la.LA_ERR_OVERFLOW),
 ])
-def test_varlen_rejects_bad_arguments(lib, cu, kw, status):
+def test_varlen_rejects_bad_descriptors(lib, kw, status):
     d = _vdesc(**kw)
-    assert la.la_prefill_varlen(d, *_P, cu, 0, 0x50000, 0, 0, 0, 0) == status
-    assert la.la_prefill_varlen_workspace_bytes(d, cu) == 0
+    assert la.la_prefill_varlen(d, *_P, _CU, 0, 0x50000, 0, 0, 0, 0) == status
+    assert la.la_prefill_varlen_workspace_bytes(d) == 0
 
 
 def test_varlen_null_alignment_aliasing(lib):
     d = _vdesc()
-    cu = [0, 100, 200, 300]
-    assert lib.la_prefill_varlen(ctypes.byref(d), *_P, None, None, 0x50000, None, None, 0,
+    assert lib.la_prefill_varlen(None, *_P, _CU, None, None, 0x50000, None, None, 0,
                                  None) == la.LA_ERR_NULL
-    assert la.la_prefill_varlen(d, 0, *_P[1:], cu, 0, 0x50000, 0, 0, 0, 0) == la.LA_ERR_NULL
-    assert la.la_prefill_varlen(d, *_P, cu, 0x7008, 0x50000, 0, 0, 0, 0) == la.LA_ERR_ALIGN
-    assert la.la_prefill_varlen(d, *_P, cu, 0, 0x50000, 0x9004, 0, 0, 0) == la.LA_ERR_ALIGN
+    assert la.la_prefill_varlen(d, *_P, 0, 0, 0x50000, 0, 0, 0, 0) == la.LA_ERR_NULL
+    assert la.la_prefill_varlen(d, 0, *_P[1:], _CU, 0, 0x50000, 0, 0, 0, 0) == la.LA_ERR_NULL
+    assert la.la_prefill_varlen(d, *_P, _CU, 0x7008, 0x50000, 0, 0, 0, 0) == la.LA_ERR_ALIGN
+    assert la.la_prefill_varlen(d, *_P, _CU, 0, 0x50000, 0x9004, 0, 0, 0) == la.LA_ERR_ALIGN
     nbytes = 300 * 2 * 128 * 2
     # out overlapping k
     assert la.la_prefill_varlen(d, 0x100000, 0x100000 + nbytes, 0x100000 + 2 * nbytes, 0x4000,
-                                cu, 0, 0x100000 + nbytes + 512, 0, 0, 0, 0) == la.LA_ERR_ALIAS
+                                _CU, 0, 0x100000 + nbytes + 512, 0, 0, 0, 0) == la.LA_ERR_ALIAS
     # state_out overlapping state_in without being the same array
     sbytes = 3 * 2 * 128 * 128 * 4
-    assert la.la_prefill_varlen(d, *_P, cu, 0x10000000, 0x50000000, 0x10000000 + sbytes // 2, 0,
+    assert la.la_prefill_varlen(d, *_P, _CU, 0x10000000, 0x50000000, 0x10000000 + sbytes // 2, 0,
                                 0, 0) == la.LA_ERR_ALIAS
 
 
-def test_varlen_workspace_sizes(lib):
-    cu = [0, 100, 200, 300]
-    # tensor path: header + a 32-byte work unit per (sequence, head, segment)
-    w = la.la_prefill_varlen_workspace_bytes(_vdesc(segments=1), cu)
-    assert w >= 256 + 3 * 2 * 32
-    # forcing several segments adds the scan flags and the state ring of every (sequence, head)
-    w2 = la.la_prefill_varlen_workspace_bytes(_vdesc(T=3000, segments=3), [0, 1000, 2000, 3000])
-    assert w2 >= 256 + 3 * 2 * 2 * 128 * 128 * 4 + 3 * 2 * 3 * 32
-    # recurrent path: header + a device copy of cu_seqlens
-    w3 = la.la_prefill_varlen_workspace_bytes(_vdesc(dtype=la.LA_F32, d=64), cu)
-    assert w3 >= 256 + 4 * 8
-    # empty sequences are allowed, including T = 0
-    assert la.la_prefill_varlen_workspace_bytes(_vdesc(T=0), [0, 0, 0, 0]) >= 256
+def test_varlen_workspace_capacity(lib):
+    # tensor path: header + one 48-byte work unit per head for every sequence and every chunk
+    T, n, H = 3000, 3, 2
+    w = la.la_prefill_varlen_workspace_bytes(_vdesc(T=T, n_seqs=n, H=H, segments=1))
+    assert w >= 256 + H * (n + -(-T // 128)) * 48
+    # forcing several segments adds the scan flags and state ring of every (sequence, head)
+    w2 = la.la_prefill_varlen_workspace_bytes(_vdesc(T=T, n_seqs=n, H=H, segments=3))
+    assert w2 >= w + n * H * 2 * 128 * 128 * 4
+    # recurrent path: the header only (it reads cu_seqlens in place)
+    w3 = la.la_prefill_varlen_workspace_bytes(_vdesc(dtype=la.LA_F32, d=64))
+    assert 256 <= w3 < 4096
+    # T = 0 (every sequence empty) is a valid problem
+    assert la.la_prefill_varlen_workspace_bytes(_vdesc(T=0)) >= 256
+
+
+def test_varlen_epilogue_checks(lib):
+    d = _vdesc()
+    ok = la.la_gate_norm(0x800000, 0x900000, 1e-6)
+
+    def call(desc, epi, out=0x50000):
+        return la.la_prefill_varlen(desc, *_P, _CU, 0, out, 0, 0, 0, 0, epilogue=epi)
+
+    # the fused norm + gate is a tensor-core epilogue
+    assert call(_vdesc(dtype=la.LA_F32, d=64), ok) == la.LA_ERR_UNSUPPORTED
+    assert call(_vdesc(path=la.LA_PATH_RECURRENT), ok) == la.LA_ERR_UNSUPPORTED
+    assert call(d, la.la_gate_norm(0, 0x900000, 1e-6)) == la.LA_ERR_NULL
+    assert call(d, la.la_gate_norm(0x800000, 0, 1e-6)) == la.LA_ERR_NULL
+    assert call(d, la.la_gate_norm(0x800008, 0x900000, 1e-6)) == la.LA_ERR_ALIGN
+    assert call(d, la.la_gate_norm(0x800000, 0x900004, 1e-6)) == la.LA_ERR_ALIGN
+    assert call(d, la.la_gate_norm(0x800000, 0x900000, float("nan"))) == la.LA_ERR_SHAPE
+    assert call(d, la.la_gate_norm(0x800000, 0x900000, -1.0)) == la.LA_ERR_SHAPE
+    # gate overlapping out
+    assert call(d, la.la_gate_norm(0x800000, 0x900000, 1e-6), out=0x800000 + 64) == la.LA_ERR_ALIAS

@@ -182,3 +182,46 @@ def test_varlen_fragmented_mix_sampled():
         a, b = cu[s], cu[s + 1]
         sub = oracle_varlen(q[a:b], k[a:b], v[a:b], sl, [0, b - a], sin[s:s + 1])
         check_all(out[a:b], st[s:s + 1], sub, [0, b - a], torch.bfloat16)
+
+
+@pytest.mark.parametrize("path", [la.LA_PATH_AUTO, la.LA_PATH_RECURRENT])
+def test_invalid_cu_seqlens_is_reported_by_the_device(path):
+    """cu_seqlens lives on the device, so a decreasing run is caught by the planning kernel:
+    the call is enqueued, the workspace status reads LA_ERR_SHAPE, and no output is written."""
+    H, d, T = 2, 128, 300
+    q, k, v = draw_packed([T], H, d, seed=91)
+    sl = synth.slopes(H, DEV)
+    cu = torch.tensor([0, 350, T], dtype=torch.int64, device=DEV)
+    out = torch.full_like(q, 7.0)
+    st = torch.full((2, H, d, d), 7.0, device=DEV)
+    desc = la.la_varlen_desc(T, 2, H, d, la.LA_BF16, 0, 0, path)
+    ws = torch.empty(la.la_prefill_varlen_workspace_bytes(desc), dtype=torch.uint8, device=DEV)
+    s = torch.cuda.current_stream().cuda_stream
+    rc = la.la_prefill_varlen(desc, q.data_ptr(), k.data_ptr(), v.data_ptr(), sl.data_ptr(),
+                              cu.data_ptr(), 0, out.data_ptr(), st.data_ptr(), ws.data_ptr(),
+                              ws.numel(), s)
+    assert rc == la.LA_OK
+    assert la.la_workspace_status(ws.data_ptr(), s) == la.LA_ERR_SHAPE
+    assert bool((out == 7.0).all()) and bool((st == 7.0).all())
+
+
+@pytest.mark.parametrize("path", [la.LA_PATH_AUTO, la.LA_PATH_RECURRENT])
+def test_all_sequences_empty(path):
+    """T = 0: nothing to read or write but the states, which pass through (or start at zero)."""
+    H, d, n = 2, 128, 3
+    buf = torch.zeros((1, H, d), dtype=torch.bfloat16, device=DEV)  # addresses only; unused
+    sl = synth.slopes(H, DEV)
+    cu = torch.zeros(n + 1, dtype=torch.int64, device=DEV)
+    desc = la.la_varlen_desc(0, n, H, d, la.LA_BF16, 0, 0, path)
+    ws = torch.empty(la.la_prefill_varlen_workspace_bytes(desc), dtype=torch.uint8, device=DEV)
+    s = torch.cuda.current_stream().cuda_stream
+    sin = draw_states(n, H, d, seed=92)
+    for state_in, want in [(sin, sin), (None, torch.zeros_like(sin))]:
+        st = torch.full_like(sin, 3.0)
+        rc = la.la_prefill_varlen(desc, buf.data_ptr(), buf.data_ptr(), buf.data_ptr(),
+                                  sl.data_ptr(), cu.data_ptr(),
+                                  0 if state_in is None else state_in.data_ptr(), buf.data_ptr(),
+                                  st.data_ptr(), ws.data_ptr(), ws.numel(), s)
+        assert rc == la.LA_OK
+        assert la.la_workspace_status(ws.data_ptr(), s) == la.LA_OK
+        assert torch.equal(st, want)
