@@ -64,6 +64,18 @@ class LaError(RuntimeError):
 _lock = threading.Lock()
 _lib = None
 
+# When True, the tensor conveniences below synchronise the stream after each call and raise on a
+# device-side error recorded in the workspace status word (a scan timeout, or a cu_seqlens the
+# planning kernel rejected).  Off by default: it costs a stream synchronisation per call.
+CHECK_STATUS = False
+
+
+def _check_device_status(ws_ptr: int, stream_ptr: int, what: str, check) -> None:
+    if ws_ptr and (CHECK_STATUS if check is None else check):
+        st = la_workspace_status(ws_ptr, stream_ptr)
+        if st != LA_OK:
+            raise LaError(st, f"{what} (device status)")
+
 
 def library(path: str | None = None):
     """The loaded libla_b200.so (raises if it has not been built)."""
@@ -182,7 +194,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Ten
             out: torch.Tensor | None = None, state_out: torch.Tensor | None = None,
             want_state: bool = True, chunk: int = 0, segments: int = 0,
             path: int = LA_PATH_AUTO, workspace: torch.Tensor | None = None,
-            stream: torch.cuda.Stream | None = None):
+            stream: torch.cuda.Stream | None = None, check: bool | None = None):
     """o, state = prefill(q, k, v, slopes): q, k, v [B, N, H, d] (bf16 or fp32, CUDA,
     contiguous), slopes float32[H].  Returns out [B, N, H, d] and the final fp32 state
     [B, H, d, d] (None if want_state is False and no state_out is given)."""
@@ -210,6 +222,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Ten
                     ws_bytes, s.cuda_stream)
     if st != LA_OK:
         raise LaError(st, "la_prefill")
+    _check_device_status(ws_ptr, s.cuda_stream, "la_prefill", check)
     return out, state_out
 
 
@@ -220,7 +233,7 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: to
                    out: torch.Tensor | None = None, state_out: torch.Tensor | None = None,
                    want_state: bool = True, chunk: int = 0, segments: int = 0,
                    path: int = LA_PATH_AUTO, workspace: torch.Tensor | None = None,
-                   stream: torch.cuda.Stream | None = None):
+                   stream: torch.cuda.Stream | None = None, check: bool | None = None):
     """o, state = prefill_varlen(q, k, v, slopes, cu_seqlens): q, k, v [T, H, d] hold n_seqs
     sequences back to back, sequence s at tokens [cu_seqlens[s], cu_seqlens[s+1]).  cu_seqlens is
     a CUDA int64 tensor of n_seqs + 1 entries (a host list or array is copied to the device
@@ -275,6 +288,7 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: to
                            ws_ptr, ws_bytes, s.cuda_stream, epi)
     if st != LA_OK:
         raise LaError(st, "la_prefill_varlen")
+    _check_device_status(ws_ptr, s.cuda_stream, "la_prefill_varlen", check)
     return out, state_out
 
 

@@ -18,9 +18,12 @@ def pytest_configure(config):
 
 @pytest.fixture(scope="session", autouse=True)
 def _built_library():
-    """Build libla_b200.so (in-tree, sm_100a) once per session if a source is newer."""
-    from long_context_attention_la_b200 import build
+    """Build libla_b200.so (in-tree, sm_100a) once per session if a source is newer, and make the
+    tensor conveniences check the device status word after every call, so that a device-side
+    error (a scan timeout) fails the test instead of leaving unwritten outputs."""
+    from long_context_attention_la_b200 import build, la
     build.build()
+    la.CHECK_STATUS = True
 
 
 def pytest_collection_modifyitems(config, items):
