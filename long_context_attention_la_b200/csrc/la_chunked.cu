@@ -251,26 +251,32 @@ __device__ __forceinline__ void decode_unit(const Params& p, int64_t u, UnitInfo
 // within each 4-lane group as the plain epilogue does, and then finishes each piece in the store
 // layout: lane t holds piece t of rows i0..i0+3, so its gate loads and stores write whole sectors
 // and its gamma slice is the same for all four rows.
+// sigmoid(x) = (1 + tanh(x / 2)) / 2: one MUFU operation (tanh.approx, max relative error
+// about 2^-11) instead of an exponential and a reciprocal.
 __device__ __forceinline__ float sigmoidf_fast(float x) {
-  return __fdividef(1.f, 1.f + __expf(-x));
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return fmaf(0.5f, t, 0.5f);
+}
+
+// Gate pieces of 32-column block cb in the 4-lane store layout: g[k] = piece t of row i0 + k
+// (zero past the segment end).
+__device__ __forceinline__ void load_gate_pieces(const __nv_bfloat16* gate_h, int32_t len,
+                                                 int32_t r0, int64_t n0, int64_t row_stride,
+                                                 uint32_t t, uint32_t cb, uint4 (&g)[4]) {
+#pragma unroll
+  for (uint32_t k = 0; k < 4; ++k) {
+    g[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (r0 + static_cast<int32_t>(k) < len)
+      g[k] = __ldcs(reinterpret_cast<const uint4*>(gate_h + (n0 + k) * row_stride + cb * 32) + t);
+  }
 }
 
 __device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint32_t trow, float f,
-                                               const UnitInfo& ui, int64_t h, int64_t b,
+                                               const UnitInfo& ui, int64_t h,
+                                               const __nv_bfloat16* gate_h, __nv_bfloat16* out_h,
                                                uint32_t t, int32_t r0, int64_t n0,
-                                               int64_t row_stride) {
-  const __nv_bfloat16* gate_h = p.gate + (b * p.N * p.H + h) * D;
-  // gate pieces of 32-column block cb in the store layout: piece t of rows i0..i0+3
-  auto load_gate = [&](uint32_t cb, uint4 (&g)[4]) {
-#pragma unroll
-    for (uint32_t k = 0; k < 4; ++k) {
-      g[k] = make_uint4(0u, 0u, 0u, 0u);
-      if (r0 + static_cast<int32_t>(k) < ui.len)
-        g[k] = __ldcs(reinterpret_cast<const uint4*>(gate_h + (n0 + k) * row_stride + cb * 32) + t);
-    }
-  };
-  uint4 g_next[4];
-  load_gate(0, g_next);  // in flight during pass 1
+                                               int64_t row_stride, uint4 (&g)[4]) {
   float ss = 0.f;
 #pragma unroll 1
   for (uint32_t cb = 0; cb < 8; ++cb) {  // 16-column blocks
@@ -289,45 +295,40 @@ __device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint
   const uint32_t lane0 = (threadIdx.x & 31u) & ~3u;
 #pragma unroll
   for (uint32_t k = 0; k < 4; ++k) rk[k] = __shfl_sync(0xffffffffu, rinv, lane0 + k);
-  __nv_bfloat16* out_h = p.out + (b * p.N * p.H + h) * D;
 #pragma unroll 1
   for (uint32_t cb = 0; cb < 4; ++cb) {
+    // this block's gate pieces are in g (block 0: loaded before O was complete; later blocks:
+    // loaded here, in flight during the accumulator reads and the exchange)
+    if (cb > 0) load_gate_pieces(gate_h, ui.len, r0, n0, row_stride, t, cb, g);
     uint4 x[4];  // bf16 O, pieces q = 0..3 of this row's 32 columns
 #pragma unroll
-    for (uint32_t hh = 0; hh < 2; ++hh) {
-      uint32_t ra[16], re[16];
-      tmem_ld16(trow + kColOintra + cb * 32 + hh * 16, ra);
-      tmem_ld16(trow + kColOinter + cb * 32 + hh * 16, re);
+    for (uint32_t q = 0; q < 4; ++q) {
+      uint32_t ra[8], re[8];
+      tmem_ld8(trow + kColOintra + cb * 32 + q * 8, ra);
+      tmem_ld8(trow + kColOinter + cb * 32 + q * 8, re);
       tmem_wait_ld();
-      if (cb == 3 && hh == 1) {
+      if (cb == 3 && q == 3) {
         // every O column of this row has been read: the accumulators may be overwritten
         tc_fence_before();
         mbar_arrive(&ctrl->o_free);
       }
+      float o[8];
 #pragma unroll
-      for (uint32_t qq = 0; qq < 2; ++qq) {
-        float o[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          o[e] = fmaf(f, __uint_as_float(re[8 * qq + e]), __uint_as_float(ra[8 * qq + e]));
-        x[2 * hh + qq].x = pack_bf16x2(o[0], o[1]);
-        x[2 * hh + qq].y = pack_bf16x2(o[2], o[3]);
-        x[2 * hh + qq].z = pack_bf16x2(o[4], o[5]);
-        x[2 * hh + qq].w = pack_bf16x2(o[6], o[7]);
-      }
+      for (int e = 0; e < 8; ++e)
+        o[e] = fmaf(f, __uint_as_float(re[e]), __uint_as_float(ra[e]));
+      x[q].x = pack_bf16x2(o[0], o[1]);
+      x[q].y = pack_bf16x2(o[2], o[3]);
+      x[q].z = pack_bf16x2(o[4], o[5]);
+      x[q].w = pack_bf16x2(o[6], o[7]);
     }
     transpose4x4_lanes(x, t);  // now x[k] = piece t of row i0 + k
-    uint4 gx[4];
-#pragma unroll
-    for (uint32_t k = 0; k < 4; ++k) gx[k] = g_next[k];
-    if (cb + 1 < 4) load_gate(cb + 1, g_next);  // the next block's pieces load meanwhile
-    const float4 ga = __ldg(reinterpret_cast<const float4*>(p.gamma + h * D + cb * 32 + 8 * t));
-    const float4 gb = __ldg(reinterpret_cast<const float4*>(p.gamma + h * D + cb * 32 + 8 * t) + 1);
-    const float gm[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+    const float4 g0 = __ldg(reinterpret_cast<const float4*>(p.gamma + h * D + cb * 32 + 8 * t));
+    const float4 g1 = __ldg(reinterpret_cast<const float4*>(p.gamma + h * D + cb * 32 + 8 * t) + 1);
+    const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
     for (uint32_t k = 0; k < 4; ++k) {
       if (r0 + static_cast<int32_t>(k) < ui.len) {
-        const uint32_t gw[4] = {gx[k].x, gx[k].y, gx[k].z, gx[k].w};
+        const uint32_t gw[4] = {g[k].x, g[k].y, g[k].z, g[k].w};
         const uint32_t ow[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
         uint32_t yw[4];
 #pragma unroll
@@ -345,6 +346,9 @@ __device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint
   }
 }
 
+// kGated: the output epilogue applies the fused norm + gate (p.gate != null).  Two instances, so
+// that the plain kernel's register allocation carries none of the gated epilogue's pressure.
+template <bool kGated>
 __global__ void __launch_bounds__(kThreads, 1)
     chunked_prefill_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -380,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&p.tm_q);
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
-    if (p.gate != nullptr) tma_prefetch_desc(&p.tm_gate);
+    if (kGated) tma_prefetch_desc(&p.tm_gate);
   }
   if (warp == 2) {
     tmem_alloc(&ctrl->tmem_base, 512);
@@ -504,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(st + kOffQ + kHalfBytes, &p.tm_q, &ctrl->full[s], 64, h, n0, b,
                         pol_first);
           }
-          if (!local_state_pass && p.gate != nullptr) {
+          if (kGated && !local_state_pass) {
             // the epilogue reads this chunk's gate rows about one chunk period from now
             tma_prefetch_l2_4d(&p.tm_gate, 0, h, n0, b, pol_normal);
             tma_prefetch_l2_4d(&p.tm_gate, 64, h, n0, b, pol_normal);
@@ -997,13 +1001,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t h = ui.bh % p.H;
       bool good = true;
       for (int32_t c = 0; c < ui.nc; ++c) {
-        ok = mbar_wait_bounded(&ctrl->o_full, n_o & 1, abort_flag, T);
-        if (!group_all(ok, kBarO, 128)) {
-          good = false;
-          break;
-        }
-        ++n_o;
-        tc_fence_after();
         // Stores go out in 4-lane groups: after a 4 x 4 exchange of 16-byte pieces among lanes
         // 4a..4a+3 (rows i0..i0+3 of the chunk), store k writes 64 contiguous bytes of row i0 + k,
         // so every 32-byte sector is written whole by one instruction.
@@ -1012,10 +1009,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t n0 = static_cast<int64_t>(ui.tok0) + static_cast<int64_t>(ui.c0) * C + r0;
         __nv_bfloat16* out_h = p.out + (b * p.N * p.H + h) * D;
         const int64_t row_stride = p.H * D;
-        if (p.gate != nullptr) {
-          gated_epilogue(p, ctrl, trow, f, ui, h, b, t, r0, n0, row_stride);
+        if (kGated) {
+          // the first column block's gate pieces load while O is being computed (the producer
+          // has already brought the chunk's gate tile into L2)
+          const __nv_bfloat16* gate_h = p.gate + (b * p.N * p.H + h) * D;
+          uint4 ga[4];
+          load_gate_pieces(gate_h, ui.len, r0, n0, row_stride, t, 0, ga);
+          ok = mbar_wait_bounded(&ctrl->o_full, n_o & 1, abort_flag, T);
+          if (!group_all(ok, kBarO, 128)) {
+            good = false;
+            break;
+          }
+          ++n_o;
+          tc_fence_after();
+          gated_epilogue(p, ctrl, trow, f, ui, h, gate_h, out_h, t, r0, n0, row_stride, ga);
           continue;
         }
+        ok = mbar_wait_bounded(&ctrl->o_full, n_o & 1, abort_flag, T);
+        if (!group_all(ok, kBarO, 128)) {
+          good = false;
+          break;
+        }
+        ++n_o;
+        tc_fence_after();
 #pragma unroll 1
         for (uint32_t cb = 0; cb < 4; ++cb) {  // 32-column blocks
           uint32_t ra[32], re[32];
@@ -1155,8 +1171,13 @@ cudaError_t launch_common(const PrefillArgs& a, Params& prm, uint8_t* ws,
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    e = cudaFuncSetAttribute(chunked_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(chunked_prefill_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemAlloc));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(chunked_prefill_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kSmemAlloc));
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -1192,7 +1213,10 @@ cudaError_t launch_common(const PrefillArgs& a, Params& prm, uint8_t* ws,
   prm.withhold_segment = a.withhold_segment;
   prm.prefetch_depth = prefetch_depth();
   const int64_t grid = std::min<int64_t>(units, num_sms);
-  chunked_prefill_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, stream>>>(prm);
+  if (prm.gate != nullptr)
+    chunked_prefill_kernel<true><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, stream>>>(prm);
+  else
+    chunked_prefill_kernel<false><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, stream>>>(prm);
   return cudaGetLastError();
 }
 
