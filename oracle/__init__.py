@@ -183,3 +183,38 @@ def gated_rmsnorm(o, gate, gamma, eps: float):
         raise ValueError("gate must match o, gamma must be [H, d]")
     ms = np.mean(o * o, axis=-1, keepdims=True)
     return gam * (o / np.sqrt(ms + float(eps))) * (1.0 / (1.0 + np.exp(-g)))
+
+
+def qk_norm_rope(x, gamma, positions, rotary_dim: int, theta: float, eps: float):
+    """The layer's step before the kernel, in fp64 ("Ling and Ring 2.6 Technical Report", §2.1
+    Fig. 2: QKV Projection -> QK Norm -> RoPE -> Linear Attention Kernel; §2.1.1: RMSNorm with
+    eps = 1e-6, partial RoPE over 64 of the 128 head dims with theta = 6,000,000; §4.3: split + QK
+    norm + RoPE run as one fused operator).  Per token t and head h:
+
+        y = gamma * x / sqrt(mean(x^2) + eps)                        (RMSNorm over d)
+        for i < r/2, w_i = theta^(-2i/r), a = positions[t] * w_i:   (rotate-half pairs)
+            (y_i, y_{i+r/2}) <- (y_i cos a - y_{i+r/2} sin a, y_{i+r/2} cos a + y_i sin a)
+
+    dims >= r pass through normalised only.  x: [T, H, d] (uint16 bf16 bits or float32);
+    gamma: float32 [d] (shared by the heads); positions: int [T]; returns fp64 [T, H, d].
+    """
+    x = _upcast(x)
+    T, H, d = x.shape
+    r = int(rotary_dim)
+    if r % 2 or r > d or r <= 0:
+        raise ValueError("rotary_dim must be even and in (0, d]")
+    gam = np.asarray(gamma, dtype=np.float32).astype(np.float64)
+    pos = np.asarray(positions, dtype=np.int64).astype(np.float64)
+    if gam.shape != (d,) or pos.shape != (T,):
+        raise ValueError("gamma must be [d] and positions [T]")
+    y = gam * x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + float(eps))
+    half = r // 2
+    w = float(theta) ** (-2.0 * np.arange(half, dtype=np.float64) / r)
+    ang = pos[:, None] * w[None, :]                      # [T, r/2]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    a = y[..., :half].copy()
+    b = y[..., half:r].copy()
+    y[..., :half] = a * c - b * s
+    y[..., half:r] = b * c + a * s
+    return y

@@ -282,3 +282,46 @@ def test_gated_rmsnorm_reads_bf16_bits_exactly():
     y = oracle.gated_rmsnorm(o, g, np.ones((1, 4), np.float32), 0.0)
     sig = 1.0 / (1.0 + np.exp(-np.array([1.0, -2.0, 0.0, 0.5])))
     assert np.array_equal(y[0, 0], sig)
+
+
+# ---------------------------------------------------------------------------------------------
+# qk_norm_rope: QK RMSNorm + partial rotary embedding before the kernel
+# ---------------------------------------------------------------------------------------------
+def test_qk_norm_rope_hand_case():
+    # d = 4, r = 2, theta irrelevant for i = 0 (w_0 = 1): x = [1, 0, 1, 1] has mean square 3/4;
+    # at position 1 the pair (y_0, y_1) turns by 1 radian, dims 2, 3 are only normalised
+    x = np.array([[[1.0, 0.0, 1.0, 1.0]]], dtype=np.float32)
+    y = oracle.qk_norm_rope(x, np.ones(4, np.float32), [1], 2, 10000.0, 0.0)
+    s = 1.0 / np.sqrt(0.75)
+    want = np.array([s * np.cos(1.0), s * np.sin(1.0), s, s])
+    assert np.allclose(y[0, 0], want, rtol=1e-15, atol=1e-15)
+    # the second frequency of r = 4: w_1 = theta^(-1/2); pair (y_1, y_3) turns by pos * w_1
+    x = np.array([[[0.0, 1.0, 0.0, 0.0]]], dtype=np.float32)
+    y = oracle.qk_norm_rope(x, np.ones(4, np.float32), [3], 4, 100.0, 0.0)
+    a = 3.0 / 10.0
+    assert np.allclose(y[0, 0], [0.0, 2.0 * np.cos(a), 0.0, 2.0 * np.sin(a)], atol=1e-15)
+
+
+def test_qk_norm_rope_invariants():
+    rng = np.random.default_rng(9)
+    T, H, d, r = 6, 3, 16, 8
+    x = rng.standard_normal((T, H, d)).astype(np.float32)
+    gamma = rng.standard_normal(d).astype(np.float32)
+    pos = rng.integers(0, 100000, T)
+    y = oracle.qk_norm_rope(x, gamma, pos, r, 6.0e6, 1e-6)
+    y0 = oracle.qk_norm_rope(x, gamma, np.zeros(T, np.int64), r, 6.0e6, 1e-6)
+    # position 0 is the plain RMSNorm
+    xd = x.astype(np.float64)
+    plain = gamma.astype(np.float64) * xd / np.sqrt(np.mean(xd * xd, -1, keepdims=True) + 1e-6)
+    assert np.allclose(y0, plain, rtol=1e-14, atol=1e-15)
+    # rotation keeps each pair's length; dims >= r are untouched by it
+    h = r // 2
+    assert np.allclose(y[..., :h] ** 2 + y[..., h:r] ** 2, plain[..., :h] ** 2 + plain[..., h:r] ** 2,
+                       rtol=1e-12)
+    assert np.array_equal(y[..., r:], plain[..., r:])
+    # relative positions: <rope(q, m), rope(k, n)> depends on m - n only
+    q = oracle.qk_norm_rope(x[:1], gamma, [1000], r, 6.0e6, 1e-6)
+    k = oracle.qk_norm_rope(x[1:2], gamma, [400], r, 6.0e6, 1e-6)
+    q2 = oracle.qk_norm_rope(x[:1], gamma, [1000 + 77777], r, 6.0e6, 1e-6)
+    k2 = oracle.qk_norm_rope(x[1:2], gamma, [400 + 77777], r, 6.0e6, 1e-6)
+    assert np.allclose(np.sum(q * k, -1), np.sum(q2 * k2, -1), rtol=1e-9)
