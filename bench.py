@@ -264,6 +264,20 @@ def run_ours(args):
         ws_bytes = la.la_prefill_varlen_workspace_bytes(desc)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
 
+    qk = None
+    if args.qk_rope:
+        # QK RMSNorm + partial RoPE (rotary dim 64, theta 6e6) turns raw projections into the
+        # prefill's q and k every step
+        gq_ = torch.Generator(device=dev)
+        gq_.manual_seed(78 + 1000 * rank)
+        q_raw = torch.randn(q.shape, generator=gq_, device=dev).to(w.dtype)
+        k_raw = torch.randn(q.shape, generator=gq_, device=dev).to(w.dtype)
+        gam_q = (1.0 + 0.1 * torch.randn(d, generator=gq_, device=dev)).float()
+        gam_k = (1.0 + 0.1 * torch.randn(d, generator=gq_, device=dev)).float()
+        positions = (torch.arange(B * N, device=dev) % N).to(torch.int64)
+        qk = la.la_qk_norm_rope_desc(B * N, H, d, H * d, H * d, 64, 6.0e6, 1e-6, 0)
+        extra_in += [q_raw, k_raw]
+
     Bd, Hd, dd = DECODE["B"], DECODE["H"], DECODE["d"]
     dstate = torch.randn(Bd, Hd, dd, dd, dtype=torch.float32, device=dev) * 0.05
     gdec = synth.decode_token_generator(4 + 1000 * rank, dev)
@@ -288,6 +302,13 @@ def run_ours(args):
         if rc != la.LA_OK:
             raise la.LaError(rc, "la_prefill")
 
+    def qk_call():
+        rc = la.la_qk_norm_rope(qk, q_raw.data_ptr(), k_raw.data_ptr(), gam_q.data_ptr(),
+                                gam_k.data_ptr(), positions.data_ptr(), q.data_ptr(),
+                                k.data_ptr(), sp)
+        if rc != la.LA_OK:
+            raise la.LaError(rc, "la_qk_norm_rope")
+
     def decode_call():
         rc = la.la_decode_step(Bd, Hd, dd, la.LA_BF16, dq.data_ptr(), dk.data_ptr(),
                                dv.data_ptr(), dsl.data_ptr(), dstate.data_ptr(),
@@ -296,6 +317,8 @@ def run_ours(args):
             raise la.LaError(rc, "la_decode_step")
 
     for _ in range(args.warmup):
+        if qk is not None:
+            qk_call()
         prefill_call()
         decode_call()
     torch.cuda.synchronize(dev)
@@ -305,7 +328,8 @@ def run_ours(args):
 
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
     t_all0 = torch.cuda.Event(enable_timing=True)
     t_all1 = torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -313,6 +337,9 @@ def run_ours(args):
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
         t_all0.record(stream)
         for i in range(K):
+            ev[i][3].record(stream)
+            if qk is not None:
+                qk_call()
             ev[i][0].record(stream)
             prefill_call()
             ev[i][1].record(stream)
@@ -322,8 +349,9 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
     barrier(world)
     total_ms = t_all0.elapsed_time(t_all1)
-    pre_ms = sum(a.elapsed_time(b) for a, b, _ in ev) / K
-    dec_ms = sum(b.elapsed_time(c) for _, b, c in ev) / K
+    pre_ms = sum(a.elapsed_time(b) for a, b, _, _ in ev) / K
+    dec_ms = sum(b.elapsed_time(c) for _, b, c, _ in ev) / K
+    qk_ms = sum(z.elapsed_time(a) for a, _, _, z in ev) / K
     st_rc = la.la_workspace_status(ws.data_ptr(), sp)
     if st_rc != la.LA_OK:
         raise la.LaError(st_rc, "device status after the timed steps")
@@ -331,6 +359,7 @@ def run_ours(args):
     total_ms = max_over_ranks(total_ms, world)
     pre_ms_max = max_over_ranks(pre_ms, world)
     dec_ms_max = max_over_ranks(dec_ms, world)
+    qk_ms_max = max_over_ranks(qk_ms, world)
 
     # ---- e2e: host buffers through the C ABI, copies inside the timed region ----
     e2e = None
@@ -368,6 +397,8 @@ def run_ours(args):
             dv.copy_(hdv, non_blocking=True)
             for x, hx in zip(extra_in, hextra):
                 x.copy_(hx, non_blocking=True)
+            if qk is not None:
+                qk_call()
             prefill_call()
             decode_call()
             hout.copy_(out, non_blocking=True)
@@ -429,12 +460,16 @@ def run_ours(args):
                                      and not args.gate else None),
                          "algorithmic_bytes": pre_bytes,
                          "kernel": "chunked_prefill_kernel", "peak_kind": peak_kind},
+            "qk_norm_rope": None if qk is None else {
+                "ms": qk_ms_max,
+                # read q, k (raw) and write q_hat, k_hat: 4 * d * 2 bytes per token-head
+                "hbm_gbs": 8 * B * N * H * d / (qk_ms_max * 1e-3) / 1e9},
             "cpu_baseline": cpu,
             "clocks": clk.summary(),
             "e2e": e2e,
             # per step: the prefill kernel (after the planning kernel for packed input) and the
             # decode kernel
-            "gpu_launches": (3 if packed else 2) * K,
+            "gpu_launches": ((3 if packed else 2) + (1 if qk is not None else 0)) * K,
         }
         print(json.dumps(line), flush=True)
     dist_teardown(world)
@@ -491,6 +526,8 @@ def main():
     ap.add_argument("--workload", choices=["prefill_32k", "prefill_4k", "prefill_256k",
                                            "varlen_64k"],
                     default="prefill_32k")
+    ap.add_argument("--qk-rope", action="store_true",
+                    help="run the QK RMSNorm + partial RoPE operator before each prefill")
     ap.add_argument("--gate", action="store_true",
                     help="fuse the grouped RMSNorm + sigmoid gate into the prefill's output")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer e2e leg")

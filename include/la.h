@@ -239,6 +239,42 @@ la_status la_prefill_varlen(const la_varlen_desc* desc, const void* q, const voi
                             float* state_out, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/* Shape and options of la_qk_norm_rope. */
+typedef struct {
+  int64_t T;          /* tokens (>= 0) */
+  int64_t H;          /* heads (>= 1) */
+  int64_t d;          /* head dimension, 64 or 128 */
+  int64_t q_stride;   /* elements from token t to token t+1 of q, >= H*d, a multiple of 8 */
+  int64_t k_stride;   /* the same for k (so q and k may be views into one fused projection) */
+  int32_t rotary_dim; /* rotated dims r: a multiple of 16 in [16, d] (the report: 64) */
+  float theta;        /* rotary base, > 0 (the report: 6,000,000) */
+  float eps;          /* RMSNorm epsilon, >= 0 (the report: 1e-6) */
+  int32_t pad;
+} la_qk_norm_rope_desc;
+
+/*
+ * la_qk_norm_rope — the fused operator before the kernel: QK RMSNorm and partial rotary
+ * embedding of q and k ("Ling and Ring 2.6 Technical Report", §2.1 Fig. 2: QK Norm -> RoPE ->
+ * Linear Attention Kernel; §2.1.1: RMSNorm eps 1e-6, rotary dim 64 of 128, theta 6e6; §4.3: split +
+ * QK norm + RoPE fused into one inference operator).  For every token t, head h and x in {q, k}:
+ *     y = gamma_x * x / sqrt(mean(x^2) + eps)                      (norm over the d channels)
+ *     (y_i, y_{i+r/2}) <- (y_i cos a - y_{i+r/2} sin a, y_{i+r/2} cos a + y_i sin a)
+ *     with a = positions[t] * theta^(-2i/r) for i < r/2; dims >= r keep the normalised value.
+ * The angle is formed and reduced modulo 2 pi in double precision before sin/cos.
+ *
+ *   desc        shape and options (host pointer, read during the call only)
+ *   q, k        bf16 device, token t of head h at q + t*q_stride + h*d (16-byte aligned)
+ *   gamma_q/_k  fp32 [d] device: the two norms' weights (shared by the heads)
+ *   positions   int64 [T] device: each token's position in its sequence (for prefill of a
+ *               cached prefix continuation, the prefix length is added by the caller)
+ *   q_out/k_out bf16 [T, H, d] device, written; each may be its input itself (in place, when that
+ *               input is contiguous), any other overlap with an input is LA_ERR_ALIAS
+ *   stream      cudaStream_t as void*
+ */
+la_status la_qk_norm_rope(const la_qk_norm_rope_desc* desc, const void* q, const void* k,
+                          const float* gamma_q, const float* gamma_k, const int64_t* positions,
+                          void* q_out, void* k_out, void* stream);
+
 /* Synchronises `stream`, then returns the device status word of a workspace that la_prefill
  * used: LA_OK, or LA_ERR_TIMEOUT if a bounded device wait gave up during the last call. */
 la_status la_workspace_status(const void* workspace, void* stream);

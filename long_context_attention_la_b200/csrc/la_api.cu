@@ -3,6 +3,7 @@
 // pointer owned by the caller.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -234,6 +235,59 @@ la_status la_prefill_varlen(const la_varlen_desc* desc, const void* q, const voi
       la::launch_prefill_varlen(a, layout, ws, desc->segments, tensor, s, sms);
   if (owned) cudaFreeAsync(ws, s);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status la_qk_norm_rope(const la_qk_norm_rope_desc* desc, const void* q, const void* k,
+                          const float* gamma_q, const float* gamma_k, const int64_t* positions,
+                          void* q_out, void* k_out, void* stream) {
+  if (desc == nullptr) return LA_ERR_NULL;
+  const la_qk_norm_rope_desc& d = *desc;
+  if (d.T < 0 || d.H < 1 || (d.d != 64 && d.d != 128)) return LA_ERR_SHAPE;
+  if (d.rotary_dim < 16 || d.rotary_dim > d.d || d.rotary_dim % 16 != 0) return LA_ERR_SHAPE;
+  if (!(d.theta > 0.f) || d.theta > 3.0e38f || !(d.eps >= 0.f) || d.eps > 3.0e38f)
+    return LA_ERR_SHAPE;
+  int64_t hd = 0, n = 0, span_q = 0, span_k = 0;
+  if (!mul_ok(d.H, d.d, &hd) || !mul_ok(d.T, hd, &n)) return LA_ERR_OVERFLOW;
+  if (d.q_stride < hd || d.k_stride < hd || d.q_stride % 8 || d.k_stride % 8) return LA_ERR_SHAPE;
+  if (!mul_ok(d.T, d.q_stride, &span_q) || !mul_ok(d.T, d.k_stride, &span_k))
+    return LA_ERR_OVERFLOW;
+  if (d.T > INT32_MAX) return LA_ERR_OVERFLOW;  // one CTA per token
+  if (!q || !k || !gamma_q || !gamma_k || !positions || !q_out || !k_out) return LA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out) ||
+      !aligned16(gamma_q) || !aligned16(gamma_k))
+    return LA_ERR_ALIGN;
+  const size_t out_bytes = static_cast<size_t>(n) * 2;
+  const size_t qb = static_cast<size_t>(span_q) * 2, kb = static_cast<size_t>(span_k) * 2;
+  if (n > 0) {
+    // in place is allowed only onto a contiguous input itself
+    const bool q_inplace = q_out == q && d.q_stride == hd;
+    const bool k_inplace = k_out == k && d.k_stride == hd;
+    if ((!q_inplace && overlaps(q_out, out_bytes, q, qb)) || overlaps(q_out, out_bytes, k, kb) ||
+        (!k_inplace && overlaps(k_out, out_bytes, k, kb)) || overlaps(k_out, out_bytes, q, qb) ||
+        overlaps(q_out, out_bytes, k_out, out_bytes))
+      return LA_ERR_ALIAS;
+  }
+  la::QkNormRopeArgs a{};
+  a.T = d.T;
+  a.H = d.H;
+  a.d = d.d;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.q_stride = d.q_stride;
+  a.k_stride = d.k_stride;
+  a.gamma_q = gamma_q;
+  a.gamma_k = gamma_k;
+  a.positions = positions;
+  a.q_out = static_cast<__nv_bfloat16*>(q_out);
+  a.k_out = static_cast<__nv_bfloat16*>(k_out);
+  a.rotary_dim = d.rotary_dim;
+  a.eps = d.eps;
+  const double log_theta = std::log(static_cast<double>(d.theta));
+  for (int i = 0; i < d.rotary_dim / 2; ++i)
+    a.inv_freq[i] = std::exp(-2.0 * i / d.rotary_dim * log_theta);
+  return la::launch_qk_norm_rope(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LA_OK
+             : LA_ERR_CUDA;
 }
 
 la_status la_decode_step(int64_t B, int64_t H, int64_t d, int32_t dtype, const void* q,

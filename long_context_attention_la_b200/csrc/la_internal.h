@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace la {
@@ -54,6 +55,23 @@ cudaError_t launch_recurrent_prefill(const PrefillArgs& a, cudaStream_t stream);
 
 // Fused decode step; one CTA per (b, h).
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// QK RMSNorm + partial rotate-half RoPE over bf16 q and k rows (la_qknorm.cu).
+struct QkNormRopeArgs {
+  int64_t T, H, d;                  // tokens, heads, head dim (64 or 128)
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  int64_t q_stride, k_stride;       // elements between consecutive tokens
+  const float* gamma_q;             // [d]
+  const float* gamma_k;             // [d]
+  const int64_t* positions;         // [T]
+  __nv_bfloat16* q_out;             // [T, H, d]
+  __nv_bfloat16* k_out;             // [T, H, d]
+  int32_t rotary_dim;               // multiple of 16, <= d
+  float eps;
+  double inv_freq[64];              // theta^(-2i / rotary_dim), i < rotary_dim / 2
+};
+cudaError_t launch_qk_norm_rope(const QkNormRopeArgs& a, cudaStream_t stream);
 
 // ---------------------------------------------------------------------------------------------
 // Chunked tensor-core prefill (bf16, d = 128, chunk C = 128).

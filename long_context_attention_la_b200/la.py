@@ -55,6 +55,13 @@ class la_gate_norm(ctypes.Structure):  # noqa: N801 - mirrors the C type name
     _fields_ = [("gate", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("eps", ctypes.c_float)]
 
 
+class la_qk_norm_rope_desc(ctypes.Structure):  # noqa: N801 - mirrors the C type name
+    _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int64), ("d", ctypes.c_int64),
+                ("q_stride", ctypes.c_int64), ("k_stride", ctypes.c_int64),
+                ("rotary_dim", ctypes.c_int32), ("theta", ctypes.c_float), ("eps", ctypes.c_float),
+                ("pad", ctypes.c_int32)]
+
+
 class LaError(RuntimeError):
     def __init__(self, status: int, what: str = ""):
         self.status = status
@@ -100,6 +107,9 @@ def library(path: str | None = None):
         lib.la_prefill_varlen.argtypes = [ctypes.POINTER(la_varlen_desc), vp, vp, vp, vp, vp, vp,
                                           ctypes.POINTER(la_gate_norm), vp, vp, vp, sz, vp]
         lib.la_prefill_varlen.restype = ctypes.c_int
+        lib.la_qk_norm_rope.argtypes = [ctypes.POINTER(la_qk_norm_rope_desc), vp, vp, vp, vp, vp,
+                                        vp, vp, vp]
+        lib.la_qk_norm_rope.restype = ctypes.c_int
         lib.la_decode_step.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp]
         lib.la_decode_step.restype = ctypes.c_int
         lib.la_workspace_status.argtypes = [vp, vp]
@@ -151,6 +161,13 @@ def la_prefill_varlen(desc: la_varlen_desc, q: int, k: int, v: int, slopes: int,
                                            None if epilogue is None else ctypes.byref(epilogue),
                                            out, state_out or None, workspace or None,
                                            workspace_bytes, stream or None))
+
+
+def la_qk_norm_rope(desc: la_qk_norm_rope_desc, q: int, k: int, gamma_q: int, gamma_k: int,
+                    positions: int, q_out: int, k_out: int, stream: int) -> int:
+    return int(library().la_qk_norm_rope(ctypes.byref(desc), q or None, k or None,
+                                         gamma_q or None, gamma_k or None, positions or None,
+                                         q_out or None, k_out or None, stream or None))
 
 
 def la_decode_step(B: int, H: int, d: int, dtype: int, q: int, k: int, v: int, slopes: int,
@@ -313,3 +330,36 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch
     if st != LA_OK:
         raise LaError(st, "la_decode_step")
     return out
+
+
+def qk_norm_rope(q: torch.Tensor, k: torch.Tensor, gamma_q: torch.Tensor, gamma_k: torch.Tensor,
+                 positions: torch.Tensor, *, rotary_dim: int = 64, theta: float = 6.0e6,
+                 eps: float = 1e-6, q_out: torch.Tensor | None = None,
+                 k_out: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None):
+    """q_hat, k_hat = qk_norm_rope(q, k, gamma_q, gamma_k, positions): q, k [T, H, d] bf16 CUDA
+    views whose head and channel dims are contiguous (the token stride may be larger, e.g. views
+    into one fused projection output); gamma_* fp32 [d]; positions int64 [T].  Returns new
+    contiguous [T, H, d] tensors (or writes q_out / k_out)."""
+    if q.dim() != 3 or q.shape != k.shape or q.dtype != torch.bfloat16 or k.dtype != q.dtype:
+        raise ValueError("q, k must be bf16 [T, H, d] of one shape")
+    T, H, d = q.shape
+    for name, t in (("q", q), ("k", k)):
+        if not t.is_cuda or t.stride(2) != 1 or t.stride(1) != d:
+            raise ValueError(f"{name} must be a CUDA view with contiguous [H, d] rows")
+    if positions.dtype != torch.int64 or tuple(positions.shape) != (T,):
+        raise ValueError("positions must be int64 [T]")
+    for name, g in (("gamma_q", gamma_q), ("gamma_k", gamma_k)):
+        if g.dtype != torch.float32 or tuple(g.shape) != (d,):
+            raise ValueError(f"{name} must be float32 [d]")
+    if q_out is None:
+        q_out = torch.empty((T, H, d), dtype=q.dtype, device=q.device)
+    if k_out is None:
+        k_out = torch.empty((T, H, d), dtype=q.dtype, device=q.device)
+    desc = la_qk_norm_rope_desc(T, H, d, q.stride(0), k.stride(0), rotary_dim, theta, eps, 0)
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    st = la_qk_norm_rope(desc, q.data_ptr(), k.data_ptr(), _cuda_ptr(gamma_q, "gamma_q"),
+                         _cuda_ptr(gamma_k, "gamma_k"), _cuda_ptr(positions, "positions"),
+                         _cuda_ptr(q_out, "q_out"), _cuda_ptr(k_out, "k_out"), s.cuda_stream)
+    if st != LA_OK:
+        raise LaError(st, "la_qk_norm_rope")
+    return q_out, k_out

@@ -21,6 +21,17 @@ def declared_functions():
     return sorted(set(names))
 
 
+# The argument checks below hand the library made-up device addresses and expect an error code
+# before any launch.  On a machine with a GPU a missed check would launch a kernel on them, so
+# this module runs only where no GPU is present.
+try:
+    import torch as _torch
+    _HAS_GPU = _torch.cuda.is_available()
+except Exception:  # pragma: no cover
+    _HAS_GPU = False
+pytestmark = pytest.mark.skipif(_HAS_GPU, reason="fake device addresses; CPU-only host checks")
+
+
 @pytest.fixture(scope="module")
 def lib():
     path = labuild.build()
@@ -189,3 +200,39 @@ def test_varlen_epilogue_checks(lib):
     assert call(d, la.la_gate_norm(0x800000, 0x900000, -1.0)) == la.LA_ERR_SHAPE
     # gate overlapping out
     assert call(d, la.la_gate_norm(0x800000, 0x900000, 1e-6), out=0x800000 + 64) == la.LA_ERR_ALIAS
+
+
+# ---------------------------------------------------------------------------------------------
+# la_qk_norm_rope: host-side argument checks
+# ---------------------------------------------------------------------------------------------
+def _qdesc(**kw):
+    base = dict(T=10, H=2, d=128, q_stride=256, k_stride=256, rotary_dim=64, theta=6e6, eps=1e-6,
+                pad=0)
+    base.update(kw)
+    return la.la_qk_norm_rope_desc(**base)
+
+
+_Q = (0x100000, 0x200000, 0x300000, 0x300400, 0x400000, 0x500000, 0x600000, 0)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), la.LA_ERR_SHAPE), (dict(H=0), la.LA_ERR_SHAPE), (dict(T=-1), la.LA_ERR_SHAPE),
+    (dict(rotary_dim=8), la.LA_ERR_SHAPE), (dict(rotary_dim=40), la.LA_ERR_SHAPE),
+    (dict(rotary_dim=144), la.LA_ERR_SHAPE), (dict(theta=0.0), la.LA_ERR_SHAPE),
+    (dict(theta=float("nan")), la.LA_ERR_SHAPE), (dict(eps=-1.0), la.LA_ERR_SHAPE),
+    (dict(q_stride=128), la.LA_ERR_SHAPE), (dict(k_stride=260), la.LA_ERR_SHAPE),
+])
+def test_qk_norm_rope_rejects_bad_descriptors(lib, kw, status):
+    assert la.la_qk_norm_rope(_qdesc(**kw), *_Q) == status
+
+
+def test_qk_norm_rope_null_alignment_alias(lib):
+    d = _qdesc()
+    assert la.la_qk_norm_rope(d, 0, *_Q[1:]) == la.LA_ERR_NULL
+    assert la.la_qk_norm_rope(d, *_Q[:4], 0, *_Q[5:]) == la.LA_ERR_NULL
+    assert la.la_qk_norm_rope(d, 0x100008, *_Q[1:]) == la.LA_ERR_ALIGN
+    assert la.la_qk_norm_rope(d, *_Q[:2], 0x300004, *_Q[3:]) == la.LA_ERR_ALIGN
+    # q_out overlapping k; k_out onto a strided k (not in place)
+    assert la.la_qk_norm_rope(d, *_Q[:5], 0x200000 + 64, *_Q[6:]) == la.LA_ERR_ALIAS
+    ds = _qdesc(k_stride=512)
+    assert la.la_qk_norm_rope(ds, *_Q[:6], 0x200000, 0) == la.LA_ERR_ALIAS
