@@ -13,10 +13,10 @@
 // square is a shuffle reduction over the row's threads and each rotary pair's partner value comes
 // from the thread r/16 positions away.  The angle pos * w_i is formed and reduced modulo 2 pi in
 // double precision (positions reach 2^18 and more, where a float angle would be off by ~0.03 rad),
-// then sin and cos are taken in float, once per token and frequency.  Each thread issues the loads
-// of 8 row sweeps before using any of them, so enough bytes are in flight to stream.
+// then sin and cos are taken in float, once per token and frequency.
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 
@@ -34,25 +34,26 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return l | (u << 16);
 }
 
-// One CTA per token: the token's r/2 rotation angles are computed once (double-precision angle and
-// reduction, float sin/cos) into shared memory, then the CTA's threads sweep the token's 2H rows
-// (q heads, then k heads), ROWS rows at a time.
+// Each CTA takes two tokens and issues the loads of both tokens' 2H rows before using any (enough
+// bytes in flight per SM to stream), computes each token's r/2 rotation angles once
+// (double-precision angle and reduction, float sin/cos) into shared memory, then sweeps the rows
+// ROWS at a time.
 template <int D>
 __global__ void __launch_bounds__(kQkThreads) qk_norm_rope_kernel(const QkNormRopeArgs a) {
   constexpr int TPR = D / 8;                   // threads per row
   constexpr int ROWS = kQkThreads / TPR;       // rows per sweep step
-  __shared__ float cs_sh[64], sn_sh[64];
-  const int64_t t = blockIdx.x;
+  constexpr int kBatch = 8;                    // sweeps per token held in registers
+  __shared__ float cs_sh[2][64], sn_sh[2][64];
   const int lt = threadIdx.x % TPR;            // position of this thread in its row
-  const int64_t rows = 2 * a.H;
-  constexpr int kBatch = 8;  // sweeps whose loads are issued together, before any is used
-  uint4 raw[kBatch];
-  auto load_batch = [&](int64_t rb) {
+  const int64_t rows = 2 * a.H;                // q heads, then k heads
+  const int half = a.rotary_dim / 2;
+
+  auto load_rows = [&](int64_t t, int64_t rb, uint4 (&raw)[kBatch]) {
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
       const int64_t row = rb + j * ROWS + threadIdx.x / TPR;
       raw[j] = make_uint4(0u, 0u, 0u, 0u);
-      if (row < rows) {
+      if (t < a.T && row < rows) {
         const bool is_k = row >= a.H;
         const int64_t h = is_k ? row - a.H : row;
         const __nv_bfloat16* src =
@@ -61,33 +62,28 @@ __global__ void __launch_bounds__(kQkThreads) qk_norm_rope_kernel(const QkNormRo
       }
     }
   };
-  load_batch(0);  // in flight while the angles are computed
-  const int half = a.rotary_dim / 2;
-  if (threadIdx.x < half) {
-    constexpr double kTwoPi = 6.283185307179586476925286766559;
-    constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
-    double ang = static_cast<double>(a.positions[t]) * a.inv_freq[threadIdx.x];
-    ang -= kTwoPi * rint(ang * kInvTwoPi);
-    float sn, cs;
-    sincosf(static_cast<float>(ang), &sn, &cs);
-    cs_sh[threadIdx.x] = cs;
-    sn_sh[threadIdx.x] = sn;
-  }
-  __syncthreads();
+  auto angles = [&](int64_t t, int buf) {
+    if (t < a.T && threadIdx.x < half) {
+      constexpr double kTwoPi = 6.283185307179586476925286766559;
+      constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+      double ang = static_cast<double>(a.positions[t]) * a.inv_freq[threadIdx.x];
+      ang -= kTwoPi * rint(ang * kInvTwoPi);
+      float sn, cs;
+      sincosf(static_cast<float>(ang), &sn, &cs);
+      cs_sh[buf][threadIdx.x] = cs;
+      sn_sh[buf][threadIdx.x] = sn;
+    }
+  };
+
   const int half_threads = a.rotary_dim / 16;  // threads per half of the rotary dims
   const bool rotary = lt < 2 * half_threads;
   const bool first = lt < half_threads;
   const int lane = threadIdx.x & 31;
   const int partner_lane = rotary ? (first ? lane + half_threads : lane - half_threads) : lane;
   const int i0 = (first ? lt : lt - half_threads) * 8;  // frequency index of element 0
-  float gq[8], gk[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    gq[e] = a.gamma_q[lt * 8 + e];
-    gk[e] = a.gamma_k[lt * 8 + e];
-  }
-  for (int64_t rb = 0; rb < rows; rb += ROWS * kBatch) {  // uniform trip counts across the CTA
-    if (rb > 0) load_batch(rb);
+
+  // normalise + rotate the rows held in raw (sweeps rb .. rb + kBatch - 1 of token t)
+  auto finish = [&](int64_t t, int64_t rb, const uint4 (&raw)[kBatch], int buf) {
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
       const int64_t row = rb + j * ROWS + threadIdx.x / TPR;
@@ -108,9 +104,10 @@ __global__ void __launch_bounds__(kQkThreads) qk_norm_rope_kernel(const QkNormRo
 #pragma unroll
       for (int o = TPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       const float rinv = rsqrtf(fmaf(ss, 1.f / D, a.eps));
+      const float* gam = (is_k ? a.gamma_k : a.gamma_q) + lt * 8;
       float y[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = (is_k ? gk[e] : gq[e]) * (x[e] * rinv);
+      for (int e = 0; e < 8; ++e) y[e] = __ldg(gam + e) * (x[e] * rinv);
       // rotate-half over the first r dims: the partner of element j is j +- r/2, held by the
       // thread r/16 positions away in the same row
       float pv[8];
@@ -119,7 +116,7 @@ __global__ void __launch_bounds__(kQkThreads) qk_norm_rope_kernel(const QkNormRo
       if (rotary) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float cs = cs_sh[i0 + e], sn = sn_sh[i0 + e];
+          const float cs = cs_sh[buf][i0 + e], sn = sn_sh[buf][i0 + e];
           y[e] = first ? fmaf(y[e], cs, -pv[e] * sn) : fmaf(y[e], cs, pv[e] * sn);
         }
       }
@@ -133,6 +130,27 @@ __global__ void __launch_bounds__(kQkThreads) qk_norm_rope_kernel(const QkNormRo
         __stcs(reinterpret_cast<uint4*>(dst), w);
       }
     }
+  };
+
+  // two tokens per CTA, all of their row loads issued before any is used
+  const int64_t t0 = 2 * static_cast<int64_t>(blockIdx.x), t1 = t0 + 1;
+  uint4 ra[kBatch], rb_[kBatch];
+  load_rows(t0, 0, ra);
+  load_rows(t1, 0, rb_);
+  angles(t0, 0);
+  angles(t1, 1);
+  __syncthreads();
+  finish(t0, 0, ra, 0);
+  for (int64_t rb = ROWS * kBatch; rb < rows; rb += ROWS * kBatch) {  // H > 64: more sweeps
+    load_rows(t0, rb, ra);
+    finish(t0, rb, ra, 0);
+  }
+  if (t1 < a.T) {  // uniform across the CTA
+    finish(t1, 0, rb_, 1);
+    for (int64_t rb = ROWS * kBatch; rb < rows; rb += ROWS * kBatch) {
+      load_rows(t1, rb, rb_);
+      finish(t1, rb, rb_, 1);
+    }
   }
 }
 
@@ -140,10 +158,11 @@ __global__ void __launch_bounds__(kQkThreads) qk_norm_rope_kernel(const QkNormRo
 
 cudaError_t launch_qk_norm_rope(const QkNormRopeArgs& a, cudaStream_t stream) {
   if (a.T == 0) return cudaSuccess;
+  const int64_t grid = (a.T + 1) / 2;  // two tokens per CTA
   if (a.d == 64)
-    qk_norm_rope_kernel<64><<<static_cast<unsigned>(a.T), kQkThreads, 0, stream>>>(a);
+    qk_norm_rope_kernel<64><<<static_cast<unsigned>(grid), kQkThreads, 0, stream>>>(a);
   else
-    qk_norm_rope_kernel<128><<<static_cast<unsigned>(a.T), kQkThreads, 0, stream>>>(a);
+    qk_norm_rope_kernel<128><<<static_cast<unsigned>(grid), kQkThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
