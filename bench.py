@@ -281,7 +281,13 @@ def run_ours(args):
     Bd, Hd, dd = DECODE["B"], DECODE["H"], DECODE["d"]
     dstate = torch.randn(Bd, Hd, dd, dd, dtype=torch.float32, device=dev) * 0.05
     gdec = synth.decode_token_generator(4 + 1000 * rank, dev)
-    dq, dk, dv = synth.draw_decode_token(gdec, Bd, Hd, dd, device=dev)
+    n_mtp = max(1, args.mtp)
+    if n_mtp == 1:
+        dq, dk, dv = synth.draw_decode_token(gdec, Bd, Hd, dd, device=dev)
+    else:
+        # n_mtp tokens per sequence in one multi-token step, [B, n, H, d]
+        toks = [synth.draw_decode_token(gdec, Bd, Hd, dd, device=dev) for _ in range(n_mtp)]
+        dq, dk, dv = (torch.stack([t[i] for t in toks], dim=1).contiguous() for i in range(3))
     dout = torch.empty_like(dq)
     dsl = synth.slopes(Hd, dev)
 
@@ -310,9 +316,14 @@ def run_ours(args):
             raise la.LaError(rc, "la_qk_norm_rope")
 
     def decode_call():
-        rc = la.la_decode_step(Bd, Hd, dd, la.LA_BF16, dq.data_ptr(), dk.data_ptr(),
-                               dv.data_ptr(), dsl.data_ptr(), dstate.data_ptr(),
-                               dout.data_ptr(), sp)
+        if n_mtp == 1:
+            rc = la.la_decode_step(Bd, Hd, dd, la.LA_BF16, dq.data_ptr(), dk.data_ptr(),
+                                   dv.data_ptr(), dsl.data_ptr(), dstate.data_ptr(),
+                                   dout.data_ptr(), sp)
+        else:
+            rc = la.la_decode_multi(Bd, Hd, dd, n_mtp, la.LA_BF16, dq.data_ptr(), dk.data_ptr(),
+                                    dv.data_ptr(), dsl.data_ptr(), dstate.data_ptr(),
+                                    dout.data_ptr(), sp)
         if rc != la.LA_OK:
             raise la.LaError(rc, "la_decode_step")
 
@@ -425,7 +436,7 @@ def run_ours(args):
         achieved = pre_bytes / (pre_ms_max * 1e-3) / 1e9
         canon = 4.0 * d * d * B * N * H  # recurrent-form flops
         executed = (4.0 * d * d + 4.0 * 128 * d) * B * N * H  # full 128 x 128 tiles
-        dec_bytes = 2 * Bd * Hd * dd * dd * 4 + 4 * Bd * Hd * dd * 2
+        dec_bytes = 2 * Bd * Hd * dd * dd * 4 + 4 * Bd * Hd * dd * 2 * n_mtp
         dec_gbs = dec_bytes / (dec_ms_max * 1e-3) / 1e9
         cpu = None
         if world == 1 and not args.no_cpu:
@@ -453,7 +464,9 @@ def run_ours(args):
                         "tflops_executed_c128": world * executed / (pre_ms_max * 1e-3) / 1e12,
                         "hbm_gbs": achieved},
             "decode": {"ms": dec_ms_max, "state_gbs": dec_gbs, "frac_of_measured": dec_gbs / hbm_peak,
-                       "frac_of_8tbs": dec_gbs / 8000.0, "tok_s": world * Bd / (dec_ms_max * 1e-3)},
+                       "frac_of_8tbs": dec_gbs / 8000.0,
+                       "tokens_per_step": n_mtp,
+                       "tok_s": world * Bd * n_mtp / (dec_ms_max * 1e-3)},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak,
                          "traffic": (measured_traffic() if args.workload == "prefill_32k"
@@ -526,6 +539,8 @@ def main():
     ap.add_argument("--workload", choices=["prefill_32k", "prefill_4k", "prefill_256k",
                                            "varlen_64k"],
                     default="prefill_32k")
+    ap.add_argument("--mtp", type=int, default=1,
+                    help="decode this many tokens per sequence per step (multi-token step)")
     ap.add_argument("--qk-rope", action="store_true",
                     help="run the QK RMSNorm + partial RoPE operator before each prefill")
     ap.add_argument("--gate", action="store_true",

@@ -128,6 +128,45 @@ la_status la_decode_step(int64_t B, int64_t H, int64_t d, int32_t dtype, const v
                          const void* k, const void* v, const float* slopes, float* state_inout,
                          void* out, void* stream);
 
+/* Optional output epilogue (la_prefill_varlen, la_decode_multi): the step the report's layer
+ * runs right after this kernel, a grouped RMSNorm of each head's output vector followed by the
+ * sigmoid gate (§2.1 Fig. 2: Linear Attention Kernel -> Grouped RMSNorm, times sigmoid(Gate
+ * Projection); §4.3 fuses "group norm + sigmoid gate" into one operator).  With it, out receives,
+ * per token t and head h,
+ *     y_j = gamma[h, j] * o_j / sqrt(mean_j(o_j^2) + eps) * sigmoid(g[t, h, j])
+ * computed from the fp32 o (each head is one norm group of d channels) and rounded once to the
+ * output dtype.  In la_prefill_varlen: tensor-core path only (bf16, d = 128). */
+typedef struct {
+  const void* gate;   /* like out, device: the gate pre-activation g = x W_gate, read only */
+  const float* gamma; /* fp32 [H, d] device: the norm's weight, read only */
+  float eps;          /* epsilon under the root, >= 0 (the report's RMSNorm uses 1e-6) */
+} la_gate_norm;
+
+/*
+ * la_decode_multi — n_tok generated tokens per sequence in one step, for speculative
+ * verification ("attention with MTP" in the report's serving path, §4.3): for every (b, h) and
+ * j = 0 .. n_tok-1 in order,
+ *     S <- lambda_h S + k_j^T v_j,   o_j = q_j S        (the la_decode_step rule per token)
+ * The state is read and written once for all n_tok tokens, so its HBM traffic per token falls
+ * as 1/n_tok.  With n_tok = 1 and no epilogue it computes exactly what la_decode_step does.
+ *
+ *   B, H, d       sequences, heads, head dim (64 or 128); n_tok >= 1 tokens per sequence
+ *   dtype         la_dtype of q, k, v, out (and of the gate)
+ *   q, k, v       [B, n_tok, H, d] device, read only
+ *   slopes        fp32[H] device
+ *   state_inout   fp32 [B, H, d, d] device, updated in place with all n_tok tokens
+ *   epilogue      NULL, or the fused grouped RMSNorm + sigmoid gate of la_gate_norm applied to
+ *                 every output row (gate [B, n_tok, H, d] of dtype, gamma fp32 [H, d])
+ *   out           [B, n_tok, H, d] device, written
+ *   stream        cudaStream_t as void*
+ * Errors as la_decode_step (LA_ERR_SHAPE also for n_tok < 1; LA_ERR_ALIAS when out or the gate
+ * overlaps another operand).
+ */
+la_status la_decode_multi(int64_t B, int64_t H, int64_t d, int64_t n_tok, int32_t dtype,
+                          const void* q, const void* k, const void* v, const float* slopes,
+                          float* state_inout, const la_gate_norm* epilogue, void* out,
+                          void* stream);
+
 /*
  * la_prefill_noalloc — la_prefill for callers that cannot allocate device memory.
  *
@@ -177,18 +216,6 @@ typedef struct {
   int32_t path;     /* la_path */
 } la_varlen_desc;
 
-/* Optional epilogue of la_prefill_varlen: the step the report's layer runs right after this
- * kernel, a grouped RMSNorm of each head's output vector followed by the sigmoid gate (§2.1
- * Fig. 2: Linear Attention Kernel -> Grouped RMSNorm, times sigmoid(Gate Projection); §4.3 fuses
- * "group norm + sigmoid gate" into one operator).  With it, out receives, per token t and head h,
- *     y_j = gamma[h, j] * o_j / sqrt(mean_j(o_j^2) + eps) * sigmoid(g[t, h, j])
- * computed from the fp32 accumulator of o (each head is one norm group of d channels), rounded
- * once to bf16.  Tensor-core path only (bf16, d = 128). */
-typedef struct {
-  const void* gate;   /* [T, H, d] device bf16: the gate pre-activation g = x W_gate, read only */
-  const float* gamma; /* fp32 [H, d] device: the norm's weight, read only */
-  float eps;          /* epsilon under the root, >= 0 (the report's RMSNorm uses 1e-6) */
-} la_gate_norm;
 
 /* Bytes of device workspace la_prefill_varlen needs (0 only for invalid arguments): an upper
  * bound over every cu_seqlens of this shape (the work-unit table holds at most

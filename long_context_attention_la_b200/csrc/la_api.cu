@@ -290,6 +290,40 @@ la_status la_qk_norm_rope(const la_qk_norm_rope_desc* desc, const void* q, const
              : LA_ERR_CUDA;
 }
 
+la_status la_decode_multi(int64_t B, int64_t H, int64_t d, int64_t n_tok, int32_t dtype,
+                          const void* q, const void* k, const void* v, const float* slopes,
+                          float* state_inout, const la_gate_norm* epilogue, void* out,
+                          void* stream) {
+  if (dtype != LA_BF16 && dtype != LA_F32) return LA_ERR_DTYPE;
+  if (B < 1 || H < 1 || n_tok < 1 || (d != 64 && d != 128)) return LA_ERR_SHAPE;
+  if (!q || !k || !v || !slopes || !state_inout || !out) return LA_ERR_NULL;
+  int64_t bh = 0, n = 0, sb = 0;
+  if (!mul_ok(B, H, &bh) || bh > INT32_MAX || !mul_ok(bh, d, &n) || !mul_ok(n, n_tok, &n) ||
+      !mul_ok(bh, d * d * 4, &sb))
+    return LA_ERR_OVERFLOW;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      !aligned16(state_inout))
+    return LA_ERR_ALIGN;
+  const size_t bytes = static_cast<size_t>(n) * (dtype == LA_BF16 ? 2 : 4);
+  if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) ||
+      overlaps(out, bytes, v, bytes) || overlaps(out, bytes, state_inout, static_cast<size_t>(sb)))
+    return LA_ERR_ALIAS;
+  la::DecodeArgs a{B, H, d, dtype, q, k, v, slopes, state_inout, out};
+  a.n_tok = n_tok;
+  if (epilogue != nullptr) {
+    if (!epilogue->gate || !epilogue->gamma) return LA_ERR_NULL;
+    if (!aligned16(epilogue->gate) || !aligned16(epilogue->gamma)) return LA_ERR_ALIGN;
+    if (!(epilogue->eps >= 0.f) || epilogue->eps > 3.0e38f) return LA_ERR_SHAPE;
+    if (overlaps(epilogue->gate, bytes, out, bytes)) return LA_ERR_ALIAS;
+    a.gate = epilogue->gate;
+    a.gamma = epilogue->gamma;
+    a.eps = epilogue->eps;
+  }
+  return la::launch_decode_multi(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LA_OK
+             : LA_ERR_CUDA;
+}
+
 la_status la_decode_step(int64_t B, int64_t H, int64_t d, int32_t dtype, const void* q,
                          const void* k, const void* v, const float* slopes, float* state_inout,
                          void* out, void* stream) {

@@ -48,7 +48,16 @@ struct DecodeArgs {
   const float* slopes;
   float* state;
   void* out;
+  // multi-token step (la_decode_multi): n_tok tokens per sequence, [B, n_tok, H, d] operands;
+  // optional fused grouped RMSNorm + sigmoid gate on each output (gate like out, gamma [H, d])
+  int64_t n_tok = 1;
+  const void* gate = nullptr;
+  const float* gamma = nullptr;
+  float eps = 0.f;
 };
+
+// n_tok tokens per sequence in one pass over the state (la_decode_multi).
+cudaError_t launch_decode_multi(const DecodeArgs& a, cudaStream_t stream);
 
 // Token-by-token CUDA-core prefill (any dtype, d in {64, 128}); one CTA per (b, h).
 cudaError_t launch_recurrent_prefill(const PrefillArgs& a, cudaStream_t stream);

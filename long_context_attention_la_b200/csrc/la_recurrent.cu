@@ -200,6 +200,113 @@ __global__ void __launch_bounds__(512) decode_kernel(const T* __restrict__ q,
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Multi-token decode step (speculative verification: the report's "attention with MTP", §4.3).
+// One CTA per (b, h), 512 threads, the state's quads held in registers as in decode_kernel, and
+// n tokens applied in order, each one: S <- lambda S + k^T v, o = q S.  The state is read and
+// written once for all n tokens.  Token j's q, k, v are staged in one of two shared buffers while
+// token j-1 is read out.  With a gate, each output row gets the fused grouped RMSNorm + sigmoid
+// gate: y = gamma * o / sqrt(mean(o^2) + eps) * sigmoid(g) (one norm group per head).
+// ---------------------------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(512) decode_multi_kernel(
+    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+    const float* __restrict__ slopes, float* __restrict__ state, T* __restrict__ out, int64_t H,
+    int64_t n_tok, const T* __restrict__ gate, const float* __restrict__ gamma, float eps) {
+  constexpr int NT = 512;
+  constexpr int Q4 = D / 4;     // column quads per row
+  constexpr int RS = NT / Q4;   // row slots
+  constexpr int RPT = D / RS;   // rows per thread
+  __shared__ float sq[2][D], sk[2][D], sv[2][D];
+  __shared__ float red[RS][D];
+  __shared__ float ss_part[D / 32];
+
+  const int tid = threadIdx.x;
+  const int c4 = tid % Q4;
+  const int r0 = tid / Q4;
+  const int64_t flat = blockIdx.x;  // b * H + h
+  const int64_t b = flat / H;
+  const int64_t h = flat % H;
+  float4* st = reinterpret_cast<float4*>(state + flat * D * D);
+
+  float4 s[RPT];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) s[r] = __ldcs(st + (r0 + r * RS) * Q4 + c4);
+  float lam_hi, lam_lo;
+  split_decay(slopes[h], lam_hi, lam_lo);
+
+  // element offset of token j's row for this head in a [B, n_tok, H, D] tensor
+  auto row_off = [&](int64_t j) { return ((b * n_tok + j) * H + h) * D; };
+  auto stage = [&](int64_t j) {
+    if (tid < 3 * D) {
+      const int which = tid / D, e = tid % D;
+      const T* src = which == 0 ? q : (which == 1 ? k : v);
+      const float x = load_as_f32<T>(src, row_off(j) + e);
+      (which == 0 ? sq : (which == 1 ? sk : sv))[j & 1][e] = x;
+    }
+  };
+  for (int64_t j = 0; j < n_tok; ++j) {
+    stage(j);
+    __syncthreads();  // token j staged; the read-out of token j-1 is done with red
+    const int buf = static_cast<int>(j & 1);
+    const float v0 = sv[buf][4 * c4 + 0], v1 = sv[buf][4 * c4 + 1];
+    const float v2 = sv[buf][4 * c4 + 2], v3 = sv[buf][4 * c4 + 3];
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+      const int i = r0 + r * RS;
+      const float ki = sk[buf][i], qi = sq[buf][i];
+      float4 x = s[r];
+      x.x = fmaf(lam_hi, x.x, fmaf(ki, v0, lam_lo * x.x));
+      x.y = fmaf(lam_hi, x.y, fmaf(ki, v1, lam_lo * x.y));
+      x.z = fmaf(lam_hi, x.z, fmaf(ki, v2, lam_lo * x.z));
+      x.w = fmaf(lam_hi, x.w, fmaf(ki, v3, lam_lo * x.w));
+      a0 = fmaf(qi, x.x, a0);
+      a1 = fmaf(qi, x.y, a1);
+      a2 = fmaf(qi, x.z, a2);
+      a3 = fmaf(qi, x.w, a3);
+      s[r] = x;
+    }
+    red[r0][4 * c4 + 0] = a0;
+    red[r0][4 * c4 + 1] = a1;
+    red[r0][4 * c4 + 2] = a2;
+    red[r0][4 * c4 + 3] = a3;
+    __syncthreads();
+    if (tid < D) {
+      float o = 0.f;
+#pragma unroll
+      for (int rr = 0; rr < RS; ++rr) o += red[rr][tid];
+      if (gate != nullptr) {
+        float ss = o * o;
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+        if ((tid & 31) == 0) ss_part[tid >> 5] = ss;
+        asm volatile("bar.sync 1, %0;" ::"r"(D) : "memory");  // the D read-out threads only
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < D / 32; ++w) tot += ss_part[w];
+        const float g = load_as_f32<T>(gate, row_off(j) + tid);
+        const float sig = 1.f / (1.f + expf(-g));
+        o = gamma[h * D + tid] * (o * rsqrtf(tot * (1.f / D) + eps)) * sig;
+        asm volatile("bar.sync 1, %0;" ::"r"(D) : "memory");  // ss_part reused by token j+1
+      }
+      store_from_f32<T>(out, row_off(j) + tid, o);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) __stcs(st + (r0 + r * RS) * Q4 + c4, s[r]);
+}
+
+template <typename T, int D>
+cudaError_t launch_decode_multi_typed(const DecodeArgs& a, cudaStream_t stream) {
+  const int64_t grid = a.B * a.H;
+  decode_multi_kernel<T, D><<<static_cast<unsigned>(grid), 512, 0, stream>>>(
+      static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
+      a.slopes, a.state, static_cast<T*>(a.out), a.H, a.n_tok, static_cast<const T*>(a.gate),
+      a.gamma, a.eps);
+  return cudaGetLastError();
+}
+
 template <typename T, int D>
 cudaError_t launch_recurrent_typed(const PrefillArgs& a, cudaStream_t stream) {
   const int64_t grid = (a.n_seqs > 0 ? a.n_seqs : a.B) * a.H;
@@ -228,6 +335,15 @@ cudaError_t launch_recurrent_prefill(const PrefillArgs& a, cudaStream_t stream) 
   }
   return a.d == 64 ? launch_recurrent_typed<__nv_bfloat16, 64>(a, stream)
                    : launch_recurrent_typed<__nv_bfloat16, 128>(a, stream);
+}
+
+cudaError_t launch_decode_multi(const DecodeArgs& a, cudaStream_t stream) {
+  if (a.dtype == kF32) {
+    return a.d == 64 ? launch_decode_multi_typed<float, 64>(a, stream)
+                     : launch_decode_multi_typed<float, 128>(a, stream);
+  }
+  return a.d == 64 ? launch_decode_multi_typed<__nv_bfloat16, 64>(a, stream)
+                   : launch_decode_multi_typed<__nv_bfloat16, 128>(a, stream);
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {

@@ -110,6 +110,9 @@ def library(path: str | None = None):
         lib.la_qk_norm_rope.argtypes = [ctypes.POINTER(la_qk_norm_rope_desc), vp, vp, vp, vp, vp,
                                         vp, vp, vp]
         lib.la_qk_norm_rope.restype = ctypes.c_int
+        lib.la_decode_multi.argtypes = [i64, i64, i64, i64, i32, vp, vp, vp, vp, vp,
+                                        ctypes.POINTER(la_gate_norm), vp, vp]
+        lib.la_decode_multi.restype = ctypes.c_int
         lib.la_decode_step.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp]
         lib.la_decode_step.restype = ctypes.c_int
         lib.la_workspace_status.argtypes = [vp, vp]
@@ -174,6 +177,15 @@ def la_decode_step(B: int, H: int, d: int, dtype: int, q: int, k: int, v: int, s
                    state_inout: int, out: int, stream: int) -> int:
     return int(library().la_decode_step(B, H, d, dtype, q, k, v, slopes, state_inout, out,
                                         stream or None))
+
+
+def la_decode_multi(B: int, H: int, d: int, n_tok: int, dtype: int, q: int, k: int, v: int,
+                    slopes: int, state_inout: int, out: int, stream: int,
+                    epilogue: la_gate_norm | None = None) -> int:
+    return int(library().la_decode_multi(B, H, d, n_tok, dtype, q or None, k or None, v or None,
+                                         slopes or None, state_inout or None,
+                                         None if epilogue is None else ctypes.byref(epilogue),
+                                         out or None, stream or None))
 
 
 def la_workspace_status(workspace: int, stream: int) -> int:
@@ -363,3 +375,36 @@ def qk_norm_rope(q: torch.Tensor, k: torch.Tensor, gamma_q: torch.Tensor, gamma_
     if st != LA_OK:
         raise LaError(st, "la_qk_norm_rope")
     return q_out, k_out
+
+
+def decode_multi(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor,
+                 state: torch.Tensor, *, gate: torch.Tensor | None = None,
+                 gamma: torch.Tensor | None = None, eps: float = 1e-6,
+                 out: torch.Tensor | None = None,
+                 stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """o = decode_multi(q, k, v, slopes, state): q, k, v [B, n, H, d]; state fp32 [B, H, d, d]
+    takes all n tokens in order, in place.  gate [B, n, H, d] and gamma fp32 [H, d] switch on
+    the fused grouped RMSNorm + sigmoid gate of each output row."""
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share one [B, n, H, d] shape")
+    if q.dtype not in _DT or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must all be bfloat16 or all float32")
+    B, n, H, d = q.shape
+    if state.dtype != torch.float32 or tuple(state.shape) != (B, H, d, d):
+        raise ValueError("state must be float32 [B, H, d, d]")
+    epi = None
+    if gate is not None or gamma is not None:
+        if gate is None or gamma is None or gate.shape != q.shape or gate.dtype != q.dtype:
+            raise ValueError("the fused norm + gate needs gate (like q) and gamma")
+        if gamma.dtype != torch.float32 or tuple(gamma.shape) != (H, d):
+            raise ValueError("gamma must be float32 [H, d]")
+        epi = la_gate_norm(_cuda_ptr(gate, "gate"), _cuda_ptr(gamma, "gamma"), float(eps))
+    if out is None:
+        out = torch.empty_like(q)
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    st = la_decode_multi(B, H, d, n, _DT[q.dtype], _cuda_ptr(q, "q"), _cuda_ptr(k, "k"),
+                         _cuda_ptr(v, "v"), _cuda_ptr(slopes, "slopes"), _cuda_ptr(state, "state"),
+                         _cuda_ptr(out, "out"), s.cuda_stream, epi)
+    if st != LA_OK:
+        raise LaError(st, "la_decode_multi")
+    return out

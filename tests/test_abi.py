@@ -236,3 +236,21 @@ def test_qk_norm_rope_null_alignment_alias(lib):
     assert la.la_qk_norm_rope(d, *_Q[:5], 0x200000 + 64, *_Q[6:]) == la.LA_ERR_ALIAS
     ds = _qdesc(k_stride=512)
     assert la.la_qk_norm_rope(ds, *_Q[:6], 0x200000, 0) == la.LA_ERR_ALIAS
+
+
+def test_decode_multi_rejects_bad_arguments(lib):
+    ok = (0x1000, 0x2000, 0x3000, 0x4000, 0x50000)  # q, k, v, slopes, state
+    out = 0x9000
+    assert la.la_decode_multi(1, 2, 128, 0, la.LA_BF16, *ok, out, 0) == la.LA_ERR_SHAPE
+    assert la.la_decode_multi(1, 2, 96, 2, la.LA_BF16, *ok, out, 0) == la.LA_ERR_SHAPE
+    assert la.la_decode_multi(1, 2, 128, 2, 7, *ok, out, 0) == la.LA_ERR_DTYPE
+    assert la.la_decode_multi(1, 2, 128, 2, la.LA_BF16, 0, *ok[1:], out, 0) == la.LA_ERR_NULL
+    assert la.la_decode_multi(1, 2, 128, 2, la.LA_BF16, 0x1004, *ok[1:], out, 0) == la.LA_ERR_ALIGN
+    # out overlapping the state
+    assert la.la_decode_multi(1, 2, 128, 2, la.LA_BF16, *ok, 0x50000 + 512, 0) == la.LA_ERR_ALIAS
+    bad = la.la_gate_norm(0x800008, 0x900000, 1e-6)
+    assert la.la_decode_multi(1, 2, 128, 2, la.LA_BF16, *ok, out, 0,
+                              epilogue=bad) == la.LA_ERR_ALIGN
+    nan = la.la_gate_norm(0x800000, 0x900000, float("nan"))
+    assert la.la_decode_multi(1, 2, 128, 2, la.LA_BF16, *ok, out, 0,
+                              epilogue=nan) == la.LA_ERR_SHAPE
