@@ -204,9 +204,10 @@ __global__ void __launch_bounds__(512) decode_kernel(const T* __restrict__ q,
 // Multi-token decode step (speculative verification: the report's "attention with MTP", §4.3).
 // One CTA per (b, h), 512 threads, the state's quads held in registers as in decode_kernel, and
 // n tokens applied in order, each one: S <- lambda S + k^T v, o = q S.  The state is read and
-// written once for all n tokens.  Token j's q, k, v are staged in one of two shared buffers while
-// token j-1 is read out.  With a gate, each output row gets the fused grouped RMSNorm + sigmoid
-// gate: y = gamma * o / sqrt(mean(o^2) + eps) * sigmoid(g) (one norm group per head).
+// written once for all n tokens.  The q, k, v (and gate) rows of up to 8 tokens are staged in
+// shared memory at once, so a group costs one load latency, and each token then costs one block
+// barrier.  With a gate, each output row gets the fused grouped RMSNorm + sigmoid gate:
+// y = gamma * o / sqrt(mean(o^2) + eps) * sigmoid(g) (one norm group per head).
 // ---------------------------------------------------------------------------------------------
 template <typename T, int D>
 __global__ void __launch_bounds__(512) decode_multi_kernel(
@@ -217,8 +218,10 @@ __global__ void __launch_bounds__(512) decode_multi_kernel(
   constexpr int Q4 = D / 4;     // column quads per row
   constexpr int RS = NT / Q4;   // row slots
   constexpr int RPT = D / RS;   // rows per thread
-  __shared__ float sq[2][D], sk[2][D], sv[2][D];
-  __shared__ float red[RS][D];
+  constexpr int NG = 8;         // tokens staged per group
+  __shared__ float sqkv[3][NG][D];   // q, k, v of the group's tokens
+  __shared__ float sg[NG][D];        // their gate pre-activations
+  __shared__ float red[2][RS][D];    // read-out partial sums, double-buffered over tokens
   __shared__ float ss_part[D / 32];
 
   const int tid = threadIdx.x;
@@ -237,61 +240,67 @@ __global__ void __launch_bounds__(512) decode_multi_kernel(
 
   // element offset of token j's row for this head in a [B, n_tok, H, D] tensor
   auto row_off = [&](int64_t j) { return ((b * n_tok + j) * H + h) * D; };
-  auto stage = [&](int64_t j) {
-    if (tid < 3 * D) {
-      const int which = tid / D, e = tid % D;
+  int64_t tok = 0;  // tokens processed so far (selects the red buffer)
+  for (int64_t j0 = 0; j0 < n_tok; j0 += NG) {
+    const int nn = static_cast<int>(min(static_cast<int64_t>(NG), n_tok - j0));
+    // stage the whole group (one load latency for nn tokens)
+    for (int idx = tid; idx < 3 * nn * D; idx += NT) {
+      const int which = idx / (nn * D), rem = idx % (nn * D), jj = rem / D, e = rem % D;
       const T* src = which == 0 ? q : (which == 1 ? k : v);
-      const float x = load_as_f32<T>(src, row_off(j) + e);
-      (which == 0 ? sq : (which == 1 ? sk : sv))[j & 1][e] = x;
+      sqkv[which][jj][e] = load_as_f32<T>(src, row_off(j0 + jj) + e);
     }
-  };
-  for (int64_t j = 0; j < n_tok; ++j) {
-    stage(j);
-    __syncthreads();  // token j staged; the read-out of token j-1 is done with red
-    const int buf = static_cast<int>(j & 1);
-    const float v0 = sv[buf][4 * c4 + 0], v1 = sv[buf][4 * c4 + 1];
-    const float v2 = sv[buf][4 * c4 + 2], v3 = sv[buf][4 * c4 + 3];
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-      const int i = r0 + r * RS;
-      const float ki = sk[buf][i], qi = sq[buf][i];
-      float4 x = s[r];
-      x.x = fmaf(lam_hi, x.x, fmaf(ki, v0, lam_lo * x.x));
-      x.y = fmaf(lam_hi, x.y, fmaf(ki, v1, lam_lo * x.y));
-      x.z = fmaf(lam_hi, x.z, fmaf(ki, v2, lam_lo * x.z));
-      x.w = fmaf(lam_hi, x.w, fmaf(ki, v3, lam_lo * x.w));
-      a0 = fmaf(qi, x.x, a0);
-      a1 = fmaf(qi, x.y, a1);
-      a2 = fmaf(qi, x.z, a2);
-      a3 = fmaf(qi, x.w, a3);
-      s[r] = x;
-    }
-    red[r0][4 * c4 + 0] = a0;
-    red[r0][4 * c4 + 1] = a1;
-    red[r0][4 * c4 + 2] = a2;
-    red[r0][4 * c4 + 3] = a3;
+    if (gate != nullptr)
+      for (int idx = tid; idx < nn * D; idx += NT)
+        sg[idx / D][idx % D] = load_as_f32<T>(gate, row_off(j0 + idx / D) + idx % D);
     __syncthreads();
-    if (tid < D) {
-      float o = 0.f;
+    for (int jj = 0; jj < nn; ++jj, ++tok) {
+      const int rb = static_cast<int>(tok & 1);
+      const float v0 = sqkv[2][jj][4 * c4 + 0], v1 = sqkv[2][jj][4 * c4 + 1];
+      const float v2 = sqkv[2][jj][4 * c4 + 2], v3 = sqkv[2][jj][4 * c4 + 3];
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-      for (int rr = 0; rr < RS; ++rr) o += red[rr][tid];
-      if (gate != nullptr) {
-        float ss = o * o;
-#pragma unroll
-        for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-        if ((tid & 31) == 0) ss_part[tid >> 5] = ss;
-        asm volatile("bar.sync 1, %0;" ::"r"(D) : "memory");  // the D read-out threads only
-        float tot = 0.f;
-#pragma unroll
-        for (int w = 0; w < D / 32; ++w) tot += ss_part[w];
-        const float g = load_as_f32<T>(gate, row_off(j) + tid);
-        const float sig = 1.f / (1.f + expf(-g));
-        o = gamma[h * D + tid] * (o * rsqrtf(tot * (1.f / D) + eps)) * sig;
-        asm volatile("bar.sync 1, %0;" ::"r"(D) : "memory");  // ss_part reused by token j+1
+      for (int r = 0; r < RPT; ++r) {
+        const int i = r0 + r * RS;
+        const float ki = sqkv[1][jj][i], qi = sqkv[0][jj][i];
+        float4 x = s[r];
+        x.x = fmaf(lam_hi, x.x, fmaf(ki, v0, lam_lo * x.x));
+        x.y = fmaf(lam_hi, x.y, fmaf(ki, v1, lam_lo * x.y));
+        x.z = fmaf(lam_hi, x.z, fmaf(ki, v2, lam_lo * x.z));
+        x.w = fmaf(lam_hi, x.w, fmaf(ki, v3, lam_lo * x.w));
+        a0 = fmaf(qi, x.x, a0);
+        a1 = fmaf(qi, x.y, a1);
+        a2 = fmaf(qi, x.z, a2);
+        a3 = fmaf(qi, x.w, a3);
+        s[r] = x;
       }
-      store_from_f32<T>(out, row_off(j) + tid, o);
+      red[rb][r0][4 * c4 + 0] = a0;
+      red[rb][r0][4 * c4 + 1] = a1;
+      red[rb][r0][4 * c4 + 2] = a2;
+      red[rb][r0][4 * c4 + 3] = a3;
+      // One barrier per token: red is double-buffered, and the read-out of this token finishes
+      // before its threads reach the next token's barrier, so red[rb] is free again two tokens on.
+      __syncthreads();
+      if (tid < D) {
+        float o = 0.f;
+#pragma unroll
+        for (int rr = 0; rr < RS; ++rr) o += red[rb][rr][tid];
+        if (gate != nullptr) {
+          float ss = o * o;
+#pragma unroll
+          for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+          if ((tid & 31) == 0) ss_part[tid >> 5] = ss;
+          asm volatile("bar.sync 1, %0;" ::"r"(D) : "memory");  // the D read-out threads only
+          float tot = 0.f;
+#pragma unroll
+          for (int w = 0; w < D / 32; ++w) tot += ss_part[w];
+          const float sig = 1.f / (1.f + expf(-sg[jj][tid]));
+          o = gamma[h * D + tid] * (o * rsqrtf(tot * (1.f / D) + eps)) * sig;
+          asm volatile("bar.sync 1, %0;" ::"r"(D) : "memory");  // ss_part reused next token
+        }
+        store_from_f32<T>(out, row_off(j0 + jj) + tid, o);
+      }
     }
+    __syncthreads();  // the group's staging buffers are read; the next group may overwrite them
   }
 #pragma unroll
   for (int r = 0; r < RPT; ++r) __stcs(st + (r0 + r * RS) * Q4 + c4, s[r]);
