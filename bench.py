@@ -230,6 +230,14 @@ def run_ours(args):
     out = torch.empty_like(q)
     extra_in = []  # further inputs copied from the host in the e2e leg
     epi = None
+    sep = None
+    if args.gate_separate:
+        gg = torch.Generator(device=dev)
+        gg.manual_seed(77 + 1000 * rank)
+        gate = (torch.randn((B * N, H, d), generator=gg, device=dev)).to(w.dtype)
+        gamma = (1.0 + 0.1 * torch.randn((H, d), generator=gg, device=dev)).float()
+        extra_in += [gate]
+        sep = la.la_gate_norm(gate.data_ptr(), gamma.data_ptr(), 1e-6)
     if args.gate:
         # fused grouped RMSNorm + sigmoid gate on the prefill output: a gate pre-activation the
         # size of q and a norm weight per head and channel (synthetic, seeded)
@@ -308,6 +316,13 @@ def run_ours(args):
         if rc != la.LA_OK:
             raise la.LaError(rc, "la_prefill")
 
+    def sep_call():
+        # the post-kernel operator on its own, in place on the prefill's output
+        rc = la.la_gate_norm_apply(B * N, H, d, la.LA_BF16, out.data_ptr(), sep, out.data_ptr(),
+                                   sp)
+        if rc != la.LA_OK:
+            raise la.LaError(rc, "la_gate_norm_apply")
+
     def qk_call():
         rc = la.la_qk_norm_rope(qk, q_raw.data_ptr(), k_raw.data_ptr(), gam_q.data_ptr(),
                                 gam_k.data_ptr(), positions.data_ptr(), q.data_ptr(),
@@ -331,6 +346,8 @@ def run_ours(args):
         if qk is not None:
             qk_call()
         prefill_call()
+        if sep is not None:
+            sep_call()
         decode_call()
     torch.cuda.synchronize(dev)
     st_rc = la.la_workspace_status(ws.data_ptr(), sp)
@@ -353,6 +370,8 @@ def run_ours(args):
                 qk_call()
             ev[i][0].record(stream)
             prefill_call()
+            if sep is not None:
+                sep_call()
             ev[i][1].record(stream)
             decode_call()
             ev[i][2].record(stream)
@@ -411,6 +430,8 @@ def run_ours(args):
             if qk is not None:
                 qk_call()
             prefill_call()
+            if sep is not None:
+                sep_call()
             decode_call()
             hout.copy_(out, non_blocking=True)
             hst.copy_(st, non_blocking=True)
@@ -431,7 +452,9 @@ def run_ours(args):
         tok_s = world * tokens / (pre_ms_max * 1e-3)
         # algorithmic bytes of one prefill launch: read q, k, v and write o (bf16), write the
         # final states (and read the initial states of the packed workload)
-        pre_bytes = (4 + (1 if args.gate else 0)) * B * N * H * d * 2 + \
+        # (the separate norm + gate pass reads o and the gate and writes y: 3 more rows)
+        pre_bytes = (4 + (1 if args.gate else 0) + (3 if args.gate_separate else 0)) * \
+            B * N * H * d * 2 + \
             n_states * H * d * d * 4 * (1 if vw is None else 2)
         achieved = pre_bytes / (pre_ms_max * 1e-3) / 1e9
         canon = 4.0 * d * d * B * N * H  # recurrent-form flops
@@ -456,6 +479,8 @@ def run_ours(args):
                                     f"(fragmented lengths), H={H} d={d} bf16, fp32 initial "
                                     f"states") + (", fused grouped RMSNorm + sigmoid gate epilogue"
                                                   if args.gate else "") +
+                                   (", then the grouped RMSNorm + sigmoid gate pass"
+                                    if args.gate_separate else "") +
                                    f" + decode step B={Bd} H={Hd} d={dd} (fp32 state)",
                        "global_batch": world * B, "seq_len": N, "parallelism": f"replicas{world}",
                        "l2": "inputs larger than L2 (no flush)"},
@@ -470,7 +495,7 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak,
                          "traffic": (measured_traffic() if args.workload == "prefill_32k"
-                                     and not args.gate else None),
+                                     and not (args.gate or args.gate_separate) else None),
                          "algorithmic_bytes": pre_bytes,
                          "kernel": "chunked_prefill_kernel", "peak_kind": peak_kind},
             "qk_norm_rope": None if qk is None else {
@@ -482,7 +507,8 @@ def run_ours(args):
             "e2e": e2e,
             # per step: the prefill kernel (after the planning kernel for packed input) and the
             # decode kernel
-            "gpu_launches": ((3 if packed else 2) + (1 if qk is not None else 0)) * K,
+            "gpu_launches": ((3 if packed else 2) + (1 if qk is not None else 0) +
+                             (1 if sep is not None else 0)) * K,
         }
         print(json.dumps(line), flush=True)
     dist_teardown(world)
@@ -543,6 +569,8 @@ def main():
                     help="decode this many tokens per sequence per step (multi-token step)")
     ap.add_argument("--qk-rope", action="store_true",
                     help="run the QK RMSNorm + partial RoPE operator before each prefill")
+    ap.add_argument("--gate-separate", action="store_true",
+                    help="run the grouped RMSNorm + sigmoid gate as its own pass after the prefill")
     ap.add_argument("--gate", action="store_true",
                     help="fuse the grouped RMSNorm + sigmoid gate into the prefill's output")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer e2e leg")

@@ -143,6 +143,23 @@ typedef struct {
 } la_gate_norm;
 
 /*
+ * la_gate_norm_apply — the report's post-kernel operator on its own: grouped RMSNorm + sigmoid
+ * gate over the kernel's output (§2.1 Fig. 2; §4.3 runs "group norm + sigmoid gate" as one fused
+ * operator after attention).  For every token t and head h:
+ *     y = gamma[h] * o / sqrt(mean(o^2) + eps) * sigmoid(g)       (one norm group per head)
+ * The same computation as the la_gate_norm epilogue of la_prefill_varlen / la_decode_multi, run
+ * as a separate memory-bound pass over o, g and y.
+ *
+ *   T, H, d     tokens (>= 0), heads, head dim (64 or 128); dtype: la_dtype of o, gate and y
+ *   o           [T, H, d] device, read only
+ *   gn          gate ([T, H, d] of dtype), gamma (fp32 [H, d]) and eps (>= 0); host pointer
+ *   y           [T, H, d] device, written; may be o itself (in place), no other overlap
+ *   stream      cudaStream_t as void*
+ */
+la_status la_gate_norm_apply(int64_t T, int64_t H, int64_t d, int32_t dtype, const void* o,
+                             const la_gate_norm* gn, void* y, void* stream);
+
+/*
  * la_decode_multi — n_tok generated tokens per sequence in one step, for speculative
  * verification ("attention with MTP" in the report's serving path, §4.3): for every (b, h) and
  * j = 0 .. n_tok-1 in order,

@@ -324,6 +324,25 @@ la_status la_decode_multi(int64_t B, int64_t H, int64_t d, int64_t n_tok, int32_
              : LA_ERR_CUDA;
 }
 
+la_status la_gate_norm_apply(int64_t T, int64_t H, int64_t d, int32_t dtype, const void* o,
+                             const la_gate_norm* gn, void* y, void* stream) {
+  if (dtype != LA_BF16 && dtype != LA_F32) return LA_ERR_DTYPE;
+  if (T < 0 || H < 1 || (d != 64 && d != 128)) return LA_ERR_SHAPE;
+  if (T > INT32_MAX) return LA_ERR_OVERFLOW;  // one CTA per token
+  if (!o || !gn || !gn->gate || !gn->gamma || !y) return LA_ERR_NULL;
+  if (!(gn->eps >= 0.f) || gn->eps > 3.0e38f) return LA_ERR_SHAPE;
+  int64_t n = 0;
+  if (!mul_ok(T, H, &n) || !mul_ok(n, d, &n)) return LA_ERR_OVERFLOW;
+  if (!aligned16(o) || !aligned16(gn->gate) || !aligned16(gn->gamma) || !aligned16(y))
+    return LA_ERR_ALIGN;
+  const size_t bytes = static_cast<size_t>(n) * (dtype == LA_BF16 ? 2 : 4);
+  if (bytes > 0 && ((y != o && overlaps(y, bytes, o, bytes)) || overlaps(y, bytes, gn->gate, bytes)))
+    return LA_ERR_ALIAS;
+  la::GateNormArgs a{T, H, d, dtype, o, gn->gate, gn->gamma, gn->eps, y};
+  return la::launch_gate_norm(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? LA_OK
+                                                                                     : LA_ERR_CUDA;
+}
+
 la_status la_decode_step(int64_t B, int64_t H, int64_t d, int32_t dtype, const void* q,
                          const void* k, const void* v, const float* slopes, float* state_inout,
                          void* out, void* stream) {

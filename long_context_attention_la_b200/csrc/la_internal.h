@@ -82,6 +82,18 @@ struct QkNormRopeArgs {
 };
 cudaError_t launch_qk_norm_rope(const QkNormRopeArgs& a, cudaStream_t stream);
 
+// Grouped RMSNorm + sigmoid gate over [T, H, d] rows (la_gatenorm.cu).
+struct GateNormArgs {
+  int64_t T, H, d;
+  int dtype;
+  const void* o;
+  const void* gate;
+  const float* gamma;  // [H, d]
+  float eps;
+  void* y;
+};
+cudaError_t launch_gate_norm(const GateNormArgs& a, cudaStream_t stream);
+
 // ---------------------------------------------------------------------------------------------
 // Chunked tensor-core prefill (bf16, d = 128, chunk C = 128).
 // ---------------------------------------------------------------------------------------------

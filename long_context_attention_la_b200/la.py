@@ -113,6 +113,9 @@ def library(path: str | None = None):
         lib.la_decode_multi.argtypes = [i64, i64, i64, i64, i32, vp, vp, vp, vp, vp,
                                         ctypes.POINTER(la_gate_norm), vp, vp]
         lib.la_decode_multi.restype = ctypes.c_int
+        lib.la_gate_norm_apply.argtypes = [i64, i64, i64, i32, vp, ctypes.POINTER(la_gate_norm),
+                                           vp, vp]
+        lib.la_gate_norm_apply.restype = ctypes.c_int
         lib.la_decode_step.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp]
         lib.la_decode_step.restype = ctypes.c_int
         lib.la_workspace_status.argtypes = [vp, vp]
@@ -186,6 +189,13 @@ def la_decode_multi(B: int, H: int, d: int, n_tok: int, dtype: int, q: int, k: i
                                          slopes or None, state_inout or None,
                                          None if epilogue is None else ctypes.byref(epilogue),
                                          out or None, stream or None))
+
+
+def la_gate_norm_apply(T: int, H: int, d: int, dtype: int, o: int, gn: la_gate_norm | None,
+                       y: int, stream: int) -> int:
+    return int(library().la_gate_norm_apply(T, H, d, dtype, o or None,
+                                            None if gn is None else ctypes.byref(gn), y or None,
+                                            stream or None))
 
 
 def la_workspace_status(workspace: int, stream: int) -> int:
@@ -407,4 +417,25 @@ def decode_multi(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torc
                          _cuda_ptr(out, "out"), s.cuda_stream, epi)
     if st != LA_OK:
         raise LaError(st, "la_decode_multi")
+    return out
+
+
+def gate_norm(o: torch.Tensor, gate: torch.Tensor, gamma: torch.Tensor, *, eps: float = 1e-6,
+              out: torch.Tensor | None = None,
+              stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """y = gate_norm(o, gate, gamma): o, gate [T, H, d] (bf16 or fp32, CUDA, contiguous), gamma
+    fp32 [H, d]; y = gamma * o / rms(o) * sigmoid(gate) per token and head (out may be o)."""
+    if o.dim() != 3 or gate.shape != o.shape or gate.dtype != o.dtype or o.dtype not in _DT:
+        raise ValueError("o and gate must share one [T, H, d] shape and dtype")
+    T, H, d = o.shape
+    if gamma.dtype != torch.float32 or tuple(gamma.shape) != (H, d):
+        raise ValueError("gamma must be float32 [H, d]")
+    if out is None:
+        out = torch.empty_like(o)
+    s = stream if stream is not None else torch.cuda.current_stream(o.device)
+    gn = la_gate_norm(_cuda_ptr(gate, "gate"), _cuda_ptr(gamma, "gamma"), float(eps))
+    st = la_gate_norm_apply(T, H, d, _DT[o.dtype], _cuda_ptr(o, "o"), gn, _cuda_ptr(out, "out"),
+                            s.cuda_stream)
+    if st != LA_OK:
+        raise LaError(st, "la_gate_norm_apply")
     return out

@@ -254,3 +254,19 @@ def test_decode_multi_rejects_bad_arguments(lib):
     nan = la.la_gate_norm(0x800000, 0x900000, float("nan"))
     assert la.la_decode_multi(1, 2, 128, 2, la.LA_BF16, *ok, out, 0,
                               epilogue=nan) == la.LA_ERR_SHAPE
+
+
+def test_gate_norm_apply_rejects_bad_arguments(lib):
+    gn = la.la_gate_norm(0x800000, 0x900000, 1e-6)
+    o, y = 0x100000, 0x200000
+    assert la.la_gate_norm_apply(4, 2, 128, 9, o, gn, y, 0) == la.LA_ERR_DTYPE
+    assert la.la_gate_norm_apply(4, 2, 96, la.LA_BF16, o, gn, y, 0) == la.LA_ERR_SHAPE
+    assert la.la_gate_norm_apply(-1, 2, 128, la.LA_BF16, o, gn, y, 0) == la.LA_ERR_SHAPE
+    assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, 0, gn, y, 0) == la.LA_ERR_NULL
+    assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, o, None, y, 0) == la.LA_ERR_NULL
+    assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, o + 8, gn, y, 0) == la.LA_ERR_ALIGN
+    nan = la.la_gate_norm(0x800000, 0x900000, float("nan"))
+    assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, o, nan, y, 0) == la.LA_ERR_SHAPE
+    # y overlapping o without being o, or overlapping the gate
+    assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, o, gn, o + 64, 0) == la.LA_ERR_ALIAS
+    assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, o, gn, 0x800000, 0) == la.LA_ERR_ALIAS

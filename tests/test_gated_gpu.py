@@ -129,3 +129,40 @@ def test_gated_epilogue_layer_width_sampled_heads():
     heads = sorted(np.random.default_rng(143).choice(H, 6, replace=False).tolist())
     ref = reference(q, k, v, sl, cu, gate, gamma, EPS, heads=heads)
     check_close(y[:, heads].float().cpu().numpy(), ref, torch.bfloat16, "y")
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 128),
+                                     (torch.bfloat16, 64)])
+def test_standalone_gate_norm_matches_oracle(dtype, d):
+    """la_gate_norm_apply (the post-kernel operator on its own) on random o."""
+    T, H = 333, 8
+    g = torch.Generator(device=DEV)
+    g.manual_seed(151)
+    o = (torch.randn((T, H, d), generator=g, device=DEV) * 0.7).to(dtype)
+    gate = (torch.randn((T, H, d), generator=g, device=DEV) * 3).to(dtype)
+    gamma = (1.0 + 0.5 * torch.randn((H, d), generator=g, device=DEV)).float()
+    y = la.gate_norm(o, gate, gamma, eps=1e-6)
+    torch.cuda.synchronize()
+    ref = oracle.gated_rmsnorm(o.double().cpu().numpy(), oracle_bits(gate), gamma.cpu().numpy(),
+                               1e-6)
+    check_close(y.float().cpu().numpy(), ref, dtype, "y")
+    # in place gives the same bits
+    o2 = o.clone()
+    la.gate_norm(o2, gate, gamma, eps=1e-6, out=o2)
+    torch.cuda.synchronize()
+    assert torch.equal(o2, y)
+
+
+def test_standalone_gate_norm_equals_fused_epilogue_path():
+    """prefill then la_gate_norm_apply agrees with the fused epilogue within the bf16 bar."""
+    H, d = 4, 128
+    lengths = [900, 300]
+    cu = synth.cu_from_lengths(lengths)
+    q, k, v = draw_packed(lengths, H, d, seed=161)
+    sl = synth.slopes(H, DEV)
+    gate, gamma = draw_gate(sum(lengths), H, d, seed=162)
+    o, _ = la.prefill_varlen(q, k, v, sl, cu)
+    y_sep = la.gate_norm(o, gate, gamma, eps=EPS)
+    y_fused, _ = la.prefill_varlen(q, k, v, sl, cu, gate=gate, gamma=gamma, eps=EPS)
+    torch.cuda.synchronize()
+    check_close(y_sep.float().cpu().numpy(), y_fused.double().cpu().numpy(), torch.bfloat16, "y")
