@@ -218,3 +218,32 @@ def qk_norm_rope(x, gamma, positions, rotary_dim: int, theta: float, eps: float)
     y[..., :half] = a * c - b * s
     y[..., half:r] = b * c + a * s
     return y
+
+
+def fold_states(parts, lengths, slopes, state_in=None):
+    """The report's "fused update h" in fp64 ("Ling and Ring 2.6 Technical Report", §4.1.1
+    Context Parallel for Lightning Attention, Fig. 10: local h of every part -> AllGather ->
+    update h): the state after consecutive parts j = 0 .. n-1 of a sequence, part j holding
+    lengths[j] tokens and having local state h_j (its state when started from zero):
+
+        S = state_in (or 0);   for j in order:  S <- lambda^lengths[j] * S + h_j
+
+    with lambda_h = exp(-slope_h) per head.  parts: [n, B, H, d, d] (any real dtype); lengths:
+    n non-negative integers; slopes: float32[H]; state_in: [B, H, d, d] or None.  Returns fp64
+    [B, H, d, d].
+    """
+    parts = np.asarray(parts, dtype=np.float64)
+    if parts.ndim != 5:
+        raise ValueError("parts must be [n, B, H, d, d]")
+    n, B, H, d, _ = parts.shape
+    lengths = [int(x) for x in lengths]
+    if len(lengths) != n or any(x < 0 for x in lengths):
+        raise ValueError("lengths must be n non-negative integers")
+    sl = np.asarray(slopes, dtype=np.float32).astype(np.float64)
+    if sl.shape != (H,):
+        raise ValueError("slopes must be float32[H]")
+    S = np.zeros((B, H, d, d)) if state_in is None else np.array(state_in, dtype=np.float64)
+    for j in range(n):
+        lam_l = np.exp(-sl * lengths[j])[None, :, None, None]
+        S = lam_l * S + parts[j]
+    return S

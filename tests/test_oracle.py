@@ -325,3 +325,65 @@ def test_qk_norm_rope_invariants():
     q2 = oracle.qk_norm_rope(x[:1], gamma, [1000 + 77777], r, 6.0e6, 1e-6)
     k2 = oracle.qk_norm_rope(x[1:2], gamma, [400 + 77777], r, 6.0e6, 1e-6)
     assert np.allclose(np.sum(q * k, -1), np.sum(q2 * k2, -1), rtol=1e-9)
+
+
+def _part_states(q, k, v, sl, cuts):
+    """Local states (each from zero) of the parts [cuts[j], cuts[j+1]) of the token axis."""
+    B, N, H, d = q.shape
+    hs = []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        if b == a:
+            hs.append(np.zeros((B, H, d, d)))
+            continue
+        _, st = oracle.prefill(q[:, a:b].copy(), k[:, a:b].copy(), v[:, a:b].copy(), sl)
+        hs.append(st.reshape(B, H, d, d))
+    return np.stack(hs)
+
+
+@pytest.mark.parametrize("cuts", [[0, 13, 40], [0, 7, 7, 25, 40], [0, 1, 2, 3, 40], [0, 40]])
+def test_fold_of_part_states_equals_sequential_state(cuts):
+    """The context-parallel invariant of §4.1.1 (local recurrence, then global correction):
+    folding the parts' local states gives the state of one sequential pass, for any cut."""
+    B, N, H, d = 2, 40, 3, 5
+    q, k, v = _rand(B, N, H, d, 31)
+    sl = np.array([0.05, 0.7, 2.5], dtype=np.float32)
+    _, st = oracle.prefill(q, k, v, sl)
+    S = oracle.fold_states(_part_states(q, k, v, sl, cuts), np.diff(cuts), sl)
+    np.testing.assert_allclose(S, st.reshape(B, H, d, d), rtol=1e-12, atol=1e-12)
+    # with an initial state (a cached prefix)
+    s0 = np.random.default_rng(32).normal(size=(B, H, d, d))
+    _, st0 = oracle.prefill(q, k, v, sl, state_in=s0.reshape(B * H, d, d))
+    S0 = oracle.fold_states(_part_states(q, k, v, sl, cuts), np.diff(cuts), sl, state_in=s0)
+    np.testing.assert_allclose(S0, st0.reshape(B, H, d, d), rtol=1e-12, atol=1e-12)
+    # the incoming state of part r continues the sequence exactly where part r starts
+    r = len(cuts) - 2
+    hs = _part_states(q, k, v, sl, cuts)
+    Sr = oracle.fold_states(hs[:r], np.diff(cuts)[:r], sl, state_in=s0)
+    a = cuts[r]
+    o_tail, _ = oracle.prefill(q[:, a:].copy(), k[:, a:].copy(), v[:, a:].copy(), sl,
+                               state_in=Sr.reshape(B * H, d, d))
+    o_all, _ = oracle.prefill(q, k, v, sl, state_in=s0.reshape(B * H, d, d))
+    np.testing.assert_allclose(o_tail, o_all[:, a:], rtol=1e-12, atol=1e-12)
+
+
+def test_fold_closed_forms():
+    """lambda = 1: the fold is state_in plus the plain sum of the parts; lambda^L = 0 (a long
+    part with a large slope): the state before that part is forgotten; no parts: state_in."""
+    rng = np.random.default_rng(33)
+    n, B, H, d = 3, 2, 2, 4
+    parts = rng.normal(size=(n, B, H, d, d))
+    s0 = rng.normal(size=(B, H, d, d))
+    np.testing.assert_allclose(oracle.fold_states(parts, [5, 9, 2], np.zeros(H, np.float32),
+                                                  state_in=s0),
+                               s0 + parts.sum(axis=0), rtol=1e-13, atol=1e-13)
+    big = np.full(H, 50.0, dtype=np.float32)  # exp(-50 * 40) underflows to exactly 0
+    np.testing.assert_array_equal(oracle.fold_states(parts, [40, 40, 40], big, state_in=s0),
+                                  parts[2])
+    np.testing.assert_array_equal(oracle.fold_states(parts[:0], [], big, state_in=s0), s0)
+    # one part: lambda^L S_in + h, per head with its own lambda
+    sl = np.array([0.1, 0.9], dtype=np.float32)
+    lam = np.exp(-sl.astype(np.float64) * 7)
+    want = lam[None, :, None, None] * s0 + parts[0]
+    np.testing.assert_allclose(oracle.fold_states(parts[:1], [7], sl, state_in=s0), want,
+                               rtol=1e-14, atol=1e-14)
+

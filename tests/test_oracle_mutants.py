@@ -66,3 +66,54 @@ def test_mutant_is_caught(name, tmp_path):
     src.write_text(text.replace(old, new, 1))  # first site: the prefill loop
     lib = oracle.open_library(oracle.compile_source(str(src), str(tmp_path / f"lib{name}.so")))
     assert not _pins_pass(lib), f"the pins did not catch the planted mistake {name}"
+
+
+# The fold of part states (oracle.fold_states): each mutant is planted in a copy of the function's
+# source, executed on the CPU, and must fail the context-parallel invariant of test_oracle.py.
+FOLD_MUTANTS = {
+    "fold_decays_h_too": ("S = lam_l * S + parts[j]", "S = lam_l * (S + parts[j])"),
+    "fold_no_decay": ("S = lam_l * S + parts[j]", "S = S + parts[j]"),
+    "fold_next_part_length": ("np.exp(-sl * lengths[j])",
+                              "np.exp(-sl * lengths[min(j + 1, n - 1)])"),
+    "fold_reversed_order": ("for j in range(n):", "for j in reversed(range(n)):"),
+    "fold_head_axis_wrong": ("[None, :, None, None]", "[None, None, :, None]"),
+}
+
+
+def _fold_from_source(src: str):
+    ns = {"np": np}
+    exec(compile(src, "<fold mutant>", "exec"), ns)  # noqa: S102 - test-only source mutation
+    return ns["fold_states"]
+
+
+def _fold_pins_pass(fold) -> bool:
+    from tests.test_oracle import _part_states
+    B, N, H, d = 2, 40, 3, 5
+    q, k, v = _rand(B, N, H, d, 31)
+    sl = np.array([0.05, 0.7, 2.5], dtype=np.float32)
+    s0 = np.random.default_rng(32).normal(size=(B, H, d, d))
+    _, st0 = oracle.prefill(q, k, v, sl, state_in=s0.reshape(B * H, d, d))
+    for cuts in ([0, 13, 40], [0, 7, 7, 25, 40], [0, 1, 2, 3, 40]):
+        S = fold(_part_states(q, k, v, sl, cuts), np.diff(cuts), sl, state_in=s0)
+        if S.shape != (B, H, d, d) or not np.allclose(S, st0.reshape(B, H, d, d), rtol=1e-12,
+                                                      atol=1e-12):
+            return False
+    return True
+
+
+def test_unmutated_fold_copy_passes():
+    import inspect
+    assert _fold_pins_pass(_fold_from_source(inspect.getsource(oracle.fold_states)))
+
+
+@pytest.mark.parametrize("name", sorted(FOLD_MUTANTS))
+def test_fold_mutant_is_caught(name):
+    import inspect
+    old, new = FOLD_MUTANTS[name]
+    text = inspect.getsource(oracle.fold_states)
+    assert text.count(old) == 1, f"mutation site for {name} not found"
+    try:
+        ok = _fold_pins_pass(_fold_from_source(text.replace(old, new)))
+    except (ValueError, IndexError):
+        ok = False  # a shape error is a failed pin too
+    assert not ok, f"the pins did not catch the planted mistake {name}"
