@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define LA_VERSION 1001 /* major*1000 + minor */
+#define LA_VERSION 1002 /* major*1000 + minor */
 
 typedef enum {
   LA_OK = 0,
@@ -318,6 +318,53 @@ typedef struct {
 la_status la_qk_norm_rope(const la_qk_norm_rope_desc* desc, const void* q, const void* k,
                           const float* gamma_q, const float* gamma_k, const int64_t* positions,
                           void* q_out, void* k_out, void* stream);
+
+/* Bytes of device workspace la_prefill_state needs for this descriptor (0 for invalid
+ * arguments or when the recurrent path runs, which needs none). */
+size_t la_prefill_state_workspace_bytes(const la_desc* desc);
+
+/*
+ * la_prefill_state — the final state of a prefill without its outputs: for every (b, h)
+ *     state_out = lambda^N state_in + sum_{t<N} lambda^(N-1-t) k_t^T v_t
+ * (state_in NULL: zero).  This is the "local h" of the report's context-parallel forward (§4.1.1,
+ * Fig. 10): each rank holding one part of a long sequence computes its part's state from its own
+ * K, V, the states are gathered, and la_state_fold turns those of the earlier parts into the
+ * rank's incoming state, from which la_prefill_varlen (state_in) computes the rank's outputs.
+ * Reads K and V once (no q, no output); on the tensor path it is one row-scaled contraction
+ * K~^T V per head (K~_t = lambda^(N-1-t) k_t) accumulated in fp32.
+ *
+ *   desc       as for la_prefill (B, N >= 1, H, d, dtype, path; chunk and segments ignored)
+ *   k, v       [B, N, H, d] device, dtype desc->dtype, read only
+ *   slopes     fp32[H] device
+ *   state_in   fp32 [B, H, d, d] device or NULL, read only
+ *   state_out  fp32 [B, H, d, d] device, written; may be state_in itself (in place)
+ *   workspace  device scratch of la_prefill_state_workspace_bytes(desc) bytes, 256-byte aligned,
+ *              or NULL (allocated and freed on `stream`)
+ *   stream     cudaStream_t as void*
+ * A device-side timeout is recorded in the workspace status word (la_workspace_status).
+ */
+la_status la_prefill_state(const la_desc* desc, const void* k, const void* v, const float* slopes,
+                           const float* state_in, float* state_out, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
+ * la_state_fold — the report's "fused update h" (§4.1.1, Fig. 10): the incoming state of part
+ * n of a sequence cut into consecutive parts of lengths[0..n-1] tokens, from the parts' local
+ * states h_j (la_prefill_state with no state_in) and the sequence's initial state:
+ *     S = state_in (or 0);   S <- lambda^lengths[j] S + h_j   for j = 0 .. n_parts-1
+ * per flat head (BH = batch * H of them).  n_parts = 0 copies state_in (or writes zeros).
+ *
+ *   n_parts    0 .. 256
+ *   BH, H, d   flat heads (a multiple of H), heads, head dim (64 or 128)
+ *   parts      fp32 [n_parts, BH, d, d] device, read only (may be NULL when n_parts = 0)
+ *   lengths    int64 [n_parts] HOST, each >= 0
+ *   slopes     fp32[H] device
+ *   state_in   fp32 [BH, d, d] device or NULL
+ *   state_out  fp32 [BH, d, d] device, written; may be state_in, must not overlap parts
+ */
+la_status la_state_fold(int64_t n_parts, int64_t BH, int64_t H, int64_t d, const float* parts,
+                        const int64_t* lengths, const float* slopes, const float* state_in,
+                        float* state_out, void* stream);
 
 /* Synchronises `stream`, then returns the device status word of a workspace that la_prefill
  * used: LA_OK, or LA_ERR_TIMEOUT if a bounded device wait gave up during the last call. */

@@ -343,6 +343,90 @@ la_status la_gate_norm_apply(int64_t T, int64_t H, int64_t d, int32_t dtype, con
                                                                                      : LA_ERR_CUDA;
 }
 
+size_t la_prefill_state_workspace_bytes(const la_desc* desc) {
+  int64_t numel = 0;
+  if (check_desc(desc, &numel) != LA_OK || !use_tensor_path(desc)) return 0;
+  const int sms = device_sms() > 0 ? device_sms() : 148;
+  return la::plan_state_pass(desc->B, desc->N, desc->H, sms).ws_bytes;
+}
+
+la_status la_prefill_state(const la_desc* desc, const void* k, const void* v, const float* slopes,
+                           const float* state_in, float* state_out, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  int64_t numel = 0;
+  const la_status st = check_desc(desc, &numel);
+  if (st != LA_OK) return st;
+  if (!k || !v || !slopes || !state_out) return LA_ERR_NULL;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(state_out) ||
+      (state_in && !aligned16(state_in)))
+    return LA_ERR_ALIGN;
+  const size_t bytes = static_cast<size_t>(numel) * (desc->dtype == LA_BF16 ? 2 : 4);
+  const size_t state_bytes =
+      static_cast<size_t>(desc->B * desc->H) * static_cast<size_t>(desc->d * desc->d) * 4;
+  if (overlaps(state_out, state_bytes, k, bytes) || overlaps(state_out, state_bytes, v, bytes))
+    return LA_ERR_ALIAS;
+  if (state_in && state_in != state_out && overlaps(state_in, state_bytes, state_out, state_bytes))
+    return LA_ERR_ALIAS;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  la::PrefillArgs a{desc->B, desc->N, desc->H, desc->d, desc->dtype, nullptr, k, v, slopes,
+                    nullptr, state_out};
+  a.state_in = state_in;
+  apply_debug_env(a);
+  if (!use_tensor_path(desc)) {
+    // token recurrence with no q and no read-out
+    return la::launch_recurrent_prefill(a, s) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+  }
+  const int sms = device_sms();
+  if (sms <= 0) return LA_ERR_CUDA;
+  const la::StatePassPlan plan = la::plan_state_pass(desc->B, desc->N, desc->H, sms);
+  void* ws = workspace;
+  bool owned = false;
+  if (ws == nullptr) {
+    if (cudaMallocAsync(&ws, plan.ws_bytes, s) != cudaSuccess) return LA_ERR_CUDA;
+    owned = true;
+  } else {
+    if (workspace_bytes < plan.ws_bytes) return LA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return LA_ERR_ALIGN;
+  }
+  const cudaError_t e = la::launch_state_pass(a, plan, ws, s);
+  if (owned) cudaFreeAsync(ws, s);
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status la_state_fold(int64_t n_parts, int64_t BH, int64_t H, int64_t d, const float* parts,
+                        const int64_t* lengths, const float* slopes, const float* state_in,
+                        float* state_out, void* stream) {
+  if (n_parts < 0 || n_parts > la::kMaxFoldParts || BH < 1 || H < 1 || BH % H != 0 ||
+      (d != 64 && d != 128))
+    return LA_ERR_SHAPE;
+  if (BH > INT32_MAX) return LA_ERR_OVERFLOW;  // grid
+  if (!slopes || !state_out || (n_parts > 0 && (!parts || !lengths))) return LA_ERR_NULL;
+  if (!aligned16(state_out) || (state_in && !aligned16(state_in)) || (parts && !aligned16(parts)))
+    return LA_ERR_ALIGN;
+  int64_t sb = 0, pb = 0;
+  if (!mul_ok(BH, d * d * 4, &sb) || !mul_ok(sb, n_parts, &pb)) return LA_ERR_OVERFLOW;
+  la::StateFoldArgs a{};
+  for (int64_t j = 0; j < n_parts; ++j) {
+    if (lengths[j] < 0) return LA_ERR_SHAPE;
+    a.lengths[j] = lengths[j];
+  }
+  if (n_parts > 0 && overlaps(state_out, static_cast<size_t>(sb), parts, static_cast<size_t>(pb)))
+    return LA_ERR_ALIAS;
+  if (state_in && state_in != state_out &&
+      overlaps(state_in, static_cast<size_t>(sb), state_out, static_cast<size_t>(sb)))
+    return LA_ERR_ALIAS;
+  a.n_parts = n_parts;
+  a.BH = BH;
+  a.H = H;
+  a.d = d;
+  a.parts = parts;
+  a.slopes = slopes;
+  a.state_in = state_in;
+  a.state_out = state_out;
+  return la::launch_state_fold(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? LA_OK
+                                                                                    : LA_ERR_CUDA;
+}
+
 la_status la_decode_step(int64_t B, int64_t H, int64_t d, int32_t dtype, const void* q,
                          const void* k, const void* v, const float* slopes, float* state_inout,
                          void* out, void* stream) {

@@ -1093,6 +1093,8 @@ int32_t prefetch_depth() {
   return v;
 }
 
+}  // namespace
+
 bool encode_map(CUtensorMap* map, const void* base, int64_t B, int64_t N, int64_t H) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (encode == nullptr) {
@@ -1118,8 +1120,6 @@ bool encode_map(CUtensorMap* map, const void* base, int64_t B, int64_t N, int64_
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
-
-}  // namespace
 
 SegmentPlan plan_segments(int64_t B, int64_t N, int64_t H, int requested_segments, int num_sms) {
   SegmentPlan pl{};

@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -94,6 +95,19 @@ struct GateNormArgs {
 };
 cudaError_t launch_gate_norm(const GateNormArgs& a, cudaStream_t stream);
 
+// Fold of per-part states (la_state.cu): S = S_in (or 0); S <- lambda^(L_j) S + h_j for the
+// parts j < n_parts in order.  parts: fp32 [n_parts, BH, d, d]; lengths travel by value.
+constexpr int kMaxFoldParts = 256;
+struct StateFoldArgs {
+  int64_t n_parts, BH, H, d;
+  const float* parts;
+  const float* slopes;
+  const float* state_in;  // [BH, d, d] or null
+  float* state_out;       // [BH, d, d]; may be state_in
+  int64_t lengths[kMaxFoldParts];
+};
+cudaError_t launch_state_fold(const StateFoldArgs& a, cudaStream_t stream);
+
 // ---------------------------------------------------------------------------------------------
 // Chunked tensor-core prefill (bf16, d = 128, chunk C = 128).
 // ---------------------------------------------------------------------------------------------
@@ -141,6 +155,24 @@ WorkspaceLayout workspace_layout(int64_t B, int64_t H, const SegmentPlan& plan);
 // Offsets inside the 256-byte header.
 constexpr size_t kWsCounter = 0;   // uint32 work-unit counter
 constexpr size_t kWsStatus = 64;   // uint32 device status (0 = ok, else a la_status code)
+
+// Tensor map of a bf16 [B, N, H, 128] activation as 4-D (d, H, N, B) tiles of 64 x 1 x C x 1
+// elements with the 128-byte swizzle (two boxes make one [C x 128] tile).
+bool encode_map(CUtensorMap* map, const void* base, int64_t B, int64_t N, int64_t H);
+
+// State-only prefill on the tensor cores (la_state.cu): the B*H*n_chunks chunk-loads, head-major,
+// in one contiguous range of `width` per CTA (`grid` CTAs).  Workspace: a 256-byte header (status
+// word at kWsStatus) and two fp32 d x d partial-state slots per CTA.
+struct StatePassPlan {
+  int64_t n_chunks;  // ceil(N / C)
+  int64_t total;     // B * H * n_chunks
+  int64_t width;     // chunk-loads per CTA
+  int64_t grid;      // CTAs
+  size_t ws_bytes;
+};
+StatePassPlan plan_state_pass(int64_t B, int64_t N, int64_t H, int num_sms);
+cudaError_t launch_state_pass(const PrefillArgs& a, const StatePassPlan& plan, void* workspace,
+                              cudaStream_t stream);
 
 cudaError_t launch_chunked_prefill(const PrefillArgs& a, const SegmentPlan& plan,
                                    void* workspace, cudaStream_t stream, int num_sms);

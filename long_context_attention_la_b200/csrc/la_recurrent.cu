@@ -77,11 +77,13 @@ __global__ void __launch_bounds__(4 * D) recurrent_prefill_kernel(
   float lam_hi, lam_lo;
   split_decay(slopes[h], lam_hi, lam_lo);
 
-  // loader role: threads [0, 3D) each fetch one element of q, k or v of a token
+  // loader role: threads [0, 3D) each fetch one element of q, k or v of a token (state only,
+  // q == nullptr and out == nullptr: the q loaders supply zeros and nothing is read out)
   const int which = tid / D;  // 0: q, 1: k, 2: v (3: idle)
   const int e = tid % D;
   const T* src = which == 0 ? q : (which == 1 ? k : v);
   auto fetch = [&](int64_t t) -> float {
+    if (src == nullptr) return 0.f;
     return load_as_f32<T>(src, ((row0 + t) * H + h) * D + e);
   };
 
@@ -111,7 +113,7 @@ __global__ void __launch_bounds__(4 * D) recurrent_prefill_kernel(
     red[rg][j] = acc;
     if (which < 3 && t + 1 < len) tok[buf ^ 1][which][e] = pf;
     __syncthreads();
-    if (rg == 0) {
+    if (rg == 0 && out != nullptr) {
       const float o = ((red[0][j] + red[1][j]) + red[2][j]) + red[3][j];
       store_from_f32<T>(out, ((row0 + t) * H + h) * D + j, o);
     }

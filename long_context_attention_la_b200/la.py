@@ -116,6 +116,13 @@ def library(path: str | None = None):
         lib.la_gate_norm_apply.argtypes = [i64, i64, i64, i32, vp, ctypes.POINTER(la_gate_norm),
                                            vp, vp]
         lib.la_gate_norm_apply.restype = ctypes.c_int
+        lib.la_prefill_state_workspace_bytes.argtypes = [ctypes.POINTER(la_desc)]
+        lib.la_prefill_state_workspace_bytes.restype = sz
+        lib.la_prefill_state.argtypes = [ctypes.POINTER(la_desc), vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.la_prefill_state.restype = ctypes.c_int
+        lib.la_state_fold.argtypes = [i64, i64, i64, i64, vp, ctypes.POINTER(ctypes.c_int64), vp,
+                                      vp, vp, vp]
+        lib.la_state_fold.restype = ctypes.c_int
         lib.la_decode_step.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp]
         lib.la_decode_step.restype = ctypes.c_int
         lib.la_workspace_status.argtypes = [vp, vp]
@@ -196,6 +203,27 @@ def la_gate_norm_apply(T: int, H: int, d: int, dtype: int, o: int, gn: la_gate_n
     return int(library().la_gate_norm_apply(T, H, d, dtype, o or None,
                                             None if gn is None else ctypes.byref(gn), y or None,
                                             stream or None))
+
+
+def la_prefill_state_workspace_bytes(desc: la_desc) -> int:
+    return int(library().la_prefill_state_workspace_bytes(ctypes.byref(desc)))
+
+
+def la_prefill_state(desc: la_desc, k: int, v: int, slopes: int, state_in: int, state_out: int,
+                     workspace: int, workspace_bytes: int, stream: int) -> int:
+    return int(library().la_prefill_state(ctypes.byref(desc), k or None, v or None,
+                                          slopes or None, state_in or None, state_out or None,
+                                          workspace or None, workspace_bytes, stream or None))
+
+
+def la_state_fold(n_parts: int, BH: int, H: int, d: int, parts: int, lengths, slopes: int,
+                  state_in: int, state_out: int, stream: int) -> int:
+    """lengths: a sequence of n_parts host integers (or None)."""
+    arr = None
+    if lengths is not None:
+        arr = (ctypes.c_int64 * max(1, len(lengths)))(*[int(x) for x in lengths])
+    return int(library().la_state_fold(n_parts, BH, H, d, parts or None, arr, slopes or None,
+                                       state_in or None, state_out or None, stream or None))
 
 
 def la_workspace_status(workspace: int, stream: int) -> int:
@@ -438,4 +466,67 @@ def gate_norm(o: torch.Tensor, gate: torch.Tensor, gamma: torch.Tensor, *, eps: 
                             s.cuda_stream)
     if st != LA_OK:
         raise LaError(st, "la_gate_norm_apply")
+    return out
+
+
+def prefill_state(k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor, *,
+                  state_in: torch.Tensor | None = None, state_out: torch.Tensor | None = None,
+                  path: int = LA_PATH_AUTO, workspace: torch.Tensor | None = None,
+                  stream: torch.cuda.Stream | None = None,
+                  check: bool | None = None) -> torch.Tensor:
+    """state = prefill_state(k, v, slopes): the final fp32 state [B, H, d, d] of a prefill of
+    k, v [B, N, H, d] (bf16 or fp32, CUDA, contiguous) from state_in (or zero), without outputs:
+    lambda^N state_in + sum_t lambda^(N-1-t) k_t^T v_t.  state_out may be state_in."""
+    if k.dim() != 4 or k.shape != v.shape or k.dtype != v.dtype or k.dtype not in _DT:
+        raise ValueError("k, v must share one [B, N, H, d] shape and dtype")
+    B, N, H, d = k.shape
+    if slopes.dtype != torch.float32 or slopes.shape != (H,):
+        raise ValueError("slopes must be float32[H]")
+    if state_in is not None and (state_in.dtype != torch.float32 or
+                                 tuple(state_in.shape) != (B, H, d, d)):
+        raise ValueError("state_in must be float32 [B, H, d, d]")
+    if state_out is None:
+        state_out = torch.empty((B, H, d, d), dtype=torch.float32, device=k.device)
+    desc = make_desc(B, N, H, d, k.dtype, 0, 0, path)
+    need = la_prefill_state_workspace_bytes(desc)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
+    ws_ptr = 0 if workspace is None else _cuda_ptr(workspace, "workspace")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    s = stream if stream is not None else torch.cuda.current_stream(k.device)
+    st = la_prefill_state(desc, _cuda_ptr(k, "k"), _cuda_ptr(v, "v"), _cuda_ptr(slopes, "slopes"),
+                          0 if state_in is None else _cuda_ptr(state_in, "state_in"),
+                          _cuda_ptr(state_out, "state_out"), ws_ptr, ws_bytes, s.cuda_stream)
+    if st != LA_OK:
+        raise LaError(st, "la_prefill_state")
+    _check_device_status(ws_ptr, s.cuda_stream, "la_prefill_state", check)
+    return state_out
+
+
+def state_fold(parts: torch.Tensor, lengths, slopes: torch.Tensor, *,
+               state_in: torch.Tensor | None = None, out: torch.Tensor | None = None,
+               stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """S = state_fold(parts, lengths, slopes): parts fp32 [n, B, H, d, d] (the local states of n
+    consecutive parts of lengths[j] tokens); returns the state after all n parts, starting from
+    state_in (fp32 [B, H, d, d], or zero): S <- lambda^lengths[j] S + parts[j] in order."""
+    if parts.dim() != 5 or parts.dtype != torch.float32:
+        raise ValueError("parts must be float32 [n_parts, B, H, d, d]")
+    n, B, H, d, _ = parts.shape
+    lengths = [int(x) for x in lengths]
+    if len(lengths) != n:
+        raise ValueError("lengths must have one entry per part")
+    if slopes.dtype != torch.float32 or slopes.shape != (H,):
+        raise ValueError("slopes must be float32[H]")
+    if state_in is not None and (state_in.dtype != torch.float32 or
+                                 tuple(state_in.shape) != (B, H, d, d)):
+        raise ValueError("state_in must be float32 [B, H, d, d]")
+    if out is None:
+        out = torch.empty((B, H, d, d), dtype=torch.float32, device=parts.device)
+    s = stream if stream is not None else torch.cuda.current_stream(parts.device)
+    st = la_state_fold(n, B * H, H, d, _cuda_ptr(parts, "parts") if n > 0 else 0, lengths,
+                       _cuda_ptr(slopes, "slopes"),
+                       0 if state_in is None else _cuda_ptr(state_in, "state_in"),
+                       _cuda_ptr(out, "out"), s.cuda_stream)
+    if st != LA_OK:
+        raise LaError(st, "la_state_fold")
     return out

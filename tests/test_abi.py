@@ -51,7 +51,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert la.la_version() == 1001
+    assert la.la_version() == 1002
     for code in range(-10, 1):
         assert la.la_status_string(code) not in ("", "unknown status")
     assert la.la_status_string(-99) == "unknown status"
@@ -270,3 +270,54 @@ def test_gate_norm_apply_rejects_bad_arguments(lib):
     # y overlapping o without being o, or overlapping the gate
     assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, o, gn, o + 64, 0) == la.LA_ERR_ALIAS
     assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, o, gn, 0x800000, 0) == la.LA_ERR_ALIAS
+
+
+def test_prefill_state_rejects_bad_arguments(lib):
+    d = _desc(N=1000, H=4)
+    ps = la.la_prefill_state
+    assert ps(_desc(N=0), 0x1000, 0x2000, 0x3000, 0, 0x40000, 0, 0, 0) == la.LA_ERR_SHAPE
+    assert ps(_desc(dtype=5), 0x1000, 0x2000, 0x3000, 0, 0x40000, 0, 0, 0) == la.LA_ERR_DTYPE
+    assert ps(d, 0, 0x2000, 0x3000, 0, 0x40000, 0, 0, 0) == la.LA_ERR_NULL
+    assert ps(d, 0x1000, 0x2000, 0x3000, 0, 0, 0, 0, 0) == la.LA_ERR_NULL
+    assert ps(d, 0x1000, 0x2000, 0, 0, 0x40000, 0, 0, 0) == la.LA_ERR_NULL
+    assert ps(d, 0x1008, 0x2000, 0x3000, 0, 0x40000, 0, 0, 0) == la.LA_ERR_ALIGN
+    assert ps(d, 0x1000, 0x2000, 0x3000, 0x5008, 0x40000, 0, 0, 0) == la.LA_ERR_ALIGN
+    # k spans 1000 * 4 * 128 * 2 bytes from 0x100000: a state_out inside it overlaps
+    assert ps(d, 0x100000, 0x900000, 0x3000, 0, 0x100100, 0, 0, 0) == la.LA_ERR_ALIAS
+    # state_in and state_out partly overlapping (identical is the in-place form, allowed)
+    assert ps(d, 0x100000, 0x900000, 0x3000, 0x2000000, 0x2000100, 0, 0, 0) == la.LA_ERR_ALIAS
+
+
+def test_prefill_state_workspace(lib):
+    # tensor path: a header and two fp32 d x d partial slots per CTA; recurrent path: none
+    need = la.la_prefill_state_workspace_bytes(_desc(N=4096, H=64))
+    assert need >= 256 + 2 * 128 * 128 * 4 and (need - 256) % (2 * 128 * 128 * 4) == 0
+    assert la.la_prefill_state_workspace_bytes(_desc(dtype=la.LA_F32)) == 0
+    assert la.la_prefill_state_workspace_bytes(_desc(d=64)) == 0
+    assert la.la_prefill_state_workspace_bytes(_desc(N=0)) == 0
+
+
+def test_state_fold_rejects_bad_arguments(lib):
+    f = la.la_state_fold
+    ok = dict(parts=0x100000, lengths=[3, 4], slopes=0x3000, state_in=0, state_out=0x40000000)
+
+    def call(n=2, BH=8, H=4, d=128, **kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(n, BH, H, d, a["parts"], a["lengths"], a["slopes"], a["state_in"],
+                 a["state_out"], 0)
+
+    assert call(n=-1) == la.LA_ERR_SHAPE
+    assert call(n=257, lengths=[1] * 257) == la.LA_ERR_SHAPE
+    assert call(BH=6) == la.LA_ERR_SHAPE  # not a multiple of H
+    assert call(d=96) == la.LA_ERR_SHAPE
+    assert call(parts=0) == la.LA_ERR_NULL
+    assert call(lengths=None) == la.LA_ERR_NULL
+    assert call(slopes=0) == la.LA_ERR_NULL
+    assert call(state_out=0) == la.LA_ERR_NULL
+    assert call(lengths=[3, -1]) == la.LA_ERR_SHAPE
+    assert call(parts=0x100008) == la.LA_ERR_ALIGN
+    assert call(state_in=0x5004) == la.LA_ERR_ALIGN
+    # parts span 2 * 8 * 128 * 128 * 4 bytes: a state_out inside them overlaps
+    assert call(state_out=0x100000 + 4096) == la.LA_ERR_ALIAS
+    assert call(state_in=0x40000000 + 256) == la.LA_ERR_ALIAS
