@@ -212,6 +212,19 @@ def oracle_sample(w, seconds_target=15.0):
 # --------------------------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------------------------
+def cp_launches(B, N, H):
+    """Kernels of one context-parallel state step: the state pass, its combine kernel when a
+    range boundary falls inside a head (the split of la_state.cu for this GPU's SM count), and
+    the fold."""
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    nc = (N + 127) // 128
+    total = B * H * nc
+    g0 = max(1, min(sms, total))
+    width = (total + g0 - 1) // g0
+    grid = (total + width - 1) // width
+    return 2 + (1 if grid > 1 and width % nc else 0)
+
+
 def run_ours(args):
     from long_context_attention_la_b200 import build as labuild
     from long_context_attention_la_b200 import la
@@ -224,6 +237,11 @@ def run_ours(args):
     w = synth.WORKLOADS[args.workload] if vw is None else synth.Workload(
         vw.name, 1, vw.T, vw.H, vw.d, vw.dtype, vw.dist, vw.seed)
     B, N, H, d = w.B, w.N, w.H, w.d
+    if args.cp:
+        # context parallel: rank r holds tokens [r N/world, (r+1) N/world) of every sequence
+        if vw is not None or args.gate or args.gate_separate or N % world:
+            raise SystemExit("--cp takes a fixed-length workload whose N divides by the ranks")
+        N = N // world
     q, k, v = synth.draw_qkv(B, N, H, d, dist=w.dist, seed=w.seed + 1000 * rank, dtype=w.dtype,
                              device=dev)
     sl = synth.slopes(H, dev)
@@ -247,11 +265,22 @@ def run_ours(args):
         gamma = (1.0 + 0.1 * torch.randn((H, d), generator=gg, device=dev)).float()
         extra_in += [gate]
         epi = la.la_gate_norm(gate.data_ptr(), gamma.data_ptr(), 1e-6)
-    if vw is None and args.gate:
-        # the fused epilogue is an option of the packed entry point: B sequences of N tokens
+    if vw is None and (args.gate or args.cp):
+        # the fused epilogue and the initial state are options of the packed entry point: B
+        # sequences of N tokens
         n_states = B
         cu = torch.arange(0, B * N + 1, N, dtype=torch.int64, device=dev)
         sin = None
+        if args.cp:
+            # the incoming state of this rank's part, folded from the gathered part states
+            sin = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+            h_loc = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+            h_all = (torch.empty(world, B, H, d, d, dtype=torch.float32, device=dev)
+                     if world > 1 else h_loc.unsqueeze(0))
+            sdesc = la.make_desc(B, N, H, d, w.dtype)
+            s_ws_bytes = la.la_prefill_state_workspace_bytes(sdesc)
+            s_ws = torch.empty(max(s_ws_bytes, 256), dtype=torch.uint8, device=dev)
+            part_lengths = [N] * world
         st = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
         desc = la.la_varlen_desc(B * N, B, H, d, la.LA_BF16, 0, 0, la.LA_PATH_AUTO)
         ws_bytes = la.la_prefill_varlen_workspace_bytes(desc)
@@ -302,7 +331,20 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
 
-    packed = vw is not None or args.gate
+    packed = vw is not None or args.gate or args.cp
+
+    def cp_state_call():
+        # local state of this rank's part, all ranks' states, the fold of those before it
+        rc = la.la_prefill_state(sdesc, k.data_ptr(), v.data_ptr(), sl.data_ptr(), 0,
+                                 h_loc.data_ptr(), s_ws.data_ptr(), s_ws_bytes, sp)
+        if rc != la.LA_OK:
+            raise la.LaError(rc, "la_prefill_state")
+        if world > 1:
+            torch.distributed.all_gather_into_tensor(h_all, h_loc)
+        rc = la.la_state_fold(rank, B * H, H, d, h_all.data_ptr() if rank > 0 else 0,
+                              part_lengths[:rank], sl.data_ptr(), 0, sin.data_ptr(), sp)
+        if rc != la.LA_OK:
+            raise la.LaError(rc, "la_state_fold")
 
     def prefill_call():
         if not packed:
@@ -345,6 +387,8 @@ def run_ours(args):
     for _ in range(args.warmup):
         if qk is not None:
             qk_call()
+        if args.cp:
+            cp_state_call()
         prefill_call()
         if sep is not None:
             sep_call()
@@ -355,9 +399,7 @@ def run_ours(args):
         raise la.LaError(st_rc, "device status after warm-up")
 
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(5)) for _ in range(K)]
     t_all0 = torch.cuda.Event(enable_timing=True)
     t_all1 = torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -369,6 +411,9 @@ def run_ours(args):
             if qk is not None:
                 qk_call()
             ev[i][0].record(stream)
+            if args.cp:
+                cp_state_call()
+            ev[i][4].record(stream)
             prefill_call()
             if sep is not None:
                 sep_call()
@@ -379,9 +424,10 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
     barrier(world)
     total_ms = t_all0.elapsed_time(t_all1)
-    pre_ms = sum(a.elapsed_time(b) for a, b, _, _ in ev) / K
-    dec_ms = sum(b.elapsed_time(c) for _, b, c, _ in ev) / K
-    qk_ms = sum(z.elapsed_time(a) for a, _, _, z in ev) / K
+    pre_ms = sum(e[4].elapsed_time(e[1]) for e in ev) / K
+    dec_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    qk_ms = sum(e[3].elapsed_time(e[0]) for e in ev) / K
+    cp_ms = sum(e[0].elapsed_time(e[4]) for e in ev) / K
     st_rc = la.la_workspace_status(ws.data_ptr(), sp)
     if st_rc != la.LA_OK:
         raise la.LaError(st_rc, "device status after the timed steps")
@@ -390,6 +436,8 @@ def run_ours(args):
     pre_ms_max = max_over_ranks(pre_ms, world)
     dec_ms_max = max_over_ranks(dec_ms, world)
     qk_ms_max = max_over_ranks(qk_ms, world)
+    cp_ms_max = max_over_ranks(cp_ms, world)
+    step_ms_max = max_over_ranks(cp_ms + pre_ms, world)  # the whole prefill of a part
 
     # ---- e2e: host buffers through the C ABI, copies inside the timed region ----
     e2e = None
@@ -429,6 +477,8 @@ def run_ours(args):
                 x.copy_(hx, non_blocking=True)
             if qk is not None:
                 qk_call()
+            if args.cp:
+                cp_state_call()
             prefill_call()
             if sep is not None:
                 sep_call()
@@ -449,13 +499,13 @@ def run_ours(args):
     if rank == 0:
         hbm_peak, tc_peak, peak_kind = load_peaks()
         tokens = B * N
-        tok_s = world * tokens / (pre_ms_max * 1e-3)
+        tok_s = world * tokens / ((step_ms_max if args.cp else pre_ms_max) * 1e-3)
         # algorithmic bytes of one prefill launch: read q, k, v and write o (bf16), write the
         # final states (and read the initial states of the packed workload)
         # (the separate norm + gate pass reads o and the gate and writes y: 3 more rows)
         pre_bytes = (4 + (1 if args.gate else 0) + (3 if args.gate_separate else 0)) * \
             B * N * H * d * 2 + \
-            n_states * H * d * d * 4 * (1 if vw is None else 2)
+            n_states * H * d * d * 4 * (1 if vw is None and not args.cp else 2)
         achieved = pre_bytes / (pre_ms_max * 1e-3) / 1e9
         canon = 4.0 * d * d * B * N * H  # recurrent-form flops
         executed = (4.0 * d * d + 4.0 * 128 * d) * B * N * H  # full 128 x 128 tiles
@@ -481,10 +531,15 @@ def run_ours(args):
                                                   if args.gate else "") +
                                    (", then the grouped RMSNorm + sigmoid gate pass"
                                     if args.gate_separate else "") +
+                                   (f", context parallel over {world} rank(s): {N} tokens per "
+                                    f"rank, state pass + all_gather + fold + prefill from the "
+                                    f"folded state" if args.cp else "") +
                                    f" + decode step B={Bd} H={Hd} d={dd} (fp32 state)",
-                       "global_batch": world * B, "seq_len": N, "parallelism": f"replicas{world}",
+                       "global_batch": world * B if not args.cp else B,
+                       "seq_len": N if not args.cp else N * world,
+                       "parallelism": f"replicas{world}" if not args.cp else f"cp{world}",
                        "l2": "inputs larger than L2 (no flush)"},
-            "prefill": {"ms": pre_ms_max, "tok_s": tok_s,
+            "prefill": {"ms": pre_ms_max, "tok_s": world * tokens / (pre_ms_max * 1e-3),
                         "tflops_canonical": world * canon / (pre_ms_max * 1e-3) / 1e12,
                         "tflops_executed_c128": world * executed / (pre_ms_max * 1e-3) / 1e12,
                         "hbm_gbs": achieved},
@@ -498,6 +553,12 @@ def run_ours(args):
                                      and not (args.gate or args.gate_separate) else None),
                          "algorithmic_bytes": pre_bytes,
                          "kernel": "chunked_prefill_kernel", "peak_kind": peak_kind},
+            "cp": None if not args.cp else {
+                "state_fold_gather_ms": cp_ms_max, "step_ms": step_ms_max,
+                # the state pass reads k and v of the part and writes the d x d states; the
+                # time also holds the gather and the fold
+                "state_step_hbm_gbs": (2 * B * N * H * d * 2 + B * H * d * d * 4) /
+                (cp_ms_max * 1e-3) / 1e9},
             "qk_norm_rope": None if qk is None else {
                 "ms": qk_ms_max,
                 # read q, k (raw) and write q_hat, k_hat: 4 * d * 2 bytes per token-head
@@ -507,8 +568,11 @@ def run_ours(args):
             "e2e": e2e,
             # per step: the prefill kernel (after the planning kernel for packed input) and the
             # decode kernel
+            # (context parallel: the state pass, its combine kernel when a head is split over
+            # CTAs, and the fold)
             "gpu_launches": ((3 if packed else 2) + (1 if qk is not None else 0) +
-                             (1 if sep is not None else 0)) * K,
+                             (1 if sep is not None else 0) +
+                             (cp_launches(B, N, H) if args.cp else 0)) * K,
         }
         print(json.dumps(line), flush=True)
     dist_teardown(world)
@@ -573,6 +637,9 @@ def main():
                     help="run the grouped RMSNorm + sigmoid gate as its own pass after the prefill")
     ap.add_argument("--gate", action="store_true",
                     help="fuse the grouped RMSNorm + sigmoid gate into the prefill's output")
+    ap.add_argument("--cp", action="store_true",
+                    help="context parallel: split each sequence over the ranks (state pass, "
+                         "all_gather of the part states, fold, prefill from the folded state)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer e2e leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     args = ap.parse_args()
