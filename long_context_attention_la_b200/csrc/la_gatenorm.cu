@@ -4,19 +4,22 @@
 // multiplied by sigmoid(Gate Projection) -> Output Projection) and §4.3 (group norm + sigmoid gate
 // run as one fused inference operator).  Per token t and head h (each head is one norm group):
 //     y = gamma[h] * o / sqrt(mean(o^2) + eps) * sigmoid(g)
-// Memory bound: read o and g, write y (3 rows of d per token-head).  One CTA per token; a row is
-// handled by d/8 threads of 16 bytes, the mean square is a shuffle reduction over them, and every
-// thread issues the loads of all its rows before using any.
+// Memory bound: read o and g, write y (3 rows of d per token-head).  A row is handled by d/8
+// threads of 16 bytes and its mean square is a shuffle reduction over them; o and g reach those
+// threads through a shared-memory ring filled two items ahead by per-thread cp.async copies.
 #include <cuda_bf16.h>
 
 #include <cstdint>
 
+#include <algorithm>
+
 #include "la_internal.h"
+#include "la_sm100.cuh"
 
 namespace la {
 namespace {
 
-constexpr int kGnThreads = 256;
+constexpr int kGnThreads = 512;
 
 template <typename T>
 struct Io;
@@ -59,91 +62,166 @@ struct Io<float> {  // 8 values = two 16-byte loads
   }
 };
 
-// bf16 rows stay packed (one uint4 per 8 values) between load and use, so a thread keeps all its
-// loads in flight with few registers; fp32 rows take two float4 each.
+// sigmoid(x).  bf16 output: (1 + tanh(x/2)) / 2 with one MUFU tanh (relative error about 2^-11,
+// far below the bf16 rounding of y).  fp32 output: 1 / (1 + e^-x) with the approximate
+// exponential and divide (a few ulp); an IEEE divide here would cost more issue slots than
+// the memory system leaves per element.
 template <typename T>
-struct Raw;
+struct Sigmoid;
 template <>
-struct Raw<__nv_bfloat16> {
-  uint4 w;
-  __device__ __forceinline__ void load(const __nv_bfloat16* src) {
-    w = __ldcs(reinterpret_cast<const uint4*>(src));
+struct Sigmoid<__nv_bfloat16> {
+  static __device__ __forceinline__ float f(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return fmaf(0.5f, t, 0.5f);
   }
-  __device__ __forceinline__ void zero() { w = make_uint4(0u, 0u, 0u, 0u); }
-  __device__ __forceinline__ void unpack(float (&x)[8]) const { Io<__nv_bfloat16>::unpack(w, x); }
 };
 template <>
-struct Raw<float> {
-  float4 a, b;
-  __device__ __forceinline__ void load(const float* src) {
-    a = __ldcs(reinterpret_cast<const float4*>(src));
-    b = __ldcs(reinterpret_cast<const float4*>(src) + 1);
-  }
-  __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
-  __device__ __forceinline__ void unpack(float (&x)[8]) const {
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-  }
+struct Sigmoid<float> {
+  static __device__ __forceinline__ float f(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 };
 
+// Pieces: a thread's 8 consecutive values of a row are kPieces 16-byte pieces (bf16 1, fp32 2).
+template <typename T>
+struct Piece {
+  static constexpr int kPieces = sizeof(T) / 2;
+  static constexpr int kElems = 16 / sizeof(T);  // elements per piece
+  static __device__ __forceinline__ void unpack(const uint4 (&w)[kPieces], float (&x)[8]);
+};
+template <>
+__device__ __forceinline__ void Piece<__nv_bfloat16>::unpack(const uint4 (&w)[1], float (&x)[8]) {
+  Io<__nv_bfloat16>::unpack(w[0], x);
+}
+template <>
+__device__ __forceinline__ void Piece<float>::unpack(const uint4 (&w)[2], float (&x)[8]) {
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    x[4 * p] = __uint_as_float(w[p].x);
+    x[4 * p + 1] = __uint_as_float(w[p].y);
+    x[4 * p + 2] = __uint_as_float(w[p].z);
+    x[4 * p + 3] = __uint_as_float(w[p].w);
+  }
+}
+
+// Work item: kSweeps x ROWS rows (head groups) of one token; a CTA takes a contiguous range of
+// items.  The loads of each item go through a kStages-deep ring in shared memory with per-thread
+// cp.async copies, two items ahead of the one being finished, so the bytes in flight are held by
+// shared memory rather than registers.  Every thread reads back only the pieces it copied itself
+// (slot [stage][piece][thread]), so the ring needs no block barrier.
+constexpr int kStages = 3;
+constexpr int kSweeps = 2;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(kGnThreads) gate_norm_kernel(const GateNormArgs a) {
-  constexpr int TPR = D / 8;                // threads per row
-  constexpr int ROWS = kGnThreads / TPR;    // rows per sweep
-  constexpr int kSweeps = 4;                // sweeps whose loads are issued together
-  const int lt = threadIdx.x % TPR;
-  const int64_t t = blockIdx.x;
+__global__ void __launch_bounds__(kGnThreads, 2) gate_norm_kernel(const GateNormArgs a,
+                                                               int64_t items_per_cta) {
+  constexpr int TPR = D / 8;              // threads per row
+  constexpr int ROWS = kGnThreads / TPR;  // rows per sweep
+  constexpr int KP = Piece<T>::kPieces;
+  constexpr int kPerItem = 2 * kSweeps * KP;  // o and g pieces per thread and item
+  extern __shared__ uint4 ring[];             // [kStages][kPerItem][kGnThreads]
+  const int tid = threadIdx.x;
+  const int lt = tid % TPR;
+  const int64_t per_token = (a.H + ROWS * kSweeps - 1) / (ROWS * kSweeps);
+  const int64_t items = a.T * per_token;
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * items_per_cta;
+  const int64_t i1 = min(i0 + items_per_cta, items);
   const T* o = static_cast<const T*>(a.o);
   const T* g = static_cast<const T*>(a.gate);
   T* y = static_cast<T*>(a.y);
-  for (int64_t hb = 0; hb < a.H; hb += ROWS * kSweeps) {  // uniform trip count across the CTA
-    Raw<T> ro[kSweeps], rg[kSweeps];
+
+  auto slot = [&](int stage, int piece) -> uint4* {
+    return ring + (stage * kPerItem + piece) * kGnThreads + tid;
+  };
+  // copy the pieces of item `it` into ring stage `st` (one commit group, empty past the range)
+  auto issue = [&](int64_t it, int st) {
+    if (it < i1) {
+      const int64_t t = it / per_token;
+      const int64_t hb = (it - t * per_token) * (ROWS * kSweeps);
 #pragma unroll
-    for (int j = 0; j < kSweeps; ++j) {
-      const int64_t h = hb + j * ROWS + threadIdx.x / TPR;
-      if (h < a.H) {
-        const int64_t off = (t * a.H + h) * D + lt * 8;
-        ro[j].load(o + off);
-        rg[j].load(g + off);
-      } else {
-        ro[j].zero();
-        rg[j].zero();
+      for (int j = 0; j < kSweeps; ++j) {
+        const int64_t h = hb + j * ROWS + tid / TPR;
+        const bool valid = h < a.H;
+        const int64_t off = valid ? (t * a.H + h) * D + lt * 8 : 0;
+#pragma unroll
+        for (int p = 0; p < KP; ++p) {
+          cp_async16(slot(st, j * KP + p), o + off + p * Piece<T>::kElems, valid);
+          cp_async16(slot(st, (kSweeps + j) * KP + p), g + off + p * Piece<T>::kElems, valid);
+        }
       }
     }
+    cp_async_commit();
+  };
+
+  issue(i0, 0);
+  issue(i0 + 1, 1);
+  int st = 0;
+  for (int64_t it = i0; it < i1; ++it) {
+    issue(it + 2, st == 0 ? 2 : st - 1);  // the stage item it - 1 used
+    cp_async_wait<2>();                   // item it's group has landed
+    const int64_t t = it / per_token;
+    const int64_t hb = (it - t * per_token) * (ROWS * kSweeps);
 #pragma unroll
     for (int j = 0; j < kSweeps; ++j) {
-      const int64_t h = hb + j * ROWS + threadIdx.x / TPR;
+      const int64_t h = hb + j * ROWS + tid / TPR;
+      uint4 wo[KP], wg[KP];
+#pragma unroll
+      for (int p = 0; p < KP; ++p) {
+        wo[p] = *slot(st, j * KP + p);
+        wg[p] = *slot(st, (kSweeps + j) * KP + p);
+      }
       float xo[8];
-      ro[j].unpack(xo);
+      Piece<T>::unpack(wo, xo);
       float ss = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) ss = fmaf(xo[e], xo[e], ss);
 #pragma unroll
       for (int m = TPR / 2; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-      if (h < a.H) {
+      if (h < a.H) {  // uniform across a row's threads
         float xg[8];
-        rg[j].unpack(xg);
+        Piece<T>::unpack(wg, xg);
         const float rinv = rsqrtf(fmaf(ss, 1.f / D, a.eps));
-        const float* gam = a.gamma + h * D + lt * 8;
+        const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gamma + h * D + lt * 8));
+        const float4 g1 = __ldg(reinterpret_cast<const float4*>(a.gamma + h * D + lt * 8) + 1);
+        const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
         float out[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float sig = 1.f / (1.f + __expf(-xg[e]));
-          out[e] = __ldg(gam + e) * (xo[e] * rinv) * sig;
-        }
+        for (int e = 0; e < 8; ++e) out[e] = gm[e] * (xo[e] * rinv) * Sigmoid<T>::f(xg[e]);
         Io<T>::store(y + (t * a.H + h) * D + lt * 8, out);
       }
     }
+    st = st == kStages - 1 ? 0 : st + 1;
   }
+  cp_async_wait<0>();  // no copy outlives the CTA
+}
+
+template <typename T, int D>
+cudaError_t launch_dim(const GateNormArgs& a, cudaStream_t stream) {
+  constexpr int ROWS = kGnThreads / (D / 8);
+  constexpr size_t kSmem = size_t(kStages) * 2 * kSweeps * Piece<T>::kPieces * kGnThreads * 16;
+  static bool attr_set[64] = {false};
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    e = cudaFuncSetAttribute(gate_norm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmem));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int64_t per_token = (a.H + ROWS * kSweeps - 1) / (ROWS * kSweeps);
+  const int64_t items = a.T * per_token;
+  const int64_t resident = kSmem <= 100 * 1024 ? 2 : 1;  // CTAs per SM that the ring allows
+  const int64_t grid0 = std::max<int64_t>(1, std::min<int64_t>(items, resident * sms));
+  const int64_t per_cta = (items + grid0 - 1) / grid0;
+  const int64_t grid = (items + per_cta - 1) / per_cta;
+  gate_norm_kernel<T, D><<<static_cast<unsigned>(grid), kGnThreads, kSmem, stream>>>(a, per_cta);
+  return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t launch_typed(const GateNormArgs& a, cudaStream_t stream) {
-  if (a.d == 64)
-    gate_norm_kernel<T, 64><<<static_cast<unsigned>(a.T), kGnThreads, 0, stream>>>(a);
-  else
-    gate_norm_kernel<T, 128><<<static_cast<unsigned>(a.T), kGnThreads, 0, stream>>>(a);
-  return cudaGetLastError();
+  return a.d == 64 ? launch_dim<T, 64>(a, stream) : launch_dim<T, 128>(a, stream);
 }
 
 }  // namespace

@@ -9,9 +9,10 @@
 //     a = pos_t * theta^(-2i/r), i < r/2 (rotate-half pairs); dims >= r pass through.
 //
 // Memory bound: one pass over q and k (read 2 rows, write 2 rows of d bf16 per token-head).  A row
-// is handled by d/8 consecutive threads, 16 bytes each, so a warp reads whole rows; the mean
-// square is a shuffle reduction over the row's threads and each rotary pair's partner value comes
-// from the thread r/16 positions away.  The angle pos * w_i is formed and reduced modulo 2 pi in
+// is handled by d/16 consecutive threads with two 16-byte pieces each, chosen so that both
+// members of every rotary pair sit in one thread (no exchange between threads), staged through
+// a shared-memory ring by per-thread cp.async copies; the mean square is a shuffle reduction over
+// the row's threads.  The angle pos * w_i is formed and reduced modulo 2 pi in
 // double precision (positions reach 2^18 and more, where a float angle would be off by ~0.03 rad),
 // then sin and cos are taken in float, once per token and frequency.
 #include <cuda_bf16.h>
@@ -21,11 +22,12 @@
 #include <cstdint>
 
 #include "la_internal.h"
+#include "la_sm100.cuh"
 
 namespace la {
 namespace {
 
-constexpr int kQkThreads = 256;
+constexpr int kQkThreads = 512;
 
 // two floats -> bf16x2 (round to nearest even), lo in the low half
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -34,136 +36,189 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return l | (u << 16);
 }
 
-// Each CTA takes two tokens and issues the loads of both tokens' 2H rows before using any (enough
-// bytes in flight per SM to stream), computes each token's r/2 rotation angles once
-// (double-precision angle and reduction, float sin/cos) into shared memory, then sweeps the rows
-// ROWS at a time.
-template <int D>
-__global__ void __launch_bounds__(kQkThreads) qk_norm_rope_kernel(const QkNormRopeArgs a) {
-  constexpr int TPR = D / 8;                   // threads per row
-  constexpr int ROWS = kQkThreads / TPR;       // rows per sweep step
-  constexpr int kBatch = 8;                    // sweeps per token held in registers
-  __shared__ float cs_sh[2][64], sn_sh[2][64];
-  const int lt = threadIdx.x % TPR;            // position of this thread in its row
-  const int64_t rows = 2 * a.H;                // q heads, then k heads
-  const int half = a.rotary_dim / 2;
+// Work item: ROWS x kBatch rows of one token (q heads first, then k heads); a CTA takes a
+// contiguous range of items.  A row is handled by D/16 threads, each holding two 16-byte pieces
+// (8 dims each) that are r/2 dims apart inside the rotary span (so both members of every
+// rotate-half pair sit in one thread) and (D - r)/2 dims apart beyond it; a warp's copies still
+// cover whole 32-byte sectors.  Row loads go through a kStages-deep shared-memory ring filled two
+// items ahead with per-thread cp.async copies (each thread reads back only its own pieces), so
+// the bytes in flight are held by shared memory rather than registers.  Every warp computes the
+// rotation angles of its item's token itself (all of a warp's rows belong to one token) into a
+// table of its own, so no block barrier is needed anywhere: a barrier per item made every warp
+// wait for the slowest warp's copies.
+constexpr int kStages = 3;
+constexpr int kBatch = 2;  // sweeps of ROWS rows per item
 
-  auto load_rows = [&](int64_t t, int64_t rb, uint4 (&raw)[kBatch]) {
+template <int D>
+__global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNormRopeArgs a,
+                                                                  int64_t items_per_cta) {
+  constexpr int TPR = D / 16;                  // threads per row
+  constexpr int ROWS = kQkThreads / TPR;       // rows per sweep
+  extern __shared__ uint4 ring[];              // [kStages][kBatch][2][kQkThreads]
+  __shared__ __align__(16) float cs_sh[kQkThreads / 32][64];  // per warp: cos, sin of the token
+  __shared__ __align__(16) float sn_sh[kQkThreads / 32][64];
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int u = tid % TPR;                     // position of this thread in its row
+  const int64_t rows = 2 * a.H;                // q heads, then k heads
+  const int64_t per_token = (rows + ROWS * kBatch - 1) / (ROWS * kBatch);
+  const int64_t items = a.T * per_token;
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * items_per_cta;
+  const int64_t i1 = min(i0 + items_per_cta, items);
+  const int half = a.rotary_dim / 2;
+  const int rot_threads = a.rotary_dim / 16;   // threads holding rotary pairs
+  const bool rotary = u < rot_threads;
+  // the thread's two pieces (8-dim units): (u, u + r/16) in the rotary span, else
+  // (r/8 + m, r/8 + m + (D - r)/16) with m = u - r/16
+  const int pa = rotary ? u : a.rotary_dim / 8 + (u - rot_threads);
+  const int pb = rotary ? u + rot_threads : pa + (D - a.rotary_dim) / 16;
+
+  auto slot = [&](int stage, int j, int w) -> uint4* {
+    return ring + ((stage * kBatch + j) * 2 + w) * kQkThreads + tid;
+  };
+  auto issue = [&](int64_t it, int st) {
+    if (it < i1) {
+      const int64_t t = it / per_token;
+      const int64_t rb = (it - t * per_token) * (ROWS * kBatch);
 #pragma unroll
-    for (int j = 0; j < kBatch; ++j) {
-      const int64_t row = rb + j * ROWS + threadIdx.x / TPR;
-      raw[j] = make_uint4(0u, 0u, 0u, 0u);
-      if (t < a.T && row < rows) {
+      for (int j = 0; j < kBatch; ++j) {
+        const int64_t row = rb + j * ROWS + tid / TPR;
+        const bool valid = row < rows;
         const bool is_k = row >= a.H;
         const int64_t h = is_k ? row - a.H : row;
         const __nv_bfloat16* src =
-            (is_k ? a.k : a.q) + t * (is_k ? a.k_stride : a.q_stride) + h * D + lt * 8;
-        raw[j] = __ldcs(reinterpret_cast<const uint4*>(src));
+            valid ? (is_k ? a.k : a.q) + t * (is_k ? a.k_stride : a.q_stride) + h * D : a.q;
+        cp_async16(slot(st, j, 0), valid ? src + pa * 8 : src, valid);
+        cp_async16(slot(st, j, 1), valid ? src + pb * 8 : src, valid);
       }
     }
+    cp_async_commit();
   };
-  auto angles = [&](int64_t t, int buf) {
-    if (t < a.T && threadIdx.x < half) {
-      constexpr double kTwoPi = 6.283185307179586476925286766559;
-      constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
-      double ang = static_cast<double>(a.positions[t]) * a.inv_freq[threadIdx.x];
+  // cos / sin of token t into this warp's table, frequency f by lane f % 32
+  auto angles = [&](int64_t t) {
+    constexpr double kTwoPi = 6.283185307179586476925286766559;
+    constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+    const double pos = static_cast<double>(a.positions[t]);
+    for (int f = lane; f < half; f += 32) {
+      double ang = pos * a.inv_freq[f];
       ang -= kTwoPi * rint(ang * kInvTwoPi);
       float sn, cs;
       sincosf(static_cast<float>(ang), &sn, &cs);
-      cs_sh[buf][threadIdx.x] = cs;
-      sn_sh[buf][threadIdx.x] = sn;
+      cs_sh[warp][f] = cs;
+      sn_sh[warp][f] = sn;
     }
   };
+  auto unpack = [](const uint4& w, float (&x)[8]) {
+    const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[2 * e] = __uint_as_float(v[e] << 16);
+      x[2 * e + 1] = __uint_as_float(v[e] & 0xffff0000u);
+    }
+  };
+  auto pack = [](const float (&y)[8]) {
+    uint4 w;
+    w.x = pack2(y[0], y[1]);
+    w.y = pack2(y[2], y[3]);
+    w.z = pack2(y[4], y[5]);
+    w.w = pack2(y[6], y[7]);
+    return w;
+  };
 
-  const int half_threads = a.rotary_dim / 16;  // threads per half of the rotary dims
-  const bool rotary = lt < 2 * half_threads;
-  const bool first = lt < half_threads;
-  const int lane = threadIdx.x & 31;
-  const int partner_lane = rotary ? (first ? lane + half_threads : lane - half_threads) : lane;
-  const int i0 = (first ? lt : lt - half_threads) * 8;  // frequency index of element 0
-
-  // normalise + rotate the rows held in raw (sweeps rb .. rb + kBatch - 1 of token t)
-  auto finish = [&](int64_t t, int64_t rb, const uint4 (&raw)[kBatch], int buf) {
+  issue(i0, 0);
+  issue(i0 + 1, 1);
+  int st = 0;
+  for (int64_t it = i0; it < i1; ++it) {
+    issue(it + 2, st == 0 ? 2 : st - 1);  // the stage item it - 1 used
+    const int64_t t = it / per_token;
+    __syncwarp();                         // the warp is done reading the previous token's table
+    angles(t);
+    __syncwarp();                         // ... and this token's table is written
+    cp_async_wait<2>();                   // item it's rows have landed (this thread's pieces)
+    const int64_t rb = (it - t * per_token) * (ROWS * kBatch);
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
-      const int64_t row = rb + j * ROWS + threadIdx.x / TPR;
+      const int64_t row = rb + j * ROWS + tid / TPR;
       const bool valid = row < rows;  // uniform across a row's threads
       const bool is_k = row >= a.H;
       const int64_t h = is_k ? row - a.H : row;
-      const uint32_t u[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
-      float x[8];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        x[2 * e] = __uint_as_float(u[e] << 16);
-        x[2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
-      }
+      float xa[8], xb[8];
+      unpack(*slot(st, j, 0), xa);
+      unpack(*slot(st, j, 1), xb);
       // mean square over the row: reduce across the TPR threads of the row (aligned groups)
       float ss = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+      for (int e = 0; e < 8; ++e) ss = fmaf(xb[e], xb[e], fmaf(xa[e], xa[e], ss));
 #pragma unroll
       for (int o = TPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       const float rinv = rsqrtf(fmaf(ss, 1.f / D, a.eps));
-      const float* gam = (is_k ? a.gamma_k : a.gamma_q) + lt * 8;
-      float y[8];
+      const float* gam = is_k ? a.gamma_k : a.gamma_q;
+      const float4 ga0 = __ldg(reinterpret_cast<const float4*>(gam + pa * 8));
+      const float4 ga1 = __ldg(reinterpret_cast<const float4*>(gam + pa * 8) + 1);
+      const float4 gb0 = __ldg(reinterpret_cast<const float4*>(gam + pb * 8));
+      const float4 gb1 = __ldg(reinterpret_cast<const float4*>(gam + pb * 8) + 1);
+      const float gma[8] = {ga0.x, ga0.y, ga0.z, ga0.w, ga1.x, ga1.y, ga1.z, ga1.w};
+      const float gmb[8] = {gb0.x, gb0.y, gb0.z, gb0.w, gb1.x, gb1.y, gb1.z, gb1.w};
+      float ya[8], yb[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = __ldg(gam + e) * (x[e] * rinv);
-      // rotate-half over the first r dims: the partner of element j is j +- r/2, held by the
-      // thread r/16 positions away in the same row
-      float pv[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) pv[e] = __shfl_sync(0xffffffffu, y[e], partner_lane);
+      for (int e = 0; e < 8; ++e) {
+        ya[e] = gma[e] * (xa[e] * rinv);
+        yb[e] = gmb[e] * (xb[e] * rinv);
+      }
       if (rotary) {
+        // rotate-half: dims (8 pa + e, 8 pa + e + r/2) with frequency index 8 pa + e
+        const float4* c4 = reinterpret_cast<const float4*>(&cs_sh[warp][pa * 8]);
+        const float4* s4 = reinterpret_cast<const float4*>(&sn_sh[warp][pa * 8]);
+        const float4 c0 = c4[0], c1 = c4[1], s0 = s4[0], s1 = s4[1];
+        const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float cs = cs_sh[buf][i0 + e], sn = sn_sh[buf][i0 + e];
-          y[e] = first ? fmaf(y[e], cs, -pv[e] * sn) : fmaf(y[e], cs, pv[e] * sn);
+          const float y0 = ya[e], y1 = yb[e];
+          ya[e] = fmaf(y0, cs[e], -y1 * sn[e]);
+          yb[e] = fmaf(y1, cs[e], y0 * sn[e]);
         }
       }
       if (valid) {
-        __nv_bfloat16* dst = (is_k ? a.k_out : a.q_out) + (t * a.H + h) * D + lt * 8;
-        uint4 w;
-        w.x = pack2(y[0], y[1]);
-        w.y = pack2(y[2], y[3]);
-        w.z = pack2(y[4], y[5]);
-        w.w = pack2(y[6], y[7]);
-        __stcs(reinterpret_cast<uint4*>(dst), w);
+        __nv_bfloat16* dst = (is_k ? a.k_out : a.q_out) + (t * a.H + h) * D;
+        __stcs(reinterpret_cast<uint4*>(dst + pa * 8), pack(ya));
+        __stcs(reinterpret_cast<uint4*>(dst + pb * 8), pack(yb));
       }
     }
-  };
+    st = st == kStages - 1 ? 0 : st + 1;
+  }
+  cp_async_wait<0>();  // no copy outlives the CTA
+}
 
-  // two tokens per CTA, all of their row loads issued before any is used
-  const int64_t t0 = 2 * static_cast<int64_t>(blockIdx.x), t1 = t0 + 1;
-  uint4 ra[kBatch], rb_[kBatch];
-  load_rows(t0, 0, ra);
-  load_rows(t1, 0, rb_);
-  angles(t0, 0);
-  angles(t1, 1);
-  __syncthreads();
-  finish(t0, 0, ra, 0);
-  for (int64_t rb = ROWS * kBatch; rb < rows; rb += ROWS * kBatch) {  // H > 64: more sweeps
-    load_rows(t0, rb, ra);
-    finish(t0, rb, ra, 0);
+template <int D>
+cudaError_t launch_dim(const QkNormRopeArgs& a, cudaStream_t stream) {
+  constexpr int ROWS = kQkThreads / (D / 16);
+  constexpr size_t kSmem = size_t(kStages) * kBatch * 2 * kQkThreads * 16;  // 96 KiB: 2 per SM
+  static bool attr_set[64] = {false};
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    e = cudaFuncSetAttribute(qk_norm_rope_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmem));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
   }
-  if (t1 < a.T) {  // uniform across the CTA
-    finish(t1, 0, rb_, 1);
-    for (int64_t rb = ROWS * kBatch; rb < rows; rb += ROWS * kBatch) {
-      load_rows(t1, rb, rb_);
-      finish(t1, rb, rb_, 1);
-    }
-  }
+  const int64_t per_token = (2 * a.H + ROWS * kBatch - 1) / (ROWS * kBatch);
+  const int64_t items = a.T * per_token;
+  const int64_t grid0 = std::max<int64_t>(1, std::min<int64_t>(items, 2 * int64_t(sms)));
+  const int64_t per_cta = (items + grid0 - 1) / grid0;
+  const int64_t grid = (items + per_cta - 1) / per_cta;
+  qk_norm_rope_kernel<D><<<static_cast<unsigned>(grid), kQkThreads, kSmem, stream>>>(a, per_cta);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_qk_norm_rope(const QkNormRopeArgs& a, cudaStream_t stream) {
   if (a.T == 0) return cudaSuccess;
-  const int64_t grid = (a.T + 1) / 2;  // two tokens per CTA
-  if (a.d == 64)
-    qk_norm_rope_kernel<64><<<static_cast<unsigned>(grid), kQkThreads, 0, stream>>>(a);
-  else
-    qk_norm_rope_kernel<128><<<static_cast<unsigned>(grid), kQkThreads, 0, stream>>>(a);
-  return cudaGetLastError();
+  return a.d == 64 ? launch_dim<64>(a, stream) : launch_dim<128>(a, stream);
 }
 
 }  // namespace la

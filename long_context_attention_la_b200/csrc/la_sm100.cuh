@@ -201,6 +201,23 @@ __device__ __forceinline__ uint64_t policy_evict_normal() {
   return p;
 }
 
+// Per-thread asynchronous 16-byte copy global -> shared (cp.async, L1 bypassed).  With
+// valid == false nothing is read and the 16 bytes are zero-filled (src must still be a valid
+// address).  Completion is tracked per thread by commit groups; the wait is a hardware wait.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
+               "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Waits until at most `kPending` of this thread's most recent commit groups are incomplete.
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+
 // ---------------------------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation tensor core
 // ---------------------------------------------------------------------------------------------
