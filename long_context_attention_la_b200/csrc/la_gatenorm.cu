@@ -25,8 +25,7 @@ template <typename T>
 struct Io;
 
 template <>
-struct Io<__nv_bfloat16> {  // 8 values = one 16-byte load
-  using Vec = uint4;
+struct Io<__nv_bfloat16> {  // 8 values = one 16-byte piece
   static __device__ __forceinline__ void unpack(const uint4& w, float (&x)[8]) {
     const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -43,19 +42,10 @@ struct Io<__nv_bfloat16> {  // 8 values = one 16-byte load
     __stcs(reinterpret_cast<uint4*>(dst),
            make_uint4(pack2(y[0], y[1]), pack2(y[2], y[3]), pack2(y[4], y[5]), pack2(y[6], y[7])));
   }
-  static __device__ __forceinline__ void load(const __nv_bfloat16* src, float (&x)[8]) {
-    unpack(__ldcs(reinterpret_cast<const uint4*>(src)), x);
-  }
 };
 
 template <>
-struct Io<float> {  // 8 values = two 16-byte loads
-  static __device__ __forceinline__ void load(const float* src, float (&x)[8]) {
-    const float4 a = __ldcs(reinterpret_cast<const float4*>(src));
-    const float4 b = __ldcs(reinterpret_cast<const float4*>(src) + 1);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-  }
+struct Io<float> {  // 8 values = two 16-byte pieces
   static __device__ __forceinline__ void store(float* dst, const float (&y)[8]) {
     __stcs(reinterpret_cast<float4*>(dst), make_float4(y[0], y[1], y[2], y[3]));
     __stcs(reinterpret_cast<float4*>(dst) + 1, make_float4(y[4], y[5], y[6], y[7]));
