@@ -14,7 +14,7 @@
 // a shared-memory ring by per-thread cp.async copies; the mean square is a shuffle reduction over
 // the row's threads.  The angle pos * w_i is formed and reduced modulo 2 pi in
 // double precision (positions reach 2^18 and more, where a float angle would be off by ~0.03 rad),
-// then sin and cos are taken in float, once per token and frequency.
+// then sin and cos are taken in float, once per token and frequency by each warp.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -94,16 +94,17 @@ __global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNor
     }
     cp_async_commit();
   };
-  // cos / sin of token t into this warp's table, frequency f by lane f % 32
-  auto angles = [&](int64_t t) {
+  // cos / sin at position `pos` into this warp's table, frequency f by lane f % 32.  The angle is
+  // reduced to [-pi, pi] in fp64 first, where the fast sin/cos (absolute error about 2^-21) is
+  // far below the bf16 rounding of the output.
+  auto angles = [&](int64_t pos) {
     constexpr double kTwoPi = 6.283185307179586476925286766559;
     constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
-    const double pos = static_cast<double>(a.positions[t]);
     for (int f = lane; f < half; f += 32) {
-      double ang = pos * a.inv_freq[f];
+      double ang = static_cast<double>(pos) * a.inv_freq[f];
       ang -= kTwoPi * rint(ang * kInvTwoPi);
       float sn, cs;
-      sincosf(static_cast<float>(ang), &sn, &cs);
+      __sincosf(static_cast<float>(ang), &sn, &cs);
       cs_sh[warp][f] = cs;
       sn_sh[warp][f] = sn;
     }
@@ -128,11 +129,14 @@ __global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNor
   issue(i0, 0);
   issue(i0 + 1, 1);
   int st = 0;
+  int64_t pos = i0 < i1 ? a.positions[i0 / per_token] : 0;
   for (int64_t it = i0; it < i1; ++it) {
     issue(it + 2, st == 0 ? 2 : st - 1);  // the stage item it - 1 used
     const int64_t t = it / per_token;
+    // the next item's position, one item ahead of its use
+    const int64_t pos_next = it + 1 < i1 ? a.positions[(it + 1) / per_token] : 0;
     __syncwarp();                         // the warp is done reading the previous token's table
-    angles(t);
+    angles(pos);
     __syncwarp();                         // ... and this token's table is written
     cp_async_wait<2>();                   // item it's rows have landed (this thread's pieces)
     const int64_t rb = (it - t * per_token) * (ROWS * kBatch);
@@ -186,6 +190,7 @@ __global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNor
       }
     }
     st = st == kStages - 1 ? 0 : st + 1;
+    pos = pos_next;
   }
   cp_async_wait<0>();  // no copy outlives the CTA
 }
