@@ -108,3 +108,49 @@ def test_prefill_cp_gloo_ranks_match_sequential_oracle(tmp_path, cuts, with_stat
                                    rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(res[-1]["st"].numpy(), st_ref.reshape(B, H, d, d), rtol=1e-10,
                                atol=1e-12)
+
+
+def _one_rank_group():
+    store = dist.TCPStore("127.0.0.1", _free_port(), 1, True,
+                          timeout=datetime.timedelta(seconds=30))
+    dist.init_process_group("gloo", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=30))
+
+
+def test_prefill_cp_rejects_inconsistent_arguments():
+    """Shape and part-length errors are raised before any exchange on the rank that sees them."""
+    _one_rank_group()
+    try:
+        x = torch.zeros((B, 5, H, d))
+        sl = torch.from_numpy(SLOPES)
+        with pytest.raises(ValueError):
+            cp.prefill_cp(x, x, x, sl, part_lengths=[4], ops=OracleOps())   # this rank holds 5
+        with pytest.raises(ValueError):
+            cp.prefill_cp(x, x, x, sl, part_lengths=[5, 5], ops=OracleOps())  # one rank only
+        with pytest.raises(ValueError):
+            cp.prefill_cp(x, torch.zeros((B, 4, H, d)), x, sl, ops=OracleOps())
+        # a one-rank group is a plain prefill from the initial state
+        rng = np.random.default_rng(5)
+        q, k, v = (torch.from_numpy(rng.normal(size=(B, 5, H, d)).astype(np.float32))
+                   for _ in range(3))
+        out, st = cp.prefill_cp(q, k, v, sl, ops=OracleOps())
+        o_ref, st_ref = oracle.prefill(q.numpy(), k.numpy(), v.numpy(), SLOPES)
+        np.testing.assert_allclose(out.numpy(), o_ref.reshape(B, H, 5, d).transpose(0, 2, 1, 3),
+                                   rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(st.numpy(), st_ref.reshape(B, H, d, d), rtol=1e-12, atol=1e-12)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_product_modules_do_not_import_the_oracle():
+    """The oracle is test infrastructure: no module of the package imports it."""
+    import ast
+    import pathlib
+    pkg = pathlib.Path(cp.__file__).parent
+    for path in pkg.glob("*.py"):
+        tree = ast.parse(path.read_text())
+        for node in ast.walk(tree):
+            if isinstance(node, ast.Import):
+                assert all(not a.name.split(".")[0] == "oracle" for a in node.names), path
+            if isinstance(node, ast.ImportFrom):
+                assert (node.module or "").split(".")[0] != "oracle", path
