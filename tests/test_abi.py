@@ -321,3 +321,18 @@ def test_state_fold_rejects_bad_arguments(lib):
     # parts span 2 * 8 * 128 * 128 * 4 bytes: a state_out inside them overlaps
     assert call(state_out=0x100000 + 4096) == la.LA_ERR_ALIAS
     assert call(state_in=0x40000000 + 256) == la.LA_ERR_ALIAS
+
+
+@pytest.mark.parametrize("B,N,H", [(1, 262144, 64), (2, 32768, 64), (1, 4096, 64), (4, 300, 64),
+                                   (1, 5, 2), (3, 128, 3)])
+def test_prefill_state_workspace_follows_the_range_split(lib, B, N, H):
+    """The state pass cuts the B*H*ceil(N/128) chunk-loads into one contiguous range per CTA (at
+    most one CTA per SM, 148 when no device is visible) and keeps two partial-state slots per CTA
+    behind a 256-byte header."""
+    total = B * H * ((N + 127) // 128)
+    grid0 = max(1, min(148, total))
+    width = -(-total // grid0)
+    grid = -(-total // width)
+    need = la.la_prefill_state_workspace_bytes(_desc(B=B, N=N, H=H))
+    assert need == 256 + 2 * grid * 128 * 128 * 4
+    assert grid <= 148 and (grid - 1) * width < total <= grid * width
