@@ -180,6 +180,24 @@ def dist_teardown(world):
 # --------------------------------------------------------------------------------------------
 # CPU baseline: the fp64 oracle on the host cores, bounded sample
 # --------------------------------------------------------------------------------------------
+def host_cpu():
+    """(cores this process may run on, CPU model string) of the host."""
+    try:
+        n = len(os.sched_getaffinity(0))
+    except Exception:  # pragma: no cover
+        n = os.cpu_count()
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except Exception:  # pragma: no cover
+        pass
+    return n, model
+
+
 def oracle_sample(w, seconds_target=15.0):
     """Times the oracle on n_threads heads x n_tok tokens of the workload's distribution.
     Returns (tok/s scaled to the workload's all-heads token, cores, description)."""
@@ -282,12 +300,13 @@ def run_ours(args):
             s_ws = torch.empty(max(s_ws_bytes, 256), dtype=torch.uint8, device=dev)
             part_lengths = [N] * world
         st = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
-        desc = la.la_varlen_desc(B * N, B, H, d, la.LA_BF16, 0, 0, la.LA_PATH_AUTO)
+        desc = la.la_varlen_desc(B * N, B, H, d, la.LA_BF16, args.chunk, args.segments,
+                                 la.LA_PATH_AUTO)
         ws_bytes = la.la_prefill_varlen_workspace_bytes(desc)
     elif vw is None:
         n_states = B
         st = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
-        desc = la.make_desc(B, N, H, d, w.dtype)
+        desc = la.make_desc(B, N, H, d, w.dtype, chunk=args.chunk, segments=args.segments)
         ws_bytes = la.la_prefill_workspace_bytes(desc)
     else:
         lengths = synth.draw_seqlens(vw.T, vw.n_seqs, seed=vw.len_seed)
@@ -297,7 +316,8 @@ def run_ours(args):
                                 device=dev)
         st = torch.empty_like(sin)
         extra_in += [sin, cu]
-        desc = la.la_varlen_desc(vw.T, vw.n_seqs, H, d, la.LA_BF16, 0, 0, la.LA_PATH_AUTO)
+        desc = la.la_varlen_desc(vw.T, vw.n_seqs, H, d, la.LA_BF16, args.chunk, args.segments,
+                                 la.LA_PATH_AUTO)
         ws_bytes = la.la_prefill_varlen_workspace_bytes(desc)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
 
@@ -316,6 +336,8 @@ def run_ours(args):
         extra_in += [q_raw, k_raw]
 
     Bd, Hd, dd = DECODE["B"], DECODE["H"], DECODE["d"]
+    if args.no_decode:
+        Bd = 1  # placeholder tensors only; the decode call is skipped
     dstate = torch.randn(Bd, Hd, dd, dd, dtype=torch.float32, device=dev) * 0.05
     gdec = synth.decode_token_generator(4 + 1000 * rank, dev)
     n_mtp = max(1, args.mtp)
@@ -373,6 +395,8 @@ def run_ours(args):
             raise la.LaError(rc, "la_qk_norm_rope")
 
     def decode_call():
+        if args.no_decode:
+            return
         if n_mtp == 1:
             rc = la.la_decode_step(Bd, Hd, dd, la.LA_BF16, dq.data_ptr(), dk.data_ptr(),
                                    dv.data_ptr(), dsl.data_ptr(), dstate.data_ptr(),
@@ -470,9 +494,10 @@ def run_ours(args):
             q.copy_(hq, non_blocking=True)
             k.copy_(hk, non_blocking=True)
             v.copy_(hv, non_blocking=True)
-            dq.copy_(hdq, non_blocking=True)
-            dk.copy_(hdk, non_blocking=True)
-            dv.copy_(hdv, non_blocking=True)
+            if not args.no_decode:
+                dq.copy_(hdq, non_blocking=True)
+                dk.copy_(hdk, non_blocking=True)
+                dv.copy_(hdv, non_blocking=True)
             for x, hx in zip(extra_in, hextra):
                 x.copy_(hx, non_blocking=True)
             if qk is not None:
@@ -485,13 +510,16 @@ def run_ours(args):
             decode_call()
             hout.copy_(out, non_blocking=True)
             hst.copy_(st, non_blocking=True)
-            hdout.copy_(dout, non_blocking=True)
+            if not args.no_decode:
+                hdout.copy_(dout, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
-        bi = 3 * q.numel() * q.element_size() + 3 * dq.numel() * dq.element_size() + sum(
+        dec_io = 0 if args.no_decode else 1
+        bi = 3 * q.numel() * q.element_size() + dec_io * 3 * dq.numel() * dq.element_size() + sum(
             x.numel() * x.element_size() for x in extra_in)
-        bo = out.numel() * out.element_size() + st.numel() * 4 + dout.numel() * dout.element_size()
+        bo = out.numel() * out.element_size() + st.numel() * 4 + \
+            dec_io * dout.numel() * dout.element_size()
         e2e = {"value": world * B * N / (e2e_ms * 1e-3), "unit": "tok/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms,
                "steps": n_e2e}
@@ -510,13 +538,14 @@ def run_ours(args):
         canon = 4.0 * d * d * B * N * H  # recurrent-form flops
         executed = (4.0 * d * d + 4.0 * 128 * d) * B * N * H  # full 128 x 128 tiles
         dec_bytes = 2 * Bd * Hd * dd * dd * 4 + 4 * Bd * Hd * dd * 2 * n_mtp
-        dec_gbs = dec_bytes / (dec_ms_max * 1e-3) / 1e9
+        dec_gbs = dec_bytes / max(dec_ms_max * 1e-3, 1e-12) / 1e9
         cpu = None
         if world == 1 and not args.no_cpu:
             try:
                 v_cpu, cores, sample = oracle_sample(w)
+                n_aff, model = host_cpu()
                 cpu = {"value": v_cpu, "unit": "tok/s", "cores": cores, "kind": "oracle",
-                       "sample": sample}
+                       "sample": sample, "affinity_cores": n_aff, "cpu_model": model}
             except Exception as exc:  # pragma: no cover - reported, not fatal
                 cpu = {"value": None, "unit": "tok/s", "cores": None, "kind": "oracle",
                        "sample": f"failed: {exc}"}
@@ -534,7 +563,11 @@ def run_ours(args):
                                    (f", context parallel over {world} rank(s): {N} tokens per "
                                     f"rank, state pass + all_gather + fold + prefill from the "
                                     f"folded state" if args.cp else "") +
-                                   f" + decode step B={Bd} H={Hd} d={dd} (fp32 state)",
+                                   ("" if args.no_decode else
+                                    f" + decode step B={Bd} H={Hd} d={dd} (fp32 state)") +
+                                   (f", chunk C={args.chunk}" if args.chunk else "") +
+                                   (f", {args.segments} segments per sequence"
+                                    if args.segments else ""),
                        "global_batch": world * B if not args.cp else B,
                        "seq_len": N if not args.cp else N * world,
                        "parallelism": f"replicas{world}" if not args.cp else f"cp{world}",
@@ -543,10 +576,10 @@ def run_ours(args):
                         "tflops_canonical": world * canon / (pre_ms_max * 1e-3) / 1e12,
                         "tflops_executed_c128": world * executed / (pre_ms_max * 1e-3) / 1e12,
                         "hbm_gbs": achieved},
-            "decode": {"ms": dec_ms_max, "state_gbs": dec_gbs, "frac_of_measured": dec_gbs / hbm_peak,
-                       "frac_of_8tbs": dec_gbs / 8000.0,
-                       "tokens_per_step": n_mtp,
-                       "tok_s": world * Bd * n_mtp / (dec_ms_max * 1e-3)},
+            "decode": None if args.no_decode else {
+                "ms": dec_ms_max, "state_gbs": dec_gbs, "frac_of_measured": dec_gbs / hbm_peak,
+                "frac_of_8tbs": dec_gbs / 8000.0, "tokens_per_step": n_mtp,
+                "tok_s": world * Bd * n_mtp / (dec_ms_max * 1e-3)},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak,
                          "traffic": (measured_traffic() if args.workload == "prefill_32k"
@@ -570,7 +603,8 @@ def run_ours(args):
             # decode kernel
             # (context parallel: the state pass, its combine kernel when a head is split over
             # CTAs, and the fold)
-            "gpu_launches": ((3 if packed else 2) + (1 if qk is not None else 0) +
+            "gpu_launches": ((2 if packed else 1) + (0 if args.no_decode else 1) +
+                             (1 if qk is not None else 0) +
                              (1 if sep is not None else 0) +
                              (cp_launches(B, N, H) if args.cp else 0)) * K,
         }
@@ -614,7 +648,8 @@ def run_reference(args):
             "config": {"workload": f"{w.name}: B={w.B} N={w.N} H={w.H} d={w.d} (sampled)",
                        "global_batch": w.B, "seq_len": w.N, "parallelism": "host cores"},
             "cpu_baseline": {"value": tok_s, "unit": "tok/s", "cores": cores, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "affinity_cores": host_cpu()[0],
+                             "cpu_model": host_cpu()[1]},
             "e2e": {"value": tok_s, "unit": "tok/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -640,6 +675,12 @@ def main():
     ap.add_argument("--cp", action="store_true",
                     help="context parallel: split each sequence over the ranks (state pass, "
                          "all_gather of the part states, fold, prefill from the folded state)")
+    ap.add_argument("--chunk", type=int, default=0,
+                    help="chunk length C of the tensor-core prefill (0: the library's default)")
+    ap.add_argument("--segments", type=int, default=0,
+                    help="segments per sequence (0: the library's automatic plan)")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="time the prefill alone (no decode state on the device)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer e2e leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     args = ap.parse_args()

@@ -28,7 +28,8 @@
  *   - stream: a cudaStream_t passed as void*; NULL means the legacy default stream.  Calls are
  *     stream-ordered and asynchronous: a return of LA_OK means the work was enqueued.
  *   - Base pointers of q, k, v, out must be 16-byte aligned (tensor-memory-accelerator rule);
- *     otherwise LA_ERR_ALIGN.  out must not overlap q, k or v (LA_ERR_ALIAS).
+ *     otherwise LA_ERR_ALIGN.  out must not overlap q, k or v, and a state that an entry point
+ *     writes (state_out, state_inout) must not overlap q, k, v or out (LA_ERR_ALIAS).
  *   - Argument errors are reported synchronously before anything is enqueued.  Launch errors
  *     map to LA_ERR_CUDA.  Nothing in the library calls exit(), abort() or a device trap.
  *   - All sizes and index arithmetic are 64-bit.
@@ -206,7 +207,10 @@ la_status la_decode_multi(int64_t B, int64_t H, int64_t d, int64_t n_tok, int32_
  *     choice once B*H exceeds half the number of SMs); the fp32 / recurrent path needs no
  *     scratch at all.
  *   - First call on a device: it looks up the device address of the array (cudaGetSymbolAddress)
- *     with that device current and caches it; make that first call before any stream capture.
+ *     with that device current and caches it for that device's CUDA context; make that first
+ *     call before any stream capture.  If the context is destroyed and recreated (for example by
+ *     cudaDeviceReset), the next call sees a new context and looks the address up again, so make
+ *     that call outside stream capture too.
  *   - Sharing: all calls on a device use the same array, which keeps the previous call's
  *     contents; each call zeroes the parts that must start at zero.  Calls whose executions
  *     overlap on the GPU (different streams, or threads without ordering) race on the array and
@@ -214,7 +218,9 @@ la_status la_decode_multi(int64_t B, int64_t H, int64_t d, int64_t n_tok, int32_
  *   - Device status: a bounded device wait that gives up (it needs the GPU to be starved for
  *     seconds) leaves the outputs invalid and is recorded only in the array, which this call
  *     offers no way to read; callers that must observe it use la_prefill with their own
- *     workspace and la_workspace_status.
+ *     workspace and la_workspace_status.  For the same reason the call returns
+ *     LA_ERR_UNSUPPORTED while the test-only failure injection (environment variable
+ *     LA_DEBUG_WITHHOLD_SEGMENT) is set.
  */
 #define LA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u + 4096u)
 la_status la_prefill_noalloc(const la_desc* desc, const void* q, const void* k, const void* v,

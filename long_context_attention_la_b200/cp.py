@@ -76,8 +76,9 @@ def prefill_cp(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.
     q, k, v: [B, L_r, H, d], this rank's consecutive tokens of every sequence (rank r of `group`
     holds part r; L_r may differ between ranks and may be 0).  slopes: fp32[H].  state_in:
     optional fp32 [B, H, d, d] initial state of the sequences, the same on every rank.
-    part_lengths: optional list of every rank's L_r (saves the length exchange and its host
-    synchronisation when the split is known).  Returns this rank's outputs [B, L_r, H, d] and
+    part_lengths: every rank's L_r.  Pass it on the hot path: without it the lengths are
+    exchanged with a collective and read back to the host, which synchronises the device on
+    every call.  Returns this rank's outputs [B, L_r, H, d] and
     the state after its part (on the last rank: after the whole sequence).  Collective: every
     rank of the group must call it with the same B, H, d.
     """

@@ -129,9 +129,14 @@ size_t la_prefill_workspace_bytes(const la_desc* desc) {
   return la::workspace_layout(desc->B, desc->H, plan).total;
 }
 
-la_status la_prefill(const la_desc* desc, const void* q, const void* k, const void* v,
-                     const float* slopes, void* out, float* state_out, void* workspace,
-                     size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Argument checks of la_prefill (and la_prefill_noalloc): descriptor, pointers, alignment and
+// overlaps, all before any CUDA call.
+la_status check_prefill_args(const la_desc* desc, const void* q, const void* k, const void* v,
+                             const float* slopes, const void* out, const float* state_out) {
   int64_t numel = 0;
   const la_status st = check_desc(desc, &numel);
   if (st != LA_OK) return st;
@@ -142,6 +147,25 @@ la_status la_prefill(const la_desc* desc, const void* q, const void* k, const vo
   if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) ||
       overlaps(out, bytes, v, bytes))
     return LA_ERR_ALIAS;
+  if (state_out != nullptr) {
+    // the final state is written while other CTAs still read q, k, v and write out
+    const size_t sb = static_cast<size_t>(desc->B * desc->H) * static_cast<size_t>(desc->d * desc->d) * 4;
+    if (overlaps(state_out, sb, q, bytes) || overlaps(state_out, sb, k, bytes) ||
+        overlaps(state_out, sb, v, bytes) || overlaps(state_out, sb, out, bytes))
+      return LA_ERR_ALIAS;
+  }
+  return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+la_status la_prefill(const la_desc* desc, const void* q, const void* k, const void* v,
+                     const float* slopes, void* out, float* state_out, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  const la_status st = check_prefill_args(desc, q, k, v, slopes, out, state_out);
+  if (st != LA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   la::PrefillArgs a{desc->B, desc->N, desc->H, desc->d, desc->dtype, q, k, v, slopes, out,
@@ -308,6 +332,11 @@ la_status la_decode_multi(int64_t B, int64_t H, int64_t d, int64_t n_tok, int32_
   if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) ||
       overlaps(out, bytes, v, bytes) || overlaps(out, bytes, state_inout, static_cast<size_t>(sb)))
     return LA_ERR_ALIAS;
+  // the state is rewritten in place while the token rows are read
+  if (overlaps(state_inout, static_cast<size_t>(sb), q, bytes) ||
+      overlaps(state_inout, static_cast<size_t>(sb), k, bytes) ||
+      overlaps(state_inout, static_cast<size_t>(sb), v, bytes))
+    return LA_ERR_ALIAS;
   la::DecodeArgs a{B, H, d, dtype, q, k, v, slopes, state_inout, out};
   a.n_tok = n_tok;
   if (epilogue != nullptr) {
@@ -443,6 +472,11 @@ la_status la_decode_step(int64_t B, int64_t H, int64_t d, int32_t dtype, const v
   if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) ||
       overlaps(out, bytes, v, bytes) || overlaps(out, bytes, state_inout, static_cast<size_t>(sb)))
     return LA_ERR_ALIAS;
+  // the state is rewritten in place while the token rows are read
+  if (overlaps(state_inout, static_cast<size_t>(sb), q, bytes) ||
+      overlaps(state_inout, static_cast<size_t>(sb), k, bytes) ||
+      overlaps(state_inout, static_cast<size_t>(sb), v, bytes))
+    return LA_ERR_ALIAS;
   la::DecodeArgs a{B, H, d, dtype, q, k, v, slopes, state_inout, out};
   return la::launch_decode(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? LA_OK
                                                                                  : LA_ERR_CUDA;
@@ -460,23 +494,66 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[LA_NOALLOC_SCRATCH_BY
 namespace {
 
 constexpr int kMaxDevices = 256;
-void* g_noalloc_ptr[kMaxDevices] = {};
+
+// The scratch array's device address in one CUDA context.  A context that is destroyed and
+// recreated (cudaDeviceReset, a primary-context reset) loads the module again, possibly at
+// another address, so the cache is keyed by the context's unique id, not the device alone.
+struct ScratchAddress {
+  unsigned long long ctx_id;
+  void* ptr;
+};
+ScratchAddress g_noalloc_addr[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
-// Device address of g_noalloc_scratch on the current device (looked up on first use).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (the runtime's primary context of the
+// current device once a runtime call has been made).
+la_status current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (get_current == nullptr || get_id == nullptr) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || f1 == nullptr ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess || f2 == nullptr)
+      return LA_ERR_CUDA;
+    get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+    get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return LA_ERR_CUDA;
+  if (get_id(ctx, id) != CUDA_SUCCESS) return LA_ERR_CUDA;
+  return LA_OK;
+}
+
+// Device address of g_noalloc_scratch on the current device, looked up with cudaGetSymbolAddress
+// once per device and context (the host-side name g_noalloc_scratch is not a device address).
 la_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return LA_ERR_UNSUPPORTED;
+  // make the device's primary context current (since CUDA 12, cudaSetDevice initialises it;
+  // a no-op once the runtime has used it); this allocates nothing
+  if (cudaSetDevice(dev) != cudaSuccess) return LA_ERR_CUDA;
+  unsigned long long ctx = 0;
+  const la_status cs = current_context_id(&ctx);
+  if (cs != LA_OK) return cs;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  ScratchAddress& a = g_noalloc_addr[dev];
+  if (a.ptr == nullptr || a.ctx_id != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_noalloc_scratch) != cudaSuccess ||
         p == nullptr)
       return LA_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
+    a.ptr = p;
+    a.ctx_id = ctx;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = a.ptr;
   return LA_OK;
 }
 
@@ -486,9 +563,12 @@ extern "C" {
 
 la_status la_prefill_noalloc(const la_desc* desc, const void* q, const void* k, const void* v,
                              const float* slopes, void* out, float* state_out, void* stream) {
-  int64_t numel = 0;
-  const la_status st = check_desc(desc, &numel);
+  const la_status st = check_prefill_args(desc, q, k, v, slopes, out, state_out);
   if (st != LA_OK) return st;
+  // The test-only failure injection (a withheld scan flag) can only be reported through the
+  // workspace status word, which callers of this entry point cannot read: refuse it here rather
+  // than return LA_OK with invalid outputs.
+  if (getenv("LA_DEBUG_WITHHOLD_SEGMENT") != nullptr) return LA_ERR_UNSUPPORTED;
   if (!use_tensor_path(desc)) {
     // the recurrent kernel uses no scratch memory
     return la_prefill(desc, q, k, v, slopes, out, state_out, nullptr, 0, stream);

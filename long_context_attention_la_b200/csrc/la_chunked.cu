@@ -1166,21 +1166,15 @@ namespace {
 cudaError_t launch_common(const PrefillArgs& a, Params& prm, uint8_t* ws,
                           const WorkspaceLayout& wl, int64_t units, cudaStream_t stream,
                           int num_sms, bool clear_header = true) {
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    e = cudaFuncSetAttribute(chunked_prefill_kernel<false>,
+  // set on every call: cheap, safe from any host thread, and it survives a context reset
+  cudaError_t e = cudaFuncSetAttribute(chunked_prefill_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemAlloc));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(chunked_prefill_kernel<true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemAlloc));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(chunked_prefill_kernel<true>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kSmemAlloc));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  if (e != cudaSuccess) return e;
   // counter, status and scan flags start at zero for every call
   if (clear_header) {
     e = cudaMemsetAsync(ws, 0, wl.flags_off + wl.flags_bytes, stream);
@@ -1485,14 +1479,9 @@ cudaError_t launch_prefill_varlen(const PrefillArgs& a, const VarlenWorkspace& l
     while (n_pad < a.n_seqs) n_pad <<= 1;
     sort_bytes = static_cast<size_t>(n_pad) * sizeof(unsigned long long);
   }
-  static bool plan_attr_set[64] = {false};
-  int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && !plan_attr_set[dev]) {
-    e = cudaFuncSetAttribute(plan_varlen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kPlanSortMax * sizeof(unsigned long long)));
-    if (e != cudaSuccess) return e;
-    plan_attr_set[dev] = true;
-  }
+  e = cudaFuncSetAttribute(plan_varlen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kPlanSortMax * sizeof(unsigned long long)));
+  if (e != cudaSuccess) return e;
   plan_varlen_kernel<<<1, kPlanThreads, sort_bytes, stream>>>(pa);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -188,17 +188,14 @@ template <typename T, int D>
 cudaError_t launch_dim(const GateNormArgs& a, cudaStream_t stream) {
   constexpr int ROWS = kGnThreads / (D / 8);
   constexpr size_t kSmem = size_t(kStages) * 2 * kSweeps * Piece<T>::kPieces * kGnThreads * 16;
-  static bool attr_set[64] = {false};
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    e = cudaFuncSetAttribute(gate_norm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmem));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  // set on every call: cheap, safe from any host thread, and it survives a context reset
+  e = cudaFuncSetAttribute(gate_norm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kSmem));
+  if (e != cudaSuccess) return e;
   const int64_t per_token = (a.H + ROWS * kSweeps - 1) / (ROWS * kSweeps);
   const int64_t items = a.T * per_token;
   const int64_t resident = kSmem <= 100 * 1024 ? 2 : 1;  // CTAs per SM that the ring allows

@@ -199,17 +199,14 @@ template <int D>
 cudaError_t launch_dim(const QkNormRopeArgs& a, cudaStream_t stream) {
   constexpr int ROWS = kQkThreads / (D / 16);
   constexpr size_t kSmem = size_t(kStages) * kBatch * 2 * kQkThreads * 16;  // 96 KiB: 2 per SM
-  static bool attr_set[64] = {false};
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    e = cudaFuncSetAttribute(qk_norm_rope_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmem));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  // set on every call: cheap, safe from any host thread, and it survives a context reset
+  e = cudaFuncSetAttribute(qk_norm_rope_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kSmem));
+  if (e != cudaSuccess) return e;
   const int64_t per_token = (2 * a.H + ROWS * kBatch - 1) / (ROWS * kBatch);
   const int64_t items = a.T * per_token;
   const int64_t grid0 = std::max<int64_t>(1, std::min<int64_t>(items, 2 * int64_t(sms)));

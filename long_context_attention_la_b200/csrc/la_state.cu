@@ -402,16 +402,10 @@ StatePassPlan plan_state_pass(int64_t B, int64_t N, int64_t H, int num_sms) {
 
 cudaError_t launch_state_pass(const PrefillArgs& a, const StatePassPlan& plan, void* workspace,
                               cudaStream_t stream) {
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  // set on every call: cheap, safe from any host thread, and it survives a context reset
+  cudaError_t e = cudaFuncSetAttribute(state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kSmemAlloc));
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    e = cudaFuncSetAttribute(state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemAlloc));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   e = cudaMemsetAsync(ws, 0, 256, stream);  // status word
   if (e != cudaSuccess) return e;

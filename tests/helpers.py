@@ -47,3 +47,53 @@ def check_close(x, ref, dtype, what=""):
     assert r <= BF16_REL_L2, f"{what}: relL2 {r:.3e} > {BF16_REL_L2}"
     assert m <= BF16_MAX_ABS_FRAC * scale + 1e-30, f"{what}: maxabs {m:.3e} > 2e-2*{scale:.3e}"
     return r, m
+
+
+class ParityAccumulator:
+    """The same bar as check_close, for a tensor compared in pieces (for example a few heads at a
+    time against the oracle): relL2 is accumulated as sums of squares over the whole tensor,
+    maxabs and max|ref| as maxima.  ``worst`` keeps the largest per-piece relL2 as a diagnostic.
+    """
+
+    def __init__(self, dtype, what=""):
+        self.dtype = dtype
+        self.what = what
+        self.num = 0.0
+        self.den = 0.0
+        self.maxabs = 0.0
+        self.scale = 0.0
+        self.worst = (0.0, None)
+        self.pieces = 0
+
+    def add(self, x, ref, tag=None):
+        x = np.asarray(x, dtype=np.float64)
+        ref = np.asarray(ref, dtype=np.float64)
+        if x.shape != ref.shape:
+            raise ValueError(f"{self.what}: shape {x.shape} != {ref.shape}")
+        diff = x - ref
+        n = float(np.sum(diff * diff))
+        d = float(np.sum(ref * ref))
+        self.num += n
+        self.den += d
+        if x.size:
+            self.maxabs = max(self.maxabs, float(np.max(np.abs(diff))))
+            self.scale = max(self.scale, float(np.max(np.abs(ref))))
+        r = (n / d) ** 0.5 if d > 0 else n ** 0.5
+        if r >= self.worst[0]:
+            self.worst = (r, tag)
+        self.pieces += 1
+
+    def rel_l2(self) -> float:
+        return (self.num / self.den) ** 0.5 if self.den > 0 else self.num ** 0.5
+
+    def check(self):
+        r = self.rel_l2()
+        if self.dtype == torch.float32:
+            assert r <= F32_REL_L2, f"{self.what}: relL2 {r:.3e} > {F32_REL_L2}"
+        else:
+            assert r <= BF16_REL_L2, f"{self.what}: relL2 {r:.3e} > {BF16_REL_L2}"
+            assert self.maxabs <= BF16_MAX_ABS_FRAC * self.scale + 1e-30, \
+                f"{self.what}: maxabs {self.maxabs:.3e} > 2e-2*{self.scale:.3e}"
+        print(f"{self.what}: relL2 {r:.3e}, maxabs {self.maxabs:.3e} (max|ref| {self.scale:.3e}), "
+              f"worst piece {self.worst[0]:.3e} at {self.worst[1]}, {self.pieces} pieces")
+        return r, self.maxabs

@@ -336,3 +336,29 @@ def test_prefill_state_workspace_follows_the_range_split(lib, B, N, H):
     need = la.la_prefill_state_workspace_bytes(_desc(B=B, N=N, H=H))
     assert need == 256 + 2 * grid * 128 * 128 * 4
     assert grid <= 148 and (grid - 1) * width < total <= grid * width
+
+
+def test_prefill_rejects_state_overlapping_an_activation(lib):
+    d = _desc(N=16, H=2, d=128)
+    nbytes = 16 * 2 * 128 * 2
+    q, k, v, out = 0x100000, 0x200000, 0x300000, 0x400000
+    for st in (q + 256, k, v + nbytes - 16, out + 512):
+        assert la.la_prefill(d, q, k, v, 0x4000, out, st, 0, 0, 0) == la.LA_ERR_ALIAS
+        assert la.la_prefill_noalloc(d, q, k, v, 0x4000, out, st, 0) == la.LA_ERR_ALIAS
+
+
+def test_decode_rejects_state_overlapping_a_token_row(lib):
+    q, k, v, out = 0x1000000, 0x2000000, 0x3000000, 0x4000000
+    sb = 2 * 128 * 128 * 4
+    for st in (q - 1024, k, v - sb + 16):
+        assert la.la_decode_step(1, 2, 128, la.LA_BF16, q, k, v, 0x4000, st, out,
+                                 0) == la.LA_ERR_ALIAS
+        assert la.la_decode_multi(1, 2, 128, 2, la.LA_BF16, q, k, v, 0x4000, st, out,
+                                  0) == la.LA_ERR_ALIAS
+
+
+def test_noalloc_refuses_the_failure_injection_it_cannot_report(lib, monkeypatch):
+    monkeypatch.setenv("LA_DEBUG_WITHHOLD_SEGMENT", "0")
+    d = _desc()
+    assert la.la_prefill_noalloc(d, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0,
+                                 0) == la.LA_ERR_UNSUPPORTED

@@ -88,7 +88,7 @@ def test_decode_multi_gated(dtype):
     torch.cuda.synchronize()
     o_ref, s_ref = oracle_steps(q, k, v, sl, state)
     y_ref = oracle.gated_rmsnorm(o_ref, oracle_bits(gate), gamma.cpu().numpy(), 1e-6)
-    check_close(y.float().cpu().numpy(), y_ref, torch.bfloat16, "y")
+    check_close(y.float().cpu().numpy(), y_ref, dtype, "y")
     check_close(st.cpu().numpy(), s_ref, dtype, "state")
 
 

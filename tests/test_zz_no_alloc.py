@@ -7,8 +7,10 @@ would fail or stall the device.  Another is a host framework that gives a kernel
 inputs and outputs but no allocator.  la_prefill_noalloc serves them from a fixed scratch array
 built into the library.  This test calls it through the C ABI twice in a row, with different
 problems, so the second call meets the first call's leftover scratch contents.  It checks each
-result against la_prefill with a workspace the test allocates, using the parity tolerances of
-the other GPU tests.  It also checks that a problem larger than the array is refused.
+result against la_prefill with a workspace the test allocates.  Both entry points run the same
+kernel with the same plan, and that kernel is deterministic, so the results must be equal bit
+for bit: any effect of stale scratch contents shows, however small.  It also checks that a
+problem larger than the array is refused.
 
 The file name sorts last, so a run that stops at the first failure has run every other test.
 """
@@ -16,7 +18,6 @@ import pytest
 import torch
 
 from long_context_attention_la_b200 import la, synth
-from tests.helpers import check_close
 
 pytestmark = pytest.mark.gpu
 
@@ -52,10 +53,10 @@ def test_noalloc_matches_allocating_entry_point_twice():
     r1, rs1 = _reference(q1, k1, v1, sl1)
     r2, rs2 = _reference(q2, k2, v2, sl2)
     torch.cuda.synchronize()
-    check_close(o1.float().cpu().numpy(), r1.float().cpu().numpy(), torch.bfloat16, "call 1 o")
-    check_close(s1.cpu().numpy(), rs1.cpu().numpy(), torch.bfloat16, "call 1 state")
-    check_close(o2.float().cpu().numpy(), r2.float().cpu().numpy(), torch.bfloat16, "call 2 o")
-    check_close(s2.cpu().numpy(), rs2.cpu().numpy(), torch.bfloat16, "call 2 state")
+    assert torch.equal(o1, r1), "call 1 o"
+    assert torch.equal(s1, rs1), "call 1 state"
+    assert torch.equal(o2, r2), "call 2 o"
+    assert torch.equal(s2, rs2), "call 2 state"
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
