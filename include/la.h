@@ -74,7 +74,10 @@ typedef struct {
   int64_t H;        /* heads, >= 1 */
   int64_t d;        /* head dimension, d_k = d_v = d, 64 or 128 */
   int32_t dtype;    /* la_dtype of q, k, v, out */
-  int32_t chunk;    /* chunk length C of the tensor-core path: 0 = default (128); 128 supported */
+  int32_t chunk;    /* chunk length C of the tensor-core path: 0 = default (128), or 64, 128,
+                       256 (every C computes the same recurrence; they differ only in where
+                       the bf16 roundings of the intra / inter split fall); the recurrent path
+                       takes 0 or 1 */
   int32_t segments; /* segments per sequence: 0 = automatic; >= 1 explicit (clamped to chunks) */
   int32_t path;     /* la_path */
 } la_desc;
@@ -87,9 +90,10 @@ size_t la_prefill_workspace_bytes(const la_desc* desc);
  * la_prefill — the whole prefill of one layer: o for every token and the final state.
  *
  * Chunked evaluation of the recurrence above ("chunk QKV", Fig. 10 of §4.1.1): within a chunk of
- * C tokens the intra-chunk term (Q K^T ⊙ M) V with M_ij = lambda^(i-j) (i >= j, else 0) and the
- * inter-chunk term diag(lambda^(i+1)) Q KV are tensor-core contractions; the fp32 state is carried
- * as KV <- lambda^C KV + (K ⊙ lambda^(C-1-i))^T V.  Long sequences are cut into segments whose
+ * C tokens (desc->chunk: 64, 128 or 256) the intra-chunk term (Q K^T ⊙ M) V with
+ * M_ij = lambda^(i-j) (i >= j, else 0) and the inter-chunk term diag(lambda^(i+1)) Q KV are
+ * tensor-core contractions (the state KV enters them rounded to bf16 once per chunk); the fp32
+ * state is carried as KV <- lambda^C KV + (K ⊙ lambda^(C-1-i))^T V.  Long sequences are cut into segments whose
  * local states are combined by a decayed prefix scan, the single-GPU form of the report's
  * "local recurrence, then global correction" (§4.1.1, Fig. 10: local h, fused update h / O).
  *

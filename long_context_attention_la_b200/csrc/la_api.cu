@@ -43,6 +43,9 @@ bool use_tensor_path(int32_t path, int32_t dtype, int64_t d) {
 }
 bool use_tensor_path(const la_desc* d) { return use_tensor_path(d->path, d->dtype, d->d); }
 
+// The tensor path's chunk length for a descriptor's `chunk` field (0: the library's default).
+int chunk_of(int32_t chunk) { return chunk == 0 ? la::kChunkDefault : chunk; }
+
 // Failure injection for tests, read on every call: LA_DEBUG_WITHHOLD_SEGMENT=k keeps segment k of
 // every sequence from publishing its scan state, so segment k+1 waits until its bounded wait
 // expires (LA_DEBUG_WAIT_LIMIT_MS, default 2000) and the call reports LA_ERR_TIMEOUT through
@@ -72,7 +75,7 @@ la_status check_desc(const la_desc* d, int64_t* numel) {
   if (d->B * d->H > INT32_MAX) return LA_ERR_OVERFLOW;  // grid / flat-head index range
   if (use_tensor_path(d)) {
     if (d->dtype != LA_BF16 || d->d != la::kHeadDim) return LA_ERR_UNSUPPORTED;
-    if (d->chunk != 0 && d->chunk != la::kChunk) return LA_ERR_UNSUPPORTED;
+    if (d->chunk != 0 && !la::chunk_supported(d->chunk)) return LA_ERR_UNSUPPORTED;
     // tensor-map coordinates are 32-bit; byte strides below 2^40
     if (d->N > INT32_MAX - la::kChunk || d->H > INT32_MAX || d->B > INT32_MAX)
       return LA_ERR_OVERFLOW;
@@ -101,7 +104,7 @@ la_status check_varlen(const la_varlen_desc* d, int64_t* numel) {
     return LA_ERR_OVERFLOW;
   if (use_tensor_path(d->path, d->dtype, d->d)) {
     if (d->dtype != LA_BF16 || d->d != la::kHeadDim) return LA_ERR_UNSUPPORTED;
-    if (d->chunk != 0 && d->chunk != la::kChunk) return LA_ERR_UNSUPPORTED;
+    if (d->chunk != 0 && !la::chunk_supported(d->chunk)) return LA_ERR_UNSUPPORTED;
     // token coordinates of the tensor maps and work units are 32-bit, and so is the unit count
     if (d->T > INT32_MAX - la::kChunk) return LA_ERR_OVERFLOW;
     int64_t cap = 0;
@@ -125,7 +128,8 @@ size_t la_prefill_workspace_bytes(const la_desc* desc) {
   if (check_desc(desc, &numel) != LA_OK) return 0;
   if (!use_tensor_path(desc)) return 0;
   const la::SegmentPlan plan =
-      la::plan_segments(desc->B, desc->N, desc->H, desc->segments, device_sms() > 0 ? device_sms() : 148);
+      la::plan_segments(desc->B, desc->N, desc->H, desc->segments,
+                        device_sms() > 0 ? device_sms() : 148, chunk_of(desc->chunk));
   return la::workspace_layout(desc->B, desc->H, plan).total;
 }
 
@@ -170,13 +174,15 @@ la_status la_prefill(const la_desc* desc, const void* q, const void* k, const vo
 
   la::PrefillArgs a{desc->B, desc->N, desc->H, desc->d, desc->dtype, q, k, v, slopes, out,
                     state_out};
+  a.chunk = chunk_of(desc->chunk);
   apply_debug_env(a);
   if (!use_tensor_path(desc)) {
     return la::launch_recurrent_prefill(a, s) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
   }
   const int sms = device_sms();
   if (sms <= 0) return LA_ERR_CUDA;
-  const la::SegmentPlan plan = la::plan_segments(desc->B, desc->N, desc->H, desc->segments, sms);
+  const la::SegmentPlan plan = la::plan_segments(desc->B, desc->N, desc->H, desc->segments, sms,
+                                                   chunk_of(desc->chunk));
   const size_t need = la::workspace_layout(desc->B, desc->H, plan).total;
   void* ws = workspace;
   bool owned = false;
@@ -246,6 +252,7 @@ la_status la_prefill_varlen(const la_varlen_desc* desc, const void* q, const voi
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return LA_ERR_ALIGN;
   }
   la::PrefillArgs a{1, desc->T, desc->H, desc->d, desc->dtype, q, k, v, slopes, out, state_out};
+  a.chunk = chunk_of(desc->chunk);
   a.n_seqs = desc->n_seqs;
   a.cu_dev = cu_seqlens;
   a.state_in = state_in;
@@ -575,7 +582,8 @@ la_status la_prefill_noalloc(const la_desc* desc, const void* q, const void* k, 
   }
   const int sms = device_sms();
   if (sms <= 0) return LA_ERR_CUDA;
-  const la::SegmentPlan plan = la::plan_segments(desc->B, desc->N, desc->H, desc->segments, sms);
+  const la::SegmentPlan plan = la::plan_segments(desc->B, desc->N, desc->H, desc->segments, sms,
+                                                   chunk_of(desc->chunk));
   const size_t need = la::workspace_layout(desc->B, desc->H, plan).total;
   if (need > LA_NOALLOC_SCRATCH_BYTES) return LA_ERR_WORKSPACE;
   void* scratch = nullptr;

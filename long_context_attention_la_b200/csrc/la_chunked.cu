@@ -2,12 +2,24 @@
 //
 // Method ("Ling and Ring 2.6 Technical Report", Chinese translation, garden.houmin.site;
 // §4.1.1 Context Parallel for Lightning Attention, Fig. 10): each (b, h) sequence is evaluated as
-// chunks of C = 128 tokens ("chunk QKV").  For chunk c with rows i, j in [0, C):
+// chunks of C tokens ("chunk QKV").  For chunk c with rows i, j in [0, C):
 //     S      = Q K^T                                   (tensor cores, fp32 in TMEM)
 //     P_ij   = lambda^(i-j) S_ij  (i >= j), 0 otherwise  (CUDA cores, bf16 back into TMEM)
 //     O      = P V + diag(lambda^(i+1)) Q KV_in          (two tensor-core accumulators)
 //     KV_out = lambda^n KV_in + (K ⊙ lambda^(n-1-j))^T V  (tensor cores, fp32 state in TMEM)
-// where n is the chunk's token count and KV_in the d x d state before the chunk.  Long sequences
+// where n is the chunk's token count and KV_in the d x d state before the chunk.  The kernel moves
+// and multiplies 128-token tiles (every MMA is M = 128); the chunk length C in {64, 128, 256} is
+// how a tile's rows split between the intra- and the inter-chunk term:
+//   C = 128  one chunk per tile (the code below calls a tile a "chunk" where C = 128 is meant);
+//   C = 64   two chunks per tile: P is block-diagonal (two 64 x 64 causal blocks), rows 0..63 read
+//            the state before the tile and rows 64..127 the state after its first half, which the
+//            state warps round to bf16 in the middle of the tile (a second Q KV product whose
+//            accumulator reuses the S columns once P V has read P);
+//   C = 256  two tiles per chunk: the second tile B adds the block below the diagonal directly,
+//            P_BA = lambda^(128+i-j) Q_B K_A^T = diag(lambda^(i+1)) Q_B K~_A^T with K~_A the first
+//            tile's keys already scaled for the state update, so the bf16 state operand is
+//            refreshed once per 256 tokens and B's inter term is lambda^(i+129) Q_B KV_in.
+// All three are the same recurrence; they differ only in where bf16 roundings fall.  Long sequences
 // are cut into segments ("local recurrence, then global correction"): a segment first computes its
 // local state h (the "local h" of Fig. 10) from K, V alone, obtains its incoming state from its
 // predecessor through a decayed prefix scan over segments (S_{k+1} = lambda^L S_k + h_k, the
@@ -71,6 +83,10 @@ constexpr int32_t kErrTimeout = -8;  // LA_ERR_TIMEOUT
 
 using UnitInfo = WorkUnit;  // one (segment, sequence, head) work unit
 
+// Chunk length of a kernel instance: C = 128 (one chunk per tile), C = 64 (two per tile) or
+// C = 256 (two tiles per chunk).
+enum ChunkMode : int { kC128 = 0, kC64 = 1, kC256 = 2 };
+
 struct Ctrl {
   uint64_t full[2];
   uint64_t empty[2];
@@ -79,6 +95,8 @@ struct Ctrl {
   uint64_t unit_empty[2];
   uint64_t s_full;
   uint64_t p_ready;
+  uint64_t s2_full;   // C = 256: the cross scores Q_B K~_A^T of a chunk's second tile are in TMEM
+  uint64_t p2_ready;  // C = 256: their scaled bf16 P_BA is in TMEM
   uint64_t o_full;
   uint64_t o_free;
   uint64_t kv_done;
@@ -272,7 +290,8 @@ __device__ __forceinline__ void load_gate_pieces(const __nv_bfloat16* gate_h, in
   }
 }
 
-__device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint32_t trow, float f,
+__device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint32_t trow,
+                                               uint32_t col_inter, float f,
                                                const UnitInfo& ui, int64_t h,
                                                const __nv_bfloat16* gate_h, __nv_bfloat16* out_h,
                                                uint32_t t, int32_t r0, int64_t n0,
@@ -282,7 +301,7 @@ __device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint
   for (uint32_t cb = 0; cb < 8; ++cb) {  // 16-column blocks
     uint32_t ra[16], re[16];
     tmem_ld16(trow + kColOintra + cb * 16, ra);
-    tmem_ld16(trow + kColOinter + cb * 16, re);
+    tmem_ld16(trow + col_inter + cb * 16, re);
     tmem_wait_ld();
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
@@ -305,7 +324,7 @@ __device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint
     for (uint32_t q = 0; q < 4; ++q) {
       uint32_t ra[8], re[8];
       tmem_ld8(trow + kColOintra + cb * 32 + q * 8, ra);
-      tmem_ld8(trow + kColOinter + cb * 32 + q * 8, re);
+      tmem_ld8(trow + col_inter + cb * 32 + q * 8, re);
       tmem_wait_ld();
       if (cb == 3 && q == 3) {
         // every O column of this row has been read: the accumulators may be overwritten
@@ -346,9 +365,10 @@ __device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint
   }
 }
 
-// kGated: the output epilogue applies the fused norm + gate (p.gate != null).  Two instances, so
-// that the plain kernel's register allocation carries none of the gated epilogue's pressure.
-template <bool kGated>
+// kGated: the output epilogue applies the fused norm + gate (p.gate != null).  Separate instances,
+// so that the plain kernel's register allocation carries none of the gated epilogue's pressure.
+// kCM: the chunk length (ChunkMode).
+template <bool kGated, int kCM>
 __global__ void __launch_bounds__(kThreads, 1)
     chunked_prefill_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -372,6 +392,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&ctrl->s_full, 1);
     mbar_init(&ctrl->p_ready, 256);
+    mbar_init(&ctrl->s2_full, 1);
+    mbar_init(&ctrl->p2_ready, 256);
     mbar_init(&ctrl->o_full, 1);
     mbar_init(&ctrl->o_free, 128);
     mbar_init(&ctrl->kv_done, 1);
@@ -545,9 +567,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idPV = make_idesc_bf16(128, 128, 0, 1);  // P (TMEM) x V (MN-major)
       constexpr uint32_t idKV = make_idesc_bf16(128, 128, 1, 1);  // K~^T (MN) x V (MN)
       uint32_t g = 0, j = 0;
-      uint32_t n_kvb = 0, n_ofree = 0, n_p = 0;
+      uint32_t n_kvb = 0, n_ofree = 0, n_p = 0, n_p2 = 0;
       bool ok = true;
-      // KV (+)= K~^T V for the chunk held in stage (gg & 1)
+      // KV (+)= K~^T V over token rows [16 kk0, 16 kk1) of the tile held in stage (gg & 1)
+      auto issue_state_update_rows = [&](uint32_t gg, uint32_t kk0, uint32_t kk1) {
+        const uint32_t kb = smem_base + (gg & 1) * kStageBytes + kOffK;
+        const uint32_t vb = smem_base + (gg & 1) * kStageBytes + kOffV;
+#pragma unroll
+        for (uint32_t kk = kk0; kk < kk1; ++kk) {
+          umma_ss(tmem + kColKV, make_sdesc_sw128(kb + kk * 2048, kHalfBytes, 1024),
+                  make_sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idKV, 1u);
+        }
+      };
+      // KV (+)= K~^T V for the whole tile held in stage (gg & 1)
       auto issue_state_update = [&](uint32_t gg, bool accumulate_first) {
         const uint32_t kb = smem_base + (gg & 1) * kStageBytes + kOffK;
         const uint32_t vb = smem_base + (gg & 1) * kStageBytes + kOffV;
@@ -605,54 +637,153 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t kb = smem_base + s * kStageBytes + kOffK;
           const uint32_t vb = smem_base + s * kStageBytes + kOffV;
           const uint32_t kvb = smem_base + kOffKVb;
-          // S_c = Q K^T
+          // C = 256: the first tile A (even c) of a two-tile chunk keeps its stage until the second
+          // tile B (odd c) has read K~_A and V_A from it (stage s ^ 1).
+          const bool tile_b = kCM == kC256 && (c & 1) != 0;
+          const bool keep_stage = kCM == kC256 && (c & 1) == 0 && c + 1 < ui.nc;
+          // D (+)= Q K^T over d = 128 (both K-major), from this tile's Q and the keys at kbase
+          auto issue_qk = [&](uint32_t d_col, uint32_t kbase) {
 #pragma unroll
-          for (uint32_t kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-            umma_ss(tmem + kColS, make_sdesc_sw128(qb + off, 16, 1024),
-                    make_sdesc_sw128(kb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+            for (uint32_t kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+              umma_ss(tmem + d_col, make_sdesc_sw128(qb + off, 16, 1024),
+                      make_sdesc_sw128(kbase + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+            }
+          };
+          // D = Q KVb (the bf16 state operand)
+          auto issue_qkv = [&](uint32_t d_col) {
+#pragma unroll
+            for (uint32_t kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+              umma_ss(tmem + d_col, make_sdesc_sw128(qb + off, 16, 1024),
+                      make_sdesc_sw128(kvb + kk * 2048, kHalfBytes, 1024), idQK,
+                      kk > 0 ? 1u : 0u);
+            }
+          };
+          // O_intra (+)= P V with P read from TMEM and the values at vbase
+          auto issue_pv = [&](uint32_t vbase, bool accumulate) {
+#pragma unroll
+            for (uint32_t kk = 0; kk < 8; ++kk) {
+              umma_ts(tmem + kColOintra, tmem + kColS + kk * 8,
+                      make_sdesc_sw128(vbase + kk * 2048, kHalfBytes, 1024), idPV,
+                      (accumulate || kk > 0) ? 1u : 0u);
+            }
+          };
+          if (kCM == kC64) {
+            // the S columns held the previous tile's second inter product until the epilogue read
+            // it, so S waits for the free accumulators here rather than before O_inter
+            if (!mbar_wait_bounded(&ctrl->o_free, n_ofree & 1, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            ++n_ofree;
+            tc_fence_after();
           }
-          umma_commit(&ctrl->s_full);
+          if (tile_b) {
+            // S_BA = Q_B K~_A^T, the scores of this tile's queries against the chunk's first tile
+            issue_qk(kColS, smem_base + (s ^ 1) * kStageBytes + kOffK);
+            umma_commit(&ctrl->s2_full);
+          } else {
+            issue_qk(kColS, kb);  // S_c = Q K^T
+            umma_commit(&ctrl->s_full);
+          }
           // O_inter = Q KV_in (needs the bf16 state operand and a free O accumulator)
-          if (!mbar_wait_bounded(&ctrl->kvb_ready, n_kvb & 1, abort_flag, T) ||
-              !mbar_wait_bounded(&ctrl->o_free, n_ofree & 1, abort_flag, T)) {
+          if (!mbar_wait_bounded(&ctrl->kvb_ready, n_kvb & 1, abort_flag, T)) {
             ok = false;
             break;
           }
           ++n_kvb;
-          ++n_ofree;
-          tc_fence_after();
-#pragma unroll
-          for (uint32_t kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-            umma_ss(tmem + kColOinter, make_sdesc_sw128(qb + off, 16, 1024),
-                    make_sdesc_sw128(kvb + kk * 2048, kHalfBytes, 1024), idQK,
-                    kk > 0 ? 1u : 0u);
-          }
-          // KV += K~_c^T V_c once K_c is row-scaled (after S_c, which read K_c unscaled).  It
-          // follows O_inter_c, so kv_done also tells the state warps that the bf16 operand O_inter
-          // read is free again.
-          if (!mbar_wait_bounded(&ctrl->kt_ready[s], ph, abort_flag, T)) {
-            ok = false;
-            break;
+          if (kCM != kC64) {
+            if (!mbar_wait_bounded(&ctrl->o_free, n_ofree & 1, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            ++n_ofree;
           }
           tc_fence_after();
-          issue_state_update(g, true);
-          umma_commit(&ctrl->kv_done);
-          // O_intra = P V, P read from TMEM
-          if (!mbar_wait_bounded(&ctrl->p_ready, n_p & 1, abort_flag, T)) {
-            ok = false;
-            break;
+          issue_qkv(kColOinter);
+          if (kCM == kC64) {
+            // first chunk of the tile: KV += K~_A^T V_A (token rows 0..63)
+            if (!mbar_wait_bounded(&ctrl->kt_ready[s], ph, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_state_update_rows(g, 0, 4);
+            umma_commit(&ctrl->kv_done);
+            // O_intra = P V with the block-diagonal P
+            if (!mbar_wait_bounded(&ctrl->p_ready, n_p & 1, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            ++n_p;
+            tc_fence_after();
+            issue_pv(vb, false);
+            // second chunk: its inter product from the state after the first chunk (rows 64..127
+            // of this D are the ones used), written over the S columns now that P has been read;
+            // then KV += K~_B^T V_B
+            if (!mbar_wait_bounded(&ctrl->kvb_ready, n_kvb & 1, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            ++n_kvb;
+            tc_fence_after();
+            issue_qkv(kColS);
+            issue_state_update_rows(g, 4, 8);
+            umma_commit(&ctrl->kv_done);
+            umma_commit(&ctrl->o_full);
+            umma_commit(&ctrl->empty[s]);
+          } else if (tile_b) {
+            // O_intra = P_BA V_A; then tile A's stage is free
+            if (!mbar_wait_bounded(&ctrl->p2_ready, n_p2 & 1, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            ++n_p2;
+            tc_fence_after();
+            issue_pv(smem_base + (s ^ 1) * kStageBytes + kOffV, false);
+            umma_commit(&ctrl->empty[s ^ 1]);
+            // S_BB = Q_B K_B^T over the S columns (in issue order after P_BA V_A read P_BA)
+            issue_qk(kColS, kb);
+            umma_commit(&ctrl->s_full);
+            if (!mbar_wait_bounded(&ctrl->kt_ready[s], ph, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_state_update(g, true);
+            umma_commit(&ctrl->kv_done);
+            if (!mbar_wait_bounded(&ctrl->p_ready, n_p & 1, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            ++n_p;
+            tc_fence_after();
+            issue_pv(vb, true);  // O_intra += P_BB V_B
+            umma_commit(&ctrl->o_full);
+            umma_commit(&ctrl->empty[s]);
+          } else {
+            // KV += K~_c^T V_c once K_c is row-scaled (after S_c, which read K_c unscaled).  It
+            // follows O_inter_c, so kv_done also tells the state warps that the bf16 operand
+            // O_inter read is free again.
+            if (!mbar_wait_bounded(&ctrl->kt_ready[s], ph, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_state_update(g, true);
+            umma_commit(&ctrl->kv_done);
+            // O_intra = P V, P read from TMEM
+            if (!mbar_wait_bounded(&ctrl->p_ready, n_p & 1, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            ++n_p;
+            tc_fence_after();
+            issue_pv(vb, false);
+            umma_commit(&ctrl->o_full);
+            if (!keep_stage) umma_commit(&ctrl->empty[s]);
           }
-          ++n_p;
-          tc_fence_after();
-#pragma unroll
-          for (uint32_t kk = 0; kk < 8; ++kk) {
-            umma_ts(tmem + kColOintra, tmem + kColS + kk * 8,
-                    make_sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idPV, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&ctrl->o_full);
-          umma_commit(&ctrl->empty[s]);
           ++g;
         }
         if (!ok) break;
@@ -675,7 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t i = wq * 32 + lane;           // row of the chunk (query token)
     const uint32_t tp = threadIdx.x - kWarpP0 * 32;  // 0..255
     const uint32_t trow = tmem + ((wq * 32) << 16);
-    uint32_t g = 0, j = 0, n_s = 0;
+    uint32_t g = 0, j = 0, n_s = 0, n_s2 = 0;
     while (true) {
       const uint32_t slot = j & 1;
       bool ok = mbar_wait_bounded(&ctrl->unit_full[slot], (j >> 1) & 1, abort_flag, T);
@@ -705,6 +836,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       for (int32_t c = 0; c < ui.nc; ++c) {
+        if (kCM == kC256 && (c & 1) != 0) {
+          // Second tile of a 256-token chunk: P_BA = lambda^(i+1) S~_BA over all 128 columns
+          // (S~_BA = Q_B K~_A^T already carries lambda^(127-j)), no causal mask.  The block split
+          // and the barrier before the first store are those of the causal pass below.
+          ok = mbar_wait_bounded(&ctrl->s2_full, n_s2 & 1, abort_flag, T);
+          if (!group_all(ok, kBarP, 256)) goto p_out;
+          ++n_s2;
+          tc_fence_after();
+          const float fr = ex2_approx(-alpha * static_cast<float>(i + 1));
+          uint32_t r[32];
+          uint32_t pk[16];
+          tmem_ld32(trow + kColS + hf * 32, r);
+          tmem_wait_ld();
+          tc_fence_before();
+          named_bar_sync(kBarP, 256);
+          tc_fence_after();
+#pragma unroll
+          for (int m = 0; m < 16; ++m)
+            pk[m] = pack_bf16x2(__uint_as_float(r[2 * m]) * fr, __uint_as_float(r[2 * m + 1]) * fr);
+          tmem_st16(trow + kColS + hf * 16, pk);
+          tmem_ld32(trow + kColS + (hf + 2) * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int m = 0; m < 16; ++m)
+            pk[m] = pack_bf16x2(__uint_as_float(r[2 * m]) * fr, __uint_as_float(r[2 * m + 1]) * fr);
+          tmem_st16(trow + kColS + (hf + 2) * 16, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&ctrl->p2_ready);
+        }
         ok = mbar_wait_bounded(&ctrl->s_full, n_s & 1, abort_flag, T);
         if (!group_all(ok, kBarP, 256)) goto p_out;
         ++n_s;
@@ -737,15 +898,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
           uint32_t r[32];
           uint32_t pk[16];
+          // C = 64: P is block-diagonal, so rows 64..127 (lane quarters 2, 3) keep nothing of
+          // columns 0..63 (S blocks 0, 1)
           const uint32_t jb0 = hf;
-          if (jb0 <= wq) {
+          const bool live0 = jb0 <= wq && !(kCM == kC64 && wq >= 2);
+          if (live0) {
             tmem_ld32(trow + kColS + jb0 * 32, r);
             tmem_wait_ld();
           }
           tc_fence_before();
           named_bar_sync(kBarP, 256);
           tc_fence_after();
-          if (jb0 <= wq) {
+          if (live0) {
             make_p(jb0, r, pk);
           } else {
 #pragma unroll
@@ -838,7 +1002,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           reinterpret_cast<const float4*>(p.ring + (rs * 2 + ((k - 1) & 1)) * (D * D));
       float4* ring_out = reinterpret_cast<float4*>(p.ring + (rs * 2 + (k & 1)) * (D * D));
       const float lam_len = exp2f(-alpha * static_cast<float>(ui.len));
-      const float lam_n0 = exp2f(-alpha * static_cast<float>(min(C, ui.len)));
+      // decay of the incoming state over the first chunk (C = 64: the first half of tile 0)
+      const float lam_n0 =
+          exp2f(-alpha * static_cast<float>(min(kCM == kC64 ? 64 : C, ui.len)));
 #pragma unroll 1
       for (uint32_t cb = 0; cb < 4; ++cb) {
         uint32_t sin[32];  // fp32 bits of the incoming state, columns [32 cb, 32 cb + 32)
@@ -906,16 +1072,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // carry the state through the segment's chunks
+      // carry the state through the segment's tiles
       bool good = true;
+      // TMEM KV <- lambda^n KV, and (write_operand) its bf16 copy -> the MMA operand beforehand
+      auto refresh = [&](bool write_operand, float lam) {
+#pragma unroll 1
+        for (uint32_t cb = 0; cb < 4; ++cb) {
+          uint32_t r[32];
+          tmem_ld32(trow + kColKV + cb * 32, r);
+          tmem_wait_ld();
+          if (write_operand) write_kvb(cb, r);
+#pragma unroll
+          for (int m = 0; m < 32; ++m) r[m] = __float_as_uint(lam * __uint_as_float(r[m]));
+          tmem_st32(trow + kColKV + cb * 32, r);
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+      };
       for (int32_t c = 0; c < ui.nc; ++c) {
         const uint32_t s = g & 1;
-        const int32_t n_c = min(C, ui.len - c * C);  // tokens in this chunk
-        // the state operand for chunk c is in place (written before the loop or by the previous
+        const int32_t n_c = min(C, ui.len - c * C);  // tokens in this tile
+        // the state operand for tile c is in place (written before the loop or by the previous
         // iteration's update)
         mbar_arrive(&ctrl->kvb_ready);
         // K~_c = diag(lambda^(n-1-j)) K_c for the state update, once S_c (the only other reader of
-        // K_c) is complete; thread i scales key row i
+        // K_c) is complete; thread i scales key row i.  C = 64: each half of the tile is a chunk
+        // of its own, scaled to its own end.
         ok = mbar_wait_bounded(&ctrl->s_full, n_s & 1, abort_flag, T);
         if (!group_all(ok, kBarS, 128)) {
           good = false;
@@ -923,8 +1106,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++n_s;
         {
-          const int32_t r = static_cast<int32_t>(i);
-          const float w = r < n_c ? exp2f(-alpha * static_cast<float>(n_c - 1 - r)) : 0.f;
+          int32_t r = static_cast<int32_t>(i);
+          int32_t n_r = n_c;
+          if (kCM == kC64) {
+            n_r = i < 64 ? min(64, n_c) : max(0, n_c - 64);
+            r = static_cast<int32_t>(i & 63u);
+          }
+          const float w = r < n_r ? exp2f(-alpha * static_cast<float>(n_r - 1 - r)) : 0.f;
           uint8_t* kt = smem + s * kStageBytes + kOffK;
           scale_half_row(kt, i, w);
           scale_half_row(kt + kHalfBytes, i, w);
@@ -938,22 +1126,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++n_kvd;
         tc_fence_after();
-        if (c + 1 < ui.nc) {
-          const int32_t n_next = min(C, ui.len - (c + 1) * C);
-          const float lam_next = exp2f(-alpha * static_cast<float>(n_next));
-#pragma unroll 1
-          for (uint32_t cb = 0; cb < 4; ++cb) {
-            uint32_t r[32];
-            tmem_ld32(trow + kColKV + cb * 32, r);
-            tmem_wait_ld();
-            write_kvb(cb, r);
-#pragma unroll
-            for (int m = 0; m < 32; ++m) r[m] = __float_as_uint(lam_next * __uint_as_float(r[m]));
-            tmem_st32(trow + kColKV + cb * 32, r);
+        if (kCM == kC64) {
+          // the state after the tile's first chunk: its bf16 copy is the second chunk's operand
+          // (the first chunk's inter product has completed: it precedes the update just waited
+          // for); the fp32 state then decays over the second chunk's tokens
+          refresh(true, exp2f(-alpha * static_cast<float>(max(0, n_c - 64))));
+          mbar_arrive(&ctrl->kvb_ready);
+          ok = mbar_wait_bounded(&ctrl->kv_done, n_kvd & 1, abort_flag, T);
+          if (!group_all(ok, kBarS, 128)) {
+            good = false;
+            break;
           }
-          tmem_wait_st();
-          fence_proxy_async_smem();
-          tc_fence_before();
+          ++n_kvd;
+          tc_fence_after();
+        }
+        if (c + 1 < ui.nc) {
+          int32_t n_next = min(C, ui.len - (c + 1) * C);
+          if (kCM == kC64) n_next = min(64, n_next);  // the next tile's first chunk
+          // C = 256: after a chunk's first tile the operand stays the chunk's initial state
+          refresh(!(kCM == kC256 && (c & 1) == 0), exp2f(-alpha * static_cast<float>(n_next)));
         } else if ((ui.flags & 2) && p.state_out != nullptr) {
           float4* so = reinterpret_cast<float4*>(p.state_out + (bh * D + i) * D);
 #pragma unroll 1
@@ -996,11 +1187,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&ctrl->unit_empty[slot]);
       if (ui.bh < 0) break;
       const float alpha = p.slopes[ui.bh % p.H] * kLog2e;
-      const float f = exp2f(-alpha * static_cast<float>(i + 1));  // lambda^(i+1)
+      // row i's inter-term factor lambda^(i'+1), i' its position in its chunk (C = 64: rows
+      // 64..127 start the tile's second chunk); C = 256 adds lambda^128 on a chunk's second tile
+      const float f_a = exp2f(-alpha * static_cast<float>((kCM == kC64 ? (i & 63u) : i) + 1));
+      const float f_b = kCM == kC256 ? exp2f(-alpha * static_cast<float>(i + 129)) : f_a;
+      // C = 64: rows 64..127 take their inter product from the S columns
+      const uint32_t col_inter = (kCM == kC64 && i >= 64) ? kColS : kColOinter;
       const int64_t b = ui.b;
       const int64_t h = ui.bh % p.H;
       bool good = true;
       for (int32_t c = 0; c < ui.nc; ++c) {
+        const float f = (c & 1) ? f_b : f_a;
         // Stores go out in 4-lane groups: after a 4 x 4 exchange of 16-byte pieces among lanes
         // 4a..4a+3 (rows i0..i0+3 of the chunk), store k writes 64 contiguous bytes of row i0 + k,
         // so every 32-byte sector is written whole by one instruction.
@@ -1022,7 +1219,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ++n_o;
           tc_fence_after();
-          gated_epilogue(p, ctrl, trow, f, ui, h, gate_h, out_h, t, r0, n0, row_stride, ga);
+          gated_epilogue(p, ctrl, trow, col_inter, f, ui, h, gate_h, out_h, t, r0, n0, row_stride,
+                         ga);
           continue;
         }
         ok = mbar_wait_bounded(&ctrl->o_full, n_o & 1, abort_flag, T);
@@ -1036,7 +1234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (uint32_t cb = 0; cb < 4; ++cb) {  // 32-column blocks
           uint32_t ra[32], re[32];
           tmem_ld32(trow + kColOintra + cb * 32, ra);
-          tmem_ld32(trow + kColOinter + cb * 32, re);
+          tmem_ld32(trow + col_inter + cb * 32, re);
           tmem_wait_ld();
           if (cb == 3) {
             // every O column of this row has been read: the accumulators may be overwritten
@@ -1121,7 +1319,8 @@ bool encode_map(CUtensorMap* map, const void* base, int64_t B, int64_t N, int64_
   return r == CUDA_SUCCESS;
 }
 
-SegmentPlan plan_segments(int64_t B, int64_t N, int64_t H, int requested_segments, int num_sms) {
+SegmentPlan plan_segments(int64_t B, int64_t N, int64_t H, int requested_segments, int num_sms,
+                          int chunk) {
   SegmentPlan pl{};
   pl.n_chunks = (N + C - 1) / C;
   const int64_t bh = B * H;
@@ -1141,6 +1340,7 @@ SegmentPlan plan_segments(int64_t B, int64_t N, int64_t H, int requested_segment
   }
   want = std::max<int64_t>(1, std::min<int64_t>(want, pl.n_chunks));
   pl.seg_chunks = (pl.n_chunks + want - 1) / want;
+  if (chunk == 256) pl.seg_chunks += pl.seg_chunks & 1;  // whole 256-token chunks per segment
   pl.segments = (pl.n_chunks + pl.seg_chunks - 1) / pl.seg_chunks;
   pl.units = pl.segments * bh;
   return pl;
@@ -1166,14 +1366,25 @@ namespace {
 cudaError_t launch_common(const PrefillArgs& a, Params& prm, uint8_t* ws,
                           const WorkspaceLayout& wl, int64_t units, cudaStream_t stream,
                           int num_sms, bool clear_header = true) {
+  // the kernel instance for this chunk length and epilogue
+  void (*kernel)(Params) = nullptr;
+  const bool gated = a.gate != nullptr;
+  switch (a.chunk) {
+    case 64:
+      kernel = gated ? chunked_prefill_kernel<true, kC64> : chunked_prefill_kernel<false, kC64>;
+      break;
+    case 128:
+      kernel = gated ? chunked_prefill_kernel<true, kC128> : chunked_prefill_kernel<false, kC128>;
+      break;
+    case 256:
+      kernel = gated ? chunked_prefill_kernel<true, kC256> : chunked_prefill_kernel<false, kC256>;
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
   // set on every call: cheap, safe from any host thread, and it survives a context reset
-  cudaError_t e = cudaFuncSetAttribute(chunked_prefill_kernel<false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemAlloc));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(chunked_prefill_kernel<true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemAlloc));
   if (e != cudaSuccess) return e;
   // counter, status and scan flags start at zero for every call
   if (clear_header) {
@@ -1207,10 +1418,7 @@ cudaError_t launch_common(const PrefillArgs& a, Params& prm, uint8_t* ws,
   prm.withhold_segment = a.withhold_segment;
   prm.prefetch_depth = prefetch_depth();
   const int64_t grid = std::min<int64_t>(units, num_sms);
-  if (prm.gate != nullptr)
-    chunked_prefill_kernel<true><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, stream>>>(prm);
-  else
-    chunked_prefill_kernel<false><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, stream>>>(prm);
+  kernel<<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, stream>>>(prm);
   return cudaGetLastError();
 }
 
@@ -1240,6 +1448,7 @@ struct PlanArgs {
   const int64_t* cu;
   int64_t n_seqs, T, H;
   int32_t requested, num_sms;
+  int32_t pair;  // 256-token chunks: segments hold whole chunks (an even number of tiles)
   int64_t unit_cap, slot_cap;
   WorkUnit* table;  // null: only check cu (recurrent path)
   int32_t* status;
@@ -1249,9 +1458,8 @@ struct PlanArgs {
 // Segments of a sequence of n_chunks chunks: the fixed-length rule of plan_segments, with B*H
 // counted over the non-empty sequences, so equal lengths plan exactly as la_prefill does.  An
 // empty sequence is one unit without chunks.
-__device__ __forceinline__ int64_t segments_of(int64_t n_chunks, int64_t nonempty_heads,
-                                               int32_t requested, int32_t sms) {
-  if (n_chunks == 0) return 1;
+__device__ __forceinline__ int64_t seg_chunks_of(int64_t n_chunks, int64_t nonempty_heads,
+                                                 int32_t requested, int32_t sms, bool pair) {
   int64_t want;
   if (requested > 0) {
     want = requested;
@@ -1261,7 +1469,15 @@ __device__ __forceinline__ int64_t segments_of(int64_t n_chunks, int64_t nonempt
     want = max(int64_t(1), min(int64_t(sms) / nonempty_heads, n_chunks / 4));
   }
   want = max(int64_t(1), min(want, n_chunks));
-  const int64_t seg_chunks = (n_chunks + want - 1) / want;
+  int64_t seg_chunks = (n_chunks + want - 1) / want;
+  if (pair) seg_chunks += seg_chunks & 1;  // whole 256-token chunks per segment
+  return seg_chunks;
+}
+
+__device__ __forceinline__ int64_t segments_of(int64_t n_chunks, int64_t nonempty_heads,
+                                               int32_t requested, int32_t sms, bool pair) {
+  if (n_chunks == 0) return 1;
+  const int64_t seg_chunks = seg_chunks_of(n_chunks, nonempty_heads, requested, sms, pair);
   return (n_chunks + seg_chunks - 1) / seg_chunks;
 }
 
@@ -1349,8 +1565,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_varlen_kernel(const PlanArg
   unsigned long long my_max = 0;
   for (int64_t s = threadIdx.x; s < a.n_seqs; s += kPlanThreads) {
     const int64_t nch = (a.cu[s + 1] - a.cu[s] + C - 1) / C;
-    my_max = max(my_max, static_cast<unsigned long long>(
-                             segments_of(nch, nonempty_heads, a.requested, a.num_sms)));
+    my_max = max(my_max, static_cast<unsigned long long>(segments_of(
+                             nch, nonempty_heads, a.requested, a.num_sms, a.pair != 0)));
   }
   atomicMax(&max_seg, my_max);
   __syncthreads();
@@ -1390,7 +1606,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_varlen_kernel(const PlanArg
       if (s < a.n_seqs) {
         len = a.cu[s + 1] - a.cu[s];
         nch = (len + C - 1) / C;
-        segs = segments_of(nch, nonempty_heads, a.requested, a.num_sms);
+        segs = segments_of(nch, nonempty_heads, a.requested, a.num_sms, a.pair != 0);
       }
       const int64_t active = (s < a.n_seqs && k < segs) ? 1 : 0;
       const int64_t multi = (s < a.n_seqs && segs > 1) ? 1 : 0;
@@ -1403,7 +1619,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_varlen_kernel(const PlanArg
         if (u0 + a.H > a.unit_cap || (multi && slot >= a.slot_cap)) {
           status = -6;  // LA_ERR_WORKSPACE (cannot happen with the host's capacities)
         } else {
-          const int64_t seg_chunks = nch > 0 ? (nch + segs - 1) / segs : 0;
+          const int64_t seg_chunks =
+              nch > 0 ? seg_chunks_of(nch, nonempty_heads, a.requested, a.num_sms, a.pair != 0) : 0;
           const int64_t c0 = k * seg_chunks;
           const int64_t nc = nch > 0 ? min(seg_chunks, nch - c0) : 0;
           const int64_t end = min(len, (c0 + nc) * C);
@@ -1468,6 +1685,7 @@ cudaError_t launch_prefill_varlen(const PrefillArgs& a, const VarlenWorkspace& l
   pa.H = a.H;
   pa.requested = requested_segments;
   pa.num_sms = num_sms;
+  pa.pair = a.chunk == 256 ? 1 : 0;
   pa.unit_cap = layout.unit_cap;
   pa.slot_cap = layout.slot_cap;
   pa.table = tensor_path ? reinterpret_cast<WorkUnit*>(ws + layout.table_off) : nullptr;

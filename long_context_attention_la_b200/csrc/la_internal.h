@@ -34,6 +34,8 @@ struct PrefillArgs {
   const void* gate = nullptr;
   const float* gamma = nullptr;
   float eps = 0.f;
+  // Chunk length of the tensor-core path: 64, 128 or 256 (the 128-token tile is fixed).
+  int32_t chunk = 128;
   // Failure injection for tests (host-side switch, see la_api.cu): the segment index whose scan
   // flag is never published (-1: none) and the limit of every device wait.
   int32_t withhold_segment = -1;
@@ -111,8 +113,12 @@ cudaError_t launch_state_fold(const StateFoldArgs& a, cudaStream_t stream);
 // ---------------------------------------------------------------------------------------------
 // Chunked tensor-core prefill (bf16, d = 128, chunk C = 128).
 // ---------------------------------------------------------------------------------------------
-constexpr int kChunk = 128;
+constexpr int kChunk = 128;  // the tile: tokens per TMA load and per M = 128 MMA
 constexpr int kHeadDim = 128;
+// Chunk lengths the tensor-core prefill supports, and the one it uses when the caller leaves
+// the choice to the library.
+constexpr int kChunkDefault = 128;
+inline bool chunk_supported(int64_t c) { return c == 64 || c == 128 || c == 256; }
 
 // One work unit of the chunked prefill, as the kernel reads it: one segment of one (sequence, head).
 struct WorkUnit {
@@ -130,15 +136,18 @@ struct WorkUnit {
 static_assert(sizeof(WorkUnit) == 48, "WorkUnit is read as three 16-byte words");
 
 // How a prefill is cut into work units: each (b, h) sequence of N tokens becomes `segments`
-// segments of `seg_chunks` chunks (the last may be shorter); one unit = one (segment, b, h).
+// segments of `seg_chunks` 128-token tiles (the last may be shorter); one unit = one
+// (segment, b, h).  With 256-token chunks a segment holds an even number of tiles, so that no
+// chunk straddles two segments.
 struct SegmentPlan {
-  int64_t n_chunks;    // ceil(N / C)
-  int64_t seg_chunks;  // chunks per segment
+  int64_t n_chunks;    // ceil(N / 128)
+  int64_t seg_chunks;  // tiles per segment
   int64_t segments;    // ceil(n_chunks / seg_chunks)
   int64_t units;       // segments * B * H
 };
 
-SegmentPlan plan_segments(int64_t B, int64_t N, int64_t H, int requested_segments, int num_sms);
+SegmentPlan plan_segments(int64_t B, int64_t N, int64_t H, int requested_segments, int num_sms,
+                          int chunk = kChunkDefault);
 
 // Workspace layout of the chunked prefill (byte offsets from the workspace base).
 struct WorkspaceLayout {
@@ -189,6 +198,7 @@ struct VarlenWorkspace {
 };
 VarlenWorkspace varlen_workspace_layout(int64_t T, int64_t n_seqs, int64_t H,
                                         int requested_segments, int num_sms, bool tensor_path);
+// (the chunk length travels in PrefillArgs::chunk)
 
 // Offset of the device-written work-unit count in the workspace header.
 constexpr size_t kWsUnits = 128;

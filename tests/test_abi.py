@@ -66,7 +66,9 @@ def _desc(**kw):
 @pytest.mark.parametrize("kw,status", [
     (dict(B=0), la.LA_ERR_SHAPE), (dict(N=0), la.LA_ERR_SHAPE), (dict(H=0), la.LA_ERR_SHAPE),
     (dict(d=96), la.LA_ERR_SHAPE), (dict(dtype=7), la.LA_ERR_DTYPE),
-    (dict(path=9), la.LA_ERR_UNSUPPORTED), (dict(chunk=64), la.LA_ERR_UNSUPPORTED),
+    (dict(path=9), la.LA_ERR_UNSUPPORTED), (dict(chunk=32), la.LA_ERR_UNSUPPORTED),
+    (dict(chunk=96), la.LA_ERR_UNSUPPORTED), (dict(chunk=512), la.LA_ERR_UNSUPPORTED),
+    (dict(chunk=64, path=la.LA_PATH_RECURRENT), la.LA_ERR_UNSUPPORTED),
     (dict(dtype=la.LA_F32, path=la.LA_PATH_TENSOR), la.LA_ERR_UNSUPPORTED),
     (dict(B=1 << 40, N=1 << 40), la.LA_ERR_OVERFLOW), (dict(segments=-1), la.LA_ERR_SHAPE),
 ])
@@ -139,7 +141,7 @@ _CU = 0x6000
 @pytest.mark.parametrize("kw,status", [
     (dict(dtype=9), la.LA_ERR_DTYPE), (dict(d=32), la.LA_ERR_SHAPE), (dict(H=0), la.LA_ERR_SHAPE),
     (dict(T=-1), la.LA_ERR_SHAPE), (dict(n_seqs=0), la.LA_ERR_SHAPE),
-    (dict(chunk=64), la.LA_ERR_UNSUPPORTED), (dict(path=5), la.LA_ERR_UNSUPPORTED),
+    (dict(chunk=32), la.LA_ERR_UNSUPPORTED), (dict(path=5), la.LA_ERR_UNSUPPORTED),
     (dict(dtype=la.LA_F32, path=la.LA_PATH_TENSOR), la.LA_ERR_UNSUPPORTED),
     (dict(segments=-2), la.LA_ERR_SHAPE), (dict(T=1 << 40, H=1 << 20), la.LA_ERR_OVERFLOW),
 ])
@@ -362,3 +364,20 @@ def test_noalloc_refuses_the_failure_injection_it_cannot_report(lib, monkeypatch
     d = _desc()
     assert la.la_prefill_noalloc(d, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0,
                                  0) == la.LA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("chunk", [0, 64, 128, 256])
+def test_every_supported_chunk_passes_the_host_checks(lib, chunk):
+    # the descriptor is valid, so the call gets as far as the pointer checks
+    d = _desc(chunk=chunk)
+    assert la.la_prefill(d, 0, 0x2000, 0x3000, 0x4000, 0x5000, 0, 0, 0, 0) == la.LA_ERR_NULL
+    assert la.la_prefill_workspace_bytes(d) > 0
+
+
+def test_256_token_chunks_keep_segments_whole(lib):
+    # 7 tiles of 128 tokens forced into 3 segments: 3 tiles each with 128-token chunks, but
+    # segments of whole 256-token chunks need 4 tiles, so only 2 segments (same ring size, since
+    # the ring holds two states per sequence whatever the count)
+    w128 = la.la_prefill_workspace_bytes(_desc(B=1, H=1, N=7 * 128, segments=3, chunk=128))
+    w256 = la.la_prefill_workspace_bytes(_desc(B=1, H=1, N=7 * 128, segments=3, chunk=256))
+    assert w128 == w256 > 256

@@ -54,8 +54,9 @@ def reference(q, k, v, sl, cu, gate, gamma, eps, state_in=None, heads=None):
     return np.concatenate(ys, axis=0)
 
 
+@pytest.mark.parametrize("chunk", [64, 128, 256])
 @pytest.mark.parametrize("segments", [0, 3])
-def test_gated_epilogue_edge_lengths(segments):
+def test_gated_epilogue_edge_lengths(segments, chunk):
     H, d = 4, 128
     lengths = [1, 127, 128, 129, 0, 300, 1000, 2049, 5]
     cu = synth.cu_from_lengths(lengths)
@@ -64,7 +65,7 @@ def test_gated_epilogue_edge_lengths(segments):
     gate, gamma = draw_gate(sum(lengths), H, d, seed=102)
     sin = synth.draw_states(len(lengths), H, d, seed=103, scale=0.3, device=DEV)
     y, st = la.prefill_varlen(q, k, v, sl, cu, state_in=sin, gate=gate, gamma=gamma, eps=EPS,
-                              segments=segments)
+                              segments=segments, chunk=chunk)
     torch.cuda.synchronize()
     ref = reference(q, k, v, sl, cu, gate, gamma, EPS, state_in=sin)
     check_close(y.float().cpu().numpy(), ref, torch.bfloat16, "y")

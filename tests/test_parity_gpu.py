@@ -102,6 +102,23 @@ def test_tensor_small(N, segments):
     check_close(state_heads(st, None), s_ref, torch.bfloat16, f"state N={N} seg={segments}")
 
 
+@pytest.mark.parametrize("chunk", [64, 256])
+@pytest.mark.parametrize("N", [1, 5, 63, 64, 65, 127, 128, 129, 255, 256, 257, 383, 1000, 2100])
+@pytest.mark.parametrize("segments", [0, 1, 2, 3])
+def test_tensor_small_chunks(chunk, N, segments):
+    """Chunk lengths 64 (two chunks per 128-token tile) and 256 (two tiles per chunk): ragged
+    lengths around both chunk sizes, with and without segments."""
+    B, H = 2, 3
+    q, k, v = draw(B, N, H, 128, 400 + N)
+    sl = synth.slopes(H, DEV)
+    out, st = la.prefill(q, k, v, sl, chunk=chunk, segments=segments, path=la.LA_PATH_TENSOR)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle_on(q, k, v, sl)
+    what = f"C={chunk} N={N} seg={segments}"
+    check_close(gpu_heads(out, None), o_ref, torch.bfloat16, f"o {what}")
+    check_close(state_heads(st, None), s_ref, torch.bfloat16, f"state {what}")
+
+
 def test_tensor_prefill_4k_full():
     w = synth.WORKLOADS["prefill_4k"]
     q, k, v = synth.draw_workload(w, device=DEV)
@@ -146,6 +163,38 @@ def test_tensor_prefill_32k_full():
     acc_s.check()
 
 
+def test_chunk_sweep_prefill_32k_full():
+    """P-chunk: the mid-context workload (B=2, N=32768, H=64) with chunk lengths 64, 128 and 256
+    on the tensor cores; each is compared with the oracle over every output and the whole final
+    state, and with the others.  The results differ only in where bf16 roundings fall."""
+    w = synth.WORKLOADS["prefill_32k"]
+    q, k, v = synth.draw_workload(w, device=DEV)
+    sl = synth.slopes(w.H, DEV)
+    chunks = [64, 128, 256]
+    res = {}
+    for c in chunks:
+        res[c] = la.prefill(q, k, v, sl, chunk=c)
+    torch.cuda.synchronize()
+    acc_o = {c: ParityAccumulator(torch.bfloat16, f"prefill_32k C={c} o") for c in chunks}
+    acc_s = {c: ParityAccumulator(torch.bfloat16, f"prefill_32k C={c} state") for c in chunks}
+    for f0 in range(0, w.B * w.H, 16):
+        heads = list(range(f0, f0 + 16))
+        o_ref, s_ref = oracle_on(q, k, v, sl, heads=heads)
+        for c in chunks:
+            out, st = res[c]
+            acc_o[c].add(gather_heads(out, heads), o_ref, tag=f"heads {f0}..{f0 + 15}")
+            acc_s[c].add(state_heads(st, heads), s_ref, tag=f"heads {f0}..{f0 + 15}")
+    for c in chunks:
+        acc_o[c].check()
+        acc_s[c].check()
+    # the chunk lengths against one another (C = 128 as the reference)
+    for c in (64, 256):
+        check_close(res[c][0].float().cpu().numpy(), res[128][0].float().cpu().numpy(),
+                    torch.bfloat16, f"o C={c} vs C=128")
+        check_close(res[c][1].cpu().numpy(), res[128][1].cpu().numpy(), torch.bfloat16,
+                    f"state C={c} vs C=128")
+
+
 def test_tensor_prefill_256k_windows_full():
     """Long context (N=262144, H=64): o of every head on 8 seeded 4096-token windows, and the
     whole final state, against the oracle (which runs the full recurrence of every head)."""
@@ -170,14 +219,15 @@ def test_tensor_prefill_256k_windows_full():
     acc_s.check()
 
 
+@pytest.mark.parametrize("chunk", [64, 128, 256])
 @pytest.mark.parametrize("slope", [0.0, 1e-6])
-def test_scan_long_no_forgetting(slope):
+def test_scan_long_no_forgetting(slope, chunk):
     """With lambda = 1 (or within 1e-6 of it) nothing is forgotten, so a segment scan that lost
     cross-segment state would fail here even though decaying heads would hide it."""
     B, N, H = 1, 65536, 2
     q, k, v = draw(B, N, H, 128, 7)
     sl = torch.full((H,), slope, dtype=torch.float32, device=DEV)
-    out, st = la.prefill(q, k, v, sl)
+    out, st = la.prefill(q, k, v, sl, chunk=chunk)
     torch.cuda.synchronize()
     t_sel = list(range(0, N, 97)) + [N - 1]
     t_sel = sorted(set(t_sel))
@@ -186,14 +236,15 @@ def test_scan_long_no_forgetting(slope):
     check_close(state_heads(st, None), s_ref, torch.bfloat16, "state")
 
 
-def test_segment_count_invariance():
+@pytest.mark.parametrize("chunk", [64, 128, 256])
+def test_segment_count_invariance(chunk):
     B, N, H = 1, 8192, 4
     q, k, v = draw(B, N, H, 128, 8)
     sl = synth.slopes(H, DEV)
     o_ref, s_ref = oracle_on(q, k, v, sl)
     outs = []
     for seg in [1, 2, 3, 7, 64]:
-        out, st = la.prefill(q, k, v, sl, segments=seg, path=la.LA_PATH_TENSOR)
+        out, st = la.prefill(q, k, v, sl, chunk=chunk, segments=seg, path=la.LA_PATH_TENSOR)
         torch.cuda.synchronize()
         check_close(gpu_heads(out, None), o_ref, torch.bfloat16, f"o seg={seg}")
         check_close(state_heads(st, None), s_ref, torch.bfloat16, f"state seg={seg}")
@@ -202,32 +253,35 @@ def test_segment_count_invariance():
         check_close(o.cpu().numpy(), outs[0].cpu().numpy(), torch.bfloat16, "segment agreement")
 
 
-def test_chunked_matches_recurrent():
-    """Chunk length 128 (tensor cores) and chunk length 1 (token recurrence) agree."""
+@pytest.mark.parametrize("chunk", [64, 128, 256])
+def test_chunked_matches_recurrent(chunk):
+    """Chunk lengths 64, 128, 256 (tensor cores) and chunk length 1 (token recurrence) agree."""
     q, k, v = draw(1, 3000, 4, 128, 9)
     sl = synth.slopes(4, DEV)
-    o1, s1 = la.prefill(q, k, v, sl, path=la.LA_PATH_TENSOR)
+    o1, s1 = la.prefill(q, k, v, sl, chunk=chunk, path=la.LA_PATH_TENSOR)
     o2, s2 = la.prefill(q, k, v, sl, path=la.LA_PATH_RECURRENT)
     torch.cuda.synchronize()
     check_close(o1.float().cpu().numpy(), o2.float().cpu().numpy(), torch.bfloat16, "o")
     check_close(s1.cpu().numpy(), s2.cpu().numpy(), torch.bfloat16, "state")
 
 
-def test_no_memory_limit():
+@pytest.mark.parametrize("chunk", [64, 128, 256])
+def test_no_memory_limit(chunk):
     """lambda -> 0 (slope 1e4): o_t = (q_t . k_t) v_t; exercises the general decay-mask path."""
     q, k, v = draw(1, 300, 2, 128, 10)
     sl = torch.full((2,), 1e4, dtype=torch.float32, device=DEV)
-    out, st = la.prefill(q, k, v, sl, path=la.LA_PATH_TENSOR)
+    out, st = la.prefill(q, k, v, sl, chunk=chunk, path=la.LA_PATH_TENSOR)
     torch.cuda.synchronize()
     o_ref, s_ref = oracle_on(q, k, v, sl)
     check_close(gpu_heads(out, None), o_ref, torch.bfloat16, "o")
     check_close(state_heads(st, None), s_ref, torch.bfloat16, "state")
 
 
-def test_silu_inputs_wide_slopes():
+@pytest.mark.parametrize("chunk", [64, 128, 256])
+def test_silu_inputs_wide_slopes(chunk):
     q, k, v = draw(1, 1500, 4, 128, 12, dist="silu_qk")
     sl = torch.tensor([0.0, 0.05, 0.9, 2.5], dtype=torch.float32, device=DEV)
-    out, st = la.prefill(q, k, v, sl, path=la.LA_PATH_TENSOR)
+    out, st = la.prefill(q, k, v, sl, chunk=chunk, path=la.LA_PATH_TENSOR)
     o_ref, s_ref = oracle_on(q, k, v, sl)
     check_close(gpu_heads(out, None), o_ref, torch.bfloat16, "o")
     check_close(state_heads(st, None), s_ref, torch.bfloat16, "state")
@@ -254,12 +308,13 @@ def test_linear_in_v():
     assert torch.equal(s2, 2 * s1)
 
 
-def test_deterministic():
+@pytest.mark.parametrize("chunk", [64, 128, 256])
+def test_deterministic(chunk):
     w = synth.WORKLOADS["prefill_4k"]
     q, k, v = synth.draw_workload(w, device=DEV)
     sl = synth.slopes(w.H, DEV)
-    o1, s1 = la.prefill(q, k, v, sl)
-    o2, s2 = la.prefill(q, k, v, sl)
+    o1, s1 = la.prefill(q, k, v, sl, chunk=chunk)
+    o2, s2 = la.prefill(q, k, v, sl, chunk=chunk)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2)
     assert torch.equal(s1, s2)

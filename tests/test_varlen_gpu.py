@@ -64,15 +64,16 @@ def check_all(out, st, ref, cu, dtype):
     check_close(st.cpu().numpy(), np.stack([r[1] for r in ref]), dtype, "state")
 
 
+@pytest.mark.parametrize("chunk", [64, 128, 256])
 @pytest.mark.parametrize("segments", [0, 1, 3])
 @pytest.mark.parametrize("with_state", [False, True])
-def test_varlen_tensor_edge_lengths(segments, with_state):
+def test_varlen_tensor_edge_lengths(segments, with_state, chunk):
     H, d = 4, 128
     cu = synth.cu_from_lengths(EDGE_LENGTHS)
     q, k, v = draw_packed(EDGE_LENGTHS, H, d, seed=21)
     sl = synth.slopes(H, DEV)
     sin = draw_states(len(EDGE_LENGTHS), H, d, seed=22) if with_state else None
-    out, st = la.prefill_varlen(q, k, v, sl, cu, state_in=sin, segments=segments)
+    out, st = la.prefill_varlen(q, k, v, sl, cu, state_in=sin, segments=segments, chunk=chunk)
     torch.cuda.synchronize()
     ref = oracle_varlen(q, k, v, sl, cu, sin)
     check_all(out, st, ref, cu, torch.bfloat16)
