@@ -206,9 +206,10 @@ la_status la_decode_multi(int64_t B, int64_t H, int64_t d, int64_t n_tok, int32_
  *
  *   - Limit: problems whose scratch need (la_prefill_workspace_bytes) exceeds
  *     LA_NOALLOC_SCRATCH_BYTES are rejected with LA_ERR_WORKSPACE before anything is enqueued.
- *     Within the limit are every problem with B*H <= 64 (for example one sequence of the 64-head
- *     layer at any length) and every problem run with one segment per sequence (the automatic
- *     choice once B*H exceeds half the number of SMs); the fp32 / recurrent path needs no
+ *     Within the limit is every problem with the automatic plan (desc->segments = 0) on a GPU of
+ *     up to 256 SMs, whatever B, N and H: that plan needs a header plus one flag and one
+ *     d x d fp32 state per SM.  An explicit segment count needs two states per sequence when it
+ *     cuts sequences, which fits for B*H up to 128.  The fp32 / recurrent path needs no
  *     scratch at all.
  *   - First call on a device: it looks up the device address of the array (cudaGetSymbolAddress)
  *     with that device current and caches it for that device's CUDA context; make that first
@@ -226,7 +227,7 @@ la_status la_decode_multi(int64_t B, int64_t H, int64_t d, int64_t n_tok, int32_
  *     LA_ERR_UNSUPPORTED while the test-only failure injection (environment variable
  *     LA_DEBUG_WITHHOLD_SEGMENT) is set.
  */
-#define LA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u + 4096u)
+#define LA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u + 4096u)
 la_status la_prefill_noalloc(const la_desc* desc, const void* q, const void* k, const void* v,
                              const float* slopes, void* out, float* state_out, void* stream);
 

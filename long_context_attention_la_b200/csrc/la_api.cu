@@ -46,6 +46,16 @@ bool use_tensor_path(const la_desc* d) { return use_tensor_path(d->path, d->dtyp
 // The tensor path's chunk length for a descriptor's `chunk` field (0: the library's default).
 int chunk_of(int32_t chunk) { return chunk == 0 ? la::kChunkDefault : chunk; }
 
+// Workspace bytes of la_prefill's tensor path: the balanced plan when the segment count is left
+// to the library, else equal segments per sequence.
+size_t prefill_workspace_need(const la_desc* d, int sms) {
+  if (d->segments == 0)
+    return la::balanced_workspace_bytes(la::plan_balanced(d->B, d->N, d->H, sms, chunk_of(d->chunk)));
+  const la::SegmentPlan plan =
+      la::plan_segments(d->B, d->N, d->H, d->segments, sms, chunk_of(d->chunk));
+  return la::workspace_layout(d->B, d->H, plan).total;
+}
+
 // Failure injection for tests, read on every call: LA_DEBUG_WITHHOLD_SEGMENT=k keeps segment k of
 // every sequence from publishing its scan state, so segment k+1 waits until its bounded wait
 // expires (LA_DEBUG_WAIT_LIMIT_MS, default 2000) and the call reports LA_ERR_TIMEOUT through
@@ -127,10 +137,7 @@ size_t la_prefill_workspace_bytes(const la_desc* desc) {
   int64_t numel = 0;
   if (check_desc(desc, &numel) != LA_OK) return 0;
   if (!use_tensor_path(desc)) return 0;
-  const la::SegmentPlan plan =
-      la::plan_segments(desc->B, desc->N, desc->H, desc->segments,
-                        device_sms() > 0 ? device_sms() : 148, chunk_of(desc->chunk));
-  return la::workspace_layout(desc->B, desc->H, plan).total;
+  return prefill_workspace_need(desc, device_sms() > 0 ? device_sms() : 148);
 }
 
 }  // extern "C"
@@ -181,9 +188,17 @@ la_status la_prefill(const la_desc* desc, const void* q, const void* k, const vo
   }
   const int sms = device_sms();
   if (sms <= 0) return LA_ERR_CUDA;
-  const la::SegmentPlan plan = la::plan_segments(desc->B, desc->N, desc->H, desc->segments, sms,
-                                                   chunk_of(desc->chunk));
-  const size_t need = la::workspace_layout(desc->B, desc->H, plan).total;
+  const bool balanced = desc->segments == 0;
+  la::BalancedPlan bplan{};
+  la::SegmentPlan splan{};
+  size_t need = 0;
+  if (balanced) {
+    bplan = la::plan_balanced(desc->B, desc->N, desc->H, sms, a.chunk);
+    need = la::balanced_workspace_bytes(bplan);
+  } else {
+    splan = la::plan_segments(desc->B, desc->N, desc->H, desc->segments, sms, a.chunk);
+    need = la::workspace_layout(desc->B, desc->H, splan).total;
+  }
   void* ws = workspace;
   bool owned = false;
   if (ws == nullptr) {
@@ -193,7 +208,8 @@ la_status la_prefill(const la_desc* desc, const void* q, const void* k, const vo
     if (workspace_bytes < need) return LA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return LA_ERR_ALIGN;
   }
-  const cudaError_t e = la::launch_chunked_prefill(a, plan, ws, s, sms);
+  const cudaError_t e = balanced ? la::launch_chunked_prefill_balanced(a, bplan, ws, s, sms)
+                                 : la::launch_chunked_prefill(a, splan, ws, s, sms);
   if (owned) cudaFreeAsync(ws, s);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
@@ -582,10 +598,7 @@ la_status la_prefill_noalloc(const la_desc* desc, const void* q, const void* k, 
   }
   const int sms = device_sms();
   if (sms <= 0) return LA_ERR_CUDA;
-  const la::SegmentPlan plan = la::plan_segments(desc->B, desc->N, desc->H, desc->segments, sms,
-                                                   chunk_of(desc->chunk));
-  const size_t need = la::workspace_layout(desc->B, desc->H, plan).total;
-  if (need > LA_NOALLOC_SCRATCH_BYTES) return LA_ERR_WORKSPACE;
+  if (prefill_workspace_need(desc, sms) > LA_NOALLOC_SCRATCH_BYTES) return LA_ERR_WORKSPACE;
   void* scratch = nullptr;
   const la_status sa = noalloc_scratch(&scratch);
   if (sa != LA_OK) return sa;

@@ -134,6 +134,10 @@ struct Params {
   uint64_t timeout_ns;
   int32_t prefetch_depth;
   int32_t withhold_segment;  // failure injection: this segment never publishes (-1: none)
+  // balanced plan (n_ranges > 0): range r covers flat tiles [range_start[r], range_start[r+1])
+  // of the head-major list of B*H sequences of n_chunks tiles
+  int32_t n_ranges;
+  int32_t range_start[kMaxRanges + 1];
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -242,9 +246,13 @@ __device__ __forceinline__ void decode_unit(const Params& p, int64_t u, UnitInfo
     ui.b = w1.z;
     ui.tok0 = w1.w;
     ui.slot = w2.x;
+    ui.in_slot = w2.y;
+    ui.in_val = w2.z;
+    ui.pub_val = w2.w;
     return;
   }
-  // fixed length: unit u = segment k of flat head bh, segment-major
+  // fixed length: unit u = segment k of flat head bh, segment-major; a two-slot state ring per
+  // sequence, segment k publishing into slot k & 1 with flag value k + 1
   const int64_t k = u / p.BH;
   const int64_t bh = u % p.BH;
   const int64_t c0 = k * p.seg_chunks;
@@ -255,10 +263,81 @@ __device__ __forceinline__ void decode_unit(const Params& p, int64_t u, UnitInfo
   ui.c0 = static_cast<int32_t>(c0);
   ui.nc = static_cast<int32_t>(nc);
   ui.len = static_cast<int32_t>(end - c0 * C);
-  ui.flags = (k + 1 < p.segments ? 1 : 0) | (k + 1 == p.segments ? 2 : 0);
+  ui.flags = (k + 1 < p.segments ? kUnitLocal : 0) | (k + 1 == p.segments ? kUnitFinal : 0);
   ui.b = static_cast<int32_t>(bh / p.H);
   ui.tok0 = 0;
-  ui.slot = static_cast<int32_t>(bh);
+  ui.slot = static_cast<int32_t>(bh * 2 + (k & 1));
+  ui.in_slot = k > 0 ? static_cast<int32_t>(bh * 2 + ((k - 1) & 1)) : -1;
+  ui.in_val = static_cast<int32_t>(k);
+  ui.pub_val = static_cast<int32_t>(k + 1);
+}
+
+// Balanced plan: the units of range r, in order.  Cursor state lives with the producer thread.
+struct RangeCursor {
+  int32_t r = -1;          // current range (-1: none yet)
+  int64_t next = 0, end = 0;  // next flat tile of the range, and its end
+  bool local_pending = false; // the cut last piece's local-state unit is still to be issued
+};
+
+// Fills ui with the piece of flat tiles [t0, t1) of one sequence (t1 inside or at its end).
+__device__ __forceinline__ void piece_unit(const Params& p, int64_t t0, int64_t t1, UnitInfo& ui) {
+  const int64_t n = p.n_chunks;
+  const int64_t sq = t0 / n;
+  const int64_t c0 = t0 - sq * n;
+  const int64_t nc = t1 - t0;
+  ui.bh = static_cast<int32_t>(sq);
+  ui.seg = c0 > 0 ? 1 : 0;
+  ui.c0 = static_cast<int32_t>(c0);
+  ui.nc = static_cast<int32_t>(nc);
+  ui.len = static_cast<int32_t>(min(p.N, (c0 + nc) * C) - c0 * C);
+  ui.b = static_cast<int32_t>(sq / p.H);
+  ui.tok0 = 0;
+}
+
+// Next unit of the balanced plan (ui.bh = -1 when every range has been taken).  A piece that
+// starts inside its sequence begins its range, and its predecessor is the cut last piece of the
+// previous range, whose local-state unit published into ring slot r - 1.
+__device__ __forceinline__ void next_balanced_unit(const Params& p, RangeCursor& cur,
+                                                   UnitInfo& ui) {
+  const int64_t n = p.n_chunks;
+  while (true) {
+    if (cur.r >= 0 && cur.local_pending) {
+      cur.local_pending = false;
+      const int64_t last0 = max(cur.next, ((cur.end - 1) / n) * n);  // the cut piece's start
+      piece_unit(p, last0, cur.end, ui);
+      ui.flags = kUnitLocal | kUnitNoOutput;
+      ui.slot = cur.r;
+      ui.pub_val = 1;
+      ui.in_slot = ui.c0 > 0 ? cur.r - 1 : -1;
+      ui.in_val = 1;
+      return;
+    }
+    if (cur.r >= 0 && cur.next < cur.end) {
+      const int64_t t0 = cur.next;
+      const int64_t seq_end = (t0 / n + 1) * n;
+      const int64_t t1 = min(cur.end, seq_end);
+      piece_unit(p, t0, t1, ui);
+      ui.flags = t1 == seq_end ? kUnitFinal : 0;
+      ui.slot = -1;
+      ui.pub_val = 0;
+      ui.in_slot = ui.c0 > 0 ? cur.r - 1 : -1;
+      ui.in_val = 1;
+      cur.next = t1;
+      return;
+    }
+    const int32_t r = static_cast<int32_t>(atomicAdd(p.counter, 1u));
+    if (r >= p.n_ranges) {
+      ui.bh = -1;
+      ui.seg = ui.c0 = ui.nc = ui.len = ui.flags = ui.b = ui.tok0 = ui.slot = 0;
+      ui.in_slot = -1;
+      ui.in_val = ui.pub_val = 0;
+      return;
+    }
+    cur.r = r;
+    cur.next = p.range_start[r];
+    cur.end = p.range_start[r + 1];
+    cur.local_pending = cur.end % n != 0;  // the range ends inside a sequence
+  }
 }
 
 // Output epilogue with the fused grouped RMSNorm and sigmoid gate ("Ling and Ring 2.6 Technical
@@ -429,7 +508,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // A unit is a stream of chunk-loads: nc local-state loads (K, V) if it has that pass,
       // then nc output loads (Q, K, V).
+      RangeCursor rcur;
       auto fetch = [&](UnitInfo& ui) {
+        if (p.n_ranges > 0) {
+          next_balanced_unit(p, rcur, ui);
+          return;
+        }
         const int64_t u = static_cast<int64_t>(atomicAdd(p.counter, 1u));
         const int64_t units = p.units_dev != nullptr ? *p.units_dev : p.units;
         if (u < units) {
@@ -437,10 +521,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           ui.bh = -1;
           ui.seg = ui.c0 = ui.nc = ui.len = ui.flags = ui.b = ui.tok0 = ui.slot = 0;
+          ui.in_slot = -1;
+          ui.in_val = ui.pub_val = 0;
         }
       };
       auto n_loads = [](const UnitInfo& ui) -> int32_t {
-        return ui.bh < 0 ? 0 : ((ui.flags & 1) ? 2 * ui.nc : ui.nc);
+        if (ui.bh < 0) return 0;
+        if (!(ui.flags & kUnitLocal)) return ui.nc;
+        return (ui.flags & kUnitNoOutput) ? ui.nc : 2 * ui.nc;
       };
       // L2 prefetch of chunk-load `pos` of `ui` (the part of it that comes from DRAM)
       auto prefetch = [&](const UnitInfo& ui, int32_t pos) {
@@ -625,7 +713,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           umma_commit(&ctrl->h_done);
         }
-        for (int32_t c = 0; c < ui.nc && ok; ++c) {
+        const int32_t n_out = (ui.flags & kUnitNoOutput) ? 0 : ui.nc;
+        for (int32_t c = 0; c < n_out && ok; ++c) {
           const uint32_t s = g & 1;
           const uint32_t ph = (g >> 1) & 1;
           if (!mbar_wait_bounded(&ctrl->full[s], ph, abort_flag, T)) {
@@ -640,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // C = 256: the first tile A (even c) of a two-tile chunk keeps its stage until the second
           // tile B (odd c) has read K~_A and V_A from it (stage s ^ 1).
           const bool tile_b = kCM == kC256 && (c & 1) != 0;
-          const bool keep_stage = kCM == kC256 && (c & 1) == 0 && c + 1 < ui.nc;
+          const bool keep_stage = kCM == kC256 && (c & 1) == 0 && c + 1 < n_out;
           // D (+)= Q K^T over d = 128 (both K-major), from this tile's Q and the keys at kbase
           auto issue_qk = [&](uint32_t d_col, uint32_t kbase) {
 #pragma unroll
@@ -835,7 +924,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++g;
         }
       }
-      for (int32_t c = 0; c < ui.nc; ++c) {
+      const int32_t n_out = (ui.flags & kUnitNoOutput) ? 0 : ui.nc;
+      for (int32_t c = 0; c < n_out; ++c) {
         if (kCM == kC256 && (c & 1) != 0) {
           // Second tile of a 256-token chunk: P_BA = lambda^(i+1) S~_BA over all 128 columns
           // (S~_BA = Q_B K~_A^T already carries lambda^(127-j)), no causal mask.  The block split
@@ -973,22 +1063,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ui.bh < 0) break;
       const float alpha = p.slopes[ui.bh % p.H] * kLog2e;
       const int64_t bh = ui.bh;    // state_in / state_out index
-      const int64_t rs = ui.slot;  // scan flags and state ring (sequences cut into segments)
       const int32_t k = ui.seg;
+      const bool publish = (ui.flags & kUnitLocal) != 0;
+      const bool outputs = (ui.flags & kUnitNoOutput) == 0;
 
-      if (ui.flags & 1) {
+      if (publish) {
         ok = mbar_wait_bounded(&ctrl->h_done, n_h & 1, abort_flag, T);
         if (!group_all(ok, kBarS, 128)) break;
         ++n_h;
         tc_fence_after();
         g += static_cast<uint32_t>(ui.nc);  // the local-state pass used these stages
       }
-      // incoming state of this segment: published by segment k-1 of the same sequence
-      if (k > 0) {
-        const uint32_t* fl = p.flags + rs * 2 + ((k - 1) & 1);
+      // incoming state of this piece: published by the previous piece of the same sequence
+      if (ui.in_slot >= 0) {
+        const uint32_t* fl = p.flags + ui.in_slot;
         const uint64_t t0 = globaltimer_ns();
         ok = true;
-        while (ld_acquire_u32(fl) != static_cast<uint32_t>(k)) {
+        while (ld_acquire_u32(fl) != static_cast<uint32_t>(ui.in_val)) {
           if (*abort_flag || ld_volatile_s32(p.status) != 0 || globaltimer_ns() - t0 > T) {
             ok = false;
             *abort_flag = 1u;
@@ -998,9 +1089,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!group_all(ok, kBarS, 128)) break;
       }
       // ring layout: float4 (state row i, columns 4q..4q+3) at index q * 128 + i
-      const float4* ring_in =
-          reinterpret_cast<const float4*>(p.ring + (rs * 2 + ((k - 1) & 1)) * (D * D));
-      float4* ring_out = reinterpret_cast<float4*>(p.ring + (rs * 2 + (k & 1)) * (D * D));
+      const float4* ring_in = reinterpret_cast<const float4*>(
+          p.ring + static_cast<int64_t>(ui.in_slot >= 0 ? ui.in_slot : 0) * (D * D));
+      float4* ring_out = reinterpret_cast<float4*>(
+          p.ring + static_cast<int64_t>(publish ? ui.slot : 0) * (D * D));
       const float lam_len = exp2f(-alpha * static_cast<float>(ui.len));
       // decay of the incoming state over the first chunk (C = 64: the first half of tile 0)
       const float lam_n0 =
@@ -1008,7 +1100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (uint32_t cb = 0; cb < 4; ++cb) {
         uint32_t sin[32];  // fp32 bits of the incoming state, columns [32 cb, 32 cb + 32)
-        if (k > 0) {
+        if (ui.in_slot >= 0) {
 #pragma unroll
           for (uint32_t q = 0; q < 8; ++q) {
             const float4 x = __ldcg(ring_in + (cb * 8 + q) * 128 + i);
@@ -1032,8 +1124,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int m = 0; m < 32; ++m) sin[m] = 0u;
         }
-        if (ui.flags & 1) {
-          // inclusive state S_{k+1} = lambda^L S_k + h_k, published for segment k+1
+        if (publish) {
+          // inclusive state S_{k+1} = lambda^L S_k + h_k, published for the next piece
           uint32_t r[32];
           tmem_ld32(trow + kColKV + cb * 32, r);
           tmem_wait_ld();
@@ -1055,20 +1147,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             so[q] = make_float4(__uint_as_float(sin[4 * q]), __uint_as_float(sin[4 * q + 1]),
                                 __uint_as_float(sin[4 * q + 2]), __uint_as_float(sin[4 * q + 3]));
         }
-        write_kvb(cb, sin);
+        if (outputs) {
+          // the incoming state: bf16 operand of the first tile's inter product, and the fp32
+          // state the tiles carry (already decayed over the first chunk)
+          write_kvb(cb, sin);
 #pragma unroll
-        for (int m = 0; m < 32; ++m) sin[m] = __float_as_uint(lam_n0 * __uint_as_float(sin[m]));
-        tmem_st32(trow + kColKV + cb * 32, sin);
+          for (int m = 0; m < 32; ++m) sin[m] = __float_as_uint(lam_n0 * __uint_as_float(sin[m]));
+          tmem_st32(trow + kColKV + cb * 32, sin);
+        }
       }
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
-      if (ui.flags & 1) {
+      if (publish) {
         __threadfence();
         named_bar_sync(kBarS, 128);
         if (wq == 0 && lane == 0 && k != p.withhold_segment) {
           __threadfence();
-          st_release_u32(p.flags + rs * 2 + (k & 1), static_cast<uint32_t>(k + 1));
+          st_release_u32(p.flags + ui.slot, static_cast<uint32_t>(ui.pub_val));
         }
       }
 
@@ -1090,7 +1186,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
       };
-      for (int32_t c = 0; c < ui.nc; ++c) {
+      const int32_t n_out = outputs ? ui.nc : 0;
+      for (int32_t c = 0; c < n_out; ++c) {
         const uint32_t s = g & 1;
         const int32_t n_c = min(C, ui.len - c * C);  // tokens in this tile
         // the state operand for tile c is in place (written before the loop or by the previous
@@ -1140,7 +1237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++n_kvd;
           tc_fence_after();
         }
-        if (c + 1 < ui.nc) {
+        if (c + 1 < n_out) {
           int32_t n_next = min(C, ui.len - (c + 1) * C);
           if (kCM == kC64) n_next = min(64, n_next);  // the next tile's first chunk
           // C = 256: after a chunk's first tile the operand stays the chunk's initial state
@@ -1196,7 +1293,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t b = ui.b;
       const int64_t h = ui.bh % p.H;
       bool good = true;
-      for (int32_t c = 0; c < ui.nc; ++c) {
+      const int32_t n_out = (ui.flags & kUnitNoOutput) ? 0 : ui.nc;
+      for (int32_t c = 0; c < n_out; ++c) {
         const float f = (c & 1) ? f_b : f_a;
         // Stores go out in 4-lane groups: after a 4 x 4 exchange of 16-byte pieces among lanes
         // 4a..4a+3 (rows i0..i0+3 of the chunk), store k writes 64 contiguous bytes of row i0 + k,
@@ -1346,6 +1444,92 @@ SegmentPlan plan_segments(int64_t B, int64_t N, int64_t H, int requested_segment
   return pl;
 }
 
+namespace {
+
+// Extra cost of a tile in a range's cut last piece (its local-state pass reads K and V once more),
+// relative to an output tile.  LA_BALANCE_LOCAL_COST (percent) overrides it: a tuning knob, every
+// value computes the same result.
+double local_pass_cost() {
+  static double v = -1.0;
+  if (v < 0.0) {
+    double c = 0.5;
+    if (const char* e = getenv("LA_BALANCE_LOCAL_COST")) c = std::max(0, std::min(300, atoi(e))) / 100.0;
+    v = c;
+  }
+  return v;
+}
+
+// The furthest end b > a of a range starting at flat tile a whose cost is at most cap: tiles
+// count 1, plus rho for each tile of a last piece that ends inside its sequence.  Ends at
+// sequence boundaries cost nothing extra; an end inside a sequence falls on an even tile offset
+// when `pair` (256-token chunks).
+int64_t range_end(int64_t a, double cap, int64_t n, int64_t total, double rho, bool pair) {
+  const int64_t seq_end = (a / n + 1) * n;
+  int64_t best = a;
+  int64_t q0 = (a / n) * n;  // start of the sequence an end inside a sequence would fall in
+  if (static_cast<double>(seq_end - a) <= cap) {
+    const int64_t k = static_cast<int64_t>((cap - static_cast<double>(seq_end - a)) / n);
+    best = std::min(total, seq_end + k * n);
+    q0 = best;
+  }
+  if (q0 < total) {
+    const int64_t p0 = std::max(a, q0);  // the last piece's first tile
+    // (b - a) + rho (b - p0) <= cap
+    int64_t b = static_cast<int64_t>((cap + static_cast<double>(a) + rho * p0) / (1.0 + rho));
+    b = std::min(b, q0 + n - 1);
+    if (pair) b = q0 + ((b - q0) & ~int64_t(1));
+    if (b > p0 && b > best) best = b;
+  }
+  return std::min(best, total);
+}
+
+}  // namespace
+
+BalancedPlan plan_balanced(int64_t B, int64_t N, int64_t H, int num_sms, int chunk) {
+  BalancedPlan pl{};
+  const int64_t n = (N + C - 1) / C;
+  const int64_t total = B * H * n;
+  pl.seq_tiles = static_cast<int32_t>(n);
+  pl.total_tiles = total;
+  const int64_t r_max = std::max<int64_t>(
+      1, std::min<int64_t>({static_cast<int64_t>(std::max(num_sms, 1)), int64_t(kMaxRanges), total}));
+  const double rho = local_pass_cost();
+  const bool pair = chunk == 256;
+  // greedy cut with a cost cap; true when it covers every tile in r_max ranges or fewer
+  auto cut = [&](double cap, BalancedPlan* out) -> bool {
+    int64_t a = 0;
+    int32_t r = 0;
+    if (out) out->start[0] = 0;
+    while (a < total) {
+      if (r >= r_max) return false;
+      int64_t b = range_end(a, cap, n, total, rho, pair);
+      if (b <= a) {  // always make progress: one tile (two inside a sequence for pairs)
+        const int64_t se = (a / n + 1) * n;
+        b = std::min(se, a + (pair ? 2 : 1));
+      }
+      a = b;
+      ++r;
+      if (out) out->start[r] = static_cast<int32_t>(a);
+    }
+    if (out) out->n_ranges = r;
+    return true;
+  };
+  double lo = static_cast<double>(total) / static_cast<double>(r_max);
+  double hi = (1.0 + rho) * (lo + static_cast<double>(n)) + 2.0;
+  while (!cut(hi, nullptr)) hi *= 2.0;
+  for (int it = 0; it < 48 && hi - lo > 0.25; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (cut(mid, nullptr)) hi = mid; else lo = mid;
+  }
+  cut(hi, &pl);
+  return pl;
+}
+
+size_t balanced_workspace_bytes(const BalancedPlan& plan) {
+  const size_t flags = (static_cast<size_t>(plan.n_ranges) * 4 + 255) / 256 * 256;
+  return 256 + flags + static_cast<size_t>(plan.n_ranges) * D * D * sizeof(float);
+}
+
 WorkspaceLayout workspace_layout(int64_t B, int64_t H, const SegmentPlan& plan) {
   WorkspaceLayout w{};
   const int64_t bh = B * H;
@@ -1428,12 +1612,42 @@ cudaError_t launch_chunked_prefill(const PrefillArgs& a, const SegmentPlan& plan
                                    void* workspace, cudaStream_t stream, int num_sms) {
   Params prm{};
   prm.unit_table = nullptr;
+  prm.n_ranges = 0;
   prm.BH = a.B * a.H;
   prm.n_chunks = plan.n_chunks;
   prm.seg_chunks = plan.seg_chunks;
   prm.segments = plan.segments;
   return launch_common(a, prm, static_cast<uint8_t*>(workspace), workspace_layout(a.B, a.H, plan),
                        plan.units, stream, num_sms);
+}
+
+cudaError_t launch_chunked_prefill_balanced(const PrefillArgs& a, const BalancedPlan& plan,
+                                            void* workspace, cudaStream_t stream, int num_sms) {
+  // the plan must cover the tile list with increasing range starts; inside a sequence a range
+  // starts on an even tile for 256-token chunks (checked here, since the kernel trusts it)
+  if (plan.n_ranges < 1 || plan.n_ranges > kMaxRanges || plan.start[0] != 0 ||
+      plan.start[plan.n_ranges] != plan.total_tiles || plan.seq_tiles < 1)
+    return cudaErrorInvalidValue;
+  for (int r = 0; r < plan.n_ranges; ++r) {
+    if (plan.start[r + 1] <= plan.start[r]) return cudaErrorInvalidValue;
+    if (a.chunk == 256 && (plan.start[r] % plan.seq_tiles) % 2 != 0) return cudaErrorInvalidValue;
+  }
+  Params prm{};
+  prm.unit_table = nullptr;
+  prm.BH = a.B * a.H;
+  prm.n_chunks = plan.seq_tiles;
+  prm.n_ranges = plan.n_ranges;
+  for (int r = 0; r <= plan.n_ranges; ++r) prm.range_start[r] = plan.start[r];
+  WorkspaceLayout wl{};
+  wl.header_bytes = 256;
+  wl.flags_off = 256;
+  wl.flags_bytes = (static_cast<size_t>(plan.n_ranges) * 4 + 255) / 256 * 256;
+  wl.ring_off = wl.flags_off + wl.flags_bytes;
+  wl.ring_bytes = static_cast<size_t>(plan.n_ranges) * D * D * sizeof(float);
+  wl.total = wl.ring_off + wl.ring_bytes;
+  // one CTA per range at most; a CTA that finishes its range takes the next untaken one
+  return launch_common(a, prm, static_cast<uint8_t*>(workspace), wl, plan.n_ranges, stream,
+                       num_sms);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -1632,10 +1846,15 @@ __global__ void __launch_bounds__(kPlanThreads) plan_varlen_kernel(const PlanArg
           w.flags = (k + 1 < segs ? 1 : 0) | (k + 1 == segs ? 2 : 0);
           w.b = 0;
           w.tok0 = static_cast<int32_t>(a.cu[s]);
-          w.pad[0] = w.pad[1] = w.pad[2] = 0;
+          // a sequence cut into segments has a two-slot state ring per head: segment k
+          // publishes into slot k & 1 with flag value k + 1
+          w.in_val = static_cast<int32_t>(k);
+          w.pub_val = static_cast<int32_t>(k + 1);
           for (int64_t h = 0; h < a.H; ++h) {
             w.bh = static_cast<int32_t>(s * a.H + h);
-            w.slot = multi ? static_cast<int32_t>(slot * a.H + h) : w.bh;
+            const int64_t rs = slot * a.H + h;
+            w.slot = multi ? static_cast<int32_t>(rs * 2 + (k & 1)) : -1;
+            w.in_slot = (multi && k > 0) ? static_cast<int32_t>(rs * 2 + ((k - 1) & 1)) : -1;
             a.table[u0 + h] = w;
           }
         }

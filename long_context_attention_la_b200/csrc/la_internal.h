@@ -120,18 +120,28 @@ constexpr int kHeadDim = 128;
 constexpr int kChunkDefault = 128;
 inline bool chunk_supported(int64_t c) { return c == 64 || c == 128 || c == 256; }
 
-// One work unit of the chunked prefill, as the kernel reads it: one segment of one (sequence, head).
+// One work unit of the chunked prefill, as the kernel reads it: one piece (a run of consecutive
+// tiles) of one (sequence, head).  A unit with kUnitLocal first computes the piece's local state
+// h = sum_j lambda^(L-1-j) k_j^T v_j, takes its incoming state S from ring slot in_slot, and
+// publishes S_out = lambda^L S + h into ring slot `slot` (flag value pub_val), so that the next
+// piece can start before this one's outputs exist; with kUnitNoOutput it stops there.  Every
+// other unit runs the output pass from its incoming state.
+constexpr int32_t kUnitLocal = 1;     // local-state pass and publish first
+constexpr int32_t kUnitFinal = 2;     // last piece of the sequence: write state_out
+constexpr int32_t kUnitNoOutput = 4;  // publish only (the outputs are another unit's)
 struct WorkUnit {
-  int32_t bh;     // state index: sequence * H + head (-1: no more work)
-  int32_t seg;    // segment index k within the sequence
-  int32_t c0;     // first chunk of the segment, counted from the sequence start
-  int32_t nc;     // chunks in the segment (0: an empty sequence, whose state passes through)
-  int32_t len;    // tokens in the segment
-  int32_t flags;  // bit 0: compute the local state first; bit 1: last segment of the sequence
-  int32_t b;      // batch coordinate of the sequence in the [B, N, H, d] tensors
-  int32_t tok0;   // token coordinate (along N) of the sequence's first token
-  int32_t slot;   // scan-flag / state-ring index of a sequence cut into segments (per head)
-  int32_t pad[3];
+  int32_t bh;       // state index: sequence * H + head (-1: no more work)
+  int32_t seg;      // piece index within the sequence (0: its first piece)
+  int32_t c0;       // first tile of the piece, counted from the sequence start
+  int32_t nc;       // tiles in the piece (0: an empty sequence, whose state passes through)
+  int32_t len;      // tokens in the piece
+  int32_t flags;    // kUnitLocal | kUnitFinal | kUnitNoOutput
+  int32_t b;        // batch coordinate of the sequence in the [B, N, H, d] tensors
+  int32_t tok0;     // token coordinate (along N) of the sequence's first token
+  int32_t slot;     // ring slot this unit publishes into (with kUnitLocal)
+  int32_t in_slot;  // ring slot of the incoming state (-1: state_in, or zero)
+  int32_t in_val;   // flag value that marks in_slot as published
+  int32_t pub_val;  // flag value this unit publishes with
 };
 static_assert(sizeof(WorkUnit) == 48, "WorkUnit is read as three 16-byte words");
 
@@ -148,6 +158,25 @@ struct SegmentPlan {
 
 SegmentPlan plan_segments(int64_t B, int64_t N, int64_t H, int requested_segments, int num_sms,
                           int chunk = kChunkDefault);
+
+// Balanced plan (the automatic plan of la_prefill): the B*H sequences' tiles, head-major, are cut
+// into at most one range per SM such that every range costs about the same, counting a tile of a
+// piece that the range's end cuts off from the rest of its sequence (1 + rho) times, since that
+// piece needs a local-state pass.  Range r runs [start[r], start[r+1]) as: the local-state pass of
+// its last piece when that piece is cut (publishing into ring slot r), then the outputs of its
+// pieces in order.  A range ends at an even tile offset within a sequence for 256-token chunks.
+constexpr int kMaxRanges = 256;
+struct BalancedPlan {
+  int32_t n_ranges;
+  int32_t seq_tiles;                  // tiles per sequence
+  int64_t total_tiles;                // B * H * seq_tiles
+  int32_t start[kMaxRanges + 1];
+};
+BalancedPlan plan_balanced(int64_t B, int64_t N, int64_t H, int num_sms, int chunk);
+// workspace: header, one scan flag and one d x d fp32 ring slot per range
+size_t balanced_workspace_bytes(const BalancedPlan& plan);
+cudaError_t launch_chunked_prefill_balanced(const PrefillArgs& a, const BalancedPlan& plan,
+                                            void* workspace, cudaStream_t stream, int num_sms);
 
 // Workspace layout of the chunked prefill (byte offsets from the workspace base).
 struct WorkspaceLayout {

@@ -156,7 +156,7 @@ def la_prefill_noalloc(desc: la_desc, q: int, k: int, v: int, slopes: int, out: 
                                             state_out or None, stream or None))
 
 
-LA_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024 + 4096
+LA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024 + 4096
 
 
 def la_prefill_varlen_workspace_bytes(desc: la_varlen_desc) -> int:

@@ -60,8 +60,8 @@ def test_noalloc_matches_allocating_entry_point_twice():
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
-    # 2 x 64 sequences cut into 2 segments each need a 16 MiB ring: more than the array holds
-    B, N, H, d = 2, 4096, 64, 128
+    # 4 x 64 sequences cut into 2 segments each need a 32 MiB ring: more than the array holds
+    B, N, H, d = 4, 4096, 64, 128
     desc = la.make_desc(B, N, H, d, torch.bfloat16, segments=2)
     assert la.la_prefill_workspace_bytes(desc) > la.LA_NOALLOC_SCRATCH_BYTES
     q = torch.zeros(B, N, H, d, dtype=torch.bfloat16, device="cuda")
