@@ -97,19 +97,25 @@ def test_varlen_recurrent(d, dtype):
     check_all(out, st, oracle_varlen(q, k, v, sl, cu, sin), cu, dtype)
 
 
-def test_varlen_equal_lengths_match_fixed_batch():
-    """B sequences of N tokens packed back to back are the [B, N, H, d] problem: same plan, same
-    bits."""
+@pytest.mark.parametrize("segments", [1, 2, 3])
+def test_varlen_equal_lengths_match_fixed_batch(segments):
+    """B sequences of N tokens packed back to back are the [B, N, H, d] problem: with the same
+    explicit segment count both forms plan the same segments, so the bits agree; the automatic
+    plans (balanced ranges for the fixed form) agree within the parity bar."""
     B, N, H, d = 3, 1000, 4, 128
     q, k, v = synth.draw_qkv(B, N, H, d, seed=41, device=DEV)
     sl = synth.slopes(H, DEV)
-    o_fixed, s_fixed = la.prefill(q, k, v, sl)
+    o_fixed, s_fixed = la.prefill(q, k, v, sl, segments=segments)
     cu = [0, N, 2 * N, 3 * N]
     o_var, s_var = la.prefill_varlen(q.view(B * N, H, d), k.view(B * N, H, d),
-                                     v.view(B * N, H, d), sl, cu)
+                                     v.view(B * N, H, d), sl, cu, segments=segments)
+    o_auto, s_auto = la.prefill(q, k, v, sl)
     torch.cuda.synchronize()
     assert torch.equal(o_var.view(B, N, H, d), o_fixed)
     assert torch.equal(s_var, s_fixed)
+    check_close(o_auto.float().cpu().numpy(), o_var.view(B, N, H, d).float().cpu().numpy(),
+                torch.bfloat16, "o automatic plan")
+    check_close(s_auto.cpu().numpy(), s_var.cpu().numpy(), torch.bfloat16, "state automatic plan")
 
 
 @pytest.mark.parametrize("split", [128, 700, 1])
