@@ -49,8 +49,13 @@ int chunk_of(int32_t chunk) { return chunk == 0 ? la::kChunkDefault : chunk; }
 // Workspace bytes of la_prefill's tensor path: the balanced plan when the segment count is left
 // to the library, else equal segments per sequence.
 size_t prefill_workspace_need(const la_desc* d, int sms) {
-  if (d->segments == 0)
-    return la::balanced_workspace_bytes(la::plan_balanced(d->B, d->N, d->H, sms, chunk_of(d->chunk)));
+  if (d->segments == 0) {
+    la::BalancedPlan bal{};
+    la::SegmentPlan seg{};
+    if (la::prefer_balanced(d->B, d->N, d->H, sms, chunk_of(d->chunk), &bal, &seg))
+      return la::balanced_workspace_bytes(bal);
+    return la::workspace_layout(d->B, d->H, seg).total;
+  }
   const la::SegmentPlan plan =
       la::plan_segments(d->B, d->N, d->H, d->segments, sms, chunk_of(d->chunk));
   return la::workspace_layout(d->B, d->H, plan).total;
@@ -188,17 +193,15 @@ la_status la_prefill(const la_desc* desc, const void* q, const void* k, const vo
   }
   const int sms = device_sms();
   if (sms <= 0) return LA_ERR_CUDA;
-  const bool balanced = desc->segments == 0;
   la::BalancedPlan bplan{};
   la::SegmentPlan splan{};
-  size_t need = 0;
-  if (balanced) {
-    bplan = la::plan_balanced(desc->B, desc->N, desc->H, sms, a.chunk);
-    need = la::balanced_workspace_bytes(bplan);
-  } else {
+  bool balanced = false;
+  if (desc->segments == 0)
+    balanced = la::prefer_balanced(desc->B, desc->N, desc->H, sms, a.chunk, &bplan, &splan);
+  else
     splan = la::plan_segments(desc->B, desc->N, desc->H, desc->segments, sms, a.chunk);
-    need = la::workspace_layout(desc->B, desc->H, splan).total;
-  }
+  const size_t need = balanced ? la::balanced_workspace_bytes(bplan)
+                               : la::workspace_layout(desc->B, desc->H, splan).total;
   void* ws = workspace;
   bool owned = false;
   if (ws == nullptr) {

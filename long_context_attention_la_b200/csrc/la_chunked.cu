@@ -46,6 +46,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdlib>
 
 #include "la_internal.h"
@@ -274,9 +275,13 @@ __device__ __forceinline__ void decode_unit(const Params& p, int64_t u, UnitInfo
 
 // Balanced plan: the units of range r, in order.  Cursor state lives with the producer thread.
 struct RangeCursor {
-  int32_t r = -1;          // current range (-1: none yet)
-  int64_t next = 0, end = 0;  // next flat tile of the range, and its end
-  bool local_pending = false; // the cut last piece's local-state unit is still to be issued
+  int32_t r = -1;           // current range (-1: none yet)
+  int32_t phase = 0;        // 0: cut piece's local state, 1: its outputs, 2: whole sequences,
+                            // 3: the piece that continues the previous range
+  int64_t a = 0, end = 0;   // the range's flat tiles [a, end)
+  int64_t cut = 0;          // first tile of the piece the range's end cuts (end: none)
+  int64_t cont_end = 0;     // end of the continuing first piece (a: none)
+  int64_t next = 0;         // next tile of phase 2 (whole sequences in [cont_end, cut))
 };
 
 // Fills ui with the piece of flat tiles [t0, t1) of one sequence (t1 inside or at its end).
@@ -292,38 +297,63 @@ __device__ __forceinline__ void piece_unit(const Params& p, int64_t t0, int64_t 
   ui.len = static_cast<int32_t>(min(p.N, (c0 + nc) * C) - c0 * C);
   ui.b = static_cast<int32_t>(sq / p.H);
   ui.tok0 = 0;
+  ui.flags = (c0 + nc == n) ? kUnitFinal : 0;
+  ui.slot = -1;
+  ui.pub_val = 0;
+  // a piece that starts inside its sequence begins its range; its predecessor is the cut last
+  // piece of the previous range, whose local-state unit published into ring slot r - 1
+  ui.in_slot = -1;
+  ui.in_val = 1;
 }
 
-// Next unit of the balanced plan (ui.bh = -1 when every range has been taken).  A piece that
-// starts inside its sequence begins its range, and its predecessor is the cut last piece of the
-// previous range, whose local-state unit published into ring slot r - 1.
+// Next unit of the balanced plan (ui.bh = -1 once every range has been taken).  A range runs,
+// in this order: the local-state pass of its cut last piece (publishing that piece's outgoing
+// state into ring slot r for the next range), that piece's outputs (its incoming state is at hand:
+// zero at a sequence start, else already awaited by the local-state unit), the outputs of the
+// whole sequences inside it, and last the piece that continues the previous range's cut, whose
+// publication (ring slot r - 1) it may have to wait for.
 __device__ __forceinline__ void next_balanced_unit(const Params& p, RangeCursor& cur,
                                                    UnitInfo& ui) {
   const int64_t n = p.n_chunks;
   while (true) {
-    if (cur.r >= 0 && cur.local_pending) {
-      cur.local_pending = false;
-      const int64_t last0 = max(cur.next, ((cur.end - 1) / n) * n);  // the cut piece's start
-      piece_unit(p, last0, cur.end, ui);
-      ui.flags = kUnitLocal | kUnitNoOutput;
-      ui.slot = cur.r;
-      ui.pub_val = 1;
-      ui.in_slot = ui.c0 > 0 ? cur.r - 1 : -1;
-      ui.in_val = 1;
-      return;
-    }
-    if (cur.r >= 0 && cur.next < cur.end) {
-      const int64_t t0 = cur.next;
-      const int64_t seq_end = (t0 / n + 1) * n;
-      const int64_t t1 = min(cur.end, seq_end);
-      piece_unit(p, t0, t1, ui);
-      ui.flags = t1 == seq_end ? kUnitFinal : 0;
-      ui.slot = -1;
-      ui.pub_val = 0;
-      ui.in_slot = ui.c0 > 0 ? cur.r - 1 : -1;
-      ui.in_val = 1;
-      cur.next = t1;
-      return;
+    if (cur.r >= 0) {
+      if (cur.phase == 0) {
+        cur.phase = 1;
+        if (cur.cut < cur.end) {
+          piece_unit(p, cur.cut, cur.end, ui);
+          ui.flags = kUnitLocal | kUnitNoOutput;
+          ui.slot = cur.r;
+          ui.pub_val = 1;
+          if (ui.c0 > 0) ui.in_slot = cur.r - 1;
+          return;
+        }
+      }
+      if (cur.phase == 1) {
+        cur.phase = 2;
+        if (cur.cut < cur.end) {
+          piece_unit(p, cur.cut, cur.end, ui);
+          if (ui.c0 > 0) ui.in_slot = cur.r - 1;
+          return;
+        }
+      }
+      if (cur.phase == 2) {
+        if (cur.next < cur.cut) {
+          const int64_t t0 = cur.next;
+          const int64_t t1 = min(cur.cut, (t0 / n + 1) * n);
+          piece_unit(p, t0, t1, ui);
+          cur.next = t1;
+          return;
+        }
+        cur.phase = 3;
+      }
+      if (cur.phase == 3) {
+        cur.phase = 4;
+        if (cur.cont_end > cur.a) {
+          piece_unit(p, cur.a, cur.cont_end, ui);
+          ui.in_slot = cur.r - 1;
+          return;
+        }
+      }
     }
     const int32_t r = static_cast<int32_t>(atomicAdd(p.counter, 1u));
     if (r >= p.n_ranges) {
@@ -334,9 +364,15 @@ __device__ __forceinline__ void next_balanced_unit(const Params& p, RangeCursor&
       return;
     }
     cur.r = r;
-    cur.next = p.range_start[r];
+    cur.phase = 0;
+    cur.a = p.range_start[r];
     cur.end = p.range_start[r + 1];
-    cur.local_pending = cur.end % n != 0;  // the range ends inside a sequence
+    // the range's end inside a sequence cuts its last piece
+    cur.cut = cur.end % n != 0 ? max(cur.a, ((cur.end - 1) / n) * n) : cur.end;
+    // a start inside a sequence continues the previous range's cut piece; when that piece is
+    // also this range's cut piece, phases 0 and 1 handle it
+    cur.cont_end = (cur.a % n != 0 && cur.cut > cur.a) ? min(cur.cut, (cur.a / n + 1) * n) : cur.a;
+    cur.next = cur.cont_end;
   }
 }
 
@@ -1446,39 +1482,77 @@ SegmentPlan plan_segments(int64_t B, int64_t N, int64_t H, int requested_segment
 
 namespace {
 
-// Extra cost of a tile in a range's cut last piece (its local-state pass reads K and V once more),
-// relative to an output tile.  LA_BALANCE_LOCAL_COST (percent) overrides it: a tuning knob, every
-// value computes the same result.
+// Relative time of a local-state tile (K and V only) against an output tile (Q, K, V in, O out).
+// LA_BALANCE_LOCAL_COST (percent) overrides it: a tuning knob; every value computes the same
+// result.
 double local_pass_cost() {
   static double v = -1.0;
   if (v < 0.0) {
-    double c = 0.5;
+    double c = 0.46;
     if (const char* e = getenv("LA_BALANCE_LOCAL_COST")) c = std::max(0, std::min(300, atoi(e))) / 100.0;
     v = c;
   }
   return v;
 }
 
-// The furthest end b > a of a range starting at flat tile a whose cost is at most cap: tiles
-// count 1, plus rho for each tile of a last piece that ends inside its sequence.  Ends at
-// sequence boundaries cost nothing extra; an end inside a sequence falls on an even tile offset
-// when `pair` (256-token chunks).
-int64_t range_end(int64_t a, double cap, int64_t n, int64_t total, double rho, bool pair) {
-  const int64_t seq_end = (a / n + 1) * n;
-  int64_t best = a;
-  int64_t q0 = (a / n) * n;  // start of the sequence an end inside a sequence would fall in
-  if (static_cast<double>(seq_end - a) <= cap) {
-    const int64_t k = static_cast<int64_t>((cap - static_cast<double>(seq_end - a)) / n);
-    best = std::min(total, seq_end + k * n);
-    q0 = best;
+// Finish time, in output-tile units, of the range [a, b) of the head-major tile list (sequences
+// of n tiles), and the time its cut last piece publishes its outgoing state (-1: no cut).  The
+// range runs the cut piece's local-state pass (rho per tile), that piece's outputs, the outputs
+// of the whole sequences inside it and last the piece that continues the previous range's cut,
+// which cannot start before that cut was published at pub_prev.  A range that is one piece cut
+// at both ends publishes only once its own local pass and its predecessor's publication are done.
+struct RangeTiming {
+  double finish, pub;
+};
+RangeTiming range_timing(int64_t a, int64_t b, int64_t n, double rho, double pub_prev) {
+  const int64_t sa = a / n, sb = (b - 1) / n;
+  const bool cont = a % n != 0;  // the first piece continues the previous range's cut
+  const bool cut = b % n != 0;   // the last piece is cut off from the rest of its sequence
+  RangeTiming t{0.0, -1.0};
+  if (sa == sb && cont && cut) {  // one piece, cut at both ends
+    const double y = static_cast<double>(b - a);
+    t.pub = std::max(rho * y, pub_prev);
+    t.finish = t.pub + y;
+    return t;
   }
+  const double x = cont ? static_cast<double>(std::min(b, (sa + 1) * n) - a) : 0.0;
+  const double y = cut ? static_cast<double>(b - std::max(a, sb * n)) : 0.0;
+  const double m = static_cast<double>(b - a) - x - y;
+  double time = (1.0 + rho) * y + m;
+  if (cut) t.pub = rho * y;
+  if (cont) time = std::max(time, pub_prev) + x;
+  t.finish = time;
+  return t;
+}
+
+// The furthest end b > a of a range that finishes by `cap`; ends at sequence boundaries are
+// considered first (no local pass), then ends inside the next sequence (binary search; the
+// finish time grows with the cut piece).  Inside a sequence the end falls on an even tile offset
+// when `pair` (256-token chunks).
+int64_t range_end(int64_t a, double cap, int64_t n, int64_t total, double rho, bool pair,
+                  double pub_prev) {
+  int64_t best = a;
+  // whole sequences: ends at seq_end(a), seq_end(a) + n, ...
+  int64_t e = (a / n + 1) * n;
+  while (e <= total && range_timing(a, e, n, rho, pub_prev).finish <= cap) {
+    best = e;
+    e += n;
+  }
+  // an end inside the sequence that starts at q0
+  const int64_t q0 = best > a ? best : (a / n) * n;
   if (q0 < total) {
-    const int64_t p0 = std::max(a, q0);  // the last piece's first tile
-    // (b - a) + rho (b - p0) <= cap
-    int64_t b = static_cast<int64_t>((cap + static_cast<double>(a) + rho * p0) / (1.0 + rho));
-    b = std::min(b, q0 + n - 1);
-    if (pair) b = q0 + ((b - q0) & ~int64_t(1));
-    if (b > p0 && b > best) best = b;
+    int64_t lo = std::max(a, q0), hi = std::min(q0 + n - 1, total);  // candidate ends (lo, hi]
+    while (hi > lo) {
+      int64_t mid = lo + (hi - lo + 1) / 2;
+      if (pair) mid = q0 + ((mid - q0) & ~int64_t(1));
+      if (mid <= lo) break;
+      if (range_timing(a, mid, n, rho, pub_prev).finish <= cap)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    if (pair) lo = q0 + ((lo - q0) & ~int64_t(1));
+    if (lo > std::max(a, q0) && lo > best) best = lo;
   }
   return std::min(best, total);
 }
@@ -1495,18 +1569,21 @@ BalancedPlan plan_balanced(int64_t B, int64_t N, int64_t H, int num_sms, int chu
       1, std::min<int64_t>({static_cast<int64_t>(std::max(num_sms, 1)), int64_t(kMaxRanges), total}));
   const double rho = local_pass_cost();
   const bool pair = chunk == 256;
-  // greedy cut with a cost cap; true when it covers every tile in r_max ranges or fewer
+  // greedy cut with a finish-time cap; true when it covers every tile in r_max ranges or fewer
   auto cut = [&](double cap, BalancedPlan* out) -> bool {
     int64_t a = 0;
     int32_t r = 0;
+    double pub_prev = 0.0;
     if (out) out->start[0] = 0;
     while (a < total) {
       if (r >= r_max) return false;
-      int64_t b = range_end(a, cap, n, total, rho, pair);
+      int64_t b = range_end(a, cap, n, total, rho, pair, pub_prev);
       if (b <= a) {  // always make progress: one tile (two inside a sequence for pairs)
         const int64_t se = (a / n + 1) * n;
         b = std::min(se, a + (pair ? 2 : 1));
       }
+      const RangeTiming t = range_timing(a, b, n, rho, pub_prev);
+      pub_prev = t.pub >= 0.0 ? t.pub : 0.0;
       a = b;
       ++r;
       if (out) out->start[r] = static_cast<int32_t>(a);
@@ -1522,7 +1599,34 @@ BalancedPlan plan_balanced(int64_t B, int64_t N, int64_t H, int num_sms, int chu
     if (cut(mid, nullptr)) hi = mid; else lo = mid;
   }
   cut(hi, &pl);
+  pl.makespan = hi;
   return pl;
+}
+
+double segments_makespan(const SegmentPlan& plan, int64_t B, int64_t H, int num_sms) {
+  const double rho = local_pass_cost();
+  const double L = static_cast<double>(plan.seg_chunks);
+  if (plan.segments <= 1) {
+    // whole sequences handed out dynamically to the CTAs
+    const double waves = std::ceil(static_cast<double>(B * H) / std::max(num_sms, 1));
+    return waves * static_cast<double>(plan.n_chunks);
+  }
+  // every segment in one wave: a cut segment runs its local pass and its outputs; the others
+  // wait for their predecessor's publication (after its local pass) and run their outputs
+  return (1.0 + rho) * L;
+}
+
+bool prefer_balanced(int64_t B, int64_t N, int64_t H, int num_sms, int chunk, BalancedPlan* bal,
+                     SegmentPlan* seg) {
+  *seg = plan_segments(B, N, H, 0, num_sms, chunk);
+  *bal = plan_balanced(B, N, H, num_sms, chunk);
+  // Short ranges pay each unit's pipeline fill and drain, which the model leaves out (measured:
+  // the balanced plan loses at 14 tiles per range and gains about 8 % at 886), so they stay on
+  // equal segments.
+  const double tiles_per_range =
+      static_cast<double>(bal->total_tiles) / std::max(bal->n_ranges, 1);
+  return tiles_per_range >= 64.0 &&
+         bal->makespan < 0.9 * segments_makespan(*seg, B, H, num_sms);
 }
 
 size_t balanced_workspace_bytes(const BalancedPlan& plan) {

@@ -170,9 +170,16 @@ struct BalancedPlan {
   int32_t n_ranges;
   int32_t seq_tiles;                  // tiles per sequence
   int64_t total_tiles;                // B * H * seq_tiles
+  double makespan;                    // modelled finish time of the slowest range, in tile times
   int32_t start[kMaxRanges + 1];
 };
 BalancedPlan plan_balanced(int64_t B, int64_t N, int64_t H, int num_sms, int chunk);
+// Modelled finish time of the equal-segment plan, in the same units.
+double segments_makespan(const SegmentPlan& plan, int64_t B, int64_t H, int num_sms);
+// The automatic plan: balanced ranges when their modelled finish time beats the equal-segment
+// plan's by a clear margin, else equal segments (sets exactly one of the two outputs).
+bool prefer_balanced(int64_t B, int64_t N, int64_t H, int num_sms, int chunk, BalancedPlan* bal,
+                     SegmentPlan* seg);
 // workspace: header, one scan flag and one d x d fp32 ring slot per range
 size_t balanced_workspace_bytes(const BalancedPlan& plan);
 cudaError_t launch_chunked_prefill_balanced(const PrefillArgs& a, const BalancedPlan& plan,
