@@ -42,11 +42,12 @@ METRIC = "lightning-attn prefill tok/s & TFLOP/s (H=64,d=128); decode state GB/s
 DECODE = dict(B=256, H=64, d=128)
 
 
-def measured_traffic():
-    """DRAM bytes per prefill launch from the committed ncu capture, or None when the kernel
-    sources changed since that capture."""
+def measured_counters():
+    """Counters of one prefill launch of the default workload from the committed ncu capture
+    (profiles/chunked_prefill_kernel_counters.json), or None when the kernel sources changed
+    since that capture: DRAM bytes and the tensor-pipe activity."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "chunked_prefill_kernel_traffic.json")
+    path = os.path.join(ROOT, "profiles", "chunked_prefill_kernel_counters.json")
     try:
         with open(path) as f:
             rec = json.load(f)
@@ -56,9 +57,16 @@ def measured_traffic():
                 h.update(f.read())
         if h.hexdigest() != rec["source_sha256"]:
             return None
-        return float(rec["dram_bytes_read"]) + float(rec["dram_bytes_write"])
+        return rec
     except Exception:
         return None
+
+
+# Tensor-core flops the prefill kernel executes per token and head at d = 128, by chunk length:
+# four 128 x 128 x 128 products per 128-token tile at C = 128 (S, the inter product, the state
+# update, P V); five at C = 64 (a second inter product) and at C = 256 (per two tiles: three
+# score blocks, two inter products, two state updates, three P V blocks).
+EXECUTED_FLOPS_PER_TOKEN_HEAD = {64: 163840.0, 128: 131072.0, 256: 163840.0}
 
 
 def load_peaks():
@@ -526,6 +534,10 @@ def run_ours(args):
 
     if rank == 0:
         hbm_peak, tc_peak, peak_kind = load_peaks()
+        # committed counters describe the default launch only (prefill_32k, plain output, the
+        # default chunk and plan)
+        counters = (measured_counters() if args.workload == "prefill_32k" and not (
+            args.gate or args.gate_separate or args.cp or args.chunk or args.segments) else None)
         tokens = B * N
         tok_s = world * tokens / ((step_ms_max if args.cp else pre_ms_max) * 1e-3)
         # algorithmic bytes of one prefill launch: read q, k, v and write o (bf16), write the
@@ -536,7 +548,8 @@ def run_ours(args):
             n_states * H * d * d * 4 * (1 if vw is None and not args.cp else 2)
         achieved = pre_bytes / (pre_ms_max * 1e-3) / 1e9
         canon = 4.0 * d * d * B * N * H  # recurrent-form flops
-        executed = (4.0 * d * d + 4.0 * 128 * d) * B * N * H  # full 128 x 128 tiles
+        chunk = args.chunk if args.chunk else 128
+        executed = EXECUTED_FLOPS_PER_TOKEN_HEAD[chunk] * B * N * H
         dec_bytes = 2 * Bd * Hd * dd * dd * 4 + 4 * Bd * Hd * dd * 2 * n_mtp
         dec_gbs = dec_bytes / max(dec_ms_max * 1e-3, 1e-12) / 1e9
         cpu = None
@@ -574,7 +587,8 @@ def run_ours(args):
                        "l2": "inputs larger than L2 (no flush)"},
             "prefill": {"ms": pre_ms_max, "tok_s": world * tokens / (pre_ms_max * 1e-3),
                         "tflops_canonical": world * canon / (pre_ms_max * 1e-3) / 1e12,
-                        "tflops_executed_c128": world * executed / (pre_ms_max * 1e-3) / 1e12,
+                        "tflops_executed": world * executed / (pre_ms_max * 1e-3) / 1e12,
+                        "chunk": chunk,
                         "hbm_gbs": achieved},
             "decode": None if args.no_decode else {
                 "ms": dec_ms_max, "state_gbs": dec_gbs, "frac_of_measured": dec_gbs / hbm_peak,
@@ -582,10 +596,23 @@ def run_ours(args):
                 "tok_s": world * Bd * n_mtp / (dec_ms_max * 1e-3)},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak,
-                         "traffic": (measured_traffic() if args.workload == "prefill_32k"
-                                     and not (args.gate or args.gate_separate) else None),
+                         "traffic": (counters["dram_bytes_read"] + counters["dram_bytes_write"]
+                                     if counters else None),
                          "algorithmic_bytes": pre_bytes,
-                         "kernel": "chunked_prefill_kernel", "peak_kind": peak_kind},
+                         "kernel": "chunked_prefill_kernel", "peak_kind": peak_kind,
+                         # the tensor pipe of the same kernel: executed MMA flops per second
+                         # against the measured bf16 burst peak, and ncu's pipe activity
+                         "tensor_pipe": {
+                             "executed_tflops": world * executed / (pre_ms_max * 1e-3) / 1e12,
+                             "peak_tflops": tc_peak,
+                             "frac": world * executed / (pre_ms_max * 1e-3) / 1e12 / tc_peak,
+                             "chunk": chunk,
+                             "ncu_pipe_tensor_active_pct": (
+                                 counters["sm__pipe_tensor_cycles_active_pct_active"]
+                                 if counters else None),
+                             "ncu_pipe_tensor_elapsed_pct": (
+                                 counters["sm__pipe_tensor_cycles_active_pct_elapsed"]
+                                 if counters else None)}},
             "cp": None if not args.cp else {
                 "state_fold_gather_ms": cp_ms_max, "step_ms": step_ms_max,
                 # the state pass reads k and v of the part and writes the d x d states; the

@@ -12,7 +12,10 @@
 // with two fused multiply-adds, so the decay is exact to fp32 rounding of each step.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "la_internal.h"
+#include "la_sm100.cuh"
 
 namespace la {
 namespace {
@@ -204,114 +207,228 @@ __global__ void __launch_bounds__(512) decode_kernel(const T* __restrict__ q,
 
 // ---------------------------------------------------------------------------------------------
 // Multi-token decode step (speculative verification: the report's "attention with MTP", §4.3).
-// One CTA per (b, h), 512 threads, the state's quads held in registers as in decode_kernel, and
-// n tokens applied in order, each one: S <- lambda S + k^T v, o = q S.  The state is read and
-// written once for all n tokens.  The q, k, v (and gate) rows of up to 8 tokens are staged in
-// shared memory at once, so a group costs one load latency, and each token then costs one block
-// barrier.  With a gate, each output row gets the fused grouped RMSNorm + sigmoid gate:
-// y = gamma * o / sqrt(mean(o^2) + eps) * sigmoid(g) (one norm group per head).
+// For every (b, h), n tokens are applied in order, each one: S <- lambda S + k^T v, o = q S.
+//
+// The n tokens are one chunk of the recurrence, evaluated in its chunked form (the same algebra
+// as the prefill's chunks): with S_0 the state before the step,
+//     o_j = lambda^(j+1) q_j S_0 + sum_{m <= j} lambda^(j-m) (q_j . k_m) v_m
+//     S_n = lambda^n S_0 + sum_m lambda^(n-1-m) k_m^T v_m
+// so the state is read once for every read-out (one multiply-add per state element per token)
+// and updated once (n + 1 per element), with a fixed number of block barriers per head instead
+// of one per token.  Groups of at most 8 tokens are applied in turn.
+//
+// One CTA per (b, h), two resident per SM: each thread loads its quads of the state into
+// registers with all its loads in flight at once (as in decode_kernel), the group's q, k, v (and
+// gate) rows are staged in shared memory, and the updated state goes back with streaming stores.
+// With a gate, each output row gets the fused grouped RMSNorm + sigmoid gate
+// y = gamma * o / sqrt(mean(o^2) + eps) * sigmoid(g).
 // ---------------------------------------------------------------------------------------------
 template <typename T, int D>
-__global__ void __launch_bounds__(512) decode_multi_kernel(
+struct MultiLayout {
+  static constexpr int NG = 8;                                    // tokens per group
+  static constexpr int RS = 512 / (D / 4);                        // row slots
+  static constexpr size_t kTok = size_t(4) * NG * D * sizeof(T);  // q, k, v, gate rows
+  static constexpr size_t kPart = size_t(NG) * RS * D * 4;        // q S_0 partial sums
+  static constexpr size_t kCtrl = 512;                            // A, norms
+  static constexpr size_t kTotal = kTok + kPart + kCtrl;
+};
+
+template <typename T>
+__device__ __forceinline__ float smem_f32(const T* p);
+template <>
+__device__ __forceinline__ float smem_f32<float>(const float* p) {
+  return *p;
+}
+template <>
+__device__ __forceinline__ float smem_f32<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+// four consecutive elements (16-byte aligned for fp32, 8-byte for bf16) as fp32
+template <typename T>
+__device__ __forceinline__ float4 smem_f32x4(const T* p);
+template <>
+__device__ __forceinline__ float4 smem_f32x4<float>(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+template <>
+__device__ __forceinline__ float4 smem_f32x4<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint2 w = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                     __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(512, 2) decode_multi_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const float* __restrict__ slopes, float* __restrict__ state, T* __restrict__ out, int64_t H,
     int64_t n_tok, const T* __restrict__ gate, const float* __restrict__ gamma, float eps) {
+  using L = MultiLayout<T, D>;
   constexpr int NT = 512;
-  constexpr int Q4 = D / 4;     // column quads per row
-  constexpr int RS = NT / Q4;   // row slots
-  constexpr int RPT = D / RS;   // rows per thread
-  constexpr int NG = 8;         // tokens staged per group
-  __shared__ float sqkv[3][NG][D];   // q, k, v of the group's tokens
-  __shared__ float sg[NG][D];        // their gate pre-activations
-  __shared__ float red[2][RS][D];    // read-out partial sums, double-buffered over tokens
-  __shared__ float ss_part[D / 32];
+  constexpr int Q4 = D / 4;       // column quads per row
+  constexpr int RS = L::RS;       // row slots
+  constexpr int RPT = D / RS;     // rows per thread
+  constexpr int NG = L::NG;
+  constexpr int TPJ = NT / NG;    // output threads per token
+  constexpr int CPT = D / TPJ;    // output columns per thread (2 at d = 128, 1 at d = 64)
+  constexpr int EPP = 16 / static_cast<int>(sizeof(T));  // elements per 16-byte piece
+  constexpr int PIECES = D / EPP;                        // pieces per token row
+  constexpr float kLog2e = 1.4426950408889634f;
+  extern __shared__ __align__(128) uint8_t sm[];
+  T* tok = reinterpret_cast<T*>(sm);                                           // [4][NG][D]
+  float(*part)[RS][D] = reinterpret_cast<float(*)[RS][D]>(sm + L::kTok);      // [NG][RS][D]
+  float* A = reinterpret_cast<float*>(sm + L::kTok + L::kPart);               // [NG][NG]
+  float* ssq = A + NG * NG;                                                    // [NG][TPJ / 32]
 
   const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
   const int c4 = tid % Q4;
   const int r0 = tid / Q4;
+  const int rows = gate != nullptr ? 4 : 3;
   const int64_t flat = blockIdx.x;  // b * H + h
-  const int64_t b = flat / H;
-  const int64_t h = flat % H;
+  const int64_t b = flat / H, h = flat % H;
   float4* st = reinterpret_cast<float4*>(state + flat * D * D);
 
+  // every state load of the thread in flight at once
   float4 s[RPT];
 #pragma unroll
   for (int r = 0; r < RPT; ++r) s[r] = __ldcs(st + (r0 + r * RS) * Q4 + c4);
-  float lam_hi, lam_lo;
-  split_decay(slopes[h], lam_hi, lam_lo);
+  const float alpha = slopes[h] * kLog2e;  // lambda^e = exp2(-alpha e)
+  const T* tq = tok;
+  const T* tkk = tok + NG * D;
+  const T* tv = tok + 2 * NG * D;
+  const T* tg = tok + 3 * NG * D;
 
-  // element offset of token j's row for this head in a [B, n_tok, H, D] tensor
-  auto row_off = [&](int64_t j) { return ((b * n_tok + j) * H + h) * D; };
-  int64_t tok = 0;  // tokens processed so far (selects the red buffer)
   for (int64_t j0 = 0; j0 < n_tok; j0 += NG) {
     const int nn = static_cast<int>(min(static_cast<int64_t>(NG), n_tok - j0));
-    // stage the whole group (one load latency for nn tokens)
-    for (int idx = tid; idx < 3 * nn * D; idx += NT) {
-      const int which = idx / (nn * D), rem = idx % (nn * D), jj = rem / D, e = rem % D;
-      const T* src = which == 0 ? q : (which == 1 ? k : v);
-      sqkv[which][jj][e] = load_as_f32<T>(src, row_off(j0 + jj) + e);
+    if (j0 > 0) __syncthreads();  // the previous group's buffers are read
+    // q, k, v (and gate) rows of the group, 16 bytes per copy
+    for (int idx = tid; idx < rows * nn * PIECES; idx += NT) {
+      const int which = idx / (nn * PIECES), rem = idx % (nn * PIECES);
+      const int jj = rem / PIECES, pc = rem % PIECES;
+      const T* src = which == 0 ? q : (which == 1 ? k : (which == 2 ? v : gate));
+      cp_async16(tok + (which * NG + jj) * D + pc * EPP,
+                 src + ((b * n_tok + j0 + jj) * H + h) * D + pc * EPP, true);
     }
-    if (gate != nullptr)
-      for (int idx = tid; idx < nn * D; idx += NT)
-        sg[idx / D][idx % D] = load_as_f32<T>(gate, row_off(j0 + idx / D) + idx % D);
+    cp_async_commit();
+    cp_async_wait<0>();
     __syncthreads();
-    for (int jj = 0; jj < nn; ++jj, ++tok) {
-      const int rb = static_cast<int>(tok & 1);
-      const float v0 = sqkv[2][jj][4 * c4 + 0], v1 = sqkv[2][jj][4 * c4 + 1];
-      const float v2 = sqkv[2][jj][4 * c4 + 2], v3 = sqkv[2][jj][4 * c4 + 3];
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    // (1) partial read-outs q_j S_0 over this thread's rows, for every token of the group
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) {
-        const int i = r0 + r * RS;
-        const float ki = sqkv[1][jj][i], qi = sqkv[0][jj][i];
-        float4 x = s[r];
-        x.x = fmaf(lam_hi, x.x, fmaf(ki, v0, lam_lo * x.x));
-        x.y = fmaf(lam_hi, x.y, fmaf(ki, v1, lam_lo * x.y));
-        x.z = fmaf(lam_hi, x.z, fmaf(ki, v2, lam_lo * x.z));
-        x.w = fmaf(lam_hi, x.w, fmaf(ki, v3, lam_lo * x.w));
-        a0 = fmaf(qi, x.x, a0);
-        a1 = fmaf(qi, x.y, a1);
-        a2 = fmaf(qi, x.z, a2);
-        a3 = fmaf(qi, x.w, a3);
-        s[r] = x;
+    for (int jj = 0; jj < NG; ++jj) {
+      if (jj < nn) {
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+          const float qi = smem_f32(tq + jj * D + r0 + r * RS);
+          y.x = fmaf(qi, s[r].x, y.x);
+          y.y = fmaf(qi, s[r].y, y.y);
+          y.z = fmaf(qi, s[r].z, y.z);
+          y.w = fmaf(qi, s[r].w, y.w);
+        }
+        *reinterpret_cast<float4*>(&part[jj][r0][4 * c4]) = y;
       }
-      red[rb][r0][4 * c4 + 0] = a0;
-      red[rb][r0][4 * c4 + 1] = a1;
-      red[rb][r0][4 * c4 + 2] = a2;
-      red[rb][r0][4 * c4 + 3] = a3;
-      // One barrier per token: red is double-buffered, and the read-out of this token finishes
-      // before its threads reach the next token's barrier, so red[rb] is free again two tokens on.
-      __syncthreads();
-      if (tid < D) {
-        float o = 0.f;
+    }
+    // (2) intra weights A[j][m] = lambda^(j-m) (q_j . k_m), m <= j, one warp per pair
+    for (int pidx = warp; pidx < nn * (nn + 1) / 2; pidx += NT / 32) {
+      int jq = 0;
+      while ((jq + 1) * (jq + 2) / 2 <= pidx) ++jq;
+      const int m = pidx - jq * (jq + 1) / 2;
+      float dot = 0.f;
 #pragma unroll
-        for (int rr = 0; rr < RS; ++rr) o += red[rb][rr][tid];
-        if (gate != nullptr) {
-          float ss = o * o;
+      for (int e = lane; e < D; e += 32)
+        dot = fmaf(smem_f32(tq + jq * D + e), smem_f32(tkk + m * D + e), dot);
 #pragma unroll
-          for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-          if ((tid & 31) == 0) ss_part[tid >> 5] = ss;
-          asm volatile("bar.sync 1, %0;" ::"r"(D) : "memory");  // the D read-out threads only
+      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      if (lane == 0) A[jq * NG + m] = exp2f(-alpha * static_cast<float>(jq - m)) * dot;
+    }
+    __syncthreads();
+    // (3) outputs: thread (j, cols) sums the row slots, adds the intra terms, scales
+    {
+      const int jj = tid / TPJ;
+      const int cbase = (tid % TPJ) * CPT;
+      float o[CPT];
+      if (jj < nn) {
+        const float fq = exp2f(-alpha * static_cast<float>(jj + 1));
+#pragma unroll
+        for (int cc = 0; cc < CPT; ++cc) {
+          const int c = cbase + cc;
+          float acc = 0.f;
+#pragma unroll
+          for (int rr = 0; rr < RS; ++rr) acc += part[jj][rr][c];
+          float intra = 0.f;
+          for (int m = 0; m <= jj; ++m)
+            intra = fmaf(A[jj * NG + m], smem_f32(tv + m * D + c), intra);
+          o[cc] = fmaf(fq, acc, intra);
+        }
+      }
+      if (gate != nullptr) {
+        // grouped RMSNorm over the token's D outputs (TPJ threads), then the sigmoid gate
+        float ss = 0.f;
+        if (jj < nn) {
+#pragma unroll
+          for (int cc = 0; cc < CPT; ++cc) ss = fmaf(o[cc], o[cc], ss);
+        }
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+        if (lane == 0) ssq[warp] = ss;  // the warps of token j are 2 j, 2 j + 1
+        __syncthreads();
+        if (jj < nn) {
           float tot = 0.f;
 #pragma unroll
-          for (int w = 0; w < D / 32; ++w) tot += ss_part[w];
-          const float sig = 1.f / (1.f + expf(-sg[jj][tid]));
-          o = gamma[h * D + tid] * (o * rsqrtf(tot * (1.f / D) + eps)) * sig;
-          asm volatile("bar.sync 1, %0;" ::"r"(D) : "memory");  // ss_part reused next token
+          for (int w = 0; w < TPJ / 32; ++w) tot += ssq[jj * (TPJ / 32) + w];
+          const float rinv = rsqrtf(tot * (1.f / D) + eps);
+#pragma unroll
+          for (int cc = 0; cc < CPT; ++cc) {
+            const int c = cbase + cc;
+            const float sig = 1.f / (1.f + expf(-smem_f32(tg + jj * D + c)));
+            o[cc] = gamma[h * D + c] * (o[cc] * rinv) * sig;
+          }
         }
-        store_from_f32<T>(out, row_off(j0 + jj) + tid, o);
+      }
+      if (jj < nn) {
+#pragma unroll
+        for (int cc = 0; cc < CPT; ++cc)
+          store_from_f32<T>(out, ((b * n_tok + j0 + jj) * H + h) * D + cbase + cc, o[cc]);
       }
     }
-    __syncthreads();  // the group's staging buffers are read; the next group may overwrite them
+    // (4) state after the group: S <- lambda^nn S + sum_m lambda^(nn-1-m) k_m^T v_m
+    {
+      const float lam_n = exp2f(-alpha * static_cast<float>(nn));
+#pragma unroll
+      for (int r = 0; r < RPT; ++r) {
+        s[r].x *= lam_n;
+        s[r].y *= lam_n;
+        s[r].z *= lam_n;
+        s[r].w *= lam_n;
+      }
+      for (int m = 0; m < nn; ++m) {
+        const float wm = exp2f(-alpha * static_cast<float>(nn - 1 - m));
+        const float4 vm = smem_f32x4(tv + m * D + 4 * c4);
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+          const float km = wm * smem_f32(tkk + m * D + r0 + r * RS);
+          s[r].x = fmaf(km, vm.x, s[r].x);
+          s[r].y = fmaf(km, vm.y, s[r].y);
+          s[r].z = fmaf(km, vm.z, s[r].z);
+          s[r].w = fmaf(km, vm.w, s[r].w);
+        }
+      }
+    }
   }
+  // the updated state back in place (a warp writes whole 512-byte rows)
 #pragma unroll
   for (int r = 0; r < RPT; ++r) __stcs(st + (r0 + r * RS) * Q4 + c4, s[r]);
 }
 
 template <typename T, int D>
 cudaError_t launch_decode_multi_typed(const DecodeArgs& a, cudaStream_t stream) {
-  const int64_t grid = a.B * a.H;
-  decode_multi_kernel<T, D><<<static_cast<unsigned>(grid), 512, 0, stream>>>(
+  using L = MultiLayout<T, D>;
+  // set on every call: cheap, safe from any host thread, and it survives a context reset
+  cudaError_t e = cudaFuncSetAttribute(decode_multi_kernel<T, D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L::kTotal));
+  if (e != cudaSuccess) return e;
+  decode_multi_kernel<T, D><<<static_cast<unsigned>(a.B * a.H), 512, L::kTotal, stream>>>(
       static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
       a.slopes, a.state, static_cast<T*>(a.out), a.H, a.n_tok, static_cast<const T*>(a.gate),
       a.gamma, a.eps);
@@ -349,6 +466,8 @@ cudaError_t launch_recurrent_prefill(const PrefillArgs& a, cudaStream_t stream) 
 }
 
 cudaError_t launch_decode_multi(const DecodeArgs& a, cudaStream_t stream) {
+  // one token and no epilogue is the plain decode step (same kernel, same bits)
+  if (a.n_tok == 1 && a.gate == nullptr) return launch_decode(a, stream);
   if (a.dtype == kF32) {
     return a.d == 64 ? launch_decode_multi_typed<float, 64>(a, stream)
                      : launch_decode_multi_typed<float, 128>(a, stream);
