@@ -98,6 +98,7 @@ struct Ctrl {
   uint64_t p_ready;
   uint64_t s2_full;   // C = 256: the cross scores Q_B K~_A^T of a chunk's second tile are in TMEM
   uint64_t p2_ready;  // C = 256: their scaled bf16 P_BA is in TMEM
+  uint64_t gate_full[2];  // fused norm + gate: the tile's gate rows are in its stage's Q slot
   uint64_t o_full;
   uint64_t o_free;
   uint64_t kv_done;
@@ -392,25 +393,23 @@ __device__ __forceinline__ float sigmoidf_fast(float x) {
   return fmaf(0.5f, t, 0.5f);
 }
 
-// Gate pieces of 32-column block cb in the 4-lane store layout: g[k] = piece t of row i0 + k
-// (zero past the segment end).
-__device__ __forceinline__ void load_gate_pieces(const __nv_bfloat16* gate_h, int32_t len,
-                                                 int32_t r0, int64_t n0, int64_t row_stride,
-                                                 uint32_t t, uint32_t cb, uint4 (&g)[4]) {
+// Gate pieces of 32-column block cb in the 4-lane store layout, from the tile's gate rows staged
+// in shared memory (two [128 x 64] halves, 128-byte swizzle): g[k] = piece t of tile row i0 + k.
+__device__ __forceinline__ void load_gate_pieces(const uint8_t* gate_tile, uint32_t i0, uint32_t t,
+                                                 uint32_t cb, uint4 (&g)[4]) {
+  const uint32_t piece = cb * 4 + t;  // 16-byte piece of the 256-byte row
+  const uint8_t* half = gate_tile + (piece >> 3) * kHalfBytes;
 #pragma unroll
-  for (uint32_t k = 0; k < 4; ++k) {
-    g[k] = make_uint4(0u, 0u, 0u, 0u);
-    if (r0 + static_cast<int32_t>(k) < len)
-      g[k] = __ldcs(reinterpret_cast<const uint4*>(gate_h + (n0 + k) * row_stride + cb * 32) + t);
-  }
+  for (uint32_t k = 0; k < 4; ++k)
+    g[k] = *reinterpret_cast<const uint4*>(half + sw128_off(i0 + k, piece & 7u));
 }
 
 __device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint32_t trow,
                                                uint32_t col_inter, float f,
                                                const UnitInfo& ui, int64_t h,
-                                               const __nv_bfloat16* gate_h, __nv_bfloat16* out_h,
-                                               uint32_t t, int32_t r0, int64_t n0,
-                                               int64_t row_stride, uint4 (&g)[4]) {
+                                               const uint8_t* gate_tile, __nv_bfloat16* out_h,
+                                               uint32_t t, int32_t r0, uint32_t i0, int64_t n0,
+                                               int64_t row_stride) {
   float ss = 0.f;
 #pragma unroll 1
   for (uint32_t cb = 0; cb < 8; ++cb) {  // 16-column blocks
@@ -431,9 +430,8 @@ __device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint
   for (uint32_t k = 0; k < 4; ++k) rk[k] = __shfl_sync(0xffffffffu, rinv, lane0 + k);
 #pragma unroll 1
   for (uint32_t cb = 0; cb < 4; ++cb) {
-    // this block's gate pieces are in g (block 0: loaded before O was complete; later blocks:
-    // loaded here, in flight during the accumulator reads and the exchange)
-    if (cb > 0) load_gate_pieces(gate_h, ui.len, r0, n0, row_stride, t, cb, g);
+    uint4 g[4];
+    load_gate_pieces(gate_tile, i0, t, cb, g);
     uint4 x[4];  // bf16 O, pieces q = 0..3 of this row's 32 columns
 #pragma unroll
     for (uint32_t q = 0; q < 4; ++q) {
@@ -500,7 +498,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctrl->full[s], 1);
-      mbar_init(&ctrl->empty[s], 1);
+      // with the fused norm + gate a stage is free once the MMAs are done with it and the
+      // epilogue has read the gate rows staged in its Q slot
+      mbar_init(&ctrl->empty[s], kGated ? 2 : 1);
+      mbar_init(&ctrl->gate_full[s], 1);
       mbar_init(&ctrl->kt_ready[s], 128);
       mbar_init(&ctrl->unit_full[s], 1);
       mbar_init(&ctrl->unit_empty[s], 1 + 256 + 128 + 128);
@@ -744,6 +745,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             issue_state_update(g, c > 0);
             umma_commit(&ctrl->empty[s]);
+            // (with the fused norm + gate a stage takes two arrivals; a local-state tile has no
+            // epilogue, so both come from here)
+            if (kGated) umma_commit(&ctrl->empty[s]);
             ++g;
           }
           if (!ok) break;
@@ -1071,6 +1075,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t trow = tmem + ((wq * 32) << 16);
     uint8_t* kvb = smem + kOffKVb;
     uint32_t g = 0, j = 0, n_kvd = 0, n_h = 0, n_s = 0;
+    uint32_t gate_issued[2] = {0u, 0u};  // fused norm + gate: gate tiles loaded per stage
     tc_fence_before();
     mbar_arrive(&ctrl->kv_free);  // the KV columns start out free
 
@@ -1273,6 +1278,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++n_kvd;
           tc_fence_after();
         }
+        if (kGated && wq == 0 && lane == 0) {
+          // every product that reads this tile's Q is complete (the update just waited for comes
+          // after them): its Q slot takes the tile's gate rows for the fused epilogue
+          const int32_t gn0 = ui.tok0 + (ui.c0 + c) * C;
+          const int32_t gh = static_cast<int32_t>(ui.bh % p.H);
+          const uint64_t pol = policy_evict_first();
+          uint8_t* qslot = smem + s * kStageBytes + kOffQ;
+          mbar_arrive_expect_tx(&ctrl->gate_full[s], kTileBytes);
+          tma_load_4d(qslot, &p.tm_gate, &ctrl->gate_full[s], 0, gh, gn0, ui.b, pol);
+          tma_load_4d(qslot + kHalfBytes, &p.tm_gate, &ctrl->gate_full[s], 64, gh, gn0, ui.b, pol);
+          ++gate_issued[s];
+        }
         if (c + 1 < n_out) {
           int32_t n_next = min(C, ui.len - (c + 1) * C);
           if (kCM == kC64) n_next = min(64, n_next);  // the next tile's first chunk
@@ -1300,6 +1317,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&ctrl->kv_free);
       ++j;
     }
+    if (kGated && wq == 0 && lane == 0 && *abort_flag) {
+      // gate loads still in flight land before the CTA's shared memory goes away
+      for (uint32_t st = 0; st < 2; ++st) {
+        if (gate_issued[st] > 0) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(&ctrl->gate_full[st], (gate_issued[st] - 1) & 1) &&
+                 globaltimer_ns() - t0 < T) {
+          }
+        }
+      }
+    }
   } else if (warp >= kWarpO0) {
     // =========================================================================================
     // output epilogue: thread i owns token row i of the chunk and writes its 256-byte output row
@@ -1310,6 +1338,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t i = wq * 32 + lane;  // token row of the chunk
     const uint32_t trow = tmem + ((wq * 32) << 16);
     uint32_t j = 0, n_o = 0;
+    uint32_t eg = 0;                  // tile loads so far (the stage of a tile is eg & 1)
+    uint32_t n_gate[2] = {0u, 0u};    // gate tiles consumed per stage
     tc_fence_before();
     mbar_arrive(&ctrl->o_free);  // the O accumulators start out free
     while (true) {
@@ -1329,6 +1359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t b = ui.b;
       const int64_t h = ui.bh % p.H;
       bool good = true;
+      if (ui.flags & kUnitLocal) eg += static_cast<uint32_t>(ui.nc);  // local-state pass loads
       const int32_t n_out = (ui.flags & kUnitNoOutput) ? 0 : ui.nc;
       for (int32_t c = 0; c < n_out; ++c) {
         const float f = (c & 1) ? f_b : f_a;
@@ -1341,20 +1372,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         __nv_bfloat16* out_h = p.out + (b * p.N * p.H + h) * D;
         const int64_t row_stride = p.H * D;
         if (kGated) {
-          // the first column block's gate pieces load while O is being computed (the producer
-          // has already brought the chunk's gate tile into L2)
-          const __nv_bfloat16* gate_h = p.gate + (b * p.N * p.H + h) * D;
-          uint4 ga[4];
-          load_gate_pieces(gate_h, ui.len, r0, n0, row_stride, t, 0, ga);
-          ok = mbar_wait_bounded(&ctrl->o_full, n_o & 1, abort_flag, T);
+          // the tile's gate rows are staged in its stage's Q slot (the state warps load them once
+          // the tile's last Q product is done); once read, the stage may be refilled
+          const uint32_t s = eg & 1;
+          ++eg;
+          ok = mbar_wait_bounded(&ctrl->o_full, n_o & 1, abort_flag, T) &&
+               mbar_wait_bounded(&ctrl->gate_full[s], n_gate[s] & 1, abort_flag, T);
           if (!group_all(ok, kBarO, 128)) {
             good = false;
             break;
           }
           ++n_o;
+          ++n_gate[s];
           tc_fence_after();
-          gated_epilogue(p, ctrl, trow, col_inter, f, ui, h, gate_h, out_h, t, r0, n0, row_stride,
-                         ga);
+          gated_epilogue(p, ctrl, trow, col_inter, f, ui, h, smem + s * kStageBytes + kOffQ,
+                         out_h, t, r0, i & ~3u, n0, row_stride);
+          named_bar_sync(kBarO, 128);
+          if (wq == 0 && lane == 0) mbar_arrive(&ctrl->empty[s]);
           continue;
         }
         ok = mbar_wait_bounded(&ctrl->o_full, n_o & 1, abort_flag, T);

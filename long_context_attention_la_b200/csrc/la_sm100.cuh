@@ -169,25 +169,6 @@ __device__ __forceinline__ void tma_store_4d(const void* tmap, const void* smem_
       : "memory");
 }
 
-// Untiled bulk copy global -> shared of `bytes` (both addresses 16-byte aligned, bytes a multiple
-// of 16); completion is signalled on `bar` as transaction bytes.
-__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Untiled bulk copy shared -> global, tracked by the issuing thread's bulk groups.
-__device__ __forceinline__ void bulk_store(void* dst, const void* smem_src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                   reinterpret_cast<uint64_t>(dst)),
-               "r"(smem_u32(smem_src)), "r"(bytes)
-               : "memory");
-}
-
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
