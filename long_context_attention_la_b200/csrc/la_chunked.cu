@@ -99,6 +99,7 @@ struct Ctrl {
   uint64_t s2_full;   // C = 256: the cross scores Q_B K~_A^T of a chunk's second tile are in TMEM
   uint64_t p2_ready;  // C = 256: their scaled bf16 P_BA is in TMEM
   uint64_t gate_full[2];  // fused norm + gate: the tile's gate rows are in its stage's Q slot
+  float row_x[128];       // fused norm + gate: a row's sum of squares / 1/rms between its two warps
   uint64_t o_full;
   uint64_t o_free;
   uint64_t kv_done;
@@ -409,10 +410,13 @@ __device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint
                                                const UnitInfo& ui, int64_t h,
                                                const uint8_t* gate_tile, __nv_bfloat16* out_h,
                                                uint32_t t, int32_t r0, uint32_t i0, int64_t n0,
-                                               int64_t row_stride) {
+                                               int64_t row_stride, uint32_t i, uint32_t eh,
+                                               uint32_t n_threads) {
+  // This thread's warp takes columns [64 eh, 64 eh + 64) of row i; the other half of the row is
+  // another warp's, so the row's mean square is completed through ctrl->row_x.
   float ss = 0.f;
 #pragma unroll 1
-  for (uint32_t cb = 0; cb < 8; ++cb) {  // 16-column blocks
+  for (uint32_t cb = 4 * eh; cb < 4 * eh + 4; ++cb) {  // 16-column blocks
     uint32_t ra[16], re[16];
     tmem_ld16(trow + kColOintra + cb * 16, ra);
     tmem_ld16(trow + col_inter + cb * 16, re);
@@ -423,13 +427,21 @@ __device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint
       ss = fmaf(o, o, ss);
     }
   }
-  const float rinv = rsqrtf(fmaf(ss, 1.f / D, p.eps));
+  if (eh == 1) ctrl->row_x[i] = ss;
+  named_bar_sync(kBarO, n_threads);
+  float rinv = 0.f;
+  if (eh == 0) {
+    rinv = rsqrtf(fmaf(ss + ctrl->row_x[i], 1.f / D, p.eps));
+    ctrl->row_x[i] = rinv;
+  }
+  named_bar_sync(kBarO, n_threads);
+  if (eh == 1) rinv = ctrl->row_x[i];
   float rk[4];  // 1 / rms of rows i0 + k, held by lanes 4a + k
   const uint32_t lane0 = (threadIdx.x & 31u) & ~3u;
 #pragma unroll
   for (uint32_t k = 0; k < 4; ++k) rk[k] = __shfl_sync(0xffffffffu, rinv, lane0 + k);
 #pragma unroll 1
-  for (uint32_t cb = 0; cb < 4; ++cb) {
+  for (uint32_t cb = 2 * eh; cb < 2 * eh + 2; ++cb) {  // 32-column blocks
     uint4 g[4];
     load_gate_pieces(gate_tile, i0, t, cb, g);
     uint4 x[4];  // bf16 O, pieces q = 0..3 of this row's 32 columns
@@ -439,8 +451,8 @@ __device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint
       tmem_ld8(trow + kColOintra + cb * 32 + q * 8, ra);
       tmem_ld8(trow + col_inter + cb * 32 + q * 8, re);
       tmem_wait_ld();
-      if (cb == 3 && q == 3) {
-        // every O column of this row has been read: the accumulators may be overwritten
+      if (cb == 2 * eh + 1 && q == 3) {
+        // every O column of this thread's half row has been read
         tc_fence_before();
         mbar_arrive(&ctrl->o_free);
       }
@@ -484,6 +496,12 @@ __device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint
 template <bool kGated, int kCM>
 __global__ void __launch_bounds__(kThreads, 1)
     chunked_prefill_kernel(const __grid_constant__ Params p) {
+  // The fused norm + gate instance runs the decay mask on 4 warps (one per TMEM lane quarter)
+  // and its heavier epilogue on 8 (warps 16-19 take columns 0..63, warps 8-11 columns 64..127);
+  // the plain instance has 8 mask warps and 4 epilogue warps.
+  constexpr uint32_t kMaskWarps = kGated ? 4 : 8;
+  constexpr uint32_t kMaskThreads = 32 * kMaskWarps;
+  constexpr uint32_t kEpiThreads = kGated ? 256 : 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -504,14 +522,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctrl->gate_full[s], 1);
       mbar_init(&ctrl->kt_ready[s], 128);
       mbar_init(&ctrl->unit_full[s], 1);
-      mbar_init(&ctrl->unit_empty[s], 1 + 256 + 128 + 128);
+      mbar_init(&ctrl->unit_empty[s], 1 + kMaskThreads + 128 + kEpiThreads);
     }
     mbar_init(&ctrl->s_full, 1);
-    mbar_init(&ctrl->p_ready, 256);
+    mbar_init(&ctrl->p_ready, kMaskThreads);
     mbar_init(&ctrl->s2_full, 1);
-    mbar_init(&ctrl->p2_ready, 256);
+    mbar_init(&ctrl->p2_ready, kMaskThreads);
     mbar_init(&ctrl->o_full, 1);
-    mbar_init(&ctrl->o_free, 128);
+    mbar_init(&ctrl->o_free, kEpiThreads);
     mbar_init(&ctrl->kv_done, 1);
     mbar_init(&ctrl->kvb_ready, 128);
     mbar_init(&ctrl->kv_free, 128);
@@ -925,21 +943,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= kWarpP0 && warp < kWarpS0) {
+  } else if (warp >= kWarpP0 && warp < kWarpP0 + kMaskWarps) {
     // =========================================================================================
     // P = decay-mask(S) -> TMEM (bf16); K -> K~ in the local-state pass
     // =========================================================================================
-    const uint32_t pw = warp - kWarpP0;          // 0..7
+    const uint32_t pw = warp - kWarpP0;          // 0..kMaskWarps-1
     const uint32_t wq = warp & 3;                // TMEM lane quarter
-    const uint32_t hf = pw >> 2;                 // column blocks hf and hf + 2
+    const uint32_t hf = pw >> 2;                 // 8 warps: column blocks hf and hf + 2
     const uint32_t i = wq * 32 + lane;           // row of the chunk (query token)
-    const uint32_t tp = threadIdx.x - kWarpP0 * 32;  // 0..255
+    const uint32_t tp = threadIdx.x - kWarpP0 * 32;  // 0..kMaskThreads-1
     const uint32_t trow = tmem + ((wq * 32) << 16);
     uint32_t g = 0, j = 0, n_s = 0, n_s2 = 0;
     while (true) {
       const uint32_t slot = j & 1;
       bool ok = mbar_wait_bounded(&ctrl->unit_full[slot], (j >> 1) & 1, abort_flag, T);
-      if (!group_all(ok, kBarP, 256)) break;
+      if (!group_all(ok, kBarP, kMaskThreads)) break;
       const UnitInfo ui = ctrl->units[slot];
       mbar_arrive(&ctrl->unit_empty[slot]);
       if (ui.bh < 0) break;
@@ -947,23 +965,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float lam1 = ex2_approx(-alpha);                 // lambda
 
       if (ui.flags & 1) {
-        // local-state pass: K~_j = lambda^(L-1-j) k_j, two threads per row (one per half)
+        // local-state pass: K~_j = lambda^(L-1-j) k_j (8 warps: two threads per row, one per
+        // half; 4 warps: one thread per row)
         const uint32_t r = tp & 127;
         const uint32_t half = tp >> 7;
         for (int32_t c = 0; c < ui.nc; ++c) {
           const uint32_t s = g & 1;
           ok = mbar_wait_bounded(&ctrl->full[s], (g >> 1) & 1, abort_flag, T);
-          if (!group_all(ok, kBarP, 256)) goto p_out;
+          if (!group_all(ok, kBarP, kMaskThreads)) goto p_out;
           const int32_t pos = c * C + static_cast<int32_t>(r);  // token within the segment
           const float w =
               pos < ui.len ? exp2f(-alpha * static_cast<float>(ui.len - 1 - pos)) : 0.f;
-          scale_half_row(smem + s * kStageBytes + kOffK + half * kHalfBytes, r, w);
+          if (kMaskWarps == 8) {
+            scale_half_row(smem + s * kStageBytes + kOffK + half * kHalfBytes, r, w);
+          } else {
+            scale_half_row(smem + s * kStageBytes + kOffK, r, w);
+            scale_half_row(smem + s * kStageBytes + kOffK + kHalfBytes, r, w);
+          }
           fence_proxy_async_smem();
-          named_bar_sync(kBarP, 256);
+          named_bar_sync(kBarP, kMaskThreads);
           if (tp < 128) mbar_arrive(&ctrl->kt_ready[s]);
           ++g;
         }
       }
+      // P_ij = lambda^(i-j) S_ij for j <= i, else 0, over S columns j = 32 jb + m.  The factor
+      // lambda^max(i-j, 0) is built per 16-column half by walking m downward from the half's
+      // last column and multiplying by lambda <= 1 once j <= i: no intermediate can overflow,
+      // for any slope, and underflow only drops terms below fp32 range.
+      auto make_p = [&](uint32_t jb, const uint32_t (&r)[32], uint32_t (&pk)[16]) {
+        const int32_t dbase = static_cast<int32_t>(i) - static_cast<int32_t>(jb * 32);
+        const int mlim = jb == wq ? static_cast<int>(lane) : 31;  // columns m > mlim: j > i
+#pragma unroll
+        for (int h = 1; h >= 0; --h) {
+          const int mtop = 16 * h + 15;
+          float f = ex2_approx(-alpha * static_cast<float>(max(dbase - mtop, 0)));
+#pragma unroll
+          for (int m = mtop; m > 16 * h; m -= 2) {
+            const float x1 = m <= mlim ? __uint_as_float(r[m]) * f : 0.f;
+            if (dbase - m >= 0) f *= lam1;
+            const float x0 = m - 1 <= mlim ? __uint_as_float(r[m - 1]) * f : 0.f;
+            if (dbase - (m - 1) >= 0) f *= lam1;
+            pk[(m - 1) >> 1] = pack_bf16x2(x0, x1);
+          }
+        }
+      };
+      // C = 64: P is block-diagonal, so rows 64..127 (lane quarters 2, 3) keep nothing of
+      // columns 0..63 (S blocks 0, 1)
+      auto live = [&](uint32_t jb) { return jb <= wq && !(kCM == kC64 && wq >= 2 && jb < 2); };
       const int32_t n_out = (ui.flags & kUnitNoOutput) ? 0 : ui.nc;
       for (int32_t c = 0; c < n_out; ++c) {
         if (kCM == kC256 && (c & 1) != 0) {
@@ -971,91 +1019,101 @@ __global__ void __launch_bounds__(kThreads, 1)
           // (S~_BA = Q_B K~_A^T already carries lambda^(127-j)), no causal mask.  The block split
           // and the barrier before the first store are those of the causal pass below.
           ok = mbar_wait_bounded(&ctrl->s2_full, n_s2 & 1, abort_flag, T);
-          if (!group_all(ok, kBarP, 256)) goto p_out;
+          if (!group_all(ok, kBarP, kMaskThreads)) goto p_out;
           ++n_s2;
           tc_fence_after();
           const float fr = ex2_approx(-alpha * static_cast<float>(i + 1));
           uint32_t r[32];
           uint32_t pk[16];
-          tmem_ld32(trow + kColS + hf * 32, r);
-          tmem_wait_ld();
-          tc_fence_before();
-          named_bar_sync(kBarP, 256);
-          tc_fence_after();
+          if (kMaskWarps == 8) {
+            tmem_ld32(trow + kColS + hf * 32, r);
+            tmem_wait_ld();
+            tc_fence_before();
+            named_bar_sync(kBarP, kMaskThreads);
+            tc_fence_after();
 #pragma unroll
-          for (int m = 0; m < 16; ++m)
-            pk[m] = pack_bf16x2(__uint_as_float(r[2 * m]) * fr, __uint_as_float(r[2 * m + 1]) * fr);
-          tmem_st16(trow + kColS + hf * 16, pk);
-          tmem_ld32(trow + kColS + (hf + 2) * 32, r);
-          tmem_wait_ld();
+            for (int m = 0; m < 16; ++m)
+              pk[m] =
+                  pack_bf16x2(__uint_as_float(r[2 * m]) * fr, __uint_as_float(r[2 * m + 1]) * fr);
+            tmem_st16(trow + kColS + hf * 16, pk);
+            tmem_ld32(trow + kColS + (hf + 2) * 32, r);
+            tmem_wait_ld();
 #pragma unroll
-          for (int m = 0; m < 16; ++m)
-            pk[m] = pack_bf16x2(__uint_as_float(r[2 * m]) * fr, __uint_as_float(r[2 * m + 1]) * fr);
-          tmem_st16(trow + kColS + (hf + 2) * 16, pk);
+            for (int m = 0; m < 16; ++m)
+              pk[m] =
+                  pack_bf16x2(__uint_as_float(r[2 * m]) * fr, __uint_as_float(r[2 * m + 1]) * fr);
+            tmem_st16(trow + kColS + (hf + 2) * 16, pk);
+          } else {
+            // one warp owns the lane quarter: the blocks in order, each read before the P
+            // store that overlaps it (P block jb lands in S block jb / 2 <= jb)
+#pragma unroll 1
+            for (uint32_t jb = 0; jb < 4; ++jb) {
+              tmem_ld32(trow + kColS + jb * 32, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int m = 0; m < 16; ++m)
+                pk[m] = pack_bf16x2(__uint_as_float(r[2 * m]) * fr,
+                                    __uint_as_float(r[2 * m + 1]) * fr);
+              tmem_st16(trow + kColS + jb * 16, pk);
+            }
+          }
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(&ctrl->p2_ready);
         }
         ok = mbar_wait_bounded(&ctrl->s_full, n_s & 1, abort_flag, T);
-        if (!group_all(ok, kBarP, 256)) goto p_out;
+        if (!group_all(ok, kBarP, kMaskThreads)) goto p_out;
         ++n_s;
         tc_fence_after();
         // P is written over S in place: P block jb -> columns [16 jb, 16 jb + 16), inside S block
-        // jb / 2.  The two warps of a lane quarter take S blocks {hf, hf + 2}; the only S blocks a
-        // P store can overwrite are 0 and 1, which the warps read first, before a barrier that
-        // precedes every P store.
-        // P_ij = lambda^(i-j) S_ij for j <= i, else 0, over S columns j = 32 jb + m.  The factor
-        // lambda^max(i-j, 0) is built per 16-column half by walking m downward from the half's
-        // last column and multiplying by lambda <= 1 once j <= i: no intermediate can overflow,
-        // for any slope, and underflow only drops terms below fp32 range.
-        auto make_p = [&](uint32_t jb, const uint32_t (&r)[32], uint32_t (&pk)[16]) {
-          const int32_t dbase = static_cast<int32_t>(i) - static_cast<int32_t>(jb * 32);
-          const int mlim = jb == wq ? static_cast<int>(lane) : 31;  // columns m > mlim: j > i
-#pragma unroll
-          for (int h = 1; h >= 0; --h) {
-            const int mtop = 16 * h + 15;
-            float f = ex2_approx(-alpha * static_cast<float>(max(dbase - mtop, 0)));
-#pragma unroll
-            for (int m = mtop; m > 16 * h; m -= 2) {
-              const float x1 = m <= mlim ? __uint_as_float(r[m]) * f : 0.f;
-              if (dbase - m >= 0) f *= lam1;
-              const float x0 = m - 1 <= mlim ? __uint_as_float(r[m - 1]) * f : 0.f;
-              if (dbase - (m - 1) >= 0) f *= lam1;
-              pk[(m - 1) >> 1] = pack_bf16x2(x0, x1);
-            }
-          }
-        };
+        // jb / 2.  With 8 warps, the two warps of a lane quarter take S blocks {hf, hf + 2}; the
+        // only S blocks a P store can overwrite are 0 and 1, which the warps read first, before a
+        // barrier that precedes every P store.  With 4 warps, each warp walks its quarter's
+        // blocks in order, reading each before the store that overlaps it.
         {
           uint32_t r[32];
           uint32_t pk[16];
-          // C = 64: P is block-diagonal, so rows 64..127 (lane quarters 2, 3) keep nothing of
-          // columns 0..63 (S blocks 0, 1)
-          const uint32_t jb0 = hf;
-          const bool live0 = jb0 <= wq && !(kCM == kC64 && wq >= 2);
-          if (live0) {
-            tmem_ld32(trow + kColS + jb0 * 32, r);
-            tmem_wait_ld();
-          }
-          tc_fence_before();
-          named_bar_sync(kBarP, 256);
-          tc_fence_after();
-          if (live0) {
-            make_p(jb0, r, pk);
-          } else {
+          if (kMaskWarps == 8) {
+            const uint32_t jb0 = hf;
+            const bool live0 = live(jb0);
+            if (live0) {
+              tmem_ld32(trow + kColS + jb0 * 32, r);
+              tmem_wait_ld();
+            }
+            tc_fence_before();
+            named_bar_sync(kBarP, kMaskThreads);
+            tc_fence_after();
+            if (live0) {
+              make_p(jb0, r, pk);
+            } else {
 #pragma unroll
-            for (int m = 0; m < 16; ++m) pk[m] = 0u;
-          }
-          tmem_st16(trow + kColS + jb0 * 16, pk);
-          const uint32_t jb1 = hf + 2;
-          if (jb1 <= wq) {
-            tmem_ld32(trow + kColS + jb1 * 32, r);
-            tmem_wait_ld();
-            make_p(jb1, r, pk);
-          } else {
+              for (int m = 0; m < 16; ++m) pk[m] = 0u;
+            }
+            tmem_st16(trow + kColS + jb0 * 16, pk);
+            const uint32_t jb1 = hf + 2;
+            if (jb1 <= wq) {
+              tmem_ld32(trow + kColS + jb1 * 32, r);
+              tmem_wait_ld();
+              make_p(jb1, r, pk);
+            } else {
 #pragma unroll
-            for (int m = 0; m < 16; ++m) pk[m] = 0u;
+              for (int m = 0; m < 16; ++m) pk[m] = 0u;
+            }
+            tmem_st16(trow + kColS + jb1 * 16, pk);
+          } else {
+#pragma unroll 1
+            for (uint32_t jb = 0; jb < 4; ++jb) {
+              if (live(jb)) {
+                tmem_ld32(trow + kColS + jb * 32, r);
+                tmem_wait_ld();
+                make_p(jb, r, pk);
+              } else {
+#pragma unroll
+                for (int m = 0; m < 16; ++m) pk[m] = 0u;
+              }
+              tmem_st16(trow + kColS + jb * 16, pk);
+            }
           }
-          tmem_st16(trow + kColS + jb1 * 16, pk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -1328,7 +1386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp >= kWarpO0) {
+  } else if (warp >= kWarpO0 || (kGated && warp >= kWarpP0 + kMaskWarps && warp < kWarpS0)) {
     // =========================================================================================
     // output epilogue: thread i owns token row i of the chunk and writes its 256-byte output row
     // straight to global memory (no shared-memory staging, so the stage is released by the MMA
@@ -1340,12 +1398,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t j = 0, n_o = 0;
     uint32_t eg = 0;                  // tile loads so far (the stage of a tile is eg & 1)
     uint32_t n_gate[2] = {0u, 0u};    // gate tiles consumed per stage
+    const uint32_t eh = warp >= kWarpO0 ? 0u : 1u;  // fused norm + gate: column half
     tc_fence_before();
     mbar_arrive(&ctrl->o_free);  // the O accumulators start out free
     while (true) {
       const uint32_t slot = j & 1;
       bool ok = mbar_wait_bounded(&ctrl->unit_full[slot], (j >> 1) & 1, abort_flag, T);
-      if (!group_all(ok, kBarO, 128)) break;
+      if (!group_all(ok, kBarO, kEpiThreads)) break;
       const UnitInfo ui = ctrl->units[slot];
       mbar_arrive(&ctrl->unit_empty[slot]);
       if (ui.bh < 0) break;
@@ -1378,7 +1437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++eg;
           ok = mbar_wait_bounded(&ctrl->o_full, n_o & 1, abort_flag, T) &&
                mbar_wait_bounded(&ctrl->gate_full[s], n_gate[s] & 1, abort_flag, T);
-          if (!group_all(ok, kBarO, 128)) {
+          if (!group_all(ok, kBarO, kEpiThreads)) {
             good = false;
             break;
           }
@@ -1386,13 +1445,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++n_gate[s];
           tc_fence_after();
           gated_epilogue(p, ctrl, trow, col_inter, f, ui, h, smem + s * kStageBytes + kOffQ,
-                         out_h, t, r0, i & ~3u, n0, row_stride);
-          named_bar_sync(kBarO, 128);
-          if (wq == 0 && lane == 0) mbar_arrive(&ctrl->empty[s]);
+                         out_h, t, r0, i & ~3u, n0, row_stride, i, eh, kEpiThreads);
+          named_bar_sync(kBarO, kEpiThreads);
+          if (warp == kWarpO0 && lane == 0) mbar_arrive(&ctrl->empty[s]);
           continue;
         }
         ok = mbar_wait_bounded(&ctrl->o_full, n_o & 1, abort_flag, T);
-        if (!group_all(ok, kBarO, 128)) {
+        if (!group_all(ok, kBarO, kEpiThreads)) {
           good = false;
           break;
         }
