@@ -381,11 +381,11 @@ __device__ __forceinline__ void next_balanced_unit(const Params& p, RangeCursor&
 // Output epilogue with the fused grouped RMSNorm and sigmoid gate ("Ling and Ring 2.6 Technical
 // Report", §2.1 Fig. 2; §4.3): thread i's row of O (one head, D channels) is one norm group,
 //     y_j = gamma_j * O_j / sqrt(mean(O^2) + eps) * sigmoid(g_j).
-// Pass 1 reads the row's fp32 accumulators once for the mean square.  Pass 2 reads them again,
-// rounds O to bf16 (the precision the unfused layer hands to its norm), exchanges 16-byte pieces
-// within each 4-lane group as the plain epilogue does, and then finishes each piece in the store
-// layout: lane t holds piece t of rows i0..i0+3, so its gate loads and stores write whole sectors
-// and its gamma slice is the same for all four rows.
+// Pass 1 reads the row's fp32 accumulators once: it sums the squares and keeps O rounded to bf16
+// (the precision the unfused layer hands to its norm) in registers.  Pass 2 exchanges 16-byte
+// pieces of that O within each 4-lane group as the plain epilogue does, and then finishes each
+// piece in the store layout: lane t holds piece t of rows i0..i0+3, so its gate reads and stores
+// cover whole sectors and its gamma slice is the same for all four rows.
 // sigmoid(x) = (1 + tanh(x / 2)) / 2: one MUFU operation (tanh.approx, max relative error
 // about 2^-11) instead of an exponential and a reciprocal.
 __device__ __forceinline__ float sigmoidf_fast(float x) {
@@ -405,28 +405,42 @@ __device__ __forceinline__ void load_gate_pieces(const uint8_t* gate_tile, uint3
     g[k] = *reinterpret_cast<const uint4*>(half + sw128_off(i0 + k, piece & 7u));
 }
 
-__device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint32_t trow,
-                                               uint32_t col_inter, float f,
-                                               const UnitInfo& ui, int64_t h,
-                                               const uint8_t* gate_tile, __nv_bfloat16* out_h,
-                                               uint32_t t, int32_t r0, uint32_t i0, int64_t n0,
-                                               int64_t row_stride, uint32_t i, uint32_t eh,
-                                               uint32_t n_threads) {
-  // This thread's warp takes columns [64 eh, 64 eh + 64) of row i; the other half of the row is
-  // another warp's, so the row's mean square is completed through ctrl->row_x.
+// Pass 1: columns [64 eh, 64 eh + 64) of this thread's row i; the other half of the row is
+// another warp's.  Returns the half row's sum of squares and its O rounded to bf16 (pairs of
+// columns 64 eh + 2m, 64 eh + 2m + 1), then gives O back to the MMA warp.
+__device__ __forceinline__ float gated_epilogue_read(Ctrl* ctrl, uint32_t trow, uint32_t col_inter,
+                                                     float f, uint32_t eh, uint32_t (&ob)[32]) {
   float ss = 0.f;
-#pragma unroll 1
-  for (uint32_t cb = 4 * eh; cb < 4 * eh + 4; ++cb) {  // 16-column blocks
+#pragma unroll
+  for (uint32_t c = 0; c < 4; ++c) {  // 16-column blocks
+    const uint32_t cb = 4 * eh + c;
     uint32_t ra[16], re[16];
     tmem_ld16(trow + kColOintra + cb * 16, ra);
     tmem_ld16(trow + col_inter + cb * 16, re);
     tmem_wait_ld();
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const float o = fmaf(f, __uint_as_float(re[m]), __uint_as_float(ra[m]));
-      ss = fmaf(o, o, ss);
+    for (int m = 0; m < 16; m += 2) {
+      const float o0 = fmaf(f, __uint_as_float(re[m]), __uint_as_float(ra[m]));
+      const float o1 = fmaf(f, __uint_as_float(re[m + 1]), __uint_as_float(ra[m + 1]));
+      ss = fmaf(o0, o0, ss);
+      ss = fmaf(o1, o1, ss);
+      ob[c * 8 + m / 2] = pack_bf16x2(o0, o1);
     }
   }
+  tc_fence_before();
+  mbar_arrive(&ctrl->o_free);  // every O column of this thread's half row has been read
+  return ss;
+}
+
+// Pass 2: completes the row's mean square through ctrl->row_x with the warp that holds the other
+// half, then writes y for this thread's half row from the gate rows staged in shared memory.
+__device__ __forceinline__ void gated_epilogue_write(const Params& p, Ctrl* ctrl, float ss,
+                                                     const uint32_t (&ob)[32],
+                                                     const UnitInfo& ui, int64_t h,
+                                                     const uint8_t* gate_tile,
+                                                     __nv_bfloat16* out_h, uint32_t t, int32_t r0,
+                                                     uint32_t i0, int64_t n0, int64_t row_stride,
+                                                     uint32_t i, uint32_t eh, uint32_t n_threads) {
   if (eh == 1) ctrl->row_x[i] = ss;
   named_bar_sync(kBarO, n_threads);
   float rinv = 0.f;
@@ -440,31 +454,16 @@ __device__ __forceinline__ void gated_epilogue(const Params& p, Ctrl* ctrl, uint
   const uint32_t lane0 = (threadIdx.x & 31u) & ~3u;
 #pragma unroll
   for (uint32_t k = 0; k < 4; ++k) rk[k] = __shfl_sync(0xffffffffu, rinv, lane0 + k);
-#pragma unroll 1
-  for (uint32_t cb = 2 * eh; cb < 2 * eh + 2; ++cb) {  // 32-column blocks
+#pragma unroll
+  for (uint32_t cc = 0; cc < 2; ++cc) {  // 32-column blocks of the half row
+    const uint32_t cb = 2 * eh + cc;
     uint4 g[4];
     load_gate_pieces(gate_tile, i0, t, cb, g);
     uint4 x[4];  // bf16 O, pieces q = 0..3 of this row's 32 columns
 #pragma unroll
-    for (uint32_t q = 0; q < 4; ++q) {
-      uint32_t ra[8], re[8];
-      tmem_ld8(trow + kColOintra + cb * 32 + q * 8, ra);
-      tmem_ld8(trow + col_inter + cb * 32 + q * 8, re);
-      tmem_wait_ld();
-      if (cb == 2 * eh + 1 && q == 3) {
-        // every O column of this thread's half row has been read
-        tc_fence_before();
-        mbar_arrive(&ctrl->o_free);
-      }
-      float o[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        o[e] = fmaf(f, __uint_as_float(re[e]), __uint_as_float(ra[e]));
-      x[q].x = pack_bf16x2(o[0], o[1]);
-      x[q].y = pack_bf16x2(o[2], o[3]);
-      x[q].z = pack_bf16x2(o[4], o[5]);
-      x[q].w = pack_bf16x2(o[6], o[7]);
-    }
+    for (uint32_t q = 0; q < 4; ++q)
+      x[q] = make_uint4(ob[cc * 16 + q * 4], ob[cc * 16 + q * 4 + 1], ob[cc * 16 + q * 4 + 2],
+                        ob[cc * 16 + q * 4 + 3]);
     transpose4x4_lanes(x, t);  // now x[k] = piece t of row i0 + k
     const float4 g0 = __ldg(reinterpret_cast<const float4*>(p.gamma + h * D + cb * 32 + 8 * t));
     const float4 g1 = __ldg(reinterpret_cast<const float4*>(p.gamma + h * D + cb * 32 + 8 * t) + 1);
@@ -1435,17 +1434,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the tile's last Q product is done); once read, the stage may be refilled
           const uint32_t s = eg & 1;
           ++eg;
-          ok = mbar_wait_bounded(&ctrl->o_full, n_o & 1, abort_flag, T) &&
-               mbar_wait_bounded(&ctrl->gate_full[s], n_gate[s] & 1, abort_flag, T);
+          ok = mbar_wait_bounded(&ctrl->o_full, n_o & 1, abort_flag, T);
           if (!group_all(ok, kBarO, kEpiThreads)) {
             good = false;
             break;
           }
           ++n_o;
-          ++n_gate[s];
           tc_fence_after();
-          gated_epilogue(p, ctrl, trow, col_inter, f, ui, h, smem + s * kStageBytes + kOffQ,
-                         out_h, t, r0, i & ~3u, n0, row_stride, i, eh, kEpiThreads);
+          uint32_t ob[32];
+          const float ss = gated_epilogue_read(ctrl, trow, col_inter, f, eh, ob);
+          // the gate rows land while O is read
+          ok = mbar_wait_bounded(&ctrl->gate_full[s], n_gate[s] & 1, abort_flag, T);
+          if (!group_all(ok, kBarO, kEpiThreads)) {
+            good = false;
+            break;
+          }
+          ++n_gate[s];
+          gated_epilogue_write(p, ctrl, ss, ob, ui, h, smem + s * kStageBytes + kOffQ, out_h, t,
+                               r0, i & ~3u, n0, row_stride, i, eh, kEpiThreads);
           named_bar_sync(kBarO, kEpiThreads);
           if (warp == kWarpO0 && lane == 0) mbar_arrive(&ctrl->empty[s]);
           continue;

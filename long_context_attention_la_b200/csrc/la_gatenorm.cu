@@ -34,9 +34,10 @@ struct Io<__nv_bfloat16> {  // 8 values = one 16-byte piece
       x[2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
     }
   }
+  // round to nearest even, one paired conversion; lo in the low half
   static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
-    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(lo))) |
-           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&p);
   }
   static __device__ __forceinline__ void store(__nv_bfloat16* dst, const float (&y)[8]) {
     __stcs(reinterpret_cast<uint4*>(dst),
@@ -123,10 +124,10 @@ __global__ void __launch_bounds__(kGnThreads, 2) gate_norm_kernel(const GateNorm
     return ring + (stage * kPerItem + piece) * kGnThreads + tid;
   };
   // copy the pieces of item `it` into ring stage `st` (one commit group, empty past the range)
-  auto issue = [&](int64_t it, int st) {
+  auto issue = [&](int64_t it, const ItemCursor& c, int st) {
     if (it < i1) {
-      const int64_t t = it / per_token;
-      const int64_t hb = (it - t * per_token) * (ROWS * kSweeps);
+      const int64_t t = c.t;
+      const int64_t hb = c.sub * (ROWS * kSweeps);
 #pragma unroll
       for (int j = 0; j < kSweeps; ++j) {
         const int64_t h = hb + j * ROWS + tid / TPR;
@@ -142,14 +143,20 @@ __global__ void __launch_bounds__(kGnThreads, 2) gate_norm_kernel(const GateNorm
     cp_async_commit();
   };
 
-  issue(i0, 0);
-  issue(i0 + 1, 1);
+  ItemCursor cur = ItemCursor::at(i0, per_token);  // item it
+  ItemCursor ahead = cur;                          // item it + 2
+  issue(i0, ahead, 0);
+  ahead.advance(per_token);
+  issue(i0 + 1, ahead, 1);
+  ahead.advance(per_token);
   int st = 0;
   for (int64_t it = i0; it < i1; ++it) {
-    issue(it + 2, st == 0 ? 2 : st - 1);  // the stage item it - 1 used
-    cp_async_wait<2>();                   // item it's group has landed
-    const int64_t t = it / per_token;
-    const int64_t hb = (it - t * per_token) * (ROWS * kSweeps);
+    issue(it + 2, ahead, st == 0 ? 2 : st - 1);  // the stage item it - 1 used
+    ahead.advance(per_token);
+    cp_async_wait<2>();                          // item it's group has landed
+    const int64_t t = cur.t;
+    const int64_t hb = cur.sub * (ROWS * kSweeps);
+    cur.advance(per_token);
 #pragma unroll
     for (int j = 0; j < kSweeps; ++j) {
       const int64_t h = hb + j * ROWS + tid / TPR;

@@ -29,11 +29,10 @@ namespace {
 
 constexpr int kQkThreads = 512;
 
-// two floats -> bf16x2 (round to nearest even), lo in the low half
+// two floats -> bf16x2 (round to nearest even, one paired conversion), lo in the low half
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
-  const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-  const uint32_t u = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-  return l | (u << 16);
+  const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&p);
 }
 
 // Work item: ROWS x kBatch rows of one token (q heads first, then k heads); a CTA takes a
@@ -76,10 +75,10 @@ __global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNor
   auto slot = [&](int stage, int j, int w) -> uint4* {
     return ring + ((stage * kBatch + j) * 2 + w) * kQkThreads + tid;
   };
-  auto issue = [&](int64_t it, int st) {
+  auto issue = [&](int64_t it, const ItemCursor& c, int st) {
     if (it < i1) {
-      const int64_t t = it / per_token;
-      const int64_t rb = (it - t * per_token) * (ROWS * kBatch);
+      const int64_t t = c.t;
+      const int64_t rb = c.sub * (ROWS * kBatch);
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
         const int64_t row = rb + j * ROWS + tid / TPR;
@@ -126,20 +125,26 @@ __global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNor
     return w;
   };
 
-  issue(i0, 0);
-  issue(i0 + 1, 1);
+  ItemCursor cur = ItemCursor::at(i0, per_token);  // item it
+  ItemCursor ahead = cur;                          // item it + 2
+  issue(i0, ahead, 0);
+  ahead.advance(per_token);
+  issue(i0 + 1, ahead, 1);
+  ahead.advance(per_token);
   int st = 0;
-  int64_t pos = i0 < i1 ? a.positions[i0 / per_token] : 0;
+  int64_t pos = i0 < i1 ? a.positions[cur.t] : 0;
   for (int64_t it = i0; it < i1; ++it) {
-    issue(it + 2, st == 0 ? 2 : st - 1);  // the stage item it - 1 used
-    const int64_t t = it / per_token;
+    issue(it + 2, ahead, st == 0 ? 2 : st - 1);  // the stage item it - 1 used
+    ahead.advance(per_token);
+    const int64_t t = cur.t;
+    const int64_t rb = cur.sub * (ROWS * kBatch);
+    cur.advance(per_token);
     // the next item's position, one item ahead of its use
-    const int64_t pos_next = it + 1 < i1 ? a.positions[(it + 1) / per_token] : 0;
+    const int64_t pos_next = it + 1 < i1 ? a.positions[cur.t] : 0;
     __syncwarp();                         // the warp is done reading the previous token's table
     angles(pos);
     __syncwarp();                         // ... and this token's table is written
     cp_async_wait<2>();                   // item it's rows have landed (this thread's pieces)
-    const int64_t rb = (it - t * per_token) * (ROWS * kBatch);
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
       const int64_t row = rb + j * ROWS + tid / TPR;

@@ -218,6 +218,22 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
 }
 
+// Position of a streaming work item as (token, block within the token), advanced one item at a
+// time, so an item loop needs no 64-bit division (a software routine of dozens of instructions).
+struct ItemCursor {
+  int64_t t, sub;
+  __device__ __forceinline__ static ItemCursor at(int64_t item, int64_t per_token) {
+    const int64_t t = item / per_token;
+    return ItemCursor{t, item - t * per_token};
+  }
+  __device__ __forceinline__ void advance(int64_t per_token) {
+    if (++sub == per_token) {
+      sub = 0;
+      ++t;
+    }
+  }
+};
+
 // ---------------------------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation tensor core
 // ---------------------------------------------------------------------------------------------
