@@ -44,13 +44,15 @@ DECODE = dict(B=256, H=64, d=128)
 
 def measured_counters():
     """Counters of one prefill launch of the default workload from the committed ncu capture
-    (profiles/chunked_prefill_kernel_counters.json), or None when the kernel sources changed
-    since that capture: DRAM bytes and the tensor-pipe activity."""
+    (the fenced json record in profiles/chunked_prefill_kernel_counters.md), or None when the
+    kernel sources changed since that capture: DRAM bytes and the tensor-pipe activity."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "chunked_prefill_kernel_counters.json")
+    path = os.path.join(ROOT, "profiles", "chunked_prefill_kernel_counters.md")
     try:
         with open(path) as f:
-            rec = json.load(f)
+            text = f.read()
+        start = text.index("```json\n") + len("```json\n")
+        rec = json.loads(text[start:text.index("\n```", start)])
         h = hashlib.sha256()
         for src in rec["sources"]:
             with open(os.path.join(ROOT, src), "rb") as f:

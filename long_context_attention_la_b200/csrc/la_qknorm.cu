@@ -12,7 +12,9 @@
 // is handled by d/16 consecutive threads with two 16-byte pieces each, chosen so that both
 // members of every rotary pair sit in one thread (no exchange between threads), staged through
 // a shared-memory ring by per-thread cp.async copies; the mean square is a shuffle reduction over
-// the row's threads.  The angle pos * w_i is formed and reduced modulo 2 pi in
+// the row's threads.  The norm weights sit in shared memory (per-row loads of them through L1
+// doubled the L1 traffic), and the row arithmetic runs on paired fp32 operations (two lanes per
+// instruction; the sum of squares keeps two partial sums).  The angle pos * w_i is formed and reduced modulo 2 pi in
 // double precision (positions reach 2^18 and more, where a float angle would be off by ~0.03 rad),
 // then sin and cos are taken in float, once per token and frequency by each warp.
 #include <cuda_bf16.h>
@@ -56,6 +58,7 @@ __global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNor
   extern __shared__ uint4 ring[];              // [kStages][kBatch][2][kQkThreads]
   __shared__ __align__(16) float cs_sh[kQkThreads / 32][64];  // per warp: cos, sin of the token
   __shared__ __align__(16) float sn_sh[kQkThreads / 32][64];
+  __shared__ __align__(16) float gam_sh[2][D];  // gamma_q, gamma_k
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int u = tid % TPR;                     // position of this thread in its row
@@ -72,6 +75,9 @@ __global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNor
   const int pa = rotary ? u : a.rotary_dim / 8 + (u - rot_threads);
   const int pb = rotary ? u + rot_threads : pa + (D - a.rotary_dim) / 16;
 
+  for (int i = threadIdx.x; i < 2 * D; i += kQkThreads)
+    gam_sh[i / D][i % D] = i < D ? a.gamma_q[i] : a.gamma_k[i - D];
+  __syncthreads();
   auto slot = [&](int stage, int j, int w) -> uint4* {
     return ring + ((stage * kBatch + j) * 2 + w) * kQkThreads + tid;
   };
@@ -108,22 +114,21 @@ __global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNor
       sn_sh[warp][f] = sn;
     }
   };
-  auto unpack = [](const uint4& w, float (&x)[8]) {
+  auto unpack = [](const uint4& w, float2 (&x)[4]) {
     const uint32_t v[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      x[2 * e] = __uint_as_float(v[e] << 16);
-      x[2 * e + 1] = __uint_as_float(v[e] & 0xffff0000u);
-    }
+    for (int e = 0; e < 4; ++e)
+      x[e] = make_float2(__uint_as_float(v[e] << 16), __uint_as_float(v[e] & 0xffff0000u));
   };
-  auto pack = [](const float (&y)[8]) {
+  auto pack_row = [](const float2 (&y)[4]) {
     uint4 w;
-    w.x = pack2(y[0], y[1]);
-    w.y = pack2(y[2], y[3]);
-    w.z = pack2(y[4], y[5]);
-    w.w = pack2(y[6], y[7]);
+    w.x = pack2(y[0].x, y[0].y);
+    w.y = pack2(y[1].x, y[1].y);
+    w.z = pack2(y[2].x, y[2].y);
+    w.w = pack2(y[3].x, y[3].y);
     return w;
   };
+
 
   ItemCursor cur = ItemCursor::at(i0, per_token);  // item it
   ItemCursor ahead = cur;                          // item it + 2
@@ -151,47 +156,54 @@ __global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNor
       const bool valid = row < rows;  // uniform across a row's threads
       const bool is_k = row >= a.H;
       const int64_t h = is_k ? row - a.H : row;
-      float xa[8], xb[8];
+      float2 xa[4], xb[4];
       unpack(*slot(st, j, 0), xa);
       unpack(*slot(st, j, 1), xb);
       // mean square over the row: reduce across the TPR threads of the row (aligned groups)
-      float ss = 0.f;
+      float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fmaf(xb[e], xb[e], fmaf(xa[e], xa[e], ss));
+      for (int e = 0; e < 4; ++e) acc = __ffma2_rn(xb[e], xb[e], __ffma2_rn(xa[e], xa[e], acc));
+      float ss = acc.x + acc.y;
 #pragma unroll
       for (int o = TPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       const float rinv = rsqrtf(fmaf(ss, 1.f / D, a.eps));
-      const float* gam = is_k ? a.gamma_k : a.gamma_q;
-      const float4 ga0 = __ldg(reinterpret_cast<const float4*>(gam + pa * 8));
-      const float4 ga1 = __ldg(reinterpret_cast<const float4*>(gam + pa * 8) + 1);
-      const float4 gb0 = __ldg(reinterpret_cast<const float4*>(gam + pb * 8));
-      const float4 gb1 = __ldg(reinterpret_cast<const float4*>(gam + pb * 8) + 1);
-      const float gma[8] = {ga0.x, ga0.y, ga0.z, ga0.w, ga1.x, ga1.y, ga1.z, ga1.w};
-      const float gmb[8] = {gb0.x, gb0.y, gb0.z, gb0.w, gb1.x, gb1.y, gb1.z, gb1.w};
-      float ya[8], yb[8];
+      const float2 r2 = make_float2(rinv, rinv);
+      const float* gam = gam_sh[is_k ? 1 : 0];
+      const float4 ga0 = *reinterpret_cast<const float4*>(gam + pa * 8);
+      const float4 ga1 = *(reinterpret_cast<const float4*>(gam + pa * 8) + 1);
+      const float4 gb0 = *reinterpret_cast<const float4*>(gam + pb * 8);
+      const float4 gb1 = *(reinterpret_cast<const float4*>(gam + pb * 8) + 1);
+      const float2 gma[4] = {make_float2(ga0.x, ga0.y), make_float2(ga0.z, ga0.w),
+                             make_float2(ga1.x, ga1.y), make_float2(ga1.z, ga1.w)};
+      const float2 gmb[4] = {make_float2(gb0.x, gb0.y), make_float2(gb0.z, gb0.w),
+                             make_float2(gb1.x, gb1.y), make_float2(gb1.z, gb1.w)};
+      float2 ya[4], yb[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        ya[e] = gma[e] * (xa[e] * rinv);
-        yb[e] = gmb[e] * (xb[e] * rinv);
+      for (int e = 0; e < 4; ++e) {
+        ya[e] = __fmul2_rn(gma[e], __fmul2_rn(xa[e], r2));
+        yb[e] = __fmul2_rn(gmb[e], __fmul2_rn(xb[e], r2));
       }
       if (rotary) {
         // rotate-half: dims (8 pa + e, 8 pa + e + r/2) with frequency index 8 pa + e
         const float4* c4 = reinterpret_cast<const float4*>(&cs_sh[warp][pa * 8]);
         const float4* s4 = reinterpret_cast<const float4*>(&sn_sh[warp][pa * 8]);
         const float4 c0 = c4[0], c1 = c4[1], s0 = s4[0], s1 = s4[1];
-        const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+        const float2 cs[4] = {make_float2(c0.x, c0.y), make_float2(c0.z, c0.w),
+                              make_float2(c1.x, c1.y), make_float2(c1.z, c1.w)};
+        const float2 sn[4] = {make_float2(s0.x, s0.y), make_float2(s0.z, s0.w),
+                              make_float2(s1.x, s1.y), make_float2(s1.z, s1.w)};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float y0 = ya[e], y1 = yb[e];
-          ya[e] = fmaf(y0, cs[e], -y1 * sn[e]);
-          yb[e] = fmaf(y1, cs[e], y0 * sn[e]);
+        for (int e = 0; e < 4; ++e) {
+          const float2 y0 = ya[e], y1 = yb[e];
+          const float2 nsn = make_float2(-sn[e].x, -sn[e].y);
+          ya[e] = __ffma2_rn(y0, cs[e], __fmul2_rn(y1, nsn));
+          yb[e] = __ffma2_rn(y1, cs[e], __fmul2_rn(y0, sn[e]));
         }
       }
       if (valid) {
         __nv_bfloat16* dst = (is_k ? a.k_out : a.q_out) + (t * a.H + h) * D;
-        __stcs(reinterpret_cast<uint4*>(dst + pa * 8), pack(ya));
-        __stcs(reinterpret_cast<uint4*>(dst + pb * 8), pack(yb));
+        __stcs(reinterpret_cast<uint4*>(dst + pa * 8), pack_row(ya));
+        __stcs(reinterpret_cast<uint4*>(dst + pb * 8), pack_row(yb));
       }
     }
     st = st == kStages - 1 ? 0 : st + 1;
