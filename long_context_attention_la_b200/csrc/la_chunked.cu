@@ -386,12 +386,12 @@ __device__ __forceinline__ void next_balanced_unit(const Params& p, RangeCursor&
 // pieces of that O within each 4-lane group as the plain epilogue does, and then finishes each
 // piece in the store layout: lane t holds piece t of rows i0..i0+3, so its gate reads and stores
 // cover whole sectors and its gamma slice is the same for all four rows.
-// sigmoid(x) = (1 + tanh(x / 2)) / 2: one MUFU operation (tanh.approx, max relative error
+// sigmoid(x) = (1 + tanh(x / 2)) / 2 takes one MUFU operation (tanh.approx, max relative error
 // about 2^-11) instead of an exponential and a reciprocal.
-__device__ __forceinline__ float sigmoidf_fast(float x) {
+__device__ __forceinline__ float tanhf_fast(float x) {
   float t;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
-  return fmaf(0.5f, t, 0.5f);
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(x));
+  return t;
 }
 
 // Gate pieces of 32-column block cb in the 4-lane store layout, from the tile's gate rows staged
@@ -473,14 +473,22 @@ __device__ __forceinline__ void gated_epilogue_write(const Params& p, Ctrl* ctrl
       if (r0 + static_cast<int32_t>(k) < ui.len) {
         const uint32_t gw[4] = {g[k].x, g[k].y, g[k].z, g[k].w};
         const uint32_t ow[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+        // y = gamma * (O * rinv) * sigmoid(g) on paired fp32 operations (two columns per
+        // instruction, the same roundings as the scalar form); the sigmoid is
+        // 1/2 + tanh(g/2)/2 with one MUFU tanh per column
         uint32_t yw[4];
+        const float2 rk2 = make_float2(rk[k], rk[k]);
+        const float2 half2 = make_float2(0.5f, 0.5f);
 #pragma unroll
         for (int e2 = 0; e2 < 4; ++e2) {
-          const float y0 = gm[2 * e2] * (bf16lo_to_f32(ow[e2]) * rk[k]) *
-                           sigmoidf_fast(bf16lo_to_f32(gw[e2]));
-          const float y1 = gm[2 * e2 + 1] * (bf16hi_to_f32(ow[e2]) * rk[k]) *
-                           sigmoidf_fast(bf16hi_to_f32(gw[e2]));
-          yw[e2] = pack_bf16x2(y0, y1);
+          const float2 ov = make_float2(bf16lo_to_f32(ow[e2]), bf16hi_to_f32(ow[e2]));
+          const float2 hg =
+              __fmul2_rn(half2, make_float2(bf16lo_to_f32(gw[e2]), bf16hi_to_f32(gw[e2])));
+          const float2 sg = __ffma2_rn(half2, make_float2(tanhf_fast(hg.x), tanhf_fast(hg.y)),
+                                       half2);
+          const float2 y = __fmul2_rn(
+              __fmul2_rn(make_float2(gm[2 * e2], gm[2 * e2 + 1]), __fmul2_rn(ov, rk2)), sg);
+          yw[e2] = pack_bf16x2(y.x, y.y);
         }
         uint4* dst = reinterpret_cast<uint4*>(out_h + (n0 + k) * row_stride + cb * 32) + t;
         __stcs(dst, make_uint4(yw[0], yw[1], yw[2], yw[3]));

@@ -58,7 +58,10 @@ __global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNor
   extern __shared__ uint4 ring[];              // [kStages][kBatch][2][kQkThreads]
   __shared__ __align__(16) float cs_sh[kQkThreads / 32][64];  // per warp: cos, sin of the token
   __shared__ __align__(16) float sn_sh[kQkThreads / 32][64];
-  __shared__ __align__(16) float gam_sh[2][D];  // gamma_q, gamma_k
+  // gamma_q, gamma_k; 4 floats of padding after every 64, so the 16-byte reads of one row's
+  // threads (pieces 0..3 and 8..11 of the row, 256 bytes apart) fall in different banks
+  constexpr int kGamStride = D + 4 * (D / 64);
+  __shared__ __align__(16) float gam_sh[2][kGamStride];
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int u = tid % TPR;                     // position of this thread in its row
@@ -75,8 +78,10 @@ __global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNor
   const int pa = rotary ? u : a.rotary_dim / 8 + (u - rot_threads);
   const int pb = rotary ? u + rot_threads : pa + (D - a.rotary_dim) / 16;
 
-  for (int i = threadIdx.x; i < 2 * D; i += kQkThreads)
-    gam_sh[i / D][i % D] = i < D ? a.gamma_q[i] : a.gamma_k[i - D];
+  for (int i = threadIdx.x; i < 2 * D; i += kQkThreads) {
+    const int dd = i % D;
+    gam_sh[i / D][dd + 4 * (dd / 64)] = i < D ? a.gamma_q[i] : a.gamma_k[i - D];
+  }
   __syncthreads();
   auto slot = [&](int stage, int j, int w) -> uint4* {
     return ring + ((stage * kBatch + j) * 2 + w) * kQkThreads + tid;
@@ -169,10 +174,10 @@ __global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNor
       const float rinv = rsqrtf(fmaf(ss, 1.f / D, a.eps));
       const float2 r2 = make_float2(rinv, rinv);
       const float* gam = gam_sh[is_k ? 1 : 0];
-      const float4 ga0 = *reinterpret_cast<const float4*>(gam + pa * 8);
-      const float4 ga1 = *(reinterpret_cast<const float4*>(gam + pa * 8) + 1);
-      const float4 gb0 = *reinterpret_cast<const float4*>(gam + pb * 8);
-      const float4 gb1 = *(reinterpret_cast<const float4*>(gam + pb * 8) + 1);
+      const float4* gpa = reinterpret_cast<const float4*>(gam + pa * 8 + 4 * (pa / 8));
+      const float4* gpb = reinterpret_cast<const float4*>(gam + pb * 8 + 4 * (pb / 8));
+      const float4 ga0 = gpa[0], ga1 = gpa[1];
+      const float4 gb0 = gpb[0], gb1 = gpb[1];
       const float2 gma[4] = {make_float2(ga0.x, ga0.y), make_float2(ga0.z, ga0.w),
                              make_float2(ga1.x, ga1.y), make_float2(ga1.z, ga1.w)};
       const float2 gmb[4] = {make_float2(gb0.x, gb0.y), make_float2(gb0.z, gb0.w),
