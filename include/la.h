@@ -78,9 +78,15 @@ typedef struct {
                        256 (every C computes the same recurrence; they differ only in where
                        the bf16 roundings of the intra / inter split fall); the recurrent path
                        takes 0 or 1 */
-  int32_t segments; /* segments per sequence: 0 = automatic; >= 1 explicit (clamped to chunks) */
+  int32_t segments; /* segments per sequence: 0 = automatic; >= 1 explicit (clamped to chunks);
+                       LA_SEGMENTS_BALANCED = the balanced range plan (the tiles of all
+                       sequences cut into one contiguous range per SM), which the automatic
+                       choice takes for few long sequences */
   int32_t path;     /* la_path */
 } la_desc;
+
+/* la_desc.segments value that selects the balanced range plan (tensor path of la_prefill). */
+#define LA_SEGMENTS_BALANCED (-1)
 
 /* Bytes of device workspace la_prefill needs for this descriptor (0 if none).  The workspace holds
  * the segment-state ring, the scan flags, a work counter and a device status word. */
@@ -206,10 +212,11 @@ la_status la_decode_multi(int64_t B, int64_t H, int64_t d, int64_t n_tok, int32_
  *
  *   - Limit: problems whose scratch need (la_prefill_workspace_bytes) exceeds
  *     LA_NOALLOC_SCRATCH_BYTES are rejected with LA_ERR_WORKSPACE before anything is enqueued.
- *     Within the limit is every problem with the automatic plan (desc->segments = 0) on a GPU of
- *     up to 256 SMs, whatever B, N and H: that plan needs a header plus one flag and one
- *     d x d fp32 state per SM.  An explicit segment count needs two states per sequence when it
- *     cuts sequences, which fits for B*H up to 128.  The fp32 / recurrent path needs no
+ *     Within the limit is every problem with the automatic plan (desc->segments = 0) or the
+ *     balanced plan (LA_SEGMENTS_BALANCED) on a GPU of up to 256 SMs, whatever B, N and H: those
+ *     plans need at most a header plus one flag and one d x d fp32 state per SM.  An explicit
+ *     segment count needs two states per sequence when it cuts sequences, which fits for B*H up
+ *     to 128.  The fp32 / recurrent path needs no
  *     scratch at all.
  *   - First call on a device: it looks up the device address of the array (cudaGetSymbolAddress)
  *     with that device current and caches it for that device's CUDA context; make that first

@@ -46,19 +46,67 @@ bool use_tensor_path(const la_desc* d) { return use_tensor_path(d->path, d->dtyp
 // The tensor path's chunk length for a descriptor's `chunk` field (0: the library's default).
 int chunk_of(int32_t chunk) { return chunk == 0 ? la::kChunkDefault : chunk; }
 
-// Workspace bytes of la_prefill's tensor path: the balanced plan when the segment count is left
-// to the library, else equal segments per sequence.
-size_t prefill_workspace_need(const la_desc* d, int sms) {
-  if (d->segments == 0) {
-    la::BalancedPlan bal{};
-    la::SegmentPlan seg{};
-    if (la::prefer_balanced(d->B, d->N, d->H, sms, chunk_of(d->chunk), &bal, &seg))
-      return la::balanced_workspace_bytes(bal);
-    return la::workspace_layout(d->B, d->H, seg).total;
+// The work plan of la_prefill's tensor path: balanced ranges (returns true, fills *bal) when asked
+// for or when the automatic choice prefers them, else equal segments per sequence (fills *seg).
+bool compute_plan(const la_desc* d, int sms, la::BalancedPlan* bal, la::SegmentPlan* seg) {
+  const int chunk = chunk_of(d->chunk);
+  if (d->segments == LA_SEGMENTS_BALANCED) {
+    *bal = la::plan_balanced(d->B, d->N, d->H, sms, chunk);
+    return true;
   }
-  const la::SegmentPlan plan =
-      la::plan_segments(d->B, d->N, d->H, d->segments, sms, chunk_of(d->chunk));
-  return la::workspace_layout(d->B, d->H, plan).total;
+  if (d->segments == 0) return la::prefer_balanced(d->B, d->N, d->H, sms, chunk, bal, seg);
+  *seg = la::plan_segments(d->B, d->N, d->H, d->segments, sms, chunk);
+  return false;
+}
+
+// The balanced plan's search takes 0.1-0.25 ms of host time, as long as a short prefill itself, so
+// the last few plans are kept, keyed by everything they depend on (shared by all host threads).
+struct PlanCacheEntry {
+  int64_t B = 0, N = 0, H = 0;
+  int32_t sms = 0, chunk = 0, segments = 0;
+  bool valid = false, balanced = false;
+  la::BalancedPlan bal{};
+  la::SegmentPlan seg{};
+};
+constexpr int kPlanCacheSize = 8;
+std::mutex g_plan_mu;
+PlanCacheEntry g_plan_cache[kPlanCacheSize];
+int g_plan_next = 0;
+
+bool choose_plan(const la_desc* d, int sms, la::BalancedPlan* bal, la::SegmentPlan* seg) {
+  const int32_t chunk = chunk_of(d->chunk);
+  {
+    std::lock_guard<std::mutex> lk(g_plan_mu);
+    for (const PlanCacheEntry& e : g_plan_cache) {
+      if (e.valid && e.B == d->B && e.N == d->N && e.H == d->H && e.sms == sms &&
+          e.chunk == chunk && e.segments == d->segments) {
+        if (e.balanced) *bal = e.bal; else *seg = e.seg;
+        return e.balanced;
+      }
+    }
+  }
+  PlanCacheEntry e;
+  e.balanced = compute_plan(d, sms, &e.bal, &e.seg);
+  e.B = d->B;
+  e.N = d->N;
+  e.H = d->H;
+  e.sms = sms;
+  e.chunk = chunk;
+  e.segments = d->segments;
+  e.valid = true;
+  if (e.balanced) *bal = e.bal; else *seg = e.seg;
+  std::lock_guard<std::mutex> lk(g_plan_mu);
+  g_plan_cache[g_plan_next] = e;
+  g_plan_next = (g_plan_next + 1) % kPlanCacheSize;
+  return e.balanced;
+}
+
+// Workspace bytes of la_prefill's tensor path for its plan.
+size_t prefill_workspace_need(const la_desc* d, int sms) {
+  la::BalancedPlan bal{};
+  la::SegmentPlan seg{};
+  if (choose_plan(d, sms, &bal, &seg)) return la::balanced_workspace_bytes(bal);
+  return la::workspace_layout(d->B, d->H, seg).total;
 }
 
 // Failure injection for tests, read on every call: LA_DEBUG_WITHHOLD_SEGMENT=k keeps segment k of
@@ -80,7 +128,7 @@ la_status check_desc(const la_desc* d, int64_t* numel) {
   if (d->B < 1 || d->N < 1 || d->H < 1 || (d->d != 64 && d->d != 128)) return LA_ERR_SHAPE;
   if (d->path != LA_PATH_AUTO && d->path != LA_PATH_TENSOR && d->path != LA_PATH_RECURRENT)
     return LA_ERR_UNSUPPORTED;
-  if (d->segments < 0) return LA_ERR_SHAPE;
+  if (d->segments < LA_SEGMENTS_BALANCED) return LA_ERR_SHAPE;
   int64_t t = 0, bytes = 0;
   if (!mul_ok(d->B, d->N, &t) || !mul_ok(t, d->H, &t) || !mul_ok(t, d->d, &t))
     return LA_ERR_OVERFLOW;
@@ -195,11 +243,7 @@ la_status la_prefill(const la_desc* desc, const void* q, const void* k, const vo
   if (sms <= 0) return LA_ERR_CUDA;
   la::BalancedPlan bplan{};
   la::SegmentPlan splan{};
-  bool balanced = false;
-  if (desc->segments == 0)
-    balanced = la::prefer_balanced(desc->B, desc->N, desc->H, sms, a.chunk, &bplan, &splan);
-  else
-    splan = la::plan_segments(desc->B, desc->N, desc->H, desc->segments, sms, a.chunk);
+  const bool balanced = choose_plan(desc, sms, &bplan, &splan);
   const size_t need = balanced ? la::balanced_workspace_bytes(bplan)
                                : la::workspace_layout(desc->B, desc->H, splan).total;
   void* ws = workspace;

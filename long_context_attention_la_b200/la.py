@@ -37,6 +37,7 @@ LA_F32 = 1
 LA_PATH_AUTO = 0
 LA_PATH_TENSOR = 1
 LA_PATH_RECURRENT = 2
+LA_SEGMENTS_BALANCED = -1  # la_desc.segments: the balanced range plan
 
 
 class la_desc(ctypes.Structure):  # noqa: N801 - mirrors the C type name

@@ -70,7 +70,7 @@ def _desc(**kw):
     (dict(chunk=96), la.LA_ERR_UNSUPPORTED), (dict(chunk=512), la.LA_ERR_UNSUPPORTED),
     (dict(chunk=64, path=la.LA_PATH_RECURRENT), la.LA_ERR_UNSUPPORTED),
     (dict(dtype=la.LA_F32, path=la.LA_PATH_TENSOR), la.LA_ERR_UNSUPPORTED),
-    (dict(B=1 << 40, N=1 << 40), la.LA_ERR_OVERFLOW), (dict(segments=-1), la.LA_ERR_SHAPE),
+    (dict(B=1 << 40, N=1 << 40), la.LA_ERR_OVERFLOW), (dict(segments=-2), la.LA_ERR_SHAPE),
 ])
 def test_prefill_rejects_bad_descriptors(lib, kw, status):
     d = _desc(**kw)
@@ -122,6 +122,30 @@ def test_tensor_path_workspace_covers_the_scan(lib):
     # single segment per sequence: only the header
     w1 = la.la_prefill_workspace_bytes(_desc(B=1, H=1, N=64 * 128, segments=1))
     assert w1 == 256 or w1 == 512
+
+
+def test_plan_cache_returns_the_same_plan(lib):
+    # the library keeps the last few plans: sizes asked for again, after the cache has turned
+    # over, must come out the same as the first time
+    shapes = [dict(B=b, H=h, N=n, segments=sg) for b, h, n in
+              [(1, 64, 1 << 18), (2, 64, 1 << 15), (1, 64, 4096), (1, 2, 1 << 16), (4, 16, 1 << 16),
+               (1, 1, 64 * 128), (3, 5, 3000)] for sg in (0, la.LA_SEGMENTS_BALANCED)]
+    first = [la.la_prefill_workspace_bytes(_desc(**kw)) for kw in shapes]
+    again = [la.la_prefill_workspace_bytes(_desc(**kw)) for kw in reversed(shapes)][::-1]
+    assert first == again
+    assert all(w >= 256 for w in first)
+
+
+def test_balanced_plan_workspace(lib):
+    # LA_SEGMENTS_BALANCED: one range per SM (at most one per tile), each with a flag and one
+    # d x d fp32 state: 64 tiles -> 64 ranges on any GPU of 64 SMs or more
+    w = la.la_prefill_workspace_bytes(_desc(B=1, H=1, N=64 * 128,
+                                            segments=la.LA_SEGMENTS_BALANCED))
+    assert w == 256 + 256 + 64 * 128 * 128 * 4
+    # many tiles: at most one range per SM (256 at most), within the no-allocation scratch
+    wl = la.la_prefill_workspace_bytes(_desc(B=4, H=64, N=1 << 18,
+                                             segments=la.LA_SEGMENTS_BALANCED))
+    assert 256 + 148 * 128 * 128 * 4 <= wl <= la.LA_NOALLOC_SCRATCH_BYTES
 
 
 # ---------------------------------------------------------------------------------------------

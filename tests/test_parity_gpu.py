@@ -219,15 +219,17 @@ def test_tensor_prefill_256k_windows_full():
     acc_s.check()
 
 
+@pytest.mark.parametrize("segments", [0, la.LA_SEGMENTS_BALANCED])
 @pytest.mark.parametrize("chunk", [64, 128, 256])
 @pytest.mark.parametrize("slope", [0.0, 1e-6])
-def test_scan_long_no_forgetting(slope, chunk):
+def test_scan_long_no_forgetting(slope, chunk, segments):
     """With lambda = 1 (or within 1e-6 of it) nothing is forgotten, so a segment scan that lost
-    cross-segment state would fail here even though decaying heads would hide it."""
+    cross-segment state would fail here even though decaying heads would hide it.  The balanced
+    plan passes each sequence's state along a chain of about 74 ranges."""
     B, N, H = 1, 65536, 2
     q, k, v = draw(B, N, H, 128, 7)
     sl = torch.full((H,), slope, dtype=torch.float32, device=DEV)
-    out, st = la.prefill(q, k, v, sl, chunk=chunk)
+    out, st = la.prefill(q, k, v, sl, chunk=chunk, segments=segments)
     torch.cuda.synchronize()
     t_sel = list(range(0, N, 97)) + [N - 1]
     t_sel = sorted(set(t_sel))
@@ -243,7 +245,9 @@ def test_segment_count_invariance(chunk):
     sl = synth.slopes(H, DEV)
     o_ref, s_ref = oracle_on(q, k, v, sl)
     outs = []
-    for seg in [1, 2, 3, 7, 64]:
+    # LA_SEGMENTS_BALANCED: one range of about 1.7 tiles per SM, so nearly every range is cut
+    # inside a sequence and hands its state to the next through the look-back ring
+    for seg in [1, 2, 3, 7, 64, la.LA_SEGMENTS_BALANCED]:
         out, st = la.prefill(q, k, v, sl, chunk=chunk, segments=seg, path=la.LA_PATH_TENSOR)
         torch.cuda.synchronize()
         check_close(gpu_heads(out, None), o_ref, torch.bfloat16, f"o seg={seg}")
@@ -253,12 +257,14 @@ def test_segment_count_invariance(chunk):
         check_close(o.cpu().numpy(), outs[0].cpu().numpy(), torch.bfloat16, "segment agreement")
 
 
+@pytest.mark.parametrize("segments", [0, la.LA_SEGMENTS_BALANCED])
 @pytest.mark.parametrize("chunk", [64, 128, 256])
-def test_chunked_matches_recurrent(chunk):
-    """Chunk lengths 64, 128, 256 (tensor cores) and chunk length 1 (token recurrence) agree."""
+def test_chunked_matches_recurrent(chunk, segments):
+    """Chunk lengths 64, 128, 256 (tensor cores) and chunk length 1 (token recurrence) agree, on
+    sequences with a ragged last tile (also under the balanced plan)."""
     q, k, v = draw(1, 3000, 4, 128, 9)
     sl = synth.slopes(4, DEV)
-    o1, s1 = la.prefill(q, k, v, sl, chunk=chunk, path=la.LA_PATH_TENSOR)
+    o1, s1 = la.prefill(q, k, v, sl, chunk=chunk, segments=segments, path=la.LA_PATH_TENSOR)
     o2, s2 = la.prefill(q, k, v, sl, path=la.LA_PATH_RECURRENT)
     torch.cuda.synchronize()
     check_close(o1.float().cpu().numpy(), o2.float().cpu().numpy(), torch.bfloat16, "o")
