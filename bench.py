@@ -494,22 +494,42 @@ def run_ours(args):
         hextra = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in extra_in]
         for hx, x in zip(hextra, extra_in):
             hx.copy_(x.cpu())
-        n_e2e = max(1, min(K, 3))
+        n_e2e = max(1, min(K, 10))
+        # The inputs copied every step are double-buffered on the device, so that the copy of
+        # step i + 1's inputs (on a copy stream) overlaps step i's kernels and the read-back of
+        # its result (on the compute stream): the link carries both directions at once.  Inputs
+        # whose address a call captured at set-up (the gate, initial states, cu_seqlens) keep
+        # one buffer, and their copy waits for the previous step's kernels.
+        copy_stream = torch.cuda.Stream(dev)
+        per_step = [(q, hq), (k, hk), (v, hv)]
+        if not args.no_decode:
+            per_step += [(dq, hdq), (dk, hdk), (dv, hdv)]
+        sets = [[x for x, _ in per_step], [torch.empty_like(x) for x, _ in per_step]]
+        landed = [torch.cuda.Event() for _ in range(n_e2e)]
+        done = [torch.cuda.Event() for _ in range(n_e2e)]
         barrier(world)
         torch.cuda.synchronize(dev)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(n_e2e):
-            q.copy_(hq, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
+        copy_stream.wait_event(e0)
+        for i in range(n_e2e):
+            bset = sets[i % 2]
+            with torch.cuda.stream(copy_stream):
+                if i >= 2:
+                    copy_stream.wait_event(done[i - 2])  # step i - 2 has read this buffer set
+                for x, (_, hx) in zip(bset, per_step):
+                    x.copy_(hx, non_blocking=True)
+                if hextra:
+                    if i >= 1:
+                        copy_stream.wait_event(done[i - 1])
+                    for x, hx in zip(extra_in, hextra):
+                        x.copy_(hx, non_blocking=True)
+                landed[i].record(copy_stream)
+            stream.wait_event(landed[i])
+            q, k, v = bset[0], bset[1], bset[2]
             if not args.no_decode:
-                dq.copy_(hdq, non_blocking=True)
-                dk.copy_(hdk, non_blocking=True)
-                dv.copy_(hdv, non_blocking=True)
-            for x, hx in zip(extra_in, hextra):
-                x.copy_(hx, non_blocking=True)
+                dq, dk, dv = bset[3], bset[4], bset[5]
             if qk is not None:
                 qk_call()
             if args.cp:
@@ -518,12 +538,16 @@ def run_ours(args):
             if sep is not None:
                 sep_call()
             decode_call()
+            done[i].record(stream)
             hout.copy_(out, non_blocking=True)
             hst.copy_(st, non_blocking=True)
             if not args.no_decode:
                 hdout.copy_(dout, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
+        q, k, v = sets[0][0], sets[0][1], sets[0][2]
+        if not args.no_decode:
+            dq, dk, dv = sets[0][3], sets[0][4], sets[0][5]
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
         dec_io = 0 if args.no_decode else 1
         bi = 3 * q.numel() * q.element_size() + dec_io * 3 * dq.numel() * dq.element_size() + sum(

@@ -185,6 +185,61 @@ def gated_rmsnorm(o, gate, gamma, eps: float):
     return gam * (o / np.sqrt(ms + float(eps))) * (1.0 / (1.0 + np.exp(-g)))
 
 
+E4M3_MAX = 448.0  # largest finite FP8 E4M3 value: 2^8 x 1.75
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """FP8 E4M3 codes of real values, rounded to nearest with ties to even and saturated to the
+    largest finite value (the 8-bit format of the report's FP8 inference path, "Ling and Ring
+    2.6 Technical Report" §4.3 and Table 7: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa
+    bits; exponent field 0 holds the subnormals m * 2^-9; no infinities; 0x7F / 0xFF are NaN, so
+    the largest finite magnitude is 0x7E = 448).  x: any real array; returns uint8 codes."""
+    x = np.asarray(x, dtype=np.float64)
+    sign = np.signbit(x).astype(np.uint8) << 7
+    a = np.minimum(np.abs(x), E4M3_MAX)  # saturate: nothing rounds past 448
+    frac, ex = np.frexp(a)  # a = frac * 2^ex, frac in [0.5, 1)
+    e = ex.astype(np.int64) - 1  # a = s * 2^e with s in [1, 2)
+    normal = a >= 2.0 ** -6
+    # normal: 3 mantissa bits of s - 1, a carry into the exponent when they round up to 8
+    mant_n = np.rint((2.0 * frac - 1.0) * 8.0).astype(np.int64)
+    e_n = e + (mant_n == 8)
+    mant_n = np.where(mant_n == 8, 0, mant_n)
+    code_n = ((e_n + 7) << 3) | mant_n
+    # subnormal: m * 2^-9; m = 8 is the smallest normal 2^-6, whose code is 8 as well
+    code_s = np.rint(a / 2.0 ** -9).astype(np.int64)
+    code = np.where(normal, code_n, code_s).astype(np.uint8)
+    return code | sign
+
+
+def e4m3_decode(code) -> np.ndarray:
+    """Real values (fp64) of FP8 E4M3 codes (NaN for 0x7F / 0xFF); the inverse of e4m3_encode on
+    the representable values."""
+    c = np.asarray(code, dtype=np.uint8).astype(np.int64)
+    sgn = np.where(c & 0x80, -1.0, 1.0)
+    ef = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(ef == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(ef - 7.0))
+    mag = np.where((ef == 15) & (m == 7), np.nan, mag)
+    return sgn * mag
+
+
+def gated_rmsnorm_fp8(o, gate, gamma, eps: float):
+    """The fused post-kernel operator with its quantize step, in fp64 ("Ling and Ring 2.6
+    Technical Report" §4.3: "group norm + sigmoid gate + quantize" fused before out_proj; the FP8
+    path quantizes the projection inputs blockwise, §4.3 and Table 7).  y is gated_rmsnorm's;
+    each head's d channels of one token are one block with one scale:
+
+        amax = max_j |y_j|,  scale = amax / 448,  code_j = E4M3(y_j * 448 / amax)
+
+    (code 0 and scale 0 for an all-zero block), so code_j * scale reproduces y_j to within half an
+    E4M3 step.  Returns (uint8 codes with o's shape, fp64 scales [..., H])."""
+    y = gated_rmsnorm(o, gate, gamma, eps)
+    amax = np.max(np.abs(y), axis=-1)
+    inv = np.where(amax > 0, E4M3_MAX / np.where(amax > 0, amax, 1.0), 0.0)
+    codes = e4m3_encode(y * inv[..., None])
+    return codes, amax / E4M3_MAX
+
+
 def qk_norm_rope(x, gamma, positions, rotary_dim: int, theta: float, eps: float):
     """The layer's step before the kernel, in fp64 ("Ling and Ring 2.6 Technical Report", §2.1
     Fig. 2: QKV Projection -> QK Norm -> RoPE -> Linear Attention Kernel; §2.1.1: RMSNorm with

@@ -285,6 +285,74 @@ def test_gated_rmsnorm_reads_bf16_bits_exactly():
 
 
 # ---------------------------------------------------------------------------------------------
+# FP8 E4M3 quantize of the fused post-kernel operator
+# ---------------------------------------------------------------------------------------------
+def test_e4m3_hand_codes():
+    # from the format: code = sign << 7 | (exponent + 7) << 3 | mantissa; exponent field 0 holds
+    # m * 2^-9; ties round to the even mantissa; magnitudes above 448 saturate to 0x7E
+    cases = [(1.0, 0x38), (-2.0, 0xC0), (448.0, 0x7E), (0.5, 0x30), (1.75, 0x3E), (2.0 ** -6, 0x08),
+             (2.0 ** -9, 0x01), (7 * 2.0 ** -9, 0x07), (0.0, 0x00), (-0.0, 0x80),
+             (1.0625, 0x38),            # halfway 1 .. 1.125: even mantissa 0
+             (1.1875, 0x3A),            # halfway 1.125 .. 1.25: even mantissa 2
+             (2.0 ** -10, 0x00),        # halfway 0 .. 2^-9: even 0
+             (3 * 2.0 ** -10, 0x02),    # halfway 2^-9 .. 2^-8: even 2
+             (15 * 2.0 ** -10, 0x08),   # halfway 7 * 2^-9 .. 2^-6: carries into the normals
+             (1.96875, 0x40),           # halfway 1.875 .. 2: carries into the next exponent
+             (464.0, 0x7E), (1.0e6, 0x7E), (-600.0, 0xFE)]
+    x = np.array([c[0] for c in cases])
+    assert oracle.e4m3_encode(x).tolist() == [c[1] for c in cases]
+
+
+def test_e4m3_round_trip_and_order():
+    codes = np.arange(256, dtype=np.uint8)
+    vals = oracle.e4m3_decode(codes)
+    finite = ~np.isnan(vals)
+    assert finite.sum() == 254 and np.isnan(vals[[0x7F, 0xFF]]).all()
+    assert np.array_equal(oracle.e4m3_encode(vals[finite]), codes[finite])
+    pos = vals[:0x7F]
+    assert np.all(np.diff(pos) > 0) and pos[-1] == 448.0 and pos[1] == 2.0 ** -9
+
+
+def test_e4m3_matches_torch_conversion():
+    # torch's float8_e4m3fn conversion (a library routine, CPU) rounds to nearest even; it does not
+    # saturate past 464, so the sweep stays within +-464
+    reps = oracle.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    mids = 0.5 * (reps[1:] + reps[:-1])
+    rng = np.random.default_rng(9)
+    x = np.concatenate([reps, mids, -mids, rng.uniform(-464, 464, 20000),
+                        rng.standard_normal(20000) * 2.0 ** -7, [464.0, -464.0]]).astype(np.float32)
+    ours = oracle.e4m3_encode(x.astype(np.float64))
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+
+
+def test_gated_rmsnorm_fp8_blocks():
+    rng = np.random.default_rng(6)
+    o = rng.standard_normal((5, 3, 16)) * rng.uniform(0.01, 100, (5, 3, 1))
+    g = rng.standard_normal((5, 3, 16)).astype(np.float32)
+    gamma = rng.standard_normal((3, 16)).astype(np.float32)
+    o[2, 1] = 0.0  # an all-zero block (eps > 0 keeps y finite: y = 0)
+    codes, scale = oracle.gated_rmsnorm_fp8(o, g, gamma, 1e-6)
+    y = oracle.gated_rmsnorm(o, g, gamma, 1e-6)
+    assert codes.shape == o.shape and codes.dtype == np.uint8 and scale.shape == (5, 3)
+    amax = np.max(np.abs(y), axis=-1)
+    assert np.allclose(scale, amax / 448.0, rtol=1e-15, atol=0)
+    assert scale[2, 1] == 0.0 and not (codes[2, 1] & 0x7F).any()  # signed zeros
+    # the block's largest magnitude maps to the largest code, with y's sign
+    j = np.argmax(np.abs(y), axis=-1)
+    top = np.take_along_axis(codes, j[..., None], axis=-1)[..., 0]
+    sgn = np.take_along_axis(y, j[..., None], axis=-1)[..., 0] < 0
+    live = amax > 0
+    assert np.array_equal(top[live] & 0x7F, np.full(live.sum(), 0x7E))
+    assert np.array_equal((top[live] >> 7).astype(bool), sgn[live])
+    # dequantized values are within half an E4M3 step of y (3 mantissa bits: relative 2^-4 for
+    # normals, absolute 2^-10 * scale for the subnormals)
+    deq = oracle.e4m3_decode(codes) * scale[..., None]
+    bound = np.maximum(np.abs(y) * 2.0 ** -4, 2.0 ** -10 * scale[..., None]) * (1 + 1e-12)
+    assert np.all(np.abs(deq - y) <= bound)
+
+
+# ---------------------------------------------------------------------------------------------
 # qk_norm_rope: QK RMSNorm + partial rotary embedding before the kernel
 # ---------------------------------------------------------------------------------------------
 def test_qk_norm_rope_hand_case():

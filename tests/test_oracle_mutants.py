@@ -117,3 +117,54 @@ def test_fold_mutant_is_caught(name):
     except (ValueError, IndexError):
         ok = False  # a shape error is a failed pin too
     assert not ok, f"the pins did not catch the planted mistake {name}"
+
+
+# The FP8 E4M3 encoder (oracle.e4m3_encode): each mutant must fail the format's hand codes or the
+# comparison with torch's conversion in test_oracle.py.
+E4M3_MUTANTS = {
+    "e4m3_bias_8": ("((e_n + 7) << 3)", "((e_n + 8) << 3)"),
+    "e4m3_round_half_up": ("np.rint((2.0 * frac - 1.0) * 8.0)", "np.floor((2.0 * frac - 1.0) * 8.0 + 0.5)"),
+    "e4m3_truncate": ("np.rint((2.0 * frac - 1.0) * 8.0)", "np.floor((2.0 * frac - 1.0) * 8.0)"),
+    "e4m3_no_carry": ("e_n = e + (mant_n == 8)", "e_n = e"),
+    "e4m3_subnormal_step": ("np.rint(a / 2.0 ** -9)", "np.rint(a / 2.0 ** -10)"),
+    "e4m3_no_saturation": ("np.minimum(np.abs(x), E4M3_MAX)", "np.abs(x)"),
+    "e4m3_sign_lost": ("return code | sign", "return code"),
+}
+
+
+def _e4m3_pins_pass(encode) -> bool:
+    import tests.test_oracle as t
+    saved = oracle.e4m3_encode
+    oracle.e4m3_encode = encode
+    try:
+        for pin in (t.test_e4m3_hand_codes, t.test_e4m3_matches_torch_conversion):
+            try:
+                pin()
+            except (AssertionError, ValueError, OverflowError):
+                return False
+        return True
+    finally:
+        oracle.e4m3_encode = saved
+
+
+def _encode_from_source(src: str):
+    ns = {"np": np, "E4M3_MAX": oracle.E4M3_MAX}
+    with np.errstate(all="ignore"):
+        exec(compile(src, "<e4m3 mutant>", "exec"), ns)  # noqa: S102 - test-only source mutation
+    return ns["e4m3_encode"]
+
+
+def test_unmutated_e4m3_copy_passes():
+    import inspect
+    assert _e4m3_pins_pass(_encode_from_source(inspect.getsource(oracle.e4m3_encode)))
+
+
+@pytest.mark.parametrize("name", sorted(E4M3_MUTANTS))
+def test_e4m3_mutant_is_caught(name):
+    import inspect
+    old, new = E4M3_MUTANTS[name]
+    text = inspect.getsource(oracle.e4m3_encode)
+    assert text.count(old) == 1, f"mutation site for {name} not found"
+    with np.errstate(all="ignore"):
+        ok = _e4m3_pins_pass(_encode_from_source(text.replace(old, new)))
+    assert not ok, f"the pins did not catch the planted mistake {name}"
