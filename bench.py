@@ -273,7 +273,16 @@ def run_ours(args):
     q, k, v = synth.draw_qkv(B, N, H, d, dist=w.dist, seed=w.seed + 1000 * rank, dtype=w.dtype,
                              device=dev)
     sl = synth.slopes(H, dev)
+    if args.fp8 and not args.gate_separate:
+        raise SystemExit("--fp8 is an output format of --gate-separate (the stand-alone "
+                         "norm + gate + quantize operator)")
+    # with --fp8 the norm + gate stores FP8 E4M3 codes (one byte per value) and one fp32 scale
+    # per (head, token) block of d values
+    fp8_scales = (torch.empty((H, B * N), dtype=torch.float32, device=dev) if args.fp8
+                  else None)
     out = torch.empty_like(q)
+    y8 = torch.empty(q.shape, dtype=torch.uint8, device=dev) if args.fp8 and \
+        args.gate_separate else None
     extra_in = []  # further inputs copied from the host in the e2e leg
     epi = None
     sep = None
@@ -283,7 +292,8 @@ def run_ours(args):
         gate = (torch.randn((B * N, H, d), generator=gg, device=dev)).to(w.dtype)
         gamma = (1.0 + 0.1 * torch.randn((H, d), generator=gg, device=dev)).float()
         extra_in += [gate]
-        sep = la.la_gate_norm(gate.data_ptr(), gamma.data_ptr(), 1e-6)
+        sep = la.la_gate_norm(gate.data_ptr(), gamma.data_ptr(), 1e-6,
+                              fp8_scales.data_ptr() if args.fp8 else None)
     if args.gate:
         # fused grouped RMSNorm + sigmoid gate on the prefill output: a gate pre-activation the
         # size of q and a norm weight per head and channel (synthetic, seeded)
@@ -391,9 +401,10 @@ def run_ours(args):
             raise la.LaError(rc, "la_prefill")
 
     def sep_call():
-        # the post-kernel operator on its own, in place on the prefill's output
-        rc = la.la_gate_norm_apply(B * N, H, d, la.LA_BF16, out.data_ptr(), sep, out.data_ptr(),
-                                   sp)
+        # the post-kernel operator on its own, in place on the prefill's output (FP8: into its
+        # own byte buffer)
+        rc = la.la_gate_norm_apply(B * N, H, d, la.LA_BF16, out.data_ptr(), sep,
+                                   (y8 if y8 is not None else out).data_ptr(), sp)
         if rc != la.LA_OK:
             raise la.LaError(rc, "la_gate_norm_apply")
 
@@ -482,7 +493,10 @@ def run_ours(args):
         hq.copy_(q.cpu())
         hk.copy_(k.cpu())
         hv.copy_(v.cpu())
-        hout = torch.empty_like(hq).pin_memory()
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        hy8 = torch.empty(y8.shape, dtype=y8.dtype, pin_memory=True) if y8 is not None else None
+        hsc = (torch.empty(fp8_scales.shape, dtype=fp8_scales.dtype, pin_memory=True)
+               if fp8_scales is not None else None)
         hst = torch.empty(st.shape, dtype=st.dtype, pin_memory=True)
         hdq = torch.empty(dq.shape, dtype=dq.dtype, pin_memory=True)
         hdk = torch.empty_like(hdq).pin_memory()
@@ -540,6 +554,10 @@ def run_ours(args):
             decode_call()
             done[i].record(stream)
             hout.copy_(out, non_blocking=True)
+            if hy8 is not None:
+                hy8.copy_(y8, non_blocking=True)
+            if hsc is not None:
+                hsc.copy_(fp8_scales, non_blocking=True)
             hst.copy_(st, non_blocking=True)
             if not args.no_decode:
                 hdout.copy_(dout, non_blocking=True)
@@ -553,7 +571,9 @@ def run_ours(args):
         bi = 3 * q.numel() * q.element_size() + dec_io * 3 * dq.numel() * dq.element_size() + sum(
             x.numel() * x.element_size() for x in extra_in)
         bo = out.numel() * out.element_size() + st.numel() * 4 + \
-            dec_io * dout.numel() * dout.element_size()
+            dec_io * dout.numel() * dout.element_size() + \
+            (y8.numel() if y8 is not None else 0) + \
+            (fp8_scales.numel() * 4 if fp8_scales is not None else 0)
         e2e = {"value": world * B * N / (e2e_ms * 1e-3), "unit": "tok/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms,
                "steps": n_e2e}
@@ -568,9 +588,17 @@ def run_ours(args):
         tok_s = world * tokens / ((step_ms_max if args.cp else pre_ms_max) * 1e-3)
         # algorithmic bytes of one prefill launch: read q, k, v and write o (bf16), write the
         # final states (and read the initial states of the packed workload)
-        # (the separate norm + gate pass reads o and the gate and writes y: 3 more rows)
-        pre_bytes = (4 + (1 if args.gate else 0) + (3 if args.gate_separate else 0)) * \
-            B * N * H * d * 2 + \
+        # (the fused norm + gate also reads the gate; the separate pass reads o and the gate and
+        # writes y; an FP8 y is d bytes plus a 4-byte scale per token-head instead of 2d bytes)
+        row = 2 * d
+        y_row = d + 4 if args.fp8 else row
+        if args.gate:
+            per_th = 3 * row + row + row
+        elif args.gate_separate:
+            per_th = 4 * row + 2 * row + y_row
+        else:
+            per_th = 4 * row
+        pre_bytes = per_th * B * N * H + \
             n_states * H * d * d * 4 * (1 if vw is None and not args.cp else 2)
         achieved = pre_bytes / (pre_ms_max * 1e-3) / 1e9
         canon = 4.0 * d * d * B * N * H  # recurrent-form flops
@@ -599,6 +627,8 @@ def run_ours(args):
                                                   if args.gate else "") +
                                    (", then the grouped RMSNorm + sigmoid gate pass"
                                     if args.gate_separate else "") +
+                                   (" with FP8 E4M3 output (one fp32 scale per token-head)"
+                                    if args.fp8 else "") +
                                    (f", context parallel over {world} rank(s): {N} tokens per "
                                     f"rank, state pass + all_gather + fold + prefill from the "
                                     f"folded state" if args.cp else "") +
@@ -725,6 +755,9 @@ def main():
                     help="run the grouped RMSNorm + sigmoid gate as its own pass after the prefill")
     ap.add_argument("--gate", action="store_true",
                     help="fuse the grouped RMSNorm + sigmoid gate into the prefill's output")
+    ap.add_argument("--fp8", action="store_true",
+                    help="with --gate-separate: store y as FP8 E4M3 with blockwise scales (the "
+                         "quantize step before out_proj)")
     ap.add_argument("--cp", action="store_true",
                     help="context parallel: split each sequence over the ranks (state pass, "
                          "all_gather of the part states, fold, prefill from the folded state)")

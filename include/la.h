@@ -151,6 +151,17 @@ typedef struct {
   const void* gate;   /* like out, device: the gate pre-activation g = x W_gate, read only */
   const float* gamma; /* fp32 [H, d] device: the norm's weight, read only */
   float eps;          /* epsilon under the root, >= 0 (the report's RMSNorm uses 1e-6) */
+  /* NULL: y is stored in out's dtype.  Otherwise the quantize step the report fuses after the
+   * gate (§4.3 "group norm + sigmoid gate + quantize", ahead of the FP8 out_proj): y goes out as
+   * FP8 E4M3 codes, one byte per value (uint8 [T, H, d]), and fp8_scales (fp32, device, 16-byte
+   * aligned) receives one scale per block of a token's d values of one head, stored head-major
+   * [H, T].  With y' = y rounded to the I/O dtype (what the unfused chain stores before its
+   * quantize step):  scale = max_j |y'_j| / 448,  code_j = E4M3(y'_j * (448 / max_j |y'_j|))
+   * (the product in fp32, rounded to nearest even, saturating at 448; an all-zero block gets
+   * scale 0 and signed-zero codes), so that y_j ~= value(code_j) * scale.  Produced by
+   * la_gate_norm_apply, the report's stand-alone post-attention operator; la_prefill_varlen and
+   * la_decode_multi return LA_ERR_UNSUPPORTED for it. */
+  float* fp8_scales;
 } la_gate_norm;
 
 /*
@@ -163,8 +174,10 @@ typedef struct {
  *
  *   T, H, d     tokens (>= 0), heads, head dim (64 or 128); dtype: la_dtype of o, gate and y
  *   o           [T, H, d] device, read only
- *   gn          gate ([T, H, d] of dtype), gamma (fp32 [H, d]) and eps (>= 0); host pointer
- *   y           [T, H, d] device, written; may be o itself (in place), no other overlap
+ *   gn          gate ([T, H, d] of dtype), gamma (fp32 [H, d]) and eps (>= 0), and optionally
+ *               fp8_scales (then y is FP8 E4M3 codes, uint8 [T, H, d]); host pointer
+ *   y           [T, H, d] device, written; may be o itself (in place, not with fp8_scales), no
+ *               other overlap
  *   stream      cudaStream_t as void*
  */
 la_status la_gate_norm_apply(int64_t T, int64_t H, int64_t d, int32_t dtype, const void* o,

@@ -295,6 +295,8 @@ la_status la_prefill_varlen(const la_varlen_desc* desc, const void* q, const voi
   const bool tensor = use_tensor_path(desc->path, desc->dtype, desc->d);
   if (epilogue != nullptr) {
     if (!tensor) return LA_ERR_UNSUPPORTED;  // the fused norm + gate lives in the chunked kernel
+    // the FP8 output is la_gate_norm_apply's (the report's separate post-attention operator)
+    if (epilogue->fp8_scales != nullptr) return LA_ERR_UNSUPPORTED;
     if (!epilogue->gate || !epilogue->gamma) return LA_ERR_NULL;
     if (!aligned16(epilogue->gate) || !aligned16(epilogue->gamma)) return LA_ERR_ALIGN;
     if (!(epilogue->eps >= 0.f) || epilogue->eps > 3.0e38f) return LA_ERR_SHAPE;  // NaN, inf
@@ -410,6 +412,7 @@ la_status la_decode_multi(int64_t B, int64_t H, int64_t d, int64_t n_tok, int32_
   la::DecodeArgs a{B, H, d, dtype, q, k, v, slopes, state_inout, out};
   a.n_tok = n_tok;
   if (epilogue != nullptr) {
+    if (epilogue->fp8_scales != nullptr) return LA_ERR_UNSUPPORTED;  // no FP8 output here
     if (!epilogue->gate || !epilogue->gamma) return LA_ERR_NULL;
     if (!aligned16(epilogue->gate) || !aligned16(epilogue->gamma)) return LA_ERR_ALIGN;
     if (!(epilogue->eps >= 0.f) || epilogue->eps > 3.0e38f) return LA_ERR_SHAPE;
@@ -435,9 +438,22 @@ la_status la_gate_norm_apply(int64_t T, int64_t H, int64_t d, int32_t dtype, con
   if (!aligned16(o) || !aligned16(gn->gate) || !aligned16(gn->gamma) || !aligned16(y))
     return LA_ERR_ALIGN;
   const size_t bytes = static_cast<size_t>(n) * (dtype == LA_BF16 ? 2 : 4);
-  if (bytes > 0 && ((y != o && overlaps(y, bytes, o, bytes)) || overlaps(y, bytes, gn->gate, bytes)))
+  const bool fp8 = gn->fp8_scales != nullptr;
+  if (fp8) {
+    // one byte per value plus [H, T] fp32 scales; y cannot be written over o in place
+    const size_t y_bytes = static_cast<size_t>(n);
+    const size_t s_bytes = static_cast<size_t>(T * H) * 4;
+    if (!aligned16(gn->fp8_scales)) return LA_ERR_ALIGN;
+    if (bytes > 0 && (overlaps(y, y_bytes, o, bytes) || overlaps(y, y_bytes, gn->gate, bytes) ||
+                      overlaps(gn->fp8_scales, s_bytes, y, y_bytes) ||
+                      overlaps(gn->fp8_scales, s_bytes, o, bytes) ||
+                      overlaps(gn->fp8_scales, s_bytes, gn->gate, bytes)))
+      return LA_ERR_ALIAS;
+  } else if (bytes > 0 &&
+             ((y != o && overlaps(y, bytes, o, bytes)) || overlaps(y, bytes, gn->gate, bytes))) {
     return LA_ERR_ALIAS;
-  la::GateNormArgs a{T, H, d, dtype, o, gn->gate, gn->gamma, gn->eps, y};
+  }
+  la::GateNormArgs a{T, H, d, dtype, o, gn->gate, gn->gamma, gn->eps, y, gn->fp8_scales};
   return la::launch_gate_norm(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? LA_OK
                                                                                      : LA_ERR_CUDA;
 }

@@ -8,6 +8,7 @@
 // threads of 16 bytes and its mean square is a shuffle reduction over them; o and g reach those
 // threads through a shared-memory ring filled two items ahead by per-thread cp.async copies.
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include <cstdint>
 
@@ -39,6 +40,10 @@ struct Io<__nv_bfloat16> {  // 8 values = one 16-byte piece
     const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&p);
   }
+  // the value as stored in this dtype (round to nearest even)
+  static __device__ __forceinline__ float round(float x) {
+    return __bfloat162float(__float2bfloat16_rn(x));
+  }
   static __device__ __forceinline__ void store(__nv_bfloat16* dst, const float (&y)[8]) {
     __stcs(reinterpret_cast<uint4*>(dst),
            make_uint4(pack2(y[0], y[1]), pack2(y[2], y[3]), pack2(y[4], y[5]), pack2(y[6], y[7])));
@@ -47,6 +52,7 @@ struct Io<__nv_bfloat16> {  // 8 values = one 16-byte piece
 
 template <>
 struct Io<float> {  // 8 values = two 16-byte pieces
+  static __device__ __forceinline__ float round(float x) { return x; }
   static __device__ __forceinline__ void store(float* dst, const float (&y)[8]) {
     __stcs(reinterpret_cast<float4*>(dst), make_float4(y[0], y[1], y[2], y[3]));
     __stcs(reinterpret_cast<float4*>(dst) + 1, make_float4(y[4], y[5], y[6], y[7]));
@@ -173,6 +179,44 @@ __global__ void __launch_bounds__(kGnThreads, 2) gate_norm_kernel(const GateNorm
       for (int e = 0; e < 8; ++e) ss = fmaf(xo[e], xo[e], ss);
 #pragma unroll
       for (int m = TPR / 2; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+      if (a.scales != nullptr) {
+        // FP8 E4M3 output: y is rounded to the I/O dtype first (the value the unfused chain would
+        // store before its quantize step); the row's (the block's) largest |y| sets its scale,
+        // amax / 448, and each value is stored as E4M3(y * 448 / amax), rounded to nearest even
+        // and saturated.  Every lane takes part in the max reduction; rows past H compute zeros.
+        const bool row_ok = h < a.H;
+        float xg[8];
+        Piece<T>::unpack(wg, xg);
+        const float rinv = rsqrtf(fmaf(ss, 1.f / D, a.eps));
+        float gm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (row_ok) {
+          const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gamma + h * D + lt * 8));
+          const float4 g1 = __ldg(reinterpret_cast<const float4*>(a.gamma + h * D + lt * 8) + 1);
+          gm[0] = g0.x; gm[1] = g0.y; gm[2] = g0.z; gm[3] = g0.w;
+          gm[4] = g1.x; gm[5] = g1.y; gm[6] = g1.z; gm[7] = g1.w;
+        }
+        float out[8];
+        float am = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          out[e] = Io<T>::round(gm[e] * (xo[e] * rinv) * Sigmoid<T>::f(xg[e]));
+          am = fmaxf(am, fabsf(out[e]));
+        }
+#pragma unroll
+        for (int m = TPR / 2; m > 0; m >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, m));
+        if (row_ok) {
+          const float inv = am > 0.f ? 448.f / am : 0.f;
+          uint32_t w[4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2)
+            w[e2] = __nv_cvt_float2_to_fp8x2(make_float2(out[2 * e2] * inv, out[2 * e2 + 1] * inv),
+                                             __NV_SATFINITE, __NV_E4M3);
+          uint8_t* y8 = static_cast<uint8_t*>(a.y) + (t * a.H + h) * D + lt * 8;
+          __stcs(reinterpret_cast<uint2*>(y8), make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16)));
+          if (lt == 0) a.scales[h * a.T + t] = am / 448.f;
+        }
+        continue;
+      }
       if (h < a.H) {  // uniform across a row's threads
         float xg[8];
         Piece<T>::unpack(wg, xg);

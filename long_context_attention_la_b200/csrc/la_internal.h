@@ -93,7 +93,8 @@ struct GateNormArgs {
   const void* gate;
   const float* gamma;  // [H, d]
   float eps;
-  void* y;
+  void* y;             // [T, H, d] of dtype, or uint8 E4M3 codes when scales is set
+  float* scales;       // FP8 output: fp32 [H, T] block scales (nullptr: y in dtype)
 };
 cudaError_t launch_gate_norm(const GateNormArgs& a, cudaStream_t stream);
 

@@ -53,7 +53,8 @@ class la_varlen_desc(ctypes.Structure):  # noqa: N801 - mirrors the C type name
 
 
 class la_gate_norm(ctypes.Structure):  # noqa: N801 - mirrors the C type name
-    _fields_ = [("gate", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("eps", ctypes.c_float)]
+    _fields_ = [("gate", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("eps", ctypes.c_float),
+                ("fp8_scales", ctypes.c_void_p)]
 
 
 class la_qk_norm_rope_desc(ctypes.Structure):  # noqa: N801 - mirrors the C type name
@@ -307,7 +308,8 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: to
     a CUDA int64 tensor of n_seqs + 1 entries (a host list or array is copied to the device
     first).  state_in: optional fp32 [n_seqs, H, d, d] initial states (state_out may be the same
     tensor).  gate [T, H, d] bf16 and gamma fp32 [H, d] switch on the fused grouped RMSNorm +
-    sigmoid gate, so out holds gamma * o / rms(o) * sigmoid(gate) per head.
+    sigmoid gate, so out holds gamma * o / rms(o) * sigmoid(gate) per head (FP8 output is
+    gate_norm's, the stand-alone operator).
     Returns out [T, H, d] and the final fp32 states [n_seqs, H, d, d].  An invalid
     cu_seqlens is reported by the device: check la_workspace_status(workspace) when it is not
     known to be valid."""
@@ -450,24 +452,29 @@ def decode_multi(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torc
 
 
 def gate_norm(o: torch.Tensor, gate: torch.Tensor, gamma: torch.Tensor, *, eps: float = 1e-6,
-              out: torch.Tensor | None = None,
-              stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+              fp8: bool = False, out: torch.Tensor | None = None,
+              stream: torch.cuda.Stream | None = None):
     """y = gate_norm(o, gate, gamma): o, gate [T, H, d] (bf16 or fp32, CUDA, contiguous), gamma
-    fp32 [H, d]; y = gamma * o / rms(o) * sigmoid(gate) per token and head (out may be o)."""
+    fp32 [H, d]; y = gamma * o / rms(o) * sigmoid(gate) per token and head (out may be o).
+    fp8=True returns (codes, scales): y as FP8 E4M3 codes (uint8 [T, H, d]) and one fp32 scale
+    per (head, token) block, [H, T]."""
     if o.dim() != 3 or gate.shape != o.shape or gate.dtype != o.dtype or o.dtype not in _DT:
         raise ValueError("o and gate must share one [T, H, d] shape and dtype")
     T, H, d = o.shape
     if gamma.dtype != torch.float32 or tuple(gamma.shape) != (H, d):
         raise ValueError("gamma must be float32 [H, d]")
     if out is None:
-        out = torch.empty_like(o)
+        out = torch.empty(o.shape, dtype=torch.uint8, device=o.device) if fp8 else \
+            torch.empty_like(o)
+    scales = torch.empty((H, T), dtype=torch.float32, device=o.device) if fp8 else None
     s = stream if stream is not None else torch.cuda.current_stream(o.device)
-    gn = la_gate_norm(_cuda_ptr(gate, "gate"), _cuda_ptr(gamma, "gamma"), float(eps))
+    gn = la_gate_norm(_cuda_ptr(gate, "gate"), _cuda_ptr(gamma, "gamma"), float(eps),
+                      _cuda_ptr(scales, "scales") if fp8 else None)
     st = la_gate_norm_apply(T, H, d, _DT[o.dtype], _cuda_ptr(o, "o"), gn, _cuda_ptr(out, "out"),
                             s.cuda_stream)
     if st != LA_OK:
         raise LaError(st, "la_gate_norm_apply")
-    return out
+    return (out, scales) if fp8 else out
 
 
 def prefill_state(k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor, *,

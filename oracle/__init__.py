@@ -232,7 +232,9 @@ def gated_rmsnorm_fp8(o, gate, gamma, eps: float):
         amax = max_j |y_j|,  scale = amax / 448,  code_j = E4M3(y_j * 448 / amax)
 
     (code 0 and scale 0 for an all-zero block), so code_j * scale reproduces y_j to within half an
-    E4M3 step.  Returns (uint8 codes with o's shape, fp64 scales [..., H])."""
+    E4M3 step.  This is the exact-arithmetic definition; the kernels quantize y after rounding it
+    to the I/O dtype, and their tests take the reference codes in that same precision.  Returns
+    (uint8 codes with o's shape, fp64 scales [..., H])."""
     y = gated_rmsnorm(o, gate, gamma, eps)
     amax = np.max(np.abs(y), axis=-1)
     inv = np.where(amax > 0, E4M3_MAX / np.where(amax > 0, amax, 1.0), 0.0)

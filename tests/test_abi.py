@@ -226,6 +226,8 @@ def test_varlen_epilogue_checks(lib):
     assert call(d, la.la_gate_norm(0x800000, 0x900000, -1.0)) == la.LA_ERR_SHAPE
     # gate overlapping out
     assert call(d, la.la_gate_norm(0x800000, 0x900000, 1e-6), out=0x800000 + 64) == la.LA_ERR_ALIAS
+    # FP8 output is the stand-alone operator's, not this epilogue's
+    assert call(d, la.la_gate_norm(0x800000, 0x900000, 1e-6, 0xA00000)) == la.LA_ERR_UNSUPPORTED
 
 
 # ---------------------------------------------------------------------------------------------
@@ -280,6 +282,10 @@ def test_decode_multi_rejects_bad_arguments(lib):
     nan = la.la_gate_norm(0x800000, 0x900000, float("nan"))
     assert la.la_decode_multi(1, 2, 128, 2, la.LA_BF16, *ok, out, 0,
                               epilogue=nan) == la.LA_ERR_SHAPE
+    # no FP8 output on the decode path
+    fp8 = la.la_gate_norm(0x800000, 0x900000, 1e-6, 0xA00000)
+    assert la.la_decode_multi(1, 2, 128, 2, la.LA_BF16, *ok, out, 0,
+                              epilogue=fp8) == la.LA_ERR_UNSUPPORTED
 
 
 def test_gate_norm_apply_rejects_bad_arguments(lib):
@@ -296,6 +302,15 @@ def test_gate_norm_apply_rejects_bad_arguments(lib):
     # y overlapping o without being o, or overlapping the gate
     assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, o, gn, o + 64, 0) == la.LA_ERR_ALIAS
     assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, o, gn, 0x800000, 0) == la.LA_ERR_ALIAS
+    # FP8 output: not in place, scales aligned and apart from o, y and the gate
+    fp8 = la.la_gate_norm(0x800000, 0x900000, 1e-6, 0xA00000)
+    assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, o, fp8, o, 0) == la.LA_ERR_ALIAS
+    assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, o, la.la_gate_norm(
+        0x800000, 0x900000, 1e-6, 0xA00008), y, 0) == la.LA_ERR_ALIGN
+    assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, o, la.la_gate_norm(
+        0x800000, 0x900000, 1e-6, y + 16), y, 0) == la.LA_ERR_ALIAS
+    assert la.la_gate_norm_apply(4, 2, 128, la.LA_BF16, o, la.la_gate_norm(
+        0x800000, 0x900000, 1e-6, 0x800000 + 16), y, 0) == la.LA_ERR_ALIAS
 
 
 def test_prefill_state_rejects_bad_arguments(lib):

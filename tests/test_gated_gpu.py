@@ -12,7 +12,7 @@ import torch
 
 import oracle
 from long_context_attention_la_b200 import la, synth
-from tests.helpers import check_close, oracle_bits
+from tests.helpers import check_close, check_fp8, oracle_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -167,3 +167,46 @@ def test_standalone_gate_norm_equals_fused_epilogue_path():
     y_fused, _ = la.prefill_varlen(q, k, v, sl, cu, gate=gate, gamma=gamma, eps=EPS)
     torch.cuda.synchronize()
     check_close(y_sep.float().cpu().numpy(), y_fused.double().cpu().numpy(), torch.bfloat16, "y")
+
+
+# ---------------------------------------------------------------------------------------------
+# FP8 E4M3 output of the fused operator ("group norm + sigmoid gate + quantize")
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 128),
+                                     (torch.bfloat16, 64)])
+def test_standalone_gate_norm_fp8_matches_oracle(dtype, d):
+    """la_gate_norm_apply with FP8 output on random o (ragged head count: rows past H in the
+    last sweep)."""
+    T, H = 333, 7
+    g = torch.Generator(device=DEV)
+    g.manual_seed(171)
+    o = (torch.randn((T, H, d), generator=g, device=DEV) * 0.7).to(dtype)
+    gate = (torch.randn((T, H, d), generator=g, device=DEV) * 3).to(dtype)
+    gamma = (1.0 + 0.5 * torch.randn((H, d), generator=g, device=DEV)).float()
+    codes, scales = la.gate_norm(o, gate, gamma, eps=1e-6, fp8=True)
+    torch.cuda.synchronize()
+    ref = oracle.gated_rmsnorm(o.double().cpu().numpy(), oracle_bits(gate), gamma.cpu().numpy(),
+                               1e-6)
+    check_fp8(codes.cpu().numpy(), scales.cpu().numpy(), ref, "standalone fp8", io_dtype=dtype)
+
+
+def test_standalone_gate_norm_fp8_zero_blocks_and_saturated_gate():
+    """All-zero o gives scale 0 and zero codes; a gate of scale 6 pushes the sigmoid into both
+    tails, so blocks mix large and tiny values; and the prefill's own output quantizes within
+    the bar (prefill, then the stand-alone operator with FP8 output)."""
+    H, d, T = 3, 128, 260
+    o = torch.zeros((T, H, d), dtype=torch.bfloat16, device=DEV)
+    gate, gamma = draw_gate(T, H, d, seed=191)
+    codes, scales = la.gate_norm(o, gate, gamma, eps=1e-6, fp8=True)
+    torch.cuda.synchronize()
+    assert bool((scales == 0).all()) and bool(((codes & 0x7F) == 0).all())
+    lengths = [700, 333]
+    cu = synth.cu_from_lengths(lengths)
+    q, k, v = draw_packed(lengths, 8, d, seed=111, dist="silu_qk")
+    sl = synth.slopes(8, DEV)
+    gate, gamma = draw_gate(sum(lengths), 8, d, seed=112, scale=6.0)
+    o, _ = la.prefill_varlen(q, k, v, sl, cu)
+    codes, scales = la.gate_norm(o, gate, gamma, eps=0.5, fp8=True)
+    torch.cuda.synchronize()
+    check_fp8(codes.cpu().numpy(), scales.cpu().numpy(),
+              reference(q, k, v, sl, cu, gate, gamma, 0.5), "prefill then fp8 operator")

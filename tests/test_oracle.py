@@ -352,6 +352,31 @@ def test_gated_rmsnorm_fp8_blocks():
     assert np.all(np.abs(deq - y) <= bound)
 
 
+def test_fp8_bar_accepts_reference_and_rejects_corruptions():
+    """The GPU tests' FP8 bar (tests.helpers.check_fp8) passes the reference quantization of y
+    itself and fails codes two steps off, a wrong scale, and codes of the wrong sign."""
+    from tests.helpers import check_fp8
+    rng = np.random.default_rng(12)
+    y = rng.standard_normal((40, 3, 128)) * rng.uniform(0.1, 10, (40, 3, 1))
+    y32 = y.astype(np.float32)
+    amax = np.max(np.abs(y32), axis=-1)
+    codes = oracle.e4m3_encode((y32 * (np.float32(448) / amax)[..., None]).astype(np.float64))
+    scales = (amax / 448.0).astype(np.float32).T.copy()
+    check_fp8(codes, scales, y, io_dtype=torch.float32)
+    bad = codes.copy()
+    mid = np.argwhere((np.abs(oracle.e4m3_decode(codes)) >= 64) &
+                      (np.abs(oracle.e4m3_decode(codes)) < 256))[0]
+    bad[tuple(mid)] = bad[tuple(mid)] + 2  # two steps up in magnitude, below saturation
+    with pytest.raises(AssertionError):
+        check_fp8(bad, scales, y, io_dtype=torch.float32)
+    s_bad = scales.copy()
+    s_bad[2, 9] *= 1.05
+    with pytest.raises(AssertionError):
+        check_fp8(codes, s_bad, y, io_dtype=torch.float32)
+    with pytest.raises(AssertionError):
+        check_fp8(codes ^ 0x80, scales, y, io_dtype=torch.float32)
+
+
 # ---------------------------------------------------------------------------------------------
 # qk_norm_rope: QK RMSNorm + partial rotary embedding before the kernel
 # ---------------------------------------------------------------------------------------------
