@@ -42,12 +42,12 @@ METRIC = "lightning-attn prefill tok/s & TFLOP/s (H=64,d=128); decode state GB/s
 DECODE = dict(B=256, H=64, d=128)
 
 
-def measured_counters():
+def measured_counters(path=None):
     """Counters of one prefill launch of the default workload from the committed ncu capture
     (the fenced json record in profiles/chunked_prefill_kernel_counters.md), or None when the
     kernel sources changed since that capture: DRAM bytes and the tensor-pipe activity."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "chunked_prefill_kernel_counters.md")
+    path = path or os.path.join(ROOT, "profiles", "chunked_prefill_kernel_counters.md")
     try:
         with open(path) as f:
             text = f.read()
@@ -62,6 +62,19 @@ def measured_counters():
         return rec
     except Exception:
         return None
+
+
+def prefill_bytes_per_token_head(d, gate=False, gate_separate=False, fp8=False):
+    """Algorithmic bytes of one token-head of the timed prefill step (bf16 rows of d values):
+    read q, k, v and write o; the fused norm + gate also reads the gate; the separate pass reads
+    o and the gate and writes y; an FP8 y is d bytes plus a 4-byte block scale."""
+    row = 2 * d
+    y_row = d + 4 if fp8 else row
+    if gate:
+        return 3 * row + row + row
+    if gate_separate:
+        return 4 * row + 2 * row + y_row
+    return 4 * row
 
 
 # Tensor-core flops the prefill kernel executes per token and head at d = 128, by chunk length:
@@ -588,16 +601,7 @@ def run_ours(args):
         tok_s = world * tokens / ((step_ms_max if args.cp else pre_ms_max) * 1e-3)
         # algorithmic bytes of one prefill launch: read q, k, v and write o (bf16), write the
         # final states (and read the initial states of the packed workload)
-        # (the fused norm + gate also reads the gate; the separate pass reads o and the gate and
-        # writes y; an FP8 y is d bytes plus a 4-byte scale per token-head instead of 2d bytes)
-        row = 2 * d
-        y_row = d + 4 if args.fp8 else row
-        if args.gate:
-            per_th = 3 * row + row + row
-        elif args.gate_separate:
-            per_th = 4 * row + 2 * row + y_row
-        else:
-            per_th = 4 * row
+        per_th = prefill_bytes_per_token_head(d, args.gate, args.gate_separate, args.fp8)
         pre_bytes = per_th * B * N * H + \
             n_states * H * d * d * 4 * (1 if vw is None and not args.cp else 2)
         achieved = pre_bytes / (pre_ms_max * 1e-3) / 1e9
