@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define LA_VERSION 1002 /* major*1000 + minor */
+#define LA_VERSION 1003 /* major*1000 + minor */
 
 typedef enum {
   LA_OK = 0,

@@ -51,7 +51,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert la.la_version() == 1002
+    assert la.la_version() == 1003
     for code in range(-10, 1):
         assert la.la_status_string(code) not in ("", "unknown status")
     assert la.la_status_string(-99) == "unknown status"
