@@ -286,6 +286,8 @@ def run_ours(args):
     q, k, v = synth.draw_qkv(B, N, H, d, dist=w.dist, seed=w.seed + 1000 * rank, dtype=w.dtype,
                              device=dev)
     sl = synth.slopes(H, dev)
+    if args.qk_fused and (args.gate or args.cp or args.qk_rope or args.chunk not in (0, 128)):
+        raise SystemExit("--qk-fused is the plain-output, 128-token-chunk prefill of raw q, k")
     if args.fp8 and not args.gate_separate:
         raise SystemExit("--fp8 is an output format of --gate-separate (the stand-alone "
                          "norm + gate + quantize operator)")
@@ -316,9 +318,9 @@ def run_ours(args):
         gamma = (1.0 + 0.1 * torch.randn((H, d), generator=gg, device=dev)).float()
         extra_in += [gate]
         epi = la.la_gate_norm(gate.data_ptr(), gamma.data_ptr(), 1e-6)
-    if vw is None and (args.gate or args.cp):
-        # the fused epilogue and the initial state are options of the packed entry point: B
-        # sequences of N tokens
+    if vw is None and (args.gate or args.cp or args.qk_fused):
+        # the fused epilogue, the in-kernel QK norm and the initial state are options of the
+        # packed entry points: B sequences of N tokens
         n_states = B
         cu = torch.arange(0, B * N + 1, N, dtype=torch.int64, device=dev)
         sin = None
@@ -367,6 +369,17 @@ def run_ours(args):
         positions = (torch.arange(B * N, device=dev) % N).to(torch.int64)
         qk = la.la_qk_norm_rope_desc(B * N, H, d, H * d, H * d, 64, 6.0e6, 1e-6, 0)
         extra_in += [q_raw, k_raw]
+    qkp = None
+    if args.qk_fused:
+        # the same operator inside the prefill kernel: q and k (as drawn) are the raw
+        # projections, normalised and rotated tile by tile in shared memory
+        gq_ = torch.Generator(device=dev)
+        gq_.manual_seed(78 + 1000 * rank)
+        gam_q = (1.0 + 0.1 * torch.randn(d, generator=gq_, device=dev)).float()
+        gam_k = (1.0 + 0.1 * torch.randn(d, generator=gq_, device=dev)).float()
+        positions = (torch.arange(B * N, device=dev) % N).to(torch.int64)
+        qkp = la.la_qk_prologue(gam_q.data_ptr(), gam_k.data_ptr(), positions.data_ptr(), 64,
+                                6.0e6, 1e-6, 0)
 
     Bd, Hd, dd = DECODE["B"], DECODE["H"], DECODE["d"]
     if args.no_decode:
@@ -386,7 +399,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
 
-    packed = vw is not None or args.gate or args.cp
+    packed = vw is not None or args.gate or args.cp or args.qk_fused
 
     def cp_state_call():
         # local state of this rank's part, all ranks' states, the fold of those before it
@@ -405,6 +418,11 @@ def run_ours(args):
         if not packed:
             rc = la.la_prefill(desc, q.data_ptr(), k.data_ptr(), v.data_ptr(), sl.data_ptr(),
                                out.data_ptr(), st.data_ptr(), ws.data_ptr(), ws_bytes, sp)
+        elif qkp is not None:
+            rc = la.la_prefill_varlen_qk(desc, qkp, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                         sl.data_ptr(), cu.data_ptr(),
+                                         0 if sin is None else sin.data_ptr(), out.data_ptr(),
+                                         st.data_ptr(), ws.data_ptr(), ws_bytes, sp)
         else:
             rc = la.la_prefill_varlen(desc, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                       sl.data_ptr(), cu.data_ptr(),
@@ -596,14 +614,16 @@ def run_ours(args):
         # committed counters describe the default launch only (prefill_32k, plain output, the
         # default chunk and plan)
         counters = (measured_counters() if args.workload == "prefill_32k" and not (
-            args.gate or args.gate_separate or args.cp or args.chunk or args.segments) else None)
+            args.gate or args.gate_separate or args.cp or args.chunk or args.segments or
+            args.qk_fused) else None)
         tokens = B * N
         tok_s = world * tokens / ((step_ms_max if args.cp else pre_ms_max) * 1e-3)
         # algorithmic bytes of one prefill launch: read q, k, v and write o (bf16), write the
         # final states (and read the initial states of the packed workload)
         per_th = prefill_bytes_per_token_head(d, args.gate, args.gate_separate, args.fp8)
         pre_bytes = per_th * B * N * H + \
-            n_states * H * d * d * 4 * (1 if vw is None and not args.cp else 2)
+            n_states * H * d * d * 4 * (1 if vw is None and not args.cp else 2) + \
+            (8 * B * N if args.qk_fused else 0)  # the in-kernel RoPE reads one position a token
         achieved = pre_bytes / (pre_ms_max * 1e-3) / 1e9
         canon = 4.0 * d * d * B * N * H  # recurrent-form flops
         chunk = args.chunk if args.chunk else 128
@@ -629,6 +649,10 @@ def run_ours(args):
                                     f"(fragmented lengths), H={H} d={d} bf16, fp32 initial "
                                     f"states") + (", fused grouped RMSNorm + sigmoid gate epilogue"
                                                   if args.gate else "") +
+                                   (", QK RMSNorm + RoPE (rotary dim 64) inside the prefill "
+                                    "kernel on raw q, k" if args.qk_fused else "") +
+                                   (", QK RMSNorm + RoPE pass (rotary dim 64) before the prefill"
+                                    if args.qk_rope else "") +
                                    (", then the grouped RMSNorm + sigmoid gate pass"
                                     if args.gate_separate else "") +
                                    (" with FP8 E4M3 output (one fp32 scale per token-head)"
@@ -679,10 +703,11 @@ def run_ours(args):
                 # time also holds the gather and the fold
                 "state_step_hbm_gbs": (2 * B * N * H * d * 2 + B * H * d * d * 4) /
                 (cp_ms_max * 1e-3) / 1e9},
-            "qk_norm_rope": None if qk is None else {
+            "qk_norm_rope": ({"in_prefill_kernel": True} if args.qk_fused else
+                             None if qk is None else {
                 "ms": qk_ms_max,
                 # read q, k (raw) and write q_hat, k_hat: 4 * d * 2 bytes per token-head
-                "hbm_gbs": 8 * B * N * H * d / (qk_ms_max * 1e-3) / 1e9},
+                "hbm_gbs": 8 * B * N * H * d / (qk_ms_max * 1e-3) / 1e9}),
             "cpu_baseline": cpu,
             "clocks": clk.summary(),
             "e2e": e2e,
@@ -755,6 +780,9 @@ def main():
                     help="decode this many tokens per sequence per step (multi-token step)")
     ap.add_argument("--qk-rope", action="store_true",
                     help="run the QK RMSNorm + partial RoPE operator before each prefill")
+    ap.add_argument("--qk-fused", action="store_true",
+                    help="apply the QK RMSNorm + partial RoPE inside the prefill kernel "
+                         "(la_prefill_varlen_qk on raw q, k)")
     ap.add_argument("--gate-separate", action="store_true",
                     help="run the grouped RMSNorm + sigmoid gate as its own pass after the prefill")
     ap.add_argument("--gate", action="store_true",

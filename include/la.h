@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define LA_VERSION 1003 /* major*1000 + minor */
+#define LA_VERSION 1004 /* major*1000 + minor */
 
 typedef enum {
   LA_OK = 0,
@@ -349,6 +349,40 @@ typedef struct {
 la_status la_qk_norm_rope(const la_qk_norm_rope_desc* desc, const void* q, const void* k,
                           const float* gamma_q, const float* gamma_k, const int64_t* positions,
                           void* q_out, void* k_out, void* stream);
+
+/* The QK RMSNorm + partial RoPE of la_qk_norm_rope, applied by la_prefill_varlen_qk inside the
+ * prefill kernel. */
+typedef struct {
+  const float* gamma_q;     /* fp32 [d] device, 16-byte aligned: q's norm weight (all heads) */
+  const float* gamma_k;     /* fp32 [d] device, 16-byte aligned: k's norm weight */
+  const int64_t* positions; /* int64 [T] device: each packed token's position in its sequence */
+  int32_t rotary_dim;       /* rotated dims r: a multiple of 16 in [16, d] (the report: 64) */
+  float theta;              /* rotary base, > 0 (the report: 6,000,000) */
+  float eps;                /* RMSNorm epsilon, >= 0 (the report: 1e-6) */
+  int32_t pad;
+} la_qk_prologue;
+
+/*
+ * la_prefill_varlen_qk — la_prefill_varlen whose q and k are the raw projections: the kernel
+ * applies the report's QK Norm and RoPE (§2.1 Fig. 2: QKV Projection -> QK Norm -> RoPE ->
+ * Linear Attention Kernel; §2.1.1) to each q and k tile in shared memory before any product
+ * reads it, so q_hat and k_hat never exist in device memory.  The result equals
+ *     la_qk_norm_rope(q, k, ... positions ...) followed by la_prefill_varlen(q_hat, k_hat, v, ...)
+ * exactly (the tiles hold the very bf16 rows la_qk_norm_rope stores), with the same segments.
+ *
+ *   desc        as for la_prefill_varlen; the tensor-core path only (bf16, d = 128, path AUTO or
+ *               TENSOR, chunk 0 or 128), else LA_ERR_UNSUPPORTED
+ *   qk          the norm + RoPE parameters (host pointer, read during the call); NULL:
+ *               LA_ERR_NULL.  positions: 8-byte aligned, one entry per packed token
+ *   q, k, v     [T, H, d] bf16 device (contiguous), read only: q and k are not modified
+ *   other arguments, the workspace (la_prefill_varlen_workspace_bytes) and the errors as for
+ *   la_prefill_varlen; there is no fused output epilogue here (out receives o).
+ */
+la_status la_prefill_varlen_qk(const la_varlen_desc* desc, const la_qk_prologue* qk,
+                               const void* q, const void* k, const void* v, const float* slopes,
+                               const int64_t* cu_seqlens, const float* state_in, void* out,
+                               float* state_out, void* workspace, size_t workspace_bytes,
+                               void* stream);
 
 /* Bytes of device workspace la_prefill_state needs for this descriptor (0 for invalid
  * arguments or when the recurrent path runs, which needs none). */

@@ -270,11 +270,25 @@ size_t la_prefill_varlen_workspace_bytes(const la_varlen_desc* desc) {
       .total;
 }
 
-la_status la_prefill_varlen(const la_varlen_desc* desc, const void* q, const void* k,
-                            const void* v, const float* slopes, const int64_t* cu_seqlens,
-                            const float* state_in, const la_gate_norm* epilogue, void* out,
-                            float* state_out, void* workspace, size_t workspace_bytes,
-                            void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Rotary frequencies theta^(-2i / r), i < r / 2, in double (one routine for both QK operators,
+// so that the in-tile form reproduces the stand-alone one exactly).
+void rope_inv_freq(double* inv_freq, int rotary_dim, float theta) {
+  const double log_theta = std::log(static_cast<double>(theta));
+  for (int i = 0; i < rotary_dim / 2; ++i)
+    inv_freq[i] = std::exp(-2.0 * i / rotary_dim * log_theta);
+}
+
+// The body of la_prefill_varlen and la_prefill_varlen_qk (qk: the in-tile QK norm + RoPE, or
+// null).
+la_status prefill_varlen_impl(const la_varlen_desc* desc, const la_qk_prologue* qk,
+                              const void* q, const void* k, const void* v, const float* slopes,
+                              const int64_t* cu_seqlens, const float* state_in,
+                              const la_gate_norm* epilogue, void* out, float* state_out,
+                              void* workspace, size_t workspace_bytes, void* stream) {
   int64_t numel = 0;
   const la_status st = check_varlen(desc, &numel);
   if (st != LA_OK) return st;
@@ -302,6 +316,18 @@ la_status la_prefill_varlen(const la_varlen_desc* desc, const void* q, const voi
     if (!(epilogue->eps >= 0.f) || epilogue->eps > 3.0e38f) return LA_ERR_SHAPE;  // NaN, inf
     if (bytes > 0 && overlaps(epilogue->gate, bytes, out, bytes)) return LA_ERR_ALIAS;
   }
+  if (qk != nullptr) {
+    // one kernel instance carries it: tensor path, 128-token chunks, plain output
+    if (!tensor || chunk_of(desc->chunk) != 128 || epilogue != nullptr) return LA_ERR_UNSUPPORTED;
+    if (!qk->gamma_q || !qk->gamma_k || !qk->positions) return LA_ERR_NULL;
+    if (!aligned16(qk->gamma_q) || !aligned16(qk->gamma_k) ||
+        (reinterpret_cast<uintptr_t>(qk->positions) & 7u) != 0)
+      return LA_ERR_ALIGN;
+    if (qk->rotary_dim < 16 || qk->rotary_dim > desc->d || qk->rotary_dim % 16 != 0)
+      return LA_ERR_SHAPE;
+    if (!(qk->theta > 0.f) || qk->theta > 3.0e38f || !(qk->eps >= 0.f) || qk->eps > 3.0e38f)
+      return LA_ERR_SHAPE;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int sms = device_sms();
   if (sms <= 0) return LA_ERR_CUDA;
@@ -326,11 +352,42 @@ la_status la_prefill_varlen(const la_varlen_desc* desc, const void* q, const voi
     a.gamma = epilogue->gamma;
     a.eps = epilogue->eps;
   }
+  if (qk != nullptr) {
+    a.qk_gamma_q = qk->gamma_q;
+    a.qk_gamma_k = qk->gamma_k;
+    a.qk_positions = qk->positions;
+    a.qk_rotary_dim = qk->rotary_dim;
+    a.qk_eps = qk->eps;
+    rope_inv_freq(a.qk_inv_freq, qk->rotary_dim, qk->theta);
+  }
   apply_debug_env(a);
   const cudaError_t e =
       la::launch_prefill_varlen(a, layout, ws, desc->segments, tensor, s, sms);
   if (owned) cudaFreeAsync(ws, s);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+la_status la_prefill_varlen(const la_varlen_desc* desc, const void* q, const void* k,
+                            const void* v, const float* slopes, const int64_t* cu_seqlens,
+                            const float* state_in, const la_gate_norm* epilogue, void* out,
+                            float* state_out, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  return prefill_varlen_impl(desc, nullptr, q, k, v, slopes, cu_seqlens, state_in, epilogue, out,
+                             state_out, workspace, workspace_bytes, stream);
+}
+
+la_status la_prefill_varlen_qk(const la_varlen_desc* desc, const la_qk_prologue* qk,
+                               const void* q, const void* k, const void* v, const float* slopes,
+                               const int64_t* cu_seqlens, const float* state_in, void* out,
+                               float* state_out, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (qk == nullptr) return LA_ERR_NULL;
+  return prefill_varlen_impl(desc, qk, q, k, v, slopes, cu_seqlens, state_in, nullptr, out,
+                             state_out, workspace, workspace_bytes, stream);
 }
 
 la_status la_qk_norm_rope(const la_qk_norm_rope_desc* desc, const void* q, const void* k,
@@ -378,9 +435,7 @@ la_status la_qk_norm_rope(const la_qk_norm_rope_desc* desc, const void* q, const
   a.k_out = static_cast<__nv_bfloat16*>(k_out);
   a.rotary_dim = d.rotary_dim;
   a.eps = d.eps;
-  const double log_theta = std::log(static_cast<double>(d.theta));
-  for (int i = 0; i < d.rotary_dim / 2; ++i)
-    a.inv_freq[i] = std::exp(-2.0 * i / d.rotary_dim * log_theta);
+  rope_inv_freq(a.inv_freq, d.rotary_dim, d.theta);
   return la::launch_qk_norm_rope(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? LA_OK
              : LA_ERR_CUDA;

@@ -39,6 +39,10 @@
 //                output pass, KV -> bf16 operand, decay rescale, final state
 //   warps 16-19  output epilogue: O = O_intra + lambda^(i+1) O_inter -> bf16 -> global, in
 //                whole 32-byte sectors
+// Two instances regroup warps 8-11: the fused norm + gate instance gives them half the epilogue's
+// columns, and the in-tile QK instance (raw q and k in) has them apply the QK RMSNorm + RoPE to
+// each tile's q and k rows in shared memory before any product reads them (and scale the keys in
+// the local-state pass); both run the decay mask on warps 4-7 alone.
 // Every wait (mbarrier or scan flag) is bounded in time; on expiry the CTA records
 // LA_ERR_TIMEOUT in the workspace status word, unwinds, frees its TMEM and exits.
 #include <cuda.h>
@@ -62,6 +66,7 @@ constexpr uint32_t kWarpP0 = 4;    // warps 4..11: decay mask / local-pass K sca
 constexpr uint32_t kWarpS0 = 12;   // warps 12..15: state
 constexpr uint32_t kWarpO0 = 16;   // warps 16..19: output epilogue
 constexpr uint32_t kBarP = 1, kBarS = 2, kBarO = 3;  // named barriers of the three groups
+constexpr uint32_t kBarT = 4;                        // ... and of the in-tile QK transform warps
 constexpr uint32_t kTileBytes = C * D * 2;           // one bf16 [128 x 128] tile
 constexpr uint32_t kHalfBytes = kTileBytes / 2;      // [128 rows x 64 cols], 128-byte rows
 constexpr uint32_t kOffQ = 0;
@@ -99,6 +104,7 @@ struct Ctrl {
   uint64_t s2_full;   // C = 256: the cross scores Q_B K~_A^T of a chunk's second tile are in TMEM
   uint64_t p2_ready;  // C = 256: their scaled bf16 P_BA is in TMEM
   uint64_t gate_full[2];  // fused norm + gate: the tile's gate rows are in its stage's Q slot
+  uint64_t qk_ready[2];   // in-tile QK norm + RoPE: the stage's q and k rows are transformed
   float row_x[128];       // fused norm + gate: a row's sum of squares / 1/rms between its two warps
   uint64_t o_full;
   uint64_t o_free;
@@ -132,6 +138,13 @@ struct Params {
   const __nv_bfloat16* gate;   // fused norm + gate: gate pre-activation like out, or null
   const float* gamma;          // fp32 [H, D] norm weight
   float eps;
+  // in-tile QK RMSNorm + RoPE (kQk instance): weights fp32 [D], positions int64 [B * N]
+  const float* qk_gamma_q;
+  const float* qk_gamma_k;
+  const int64_t* qk_positions;
+  int32_t qk_rotary_dim;
+  float qk_eps;
+  double qk_inv_freq[64];      // theta^(-2i / rotary_dim), i < rotary_dim / 2
   int64_t N, H, BH;
   int64_t n_chunks, seg_chunks, segments, units;
   uint64_t timeout_ns;
@@ -198,6 +211,133 @@ __device__ __forceinline__ void scale_half_row(uint8_t* half_tile, uint32_t r, f
       x[c].w = pack_bf16x2(bf16lo_to_f32(x[c].w) * w, bf16hi_to_f32(x[c].w) * w);
       *reinterpret_cast<uint4*>(row + (((c0 + c) ^ (r & 7u)) << 4)) = x[c];
     }
+  }
+}
+
+// 16-byte chunk gc (0..15, dims 8 gc .. 8 gc + 7) of row r of a swizzled [128 x 128] tile
+__device__ __forceinline__ uint8_t* tile_chunk(uint8_t* tile, uint32_t r, uint32_t gc) {
+  return tile + (gc >> 3) * kHalfBytes + sw128_off(r, gc & 7u);
+}
+
+// the 8 bf16 of a chunk as 4 fp32 pairs
+__device__ __forceinline__ void unpack_chunk(const uint4& w, float2 (&x)[4]) {
+  const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] = make_float2(bf16lo_to_f32(v[e]), bf16hi_to_f32(v[e]));
+}
+
+// QK RMSNorm + partial rotate-half RoPE, in place, of row r of the k tile and (kWithQ) of the q
+// tile in the same stage: both rows are one token's, so they share its rotation angles.
+//     y = gamma * x / sqrt(mean(x^2) + eps);  (y_i, y_{i+R/2}) <- (y_i cos a - y_{i+R/2} sin a,
+//     y_{i+R/2} cos a + y_i sin a), a = pos * theta^(-2i/R), i < R/2 (R = rotary_dim)
+// ("Ling and Ring 2.6 Technical Report", §2.1 Fig. 2 and §2.1.1).  The row's 16 chunks are taken
+// in the pairs the stand-alone operator (la_qknorm.cu) gives to each of a row's 8 threads,
+// piece (u, u + R/16) for u < R/16, else two chunks (128 - R)/16 apart past the rotary span, and
+// every rounding follows that operator: per-pair partial sums of squares on paired fp32 FMAs,
+// added in its shuffle-tree order; y = gamma (x rinv); the rotation and the angle reduction as
+// there.  The tiles therefore hold exactly the bf16 rows that operator would have stored.
+template <bool kWithQ>
+__device__ __forceinline__ void qk_norm_rope_rows(uint8_t* q_tile, uint8_t* k_tile, uint32_t r,
+                                                  int64_t pos, const float* gamma_q,
+                                                  const float* gamma_k, const double* inv_freq,
+                                                  int32_t rotary_dim, float eps) {
+  const int rot = rotary_dim / 16;      // chunk pairs inside the rotary span
+  const int rd8 = rotary_dim / 8;       // first chunk past it
+  const int far = 8 - rot;              // distance of a pass-through pair's two chunks
+  auto piece_a = [&](int u) { return u < rot ? u : rd8 + (u - rot); };
+  auto piece_b = [&](int u) { return u < rot ? u + rot : rd8 + (u - rot) + far; };
+  auto pair_ss = [&](uint8_t* tile, int u) {
+    float2 xa[4], xb[4];
+    unpack_chunk(*reinterpret_cast<const uint4*>(tile_chunk(tile, r, piece_a(u))), xa);
+    unpack_chunk(*reinterpret_cast<const uint4*>(tile_chunk(tile, r, piece_b(u))), xb);
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc = __ffma2_rn(xb[e], xb[e], __ffma2_rn(xa[e], xa[e], acc));
+    return acc.x + acc.y;
+  };
+  // the pairs' partial sums in the order of a butterfly over 8 lanes (xor 4, then 2, then 1)
+  auto tree = [](const float (&s)[8]) {
+    return ((s[0] + s[4]) + (s[2] + s[6])) + ((s[1] + s[5]) + (s[3] + s[7]));
+  };
+  float sq[8] = {}, sk[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    if constexpr (kWithQ) sq[u] = pair_ss(q_tile, u);
+    sk[u] = pair_ss(k_tile, u);
+  }
+  float rq = 0.f;
+  if constexpr (kWithQ) rq = rsqrtf(fmaf(tree(sq), 1.f / D, eps));
+  const float rk = rsqrtf(fmaf(tree(sk), 1.f / D, eps));
+
+  // one pair of chunks of one row: normalise, weight, rotate (rotary pairs), store as bf16
+  auto apply = [&](uint8_t* tile, const float* gamma, float rinv, int ca, int cb, bool rotary,
+                   const float2 (&cs)[4], const float2 (&sn)[4]) {
+    uint4* pa = reinterpret_cast<uint4*>(tile_chunk(tile, r, ca));
+    uint4* pb = reinterpret_cast<uint4*>(tile_chunk(tile, r, cb));
+    float2 ya[4], yb[4];
+    unpack_chunk(*pa, ya);
+    unpack_chunk(*pb, yb);
+    const float4* gpa = reinterpret_cast<const float4*>(gamma + 8 * ca);
+    const float4* gpb = reinterpret_cast<const float4*>(gamma + 8 * cb);
+    const float4 ga0 = __ldg(gpa), ga1 = __ldg(gpa + 1), gb0 = __ldg(gpb), gb1 = __ldg(gpb + 1);
+    const float2 gma[4] = {make_float2(ga0.x, ga0.y), make_float2(ga0.z, ga0.w),
+                           make_float2(ga1.x, ga1.y), make_float2(ga1.z, ga1.w)};
+    const float2 gmb[4] = {make_float2(gb0.x, gb0.y), make_float2(gb0.z, gb0.w),
+                           make_float2(gb1.x, gb1.y), make_float2(gb1.z, gb1.w)};
+    const float2 r2 = make_float2(rinv, rinv);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      ya[e] = __fmul2_rn(gma[e], __fmul2_rn(ya[e], r2));
+      yb[e] = __fmul2_rn(gmb[e], __fmul2_rn(yb[e], r2));
+    }
+    if (rotary) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 y0 = ya[e], y1 = yb[e];
+        const float2 nsn = make_float2(-sn[e].x, -sn[e].y);
+        ya[e] = __ffma2_rn(y0, cs[e], __fmul2_rn(y1, nsn));
+        yb[e] = __ffma2_rn(y1, cs[e], __fmul2_rn(y0, sn[e]));
+      }
+    }
+    uint4 wa, wb;
+    wa.x = pack_bf16x2(ya[0].x, ya[0].y);
+    wa.y = pack_bf16x2(ya[1].x, ya[1].y);
+    wa.z = pack_bf16x2(ya[2].x, ya[2].y);
+    wa.w = pack_bf16x2(ya[3].x, ya[3].y);
+    wb.x = pack_bf16x2(yb[0].x, yb[0].y);
+    wb.y = pack_bf16x2(yb[1].x, yb[1].y);
+    wb.z = pack_bf16x2(yb[2].x, yb[2].y);
+    wb.w = pack_bf16x2(yb[3].x, yb[3].y);
+    *pa = wa;
+    *pb = wb;
+  };
+#pragma unroll 1
+  for (int u = 0; u < 8; ++u) {
+    const bool rotary = u < rot;
+    float2 cs[4], sn[4];
+    if (rotary) {
+      // the angle pos * w_f, reduced modulo 2 pi in fp64, then sin and cos in fp32
+      constexpr double kTwoPi = 6.283185307179586476925286766559;
+      constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float s0, c0, s1, c1;
+        const double a0 = __dmul_rn(static_cast<double>(pos), inv_freq[8 * u + 2 * e]);
+        const double a1 = __dmul_rn(static_cast<double>(pos), inv_freq[8 * u + 2 * e + 1]);
+        __sincosf(static_cast<float>(__fma_rn(-kTwoPi, rint(__dmul_rn(a0, kInvTwoPi)), a0)), &s0,
+                  &c0);
+        __sincosf(static_cast<float>(__fma_rn(-kTwoPi, rint(__dmul_rn(a1, kInvTwoPi)), a1)), &s1,
+                  &c1);
+        cs[e] = make_float2(c0, c1);
+        sn[e] = make_float2(s0, s1);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) cs[e] = sn[e] = make_float2(0.f, 0.f);
+    }
+    const int ca = piece_a(u), cb = piece_b(u);
+    if constexpr (kWithQ) apply(q_tile, gamma_q, rq, ca, cb, rotary, cs, sn);
+    apply(k_tile, gamma_k, rk, ca, cb, rotary, cs, sn);
   }
 }
 
@@ -499,14 +639,18 @@ __device__ __forceinline__ void gated_epilogue_write(const Params& p, Ctrl* ctrl
 
 // kGated: the output epilogue applies the fused norm + gate (p.gate != null).  Separate instances,
 // so that the plain kernel's register allocation carries none of the gated epilogue's pressure.
-// kCM: the chunk length (ChunkMode).
-template <bool kGated, int kCM>
+// kCM: the chunk length (ChunkMode).  kQk: q and k arrive raw and get their QK RMSNorm + RoPE in
+// shared memory first (C = 128, plain output only).
+template <bool kGated, int kCM, bool kQk = false>
 __global__ void __launch_bounds__(kThreads, 1)
     chunked_prefill_kernel(const __grid_constant__ Params p) {
+  static_assert(!kQk || (!kGated && kCM == kC128), "in-tile QK norm: C = 128, plain output");
   // The fused norm + gate instance runs the decay mask on 4 warps (one per TMEM lane quarter)
   // and its heavier epilogue on 8 (warps 16-19 take columns 0..63, warps 8-11 columns 64..127);
-  // the plain instance has 8 mask warps and 4 epilogue warps.
-  constexpr uint32_t kMaskWarps = kGated ? 4 : 8;
+  // the in-tile QK instance gives warps 8-11 the QK transform instead; the plain instance has 8
+  // mask warps and 4 epilogue warps.
+  constexpr uint32_t kMaskWarps = (kGated || kQk) ? 4 : 8;
+  constexpr uint32_t kQkThreads = kQk ? 128 : 0;
   constexpr uint32_t kMaskThreads = 32 * kMaskWarps;
   constexpr uint32_t kEpiThreads = kGated ? 256 : 128;
   extern __shared__ uint8_t smem_raw[];
@@ -527,9 +671,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // epilogue has read the gate rows staged in its Q slot
       mbar_init(&ctrl->empty[s], kGated ? 2 : 1);
       mbar_init(&ctrl->gate_full[s], 1);
+      mbar_init(&ctrl->qk_ready[s], 128);
       mbar_init(&ctrl->kt_ready[s], 128);
       mbar_init(&ctrl->unit_full[s], 1);
-      mbar_init(&ctrl->unit_empty[s], 1 + kMaskThreads + 128 + kEpiThreads);
+      mbar_init(&ctrl->unit_empty[s], 1 + kMaskThreads + 128 + kEpiThreads + kQkThreads);
     }
     mbar_init(&ctrl->s_full, 1);
     mbar_init(&ctrl->p_ready, kMaskThreads);
@@ -782,7 +927,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int32_t c = 0; c < n_out && ok; ++c) {
           const uint32_t s = g & 1;
           const uint32_t ph = (g >> 1) & 1;
-          if (!mbar_wait_bounded(&ctrl->full[s], ph, abort_flag, T)) {
+          if (!mbar_wait_bounded(&ctrl->full[s], ph, abort_flag, T) ||
+              (kQk && !mbar_wait_bounded(&ctrl->qk_ready[s], ph, abort_flag, T))) {
             ok = false;
             break;
           }
@@ -971,7 +1117,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float alpha = p.slopes[ui.bh % p.H] * kLog2e;  // lambda^n = exp2(-alpha n)
       const float lam1 = ex2_approx(-alpha);                 // lambda
 
-      if (ui.flags & 1) {
+      if ((ui.flags & 1) && kQk) {
+        g += static_cast<uint32_t>(ui.nc);  // (the QK transform warps scale these tiles' keys)
+      } else if (ui.flags & 1) {
         // local-state pass: K~_j = lambda^(L-1-j) k_j (8 warps: two threads per row, one per
         // half; 4 warps: one thread per row)
         const uint32_t r = tp & 127;
@@ -1130,6 +1278,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++j;
     }
   p_out:;
+  } else if (kQk && warp >= kWarpP0 + kMaskWarps && warp < kWarpS0) {
+    // =========================================================================================
+    // in-tile QK RMSNorm + RoPE: thread r transforms row r of the stage's q and k tiles as soon
+    // as they land, before any product reads them; in the local-state pass it also scales its
+    // key row to K~ (the mask warps' job in the other instances)
+    // =========================================================================================
+    const uint32_t r = (warp - (kWarpP0 + kMaskWarps)) * 32 + lane;  // tile row 0..127
+    uint32_t g = 0, j = 0;
+    while (true) {
+      const uint32_t slot = j & 1;
+      bool ok = mbar_wait_bounded(&ctrl->unit_full[slot], (j >> 1) & 1, abort_flag, T);
+      if (!group_all(ok, kBarT, kQkThreads)) break;
+      const UnitInfo ui = ctrl->units[slot];
+      mbar_arrive(&ctrl->unit_empty[slot]);
+      if (ui.bh < 0) break;
+      const float alpha = p.slopes[ui.bh % p.H] * kLog2e;
+      const int32_t n_local = (ui.flags & kUnitLocal) ? ui.nc : 0;
+      const int32_t n_tiles = n_local + ((ui.flags & kUnitNoOutput) ? 0 : ui.nc);
+      // index along the B * N token axis of row r of the piece's first tile
+      const int64_t tok_r = static_cast<int64_t>(ui.b) * p.N + ui.tok0 +
+                            static_cast<int64_t>(ui.c0) * C + r;
+      for (int32_t q = 0; q < n_tiles; ++q) {
+        const bool local = q < n_local;
+        const int32_t c = local ? q : q - n_local;
+        const int32_t row = c * C + static_cast<int32_t>(r);  // token of the piece
+        const bool valid = row < ui.len;  // rows past the piece are never output nor summed
+        const int64_t pos = valid ? p.qk_positions[tok_r + static_cast<int64_t>(c) * C] : 0;
+        const uint32_t s = g & 1;
+        ok = mbar_wait_bounded(&ctrl->full[s], (g >> 1) & 1, abort_flag, T);
+        if (!group_all(ok, kBarT, kQkThreads)) goto t_out;
+        uint8_t* st = smem + s * kStageBytes;
+        if (local) {
+          // K~_j = lambda^(L-1-j) k_hat_j: the transformed row is rounded to bf16 and then
+          // scaled with one more rounding, as when k_hat comes from memory
+          if (valid)
+            qk_norm_rope_rows<false>(nullptr, st + kOffK, r, pos, p.qk_gamma_q, p.qk_gamma_k,
+                                     p.qk_inv_freq, p.qk_rotary_dim, p.qk_eps);
+          const float w = valid ? exp2f(-alpha * static_cast<float>(ui.len - 1 - row)) : 0.f;
+          scale_half_row(st + kOffK, r, w);
+          scale_half_row(st + kOffK + kHalfBytes, r, w);
+        } else if (valid) {
+          qk_norm_rope_rows<true>(st + kOffQ, st + kOffK, r, pos, p.qk_gamma_q, p.qk_gamma_k,
+                                  p.qk_inv_freq, p.qk_rotary_dim, p.qk_eps);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&ctrl->qk_ready[s]);
+        if (local) mbar_arrive(&ctrl->kt_ready[s]);
+        ++g;
+      }
+      ++j;
+    }
+  t_out:;
   } else if (warp >= kWarpS0 && warp < kWarpO0) {
     // =========================================================================================
     // state: look-back scan over segments, bf16 operand, decay rescale, final state; K -> K~
@@ -1317,6 +1517,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float w = r < n_r ? exp2f(-alpha * static_cast<float>(n_r - 1 - r)) : 0.f;
           uint8_t* kt = smem + s * kStageBytes + kOffK;
+          // in-tile QK instance: the transform of this tile completed before S_c was issued, so
+          // this wait returns at once; it orders those shared-memory writes before this row's
+          if (kQk) (void)mbar_wait_bounded(&ctrl->qk_ready[s], (g >> 1) & 1, abort_flag, T);
           scale_half_row(kt, i, w);
           scale_half_row(kt + kHalfBytes, i, w);
           fence_proxy_async_smem();
@@ -1777,6 +1980,14 @@ cudaError_t launch_common(const PrefillArgs& a, Params& prm, uint8_t* ws,
     default:
       return cudaErrorInvalidValue;
   }
+  const bool qk = a.qk_positions != nullptr;
+  if (qk) {
+    // the in-tile QK norm + RoPE instance: C = 128, plain output, 16-row chunk pairs
+    if (a.chunk != 128 || gated || a.qk_gamma_q == nullptr || a.qk_gamma_k == nullptr ||
+        a.qk_rotary_dim < 16 || a.qk_rotary_dim > D || a.qk_rotary_dim % 16 != 0)
+      return cudaErrorInvalidValue;
+    kernel = chunked_prefill_kernel<false, kC128, true>;
+  }
   // set on every call: cheap, safe from any host thread, and it survives a context reset
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemAlloc));
@@ -1802,6 +2013,12 @@ cudaError_t launch_common(const PrefillArgs& a, Params& prm, uint8_t* ws,
     return cudaErrorInvalidValue;
   prm.gamma = a.gamma;
   prm.eps = a.eps;
+  prm.qk_gamma_q = a.qk_gamma_q;
+  prm.qk_gamma_k = a.qk_gamma_k;
+  prm.qk_positions = a.qk_positions;
+  prm.qk_rotary_dim = a.qk_rotary_dim;
+  prm.qk_eps = a.qk_eps;
+  for (int f = 0; f < 64; ++f) prm.qk_inv_freq[f] = a.qk_inv_freq[f];
   prm.counter = reinterpret_cast<uint32_t*>(ws + kWsCounter);
   prm.status = reinterpret_cast<int32_t*>(ws + kWsStatus);
   prm.flags = reinterpret_cast<uint32_t*>(ws + wl.flags_off);

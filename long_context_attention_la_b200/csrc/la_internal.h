@@ -34,6 +34,15 @@ struct PrefillArgs {
   const void* gate = nullptr;
   const float* gamma = nullptr;
   float eps = 0.f;
+  // QK RMSNorm + partial rotate-half RoPE applied to each q and k tile inside the chunked kernel
+  // before any product reads it (la_prefill_varlen_qk; tensor path, C = 128, no gate): weights
+  // fp32 [d], positions int64 over the token axis (index b * N + n).  Null: q and k as given.
+  const float* qk_gamma_q = nullptr;
+  const float* qk_gamma_k = nullptr;
+  const int64_t* qk_positions = nullptr;
+  int32_t qk_rotary_dim = 0;
+  float qk_eps = 0.f;
+  double qk_inv_freq[64] = {};  // theta^(-2i / rotary_dim), i < rotary_dim / 2
   // Chunk length of the tensor-core path: 64, 128 or 256 (the 128-token tile is fixed).
   int32_t chunk = 128;
   // Failure injection for tests (host-side switch, see la_api.cu): the segment index whose scan

@@ -111,10 +111,12 @@ __global__ void __launch_bounds__(kQkThreads, 2) qk_norm_rope_kernel(const QkNor
     constexpr double kTwoPi = 6.283185307179586476925286766559;
     constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
     for (int f = lane; f < half; f += 32) {
-      double ang = static_cast<double>(pos) * a.inv_freq[f];
-      ang -= kTwoPi * rint(ang * kInvTwoPi);
+      // explicit roundings (no contraction left to the compiler), so that the prefill kernel's
+      // in-tile form of this operator reproduces the angles bit for bit
+      const double a0 = __dmul_rn(static_cast<double>(pos), a.inv_freq[f]);
       float sn, cs;
-      __sincosf(static_cast<float>(ang), &sn, &cs);
+      __sincosf(static_cast<float>(__fma_rn(-kTwoPi, rint(__dmul_rn(a0, kInvTwoPi)), a0)), &sn,
+                &cs);
       cs_sh[warp][f] = cs;
       sn_sh[warp][f] = sn;
     }

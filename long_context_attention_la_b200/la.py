@@ -64,6 +64,12 @@ class la_qk_norm_rope_desc(ctypes.Structure):  # noqa: N801 - mirrors the C type
                 ("pad", ctypes.c_int32)]
 
 
+class la_qk_prologue(ctypes.Structure):  # noqa: N801 - mirrors the C type name
+    _fields_ = [("gamma_q", ctypes.c_void_p), ("gamma_k", ctypes.c_void_p),
+                ("positions", ctypes.c_void_p), ("rotary_dim", ctypes.c_int32),
+                ("theta", ctypes.c_float), ("eps", ctypes.c_float), ("pad", ctypes.c_int32)]
+
+
 class LaError(RuntimeError):
     def __init__(self, status: int, what: str = ""):
         self.status = status
@@ -109,6 +115,10 @@ def library(path: str | None = None):
         lib.la_prefill_varlen.argtypes = [ctypes.POINTER(la_varlen_desc), vp, vp, vp, vp, vp, vp,
                                           ctypes.POINTER(la_gate_norm), vp, vp, vp, sz, vp]
         lib.la_prefill_varlen.restype = ctypes.c_int
+        lib.la_prefill_varlen_qk.argtypes = [ctypes.POINTER(la_varlen_desc),
+                                             ctypes.POINTER(la_qk_prologue), vp, vp, vp, vp, vp,
+                                             vp, vp, vp, vp, sz, vp]
+        lib.la_prefill_varlen_qk.restype = ctypes.c_int
         lib.la_qk_norm_rope.argtypes = [ctypes.POINTER(la_qk_norm_rope_desc), vp, vp, vp, vp, vp,
                                         vp, vp, vp]
         lib.la_qk_norm_rope.restype = ctypes.c_int
@@ -176,6 +186,18 @@ def la_prefill_varlen(desc: la_varlen_desc, q: int, k: int, v: int, slopes: int,
                                            None if epilogue is None else ctypes.byref(epilogue),
                                            out, state_out or None, workspace or None,
                                            workspace_bytes, stream or None))
+
+
+def la_prefill_varlen_qk(desc: la_varlen_desc, qk: la_qk_prologue | None, q: int, k: int, v: int,
+                         slopes: int, cu_seqlens: int, state_in: int, out: int, state_out: int,
+                         workspace: int, workspace_bytes: int, stream: int) -> int:
+    """la_prefill_varlen with the QK norm + RoPE applied inside the kernel (qk: la_qk_prologue)."""
+    return int(library().la_prefill_varlen_qk(ctypes.byref(desc),
+                                              None if qk is None else ctypes.byref(qk),
+                                              q or None, k or None, v or None, slopes or None,
+                                              cu_seqlens or None, state_in or None, out or None,
+                                              state_out or None, workspace or None,
+                                              workspace_bytes, stream or None))
 
 
 def la_qk_norm_rope(desc: la_qk_norm_rope_desc, q: int, k: int, gamma_q: int, gamma_k: int,
@@ -295,24 +317,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Ten
     return out, state_out
 
 
-def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor,
-                   cu_seqlens, *, state_in: torch.Tensor | None = None,
-                   gate: torch.Tensor | None = None, gamma: torch.Tensor | None = None,
-                   eps: float = 1e-6,
-                   out: torch.Tensor | None = None, state_out: torch.Tensor | None = None,
-                   want_state: bool = True, chunk: int = 0, segments: int = 0,
-                   path: int = LA_PATH_AUTO, workspace: torch.Tensor | None = None,
-                   stream: torch.cuda.Stream | None = None, check: bool | None = None):
-    """o, state = prefill_varlen(q, k, v, slopes, cu_seqlens): q, k, v [T, H, d] hold n_seqs
-    sequences back to back, sequence s at tokens [cu_seqlens[s], cu_seqlens[s+1]).  cu_seqlens is
-    a CUDA int64 tensor of n_seqs + 1 entries (a host list or array is copied to the device
-    first).  state_in: optional fp32 [n_seqs, H, d, d] initial states (state_out may be the same
-    tensor).  gate [T, H, d] bf16 and gamma fp32 [H, d] switch on the fused grouped RMSNorm +
-    sigmoid gate, so out holds gamma * o / rms(o) * sigmoid(gate) per head (FP8 output is
-    gate_norm's, the stand-alone operator).
-    Returns out [T, H, d] and the final fp32 states [n_seqs, H, d, d].  An invalid
-    cu_seqlens is reported by the device: check la_workspace_status(workspace) when it is not
-    known to be valid."""
+def _varlen_operands(q, k, v, slopes, cu_seqlens, state_in, out, state_out, want_state):
+    """Checks of the packed operands; returns cu_seqlens on the device, out and state_out."""
     if q.dim() != 3 or q.shape != k.shape or q.shape != v.shape:
         raise ValueError("q, k, v must share one [T, H, d] shape")
     if q.dtype not in _DT or k.dtype != q.dtype or v.dtype != q.dtype:
@@ -334,6 +340,31 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: to
         out = torch.empty_like(q)
     if state_out is None and want_state:
         state_out = torch.empty((n, H, d, d), dtype=torch.float32, device=q.device)
+    return cu_seqlens, out, state_out
+
+
+def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor,
+                   cu_seqlens, *, state_in: torch.Tensor | None = None,
+                   gate: torch.Tensor | None = None, gamma: torch.Tensor | None = None,
+                   eps: float = 1e-6,
+                   out: torch.Tensor | None = None, state_out: torch.Tensor | None = None,
+                   want_state: bool = True, chunk: int = 0, segments: int = 0,
+                   path: int = LA_PATH_AUTO, workspace: torch.Tensor | None = None,
+                   stream: torch.cuda.Stream | None = None, check: bool | None = None):
+    """o, state = prefill_varlen(q, k, v, slopes, cu_seqlens): q, k, v [T, H, d] hold n_seqs
+    sequences back to back, sequence s at tokens [cu_seqlens[s], cu_seqlens[s+1]).  cu_seqlens is
+    a CUDA int64 tensor of n_seqs + 1 entries (a host list or array is copied to the device
+    first).  state_in: optional fp32 [n_seqs, H, d, d] initial states (state_out may be the same
+    tensor).  gate [T, H, d] bf16 and gamma fp32 [H, d] switch on the fused grouped RMSNorm +
+    sigmoid gate, so out holds gamma * o / rms(o) * sigmoid(gate) per head (FP8 output is
+    gate_norm's, the stand-alone operator).
+    Returns out [T, H, d] and the final fp32 states [n_seqs, H, d, d].  An invalid
+    cu_seqlens is reported by the device: check la_workspace_status(workspace) when it is not
+    known to be valid."""
+    cu_seqlens, out, state_out = _varlen_operands(q, k, v, slopes, cu_seqlens, state_in, out,
+                                                  state_out, want_state)
+    T, H, d = q.shape
+    n = cu_seqlens.numel() - 1
     epi = None
     if gate is not None or gamma is not None:
         if gate is None or gamma is None:
@@ -359,6 +390,49 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: to
     if st != LA_OK:
         raise LaError(st, "la_prefill_varlen")
     _check_device_status(ws_ptr, s.cuda_stream, "la_prefill_varlen", check)
+    return out, state_out
+
+
+def prefill_varlen_qk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor,
+                      cu_seqlens, gamma_q: torch.Tensor, gamma_k: torch.Tensor,
+                      positions: torch.Tensor, *, rotary_dim: int = 64, theta: float = 6.0e6,
+                      eps: float = 1e-6, state_in: torch.Tensor | None = None,
+                      out: torch.Tensor | None = None, state_out: torch.Tensor | None = None,
+                      want_state: bool = True, segments: int = 0,
+                      workspace: torch.Tensor | None = None,
+                      stream: torch.cuda.Stream | None = None, check: bool | None = None):
+    """o, state = prefill_varlen_qk(q, k, v, slopes, cu_seqlens, gamma_q, gamma_k, positions):
+    prefill_varlen of the raw q and k projections, with qk_norm_rope (gamma_* fp32 [d],
+    positions int64 [T], rotary_dim, theta, eps) applied inside the kernel to each tile before
+    use.  bf16, d = 128, tensor-core path, 128-token chunks.  Equals qk_norm_rope followed by
+    prefill_varlen exactly."""
+    cu_seqlens, out, state_out = _varlen_operands(q, k, v, slopes, cu_seqlens, state_in, out,
+                                                  state_out, want_state)
+    T, H, d = q.shape
+    n = cu_seqlens.numel() - 1
+    if positions.dtype != torch.int64 or tuple(positions.shape) != (T,):
+        raise ValueError("positions must be int64 [T]")
+    for name, g in (("gamma_q", gamma_q), ("gamma_k", gamma_k)):
+        if g.dtype != torch.float32 or tuple(g.shape) != (d,):
+            raise ValueError(f"{name} must be float32 [d]")
+    qk = la_qk_prologue(_cuda_ptr(gamma_q, "gamma_q"), _cuda_ptr(gamma_k, "gamma_k"),
+                        _cuda_ptr(positions, "positions"), rotary_dim, theta, eps, 0)
+    desc = la_varlen_desc(T, n, H, d, _DT[q.dtype], 0, segments, LA_PATH_AUTO)
+    need = la_prefill_varlen_workspace_bytes(desc)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = 0 if workspace is None else _cuda_ptr(workspace, "workspace")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    st = la_prefill_varlen_qk(desc, qk, _cuda_ptr(q, "q"), _cuda_ptr(k, "k"), _cuda_ptr(v, "v"),
+                              _cuda_ptr(slopes, "slopes"), _cuda_ptr(cu_seqlens, "cu_seqlens"),
+                              0 if state_in is None else _cuda_ptr(state_in, "state_in"),
+                              _cuda_ptr(out, "out"),
+                              0 if state_out is None else _cuda_ptr(state_out, "state_out"),
+                              ws_ptr, ws_bytes, s.cuda_stream)
+    if st != LA_OK:
+        raise LaError(st, "la_prefill_varlen_qk")
+    _check_device_status(ws_ptr, s.cuda_stream, "la_prefill_varlen_qk", check)
     return out, state_out
 
 

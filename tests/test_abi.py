@@ -51,7 +51,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert la.la_version() == 1003
+    assert la.la_version() == 1004
     for code in range(-10, 1):
         assert la.la_status_string(code) not in ("", "unknown status")
     assert la.la_status_string(-99) == "unknown status"
@@ -228,6 +228,43 @@ def test_varlen_epilogue_checks(lib):
     assert call(d, la.la_gate_norm(0x800000, 0x900000, 1e-6), out=0x800000 + 64) == la.LA_ERR_ALIAS
     # FP8 output is the stand-alone operator's, not this epilogue's
     assert call(d, la.la_gate_norm(0x800000, 0x900000, 1e-6, 0xA00000)) == la.LA_ERR_UNSUPPORTED
+
+
+def test_varlen_qk_prologue_checks(lib):
+    """la_prefill_varlen_qk: the in-tile QK norm + RoPE has one kernel instance (bf16, d = 128,
+    tensor path, 128-token chunks); its parameters are checked like la_qk_norm_rope's."""
+    ok = dict(gamma_q=0x800000, gamma_k=0x900000, positions=0xA00000, rotary_dim=64, theta=6e6,
+              eps=1e-6, pad=0)
+
+    def call(desc=None, out=0x50000, **kw):
+        qk = la.la_qk_prologue(**{**ok, **kw})
+        return la.la_prefill_varlen_qk(desc or _vdesc(), qk, *_P, _CU, 0, out, 0, 0, 0, 0)
+
+    assert la.la_prefill_varlen_qk(_vdesc(), None, *_P, _CU, 0, 0x50000, 0, 0, 0,
+                                   0) == la.LA_ERR_NULL
+    # descriptor errors first, as for la_prefill_varlen
+    assert call(_vdesc(d=32)) == la.LA_ERR_SHAPE
+    assert call(_vdesc(dtype=9)) == la.LA_ERR_DTYPE
+    # only the bf16, d = 128, C = 128 tensor-core instance carries it
+    assert call(_vdesc(dtype=la.LA_F32)) == la.LA_ERR_UNSUPPORTED
+    assert call(_vdesc(d=64)) == la.LA_ERR_UNSUPPORTED
+    assert call(_vdesc(path=la.LA_PATH_RECURRENT)) == la.LA_ERR_UNSUPPORTED
+    for chunk in (64, 256):
+        assert call(_vdesc(chunk=chunk)) == la.LA_ERR_UNSUPPORTED
+    assert call(gamma_q=0) == la.LA_ERR_NULL
+    assert call(gamma_k=0) == la.LA_ERR_NULL
+    assert call(positions=0) == la.LA_ERR_NULL
+    assert call(gamma_q=0x800004) == la.LA_ERR_ALIGN
+    assert call(gamma_k=0x900008) == la.LA_ERR_ALIGN
+    assert call(positions=0xA00004) == la.LA_ERR_ALIGN
+    for r in (0, 8, 24, 144):
+        assert call(rotary_dim=r) == la.LA_ERR_SHAPE
+    for theta in (0.0, -1.0, float("nan"), float("inf")):
+        assert call(theta=theta) == la.LA_ERR_SHAPE
+    for eps in (-1e-6, float("nan")):
+        assert call(eps=eps) == la.LA_ERR_SHAPE
+    # q, k, v are only read: out must still not overlap them
+    assert call(out=0x1000 + 64) == la.LA_ERR_ALIAS
 
 
 # ---------------------------------------------------------------------------------------------
