@@ -377,6 +377,11 @@ typedef struct {
  *   q, k, v     [T, H, d] bf16 device (contiguous), read only: q and k are not modified
  *   other arguments, the workspace (la_prefill_varlen_workspace_bytes) and the errors as for
  *   la_prefill_varlen; there is no fused output epilogue here (out receives o).
+ *
+ * Speed: the transform runs on four warps between a tile's arrival and its first product, so
+ * this call is currently slower than la_qk_norm_rope (which may write q_hat, k_hat in place over
+ * q, k) followed by la_prefill_varlen.  It is for callers whose q and k must stay as they are and
+ * who cannot hold a second copy of them.
  */
 la_status la_prefill_varlen_qk(const la_varlen_desc* desc, const la_qk_prologue* qk,
                                const void* q, const void* k, const void* v, const float* slopes,
